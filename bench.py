@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Masked MoE-layer throughput of the BEAM layer on B200, with roofline and CPU-oracle baselines.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one forward of the whole layer (router, Top-K/softmax/mask, compaction, kept experts,
+shared experts, combine) over one synthetic token batch resident in HBM.  N > 1 runs N
+independent replicas (one per GPU, launched with torchrun), each on its own batch: the layer
+has no cross-token exchange, so there is no collective on the data path (weak scaling).
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# name -> (layer spec, tokens, keep rate; None = mask off / plain Top-K)
+WORKLOADS = {
+    "mixtral-prefill": ("mixtral", 4096, 0.5),
+    "mixtral-prefill-high": ("mixtral", 4096, 0.25),
+    "mixtral-decode1": ("mixtral", 1, 0.5),
+    "mixtral-decode8": ("mixtral", 8, 0.5),
+    "mixtral-decode64": ("mixtral", 64, 0.5),
+    "dsv2lite-prefill": ("dsv2lite", 8192, 0.45),
+    "dsv2lite-decode1": ("dsv2lite", 1, 0.07),
+    "dsv2lite-decode64": ("dsv2lite", 64, 0.45),
+    "qwenmoe-prefill": ("qwenmoe", 16384, 0.5),
+    "fine-prefill": ("fine", 8192, 0.25),
+    "fine-decode32": ("fine", 32, 0.5),
+    "tiny": ("tiny", 64, 0.5),
+}
+DEFAULT_WORKLOAD = "mixtral-prefill"
+# supplementary points measured after the headline in the default run
+EXTRA_POINTS = ["mixtral-decode1", "mixtral-decode8", "mixtral-decode64"]
+
+
+# ------------------------------------------------------------------ environment helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), tc=float(d["bf16_tflops"]),
+                    tc_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm=FALLBACK_HBM_GBS, tc=FALLBACK_BF16_TFLOPS,
+                    tc_sustained=FALLBACK_BF16_TFLOPS, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dynamic_expert_routing_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from a committed ncu summary, if it still matches the
+    current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    rec = d.get(workload, {}).get(kernel)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of the SM clock and throttle reasons of one GPU."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu_id], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        try:
+            rows = [l.split(",") for l in open(self.path).read().strip().splitlines()]
+        except Exception:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(dev)
+
+
+# ------------------------------------------------------------------ algorithmic work
+def layer_work(spec, T, st):
+    """Algorithmic bytes and FLOPs of one forward (what the method must move / compute)."""
+    D, E, K, F = spec.d_model, spec.n_experts, spec.top_k, spec.d_ff
+    es = 4 if spec.storage == "fp32" else 2
+    Fsh = spec.n_shared * spec.d_ff_shared
+    na, nk = st["n_active_experts"], st["n_kept"]
+    Tr = math.ceil(T / spec.segment_len) if spec.segment_len > 1 else T
+    w = {}
+    w["router_logits"] = dict(bytes=2 * E * D * es + Tr * D * es + Tr * 2 * E * 4,
+                              flops=2 * Tr * D * 2 * E)
+    gu_bytes = (na * 2 * F * D + 2 * Fsh * D) * es + (nk + (T if Fsh else 0)) * D * es \
+        + (nk * F + T * Fsh) * es
+    gu_flops = 2 * (nk * 2 * F * D + T * 2 * Fsh * D)
+    dn_bytes = (na * D * F + D * Fsh) * es + (nk * F + T * Fsh) * es + (nk + (T if Fsh else 0)) * D * 4
+    dn_flops = 2 * (nk * F * D + T * Fsh * D)
+    for s in ("stream_gateup", "tc_gateup"):
+        w[s] = dict(bytes=gu_bytes, flops=gu_flops)
+    for s in ("stream_down", "tc_down"):
+        w[s] = dict(bytes=dn_bytes, flops=dn_flops)
+    w["combine"] = dict(bytes=nk * D * 4 + (T * D * 4 if Fsh else 0) + T * D * 4 + T * K * 8,
+                        flops=2 * nk * D)
+    w["scatter_gather"] = dict(bytes=2 * nk * D * es + T * K * 12, flops=0)
+    total_bytes = (na * 3 * F * D + 3 * Fsh * D + 2 * E * D) * es + T * D * es + T * D * 4
+    total_flops = 2 * (nk * 3 * F * D + T * 3 * Fsh * D + Tr * D * 2 * E)
+    return w, dict(bytes=total_bytes, flops=total_flops)
+
+
+TENSOR_STAGES = {"tc_gateup", "tc_down", "tc_router"}
+
+
+def roofline_for(stage, work, ms_per_launch, peaks, workload):
+    if stage in TENSOR_STAGES:
+        achieved = work["flops"] / (ms_per_launch * 1e-3) / 1e12
+        peak = peaks["tc_sustained"]
+        out = dict(bound="tensor", achieved=round(achieved, 2), peak=peak, unit="TFLOP/s")
+    else:
+        achieved = work["bytes"] / (ms_per_launch * 1e-3) / 1e9
+        peak = peaks["hbm"]
+        out = dict(bound="hbm", achieved=round(achieved, 1), peak=peak, unit="GB/s")
+    out["frac"] = round(achieved / peak, 4)
+    out["traffic"] = recorded_traffic(stage, workload)
+    out["kernel"] = stage
+    out["ms_per_launch"] = round(ms_per_launch, 5)
+    out["algorithmic_bytes"] = int(work["bytes"])
+    out["algorithmic_flops"] = int(work["flops"])
+    out["peak_source"] = peaks["source"] + (" (sustained bf16)" if stage in TENSOR_STAGES else "")
+    return out
+
+
+# ------------------------------------------------------------------ our arm
+def build_layer(torch, name, device, seed=0):
+    import synth
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec_name, T, keep = WORKLOADS[name]
+    spec = synth.SPECS[spec_name]
+    w = synth.make_layer(spec, seed=seed, keep_rate=keep if keep else 0.5, device=device)
+    wd = {k: v for k, v in w.items() if isinstance(v, torch.Tensor)}
+    layer = BeamMoE(wd, spec.top_k, max_tokens=T, segment_len=spec.segment_len)
+    x = synth.make_tokens(spec, T, seed=seed, device=device)
+    del w, wd
+    torch.cuda.empty_cache()
+    return spec, T, keep, layer, x
+
+
+def time_steps(torch, dist, layer, x, y, steps, warmup, mask_off, world):
+    for _ in range(warmup):
+        layer.forward(x, mask_off=mask_off, out=y)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    st = torch.cuda.current_stream()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    n0 = layer.launch_count()
+    a.record(st)
+    for _ in range(steps):
+        layer.forward(x, mask_off=mask_off, out=y)
+    b.record(st)
+    torch.cuda.synchronize()
+    launches = layer.launch_count() - n0
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, launches
+
+
+def point(torch, dist, name, steps, warmup, world, device, peaks, mask_off=False):
+    """Measure one supplementary point (tokens/s, roofline of its dominant kernel)."""
+    spec, T, keep, layer, x = build_layer(torch, name, device)
+    y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
+    mo = mask_off or keep is None
+    ms, _ = time_steps(torch, dist, layer, x, y, steps, warmup, mo, world)
+    st = layer.stats()
+    layer.profile_begin(steps)
+    for _ in range(steps):
+        layer.forward(x, mask_off=mo, out=y)
+    prof = layer.profile_end()
+    work, total = layer_work(spec, T, st)
+    stage = max((k for k in prof if k != "forwards"), key=lambda k: prof[k][0])
+    rl = roofline_for(stage, work.get(stage, dict(bytes=0, flops=0)),
+                      prof[stage][0] / prof[stage][1], peaks, name)
+    t_roof = max(total["bytes"] / (peaks["hbm"] * 1e9), total["flops"] / (peaks["tc"] * 1e12))
+    layer.close()
+    return dict(workload=name, tokens=T, keep_rate=keep, mask="off" if mo else "on",
+                value=round(T * world / (ms * 1e-3), 2), ms_per_step=round(ms, 5),
+                avg_k=round(st["avg_k"], 4), n_active_experts=st["n_active_experts"],
+                layer_roofline_frac=round(t_roof / (ms * 1e-3), 4), roofline=rl)
+
+
+def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_steps=None):
+    """Time the fp64 oracle on a bounded sample of the workload (tokens/s on host cores)."""
+    import numpy as np
+    import torch
+    import oracle
+    w = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in weights_dev.items()}
+    x = x_dev.cpu()
+    # probe the cost of one token, then size the sample to the budget
+    t0 = time.perf_counter()
+    r1 = oracle.route(x[:1], w["w_router"], w["w_mask"], spec.top_k,
+                      segment_len=spec.segment_len, mask_off=keep is None)
+    oracle.layer(x[:1], w, r1)
+    per_tok = max(time.perf_counter() - t0, 1e-4)
+    threads = oracle.num_threads()
+    n = int(max(1, min(T, budget_s * threads / per_tok)))
+    stride = max(1, T // n)
+    sel = np.arange(0, T, stride, dtype=np.int32)[:n]
+    t0 = time.perf_counter()
+    xs = x[torch.from_numpy(sel).long()]
+    r = oracle.route(xs, w["w_router"], w["w_mask"], spec.top_k, mask_off=keep is None)
+    oracle.layer(xs, w, r)
+    dt = time.perf_counter() - t0
+    return dict(value=round(len(sel) / dt, 4), unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"{len(sel)} of {T} tokens (every {stride}th), routing + experts, fp64")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+
+    name = args.workload
+    spec, T, keep, layer, x = build_layer(torch, name, device)
+    y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
+    mask_off = keep is None
+    sampler = ClockSampler(gpu_uuid(torch, device))
+    with sampler:
+        ms, launches = time_steps(torch, dist, layer, x, y, args.steps, args.warmup, mask_off, world)
+    clocks = sampler.summary()
+    st = layer.stats()
+    # per-kernel timing pass (same K steps, events around every kernel)
+    layer.profile_begin(args.steps)
+    for _ in range(args.steps):
+        layer.forward(x, mask_off=mask_off, out=y)
+    prof = layer.profile_end()
+    work, total = layer_work(spec, T, st)
+    stages = {k: v for k, v in prof.items() if k != "forwards"}
+    tot_ms = sum(v[0] for v in stages.values())
+    dom = max(stages, key=lambda k: stages[k][0])
+    rl = roofline_for(dom, work.get(dom, dict(bytes=0, flops=0)), stages[dom][0] / stages[dom][1],
+                      peaks, name)
+    rl["share"] = round(stages[dom][0] / tot_ms, 4)
+    t_roof = max(total["bytes"] / (peaks["hbm"] * 1e9), total["flops"] / (peaks["tc"] * 1e12))
+
+    # end to end through the host-buffer entry point (pinned memory, copies inside the region)
+    es = 2 if spec.storage == "bf16" else 4
+    xh = x.cpu().pin_memory()
+    yh = torch.empty((T, spec.d_model), dtype=torch.float32).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        layer.forward_host(xh, yh, mask_off=mask_off)
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps // 2)
+    a.record()
+    for _ in range(e2e_steps):
+        layer.forward_host(xh, yh, mask_off=mask_off)
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # mask off through the same library at the headline shape: the layer speedup from skipping
+    y.zero_()
+    ms_off, _ = time_steps(torch, dist, layer, x, y, args.steps, args.warmup, True, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import synth
+        wcpu = synth.make_layer(spec, seed=0, keep_rate=keep if keep else 0.5, device=device)
+        cpu = cpu_baseline(spec, T, keep, wcpu, x, budget_s=args.cpu_budget)
+        del wcpu
+    layer.close()
+    del layer, x, y
+    torch.cuda.empty_cache()
+
+    points = []
+    if not args.no_points:
+        for p in EXTRA_POINTS:
+            if p == name:
+                continue
+            points.append(point(torch, dist, p, max(10, args.steps), args.warmup, world, device, peaks))
+
+    if rank == 0:
+        line = {
+            "metric": "masked MoE-layer tokens/s",
+            "value": round(T * world / (ms * 1e-3), 2),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if spec.storage == "bf16" else "f32",
+            "data": "synthetic (seeded; random-init weights of the layer shape)",
+            "config": {
+                "workload": f"{spec.name}-like layer, {'prefill' if T > 64 else 'decode'} T={T}, "
+                            f"keep rate {keep if keep else 1.0}",
+                "d_model": spec.d_model, "n_experts": spec.n_experts, "top_k": spec.top_k,
+                "d_ff": spec.d_ff, "n_shared": spec.n_shared, "d_ff_shared": spec.d_ff_shared,
+                "tokens_per_gpu": T, "keep_rate": keep, "mask": "off" if mask_off else "on",
+                "avg_k": round(st["avg_k"], 4), "n_active_experts": st["n_active_experts"],
+                "l2": "expert weights exceed the 126 MB L2; no flush between steps",
+                "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
+            },
+            "roofline": rl,
+            "layer_roofline_frac": round(t_roof / (ms * 1e-3), 4),
+            "mask_off": {"value": round(T * world / (ms_off * 1e-3), 2),
+                         "ms_per_step": round(ms_off, 5),
+                         "layer_speedup_from_mask": round(ms_off / ms, 4)},
+            "stage_ms_per_forward": {k: round(v[0] / prof["forwards"], 5) for k, v in stages.items()},
+            "e2e": {"value": round(T * world / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * spec.d_model * es,
+                    "d2h_bytes_per_step": T * spec.d_model * 4},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "points": points,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    spec_name, T, keep = WORKLOADS[args.workload]
+    spec = synth.SPECS[spec_name]
+    oracle.build()
+    w = synth.make_layer(spec, seed=0, keep_rate=keep if keep else 0.5,
+                         device="cuda" if torch.cuda.is_available() else "cpu")
+    w = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in w.items()}
+    x = synth.make_tokens(spec, T, seed=0, device="cuda" if torch.cuda.is_available() else "cpu").cpu()
+    threads = oracle.num_threads()
+    # one step = the oracle on a fixed sample of tokens of the batch, end to end
+    t0 = time.perf_counter()
+    r1 = oracle.route(x[:1], w["w_router"], w["w_mask"], spec.top_k, mask_off=keep is None)
+    oracle.layer(x[:1], w, r1)
+    per_tok = max(time.perf_counter() - t0, 1e-4) / threads
+    budget = 150.0 / (args.steps + args.warmup)
+    n = int(max(1, min(T, budget / per_tok)))
+    stride = max(1, T // n)
+    sel = torch.from_numpy(np.arange(0, T, stride)[:n]).long()
+    xs = x[sel]
+
+    def step():
+        r = oracle.route(xs, w["w_router"], w["w_mask"], spec.top_k,
+                         segment_len=0, mask_off=keep is None)
+        oracle.layer(xs, w, r)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = round(len(sel) / dt, 4)
+    line = {
+        "impl": "reference",
+        "metric": "masked MoE-layer tokens/s",
+        "value": value, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; random-init weights of the layer shape)",
+        "config": {"workload": f"{spec.name}-like layer, T={T}, keep rate {keep}",
+                   "d_model": spec.d_model, "n_experts": spec.n_experts, "top_k": spec.top_k,
+                   "d_ff": spec.d_ff, "tokens_per_gpu": T, "keep_rate": keep},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{len(sel)} of {T} tokens per step (every {stride}th), "
+                                   "routing + experts, fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-points", action="store_true", help="skip the supplementary points")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

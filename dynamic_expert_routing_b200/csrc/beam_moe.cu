@@ -1,0 +1,719 @@
+// beam_moe.cu -- C ABI and host orchestration of the BEAM masked MoE-layer forward (sm_100a).
+//
+// One handle owns the repacked weights and every workspace buffer, sized at create time for
+// max_tokens, so the forward allocates nothing and never synchronises with the host: the
+// per-expert token counts are produced and consumed on the device.  Kernels are chained with
+// programmatic dependent launch (each waits on griddepcontrol before reading its producer's
+// output), so a kernel's launch overlaps the tail of the one before it.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/beam_moe.h"
+#include "common.cuh"
+#include "router.cuh"
+#include "compact.cuh"
+#include "stream_experts.cuh"
+#include "tc_experts.cuh"
+
+using namespace beam;
+
+// ---------------------------------------------------------------- errors
+static thread_local char g_err[512] = "";
+
+static beam_status_t fail(beam_status_t st, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+#define BEAM_CUDA(call)                                                                   \
+    do {                                                                                  \
+        cudaError_t e_ = (call);                                                          \
+        if (e_ != cudaSuccess)                                                            \
+            return fail(BEAM_ERR_CUDA, "%s failed: %s (%s:%d)", #call,                    \
+                        cudaGetErrorString(e_), __FILE__, __LINE__);                      \
+    } while (0)
+
+// ---------------------------------------------------------------- repack kernels
+// Wrm [n2E_pad][D]: row j < E is column j of W_r, row E + j is column j of W_m, rest zero.
+template <typename T>
+__global__ void repack_router_kernel(const T* __restrict__ wr, const T* __restrict__ wm, int D,
+                                     int E, int n2E_pad, T* __restrict__ out)
+{
+    const size_t n = (size_t)n2E_pad * D;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const int j = (int)(i / D), d = (int)(i % D);
+        T v = from_float<T>(0.f);
+        if (j < E) v = wr[(size_t)d * E + j];
+        else if (j < 2 * E) v = wm[(size_t)d * E + (j - E)];
+        out[i] = v;
+    }
+}
+
+// Gate/up interleaving in blocks of 128 rows: out[e][b][0][r][:] = wg[e][128b + r][:],
+// out[e][b][1][r][:] = wu[e][128b + r][:].  One block of 128 threads per output row.
+template <typename T>
+__global__ void repack_gateup_kernel(const T* __restrict__ wg, const T* __restrict__ wu, int nE,
+                                     int F, int D, T* __restrict__ out)
+{
+    const long long row = blockIdx.x;  // output row in [nE][F/128][2][128]
+    const long long nrows = (long long)nE * 2 * F;
+    if (row >= nrows) return;
+    const int r = (int)(row % 128);
+    const int half = (int)((row / 128) % 2);
+    const long long b = row / 256;       // global 128-row block index (e * F/128 + block)
+    const long long src_row = b * 128 + r;  // row of [nE*F][D]
+    const uint4* s = reinterpret_cast<const uint4*>((half ? wu : wg) + src_row * D);
+    uint4* d = reinterpret_cast<uint4*>(out + row * D);
+    const int nv = D * (int)sizeof(T) / 16;
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) d[v] = s[v];
+}
+
+// Down projection into the type of H (fp16 for bf16 layers: exact for every bf16 value of
+// magnitude >= 2^-14, within 2^-25 absolute below it; a magnitude >= 65504 sets *bad).
+// Routed: out[e][j][f] = w[e][j][f] (S = 1, Fs = F, n = E*D*F).  Shared concatenation:
+// out[j][s*Fs + f] = w[s][j][f].
+template <typename TI, typename TO>
+__global__ void repack_down_kernel(const TI* __restrict__ w, long long n, int S, int D, int Fs,
+                                   int concat, TO* __restrict__ out, int* __restrict__ bad)
+{
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float v = to_float(w[i]);
+        if (!(fabsf(v) < 65504.f) && sizeof(TO) == 2) atomicOr(bad, 1);
+        long long o = i;
+        if (concat) {
+            const long long f = i % Fs;
+            const long long j = (i / Fs) % D;
+            const long long s = i / ((long long)Fs * D);
+            o = j * S * Fs + s * Fs + f;
+        }
+        out[o] = from_float<TO>(v);
+    }
+}
+
+// ---------------------------------------------------------------- the handle
+struct beam_moe {
+    beam_moe_config_t cfg;
+    int E, K, D, F, Fsh, Tmax, S;
+    int n2E;
+    size_t esz;
+    int num_sms;
+    int max_nch;
+    // repacked weights
+    void *wrm = nullptr, *wgu = nullptr, *wd = nullptr, *wsgu = nullptr, *wsd = nullptr;
+    // routing workspace
+    float* L = nullptr;
+    int* topk_id = nullptr;
+    float *gate = nullptr, *mlogit = nullptr, *ghat = nullptr;
+    uint8_t* keep = nullptr;
+    int* nkeep_tok = nullptr;
+    float* lreg_tok = nullptr;
+    uint32_t* bits = nullptr;
+    int *chunk_base = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
+    Group* groups = nullptr;
+    int* n_groups = nullptr;
+    DevStats* dstats = nullptr;
+    // expert workspace
+    void *xperm = nullptr, *hbuf = nullptr, *hsh = nullptr;
+    float *yperm = nullptr, *ysh = nullptr;
+    // host-call staging
+    void* x_stage = nullptr;
+    float* y_stage = nullptr;
+    size_t hsz;          // bytes per element of H and of the stored down projections
+    bool tc_ok = false;  // tensor-core expert path available (bf16, D % 256 == 0)
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    tc::TcParams p1, p2;  // GEMM1 / GEMM2 parameters (the x map of GEMM1 is set per forward)
+    int* range_flag = nullptr;
+    cudaEvent_t done = nullptr;
+    int last_T = -1;
+    std::vector<void*> allocs;
+    // launch accounting and optional per-stage timing
+    long long launches = 0;
+    bool prof = false;
+    int prof_max = 0, prof_forwards = 0;
+    std::vector<cudaEvent_t> prof_pool;   // free events
+    struct ProfRec { int stage; cudaEvent_t a, b; };
+    std::vector<ProfRec> prof_recs;
+};
+
+enum Stage {
+    ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
+    ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
+    ST_RESERVED, ST_COUNT
+};
+static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
+static const char* kStageNames[ST_COUNT] = {
+    "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
+    "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router", "reserved"};
+
+static void prof_release(beam_moe* h)
+{
+    for (auto& r : h->prof_recs) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+    h->prof_recs.clear();
+    for (cudaEvent_t e : h->prof_pool) cudaEventDestroy(e);
+    h->prof_pool.clear();
+    h->prof = false;
+}
+
+static void free_all(beam_moe* h)
+{
+    prof_release(h);
+    for (void* p : h->allocs) cudaFree(p);
+    h->allocs.clear();
+    if (h->done) cudaEventDestroy(h->done);
+    h->done = nullptr;
+}
+
+template <typename P>
+static beam_status_t dalloc(beam_moe* h, P** out, size_t bytes)
+{
+    void* p = nullptr;
+    if (bytes == 0) bytes = 16;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(BEAM_ERR_OOM, "cudaMalloc of %zu bytes failed: %s", bytes, cudaGetErrorString(e));
+    }
+    h->allocs.push_back(p);
+    *out = static_cast<P*>(p);
+    return BEAM_OK;
+}
+
+#define BEAM_TRY(x)                              \
+    do {                                         \
+        beam_status_t s_ = (x);                  \
+        if (s_ != BEAM_OK) return s_;            \
+    } while (0)
+
+static beam_status_t validate(const beam_moe_config_t* c)
+{
+    if (!c) return fail(BEAM_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->dtype != BEAM_DTYPE_F32 && c->dtype != BEAM_DTYPE_BF16)
+        return fail(BEAM_ERR_INVALID_ARG, "dtype must be BEAM_DTYPE_F32 or BEAM_DTYPE_BF16");
+    const int dmul = c->dtype == BEAM_DTYPE_BF16 ? 64 : 4;
+    const int dmax = c->dtype == BEAM_DTYPE_BF16 ? 8192 : 4096;
+    if (c->d_model <= 0 || c->d_model % dmul || c->d_model > dmax)
+        return fail(BEAM_ERR_INVALID_ARG, "d_model=%d must be a positive multiple of %d, <= %d",
+                    c->d_model, dmul, dmax);
+    if (c->n_experts < 1 || c->n_experts > kMaxE)
+        return fail(BEAM_ERR_INVALID_ARG, "n_experts=%d must be in [1, %d]", c->n_experts, kMaxE);
+    if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > 32)
+        return fail(BEAM_ERR_INVALID_ARG, "top_k=%d must be in [1, min(n_experts, 32)]", c->top_k);
+    if (c->d_ff <= 0 || c->d_ff % 128 || c->d_ff > 65536)
+        return fail(BEAM_ERR_INVALID_ARG, "d_ff=%d must be a positive multiple of 128", c->d_ff);
+    if (c->n_shared < 0 || c->n_shared > 16)
+        return fail(BEAM_ERR_INVALID_ARG, "n_shared=%d must be in [0, 16]", c->n_shared);
+    if (c->n_shared > 0 && (c->d_ff_shared <= 0 || c->d_ff_shared % 128))
+        return fail(BEAM_ERR_INVALID_ARG, "d_ff_shared=%d must be a positive multiple of 128",
+                    c->d_ff_shared);
+    if (c->segment_len < 0 || c->segment_len > 65536)
+        return fail(BEAM_ERR_INVALID_ARG, "segment_len=%d out of range", c->segment_len);
+    if (c->max_tokens < 1 || c->max_tokens > 65536)
+        return fail(BEAM_ERR_INVALID_ARG, "max_tokens=%d must be in [1, 65536]", c->max_tokens);
+    return BEAM_OK;
+}
+
+static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Automatic path choice: up to this many tokens per forward the experts run as
+// weight-streaming GEMVs, above it on the tensor cores.
+constexpr int kStreamMaxTokens = 16;
+
+template <typename T>
+static beam_status_t repack(beam_moe* h, const beam_moe_weights_t* w, cudaStream_t st)
+{
+    using TH = typename HType<T>::type;
+    const int D = h->D, E = h->E, F = h->F;
+    repack_router_kernel<T><<<1024, 256, 0, st>>>(static_cast<const T*>(w->w_router),
+                                                  static_cast<const T*>(w->w_mask), D, E, h->n2E,
+                                                  static_cast<T*>(h->wrm));
+    BEAM_CUDA(cudaGetLastError());
+    repack_gateup_kernel<T><<<(unsigned)((long long)E * 2 * F), 128, 0, st>>>(
+        static_cast<const T*>(w->w_gate), static_cast<const T*>(w->w_up), E, F, D,
+        static_cast<T*>(h->wgu));
+    BEAM_CUDA(cudaGetLastError());
+    repack_down_kernel<T, TH><<<2048, 256, 0, st>>>(static_cast<const T*>(w->w_down),
+                                                    (long long)E * D * F, 1, D, F, 0,
+                                                    static_cast<TH*>(h->wd), h->range_flag);
+    BEAM_CUDA(cudaGetLastError());
+    if (h->Fsh > 0) {
+        repack_gateup_kernel<T><<<(unsigned)(2LL * h->Fsh), 128, 0, st>>>(
+            static_cast<const T*>(w->ws_gate), static_cast<const T*>(w->ws_up), 1, h->Fsh, D,
+            static_cast<T*>(h->wsgu));
+        BEAM_CUDA(cudaGetLastError());
+        repack_down_kernel<T, TH><<<1024, 256, 0, st>>>(
+            static_cast<const T*>(w->ws_down), (long long)h->cfg.n_shared * D * h->cfg.d_ff_shared,
+            h->cfg.n_shared, D, h->cfg.d_ff_shared, 1, static_cast<TH*>(h->wsd), h->range_flag);
+        BEAM_CUDA(cudaGetLastError());
+    }
+    return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- tensor-core path set-up
+static beam_status_t encode_map(beam_moe* h, CUtensorMap* m, CUtensorMapDataType dt,
+                                const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)tc::BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = h->encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(BEAM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a %llu x %llu tensor",
+                    (int)r, (unsigned long long)rows, (unsigned long long)cols);
+    return BEAM_OK;
+}
+
+static beam_status_t setup_tc(beam_moe* h)
+{
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    BEAM_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (!fn || q != cudaDriverEntryPointSuccess)
+        return fail(BEAM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    h->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    const uint64_t D = h->D, E = h->E, F = h->F, Fsh = h->Fsh, Tm = h->Tmax;
+    const uint64_t rows = Tm * h->K;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, HF = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    tc::TcParams& a = h->p1;
+    tc::TcParams& b = h->p2;
+    memset(&a, 0, sizeof a);
+    memset(&b, 0, sizeof b);
+    // GEMM1: X_perm [rows][D] x W_gu [E*2F][D] -> H (fp16) [rows][F]
+    BEAM_TRY(encode_map(h, &a.a_routed, BF, h->xperm, rows, D, tc::BM));
+    BEAM_TRY(encode_map(h, &a.b_routed, BF, h->wgu, E * 2 * F, D, tc::BN));
+    // GEMM2: H [rows][F] x W_d [E*D][F] -> Y_perm (f32) [rows][D]
+    BEAM_TRY(encode_map(h, &b.a_routed, HF, h->hbuf, rows, F, tc::BM));
+    BEAM_TRY(encode_map(h, &b.b_routed, HF, h->wd, E * D, F, tc::BN));
+    if (Fsh) {
+        BEAM_TRY(encode_map(h, &a.b_shared, BF, h->wsgu, 2 * Fsh, D, tc::BN));
+        BEAM_TRY(encode_map(h, &b.a_shared, HF, h->hsh, Tm, Fsh, tc::BM));
+        BEAM_TRY(encode_map(h, &b.b_shared, HF, h->wsd, D, Fsh, tc::BN));
+    } else {
+        a.b_shared = a.b_routed;
+        b.a_shared = b.a_routed;
+        b.b_shared = b.b_routed;
+    }
+    a.a_shared = a.a_routed;  // replaced by the map of x in every forward
+    a.groups = b.groups = h->groups;
+    a.n_groups = b.n_groups = h->n_groups;
+    a.out_routed = h->hbuf; a.ld_routed = (int)F;
+    a.out_shared = h->hsh;  a.ld_shared = (int)Fsh;
+    b.out_routed = h->yperm; b.ld_routed = (int)D;
+    b.out_shared = h->ysh;   b.ld_shared = (int)D;
+    a.b_rows_per_expert = (int)(2 * F);
+    b.b_rows_per_expert = (int)D;
+    a.n_tiles_routed = (int)(2 * F / tc::BN);
+    a.n_tiles_shared = (int)(2 * Fsh / tc::BN);
+    b.n_tiles_routed = b.n_tiles_shared = (int)(D / tc::BN);
+    a.k_steps_routed = a.k_steps_shared = (int)(D / tc::BK);
+    b.k_steps_routed = (int)(F / tc::BK);
+    b.k_steps_shared = (int)(Fsh / tc::BK);
+    a.err = b.err = &h->dstats->err;
+    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+    h->tc_ok = true;
+    return BEAM_OK;
+}
+
+static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_weights_t* w,
+                                 cudaStream_t st, beam_moe* h)
+{
+    h->cfg = *cfg;
+    h->E = cfg->n_experts; h->K = cfg->top_k; h->D = cfg->d_model; h->F = cfg->d_ff;
+    h->Fsh = cfg->n_shared * cfg->d_ff_shared;
+    h->Tmax = cfg->max_tokens;
+    h->S = cfg->segment_len > 1 ? cfg->segment_len : 1;
+    h->n2E = 2 * h->E;
+    h->esz = cfg->dtype == BEAM_DTYPE_BF16 ? 2 : 4;
+    h->hsz = cfg->dtype == BEAM_DTYPE_BF16 ? 2 : 4;
+    h->max_nch = ceil_div(h->Tmax, 32);
+    int dev = 0;
+    BEAM_CUDA(cudaGetDevice(&dev));
+    BEAM_CUDA(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
+
+    const size_t D = h->D, E = h->E, K = h->K, F = h->F, Fsh = h->Fsh, Tm = h->Tmax;
+    const size_t es = h->esz, hs = h->hsz;
+    const size_t rows = Tm * K;  // upper bound on kept pairs
+    BEAM_TRY(dalloc(h, &h->wrm, (size_t)h->n2E * D * es));
+    BEAM_TRY(dalloc(h, &h->wgu, E * 2 * F * D * es));
+    BEAM_TRY(dalloc(h, &h->wd, E * D * F * hs));
+    BEAM_TRY(dalloc(h, &h->range_flag, sizeof(int)));
+    if (Fsh) {
+        BEAM_TRY(dalloc(h, &h->wsgu, 2 * Fsh * D * es));
+        BEAM_TRY(dalloc(h, &h->wsd, D * Fsh * hs));
+        BEAM_TRY(dalloc(h, &h->hsh, Tm * Fsh * hs));
+        BEAM_TRY(dalloc(h, &h->ysh, Tm * D * sizeof(float)));
+    }
+    BEAM_TRY(dalloc(h, &h->L, Tm * h->n2E * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->topk_id, rows * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->gate, rows * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->mlogit, rows * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->ghat, rows * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->keep, rows));
+    BEAM_TRY(dalloc(h, &h->nkeep_tok, Tm * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->lreg_tok, Tm * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->bits, E * h->max_nch * sizeof(uint32_t)));
+    BEAM_TRY(dalloc(h, &h->chunk_base, E * h->max_nch * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->counts, E * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->offsets, (E + 1) * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->perm, rows * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->inv, rows * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->groups, E * sizeof(Group)));
+    BEAM_TRY(dalloc(h, &h->n_groups, sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->dstats, sizeof(DevStats)));
+    BEAM_TRY(dalloc(h, &h->xperm, rows * D * es));
+    BEAM_TRY(dalloc(h, &h->hbuf, rows * F * hs));
+    BEAM_TRY(dalloc(h, &h->yperm, rows * D * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->x_stage, Tm * D * es));
+    BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
+    BEAM_CUDA(cudaMemsetAsync(h->dstats, 0, sizeof(DevStats), st));
+    BEAM_CUDA(cudaMemsetAsync(h->range_flag, 0, sizeof(int), st));
+    BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
+
+    if (cfg->dtype == BEAM_DTYPE_BF16) BEAM_TRY(repack<__nv_bfloat16>(h, w, st));
+    else BEAM_TRY(repack<float>(h, w, st));
+
+    const int smem_gu = kStreamMT * h->D * (int)h->esz;
+    if (cfg->dtype == BEAM_DTYPE_BF16) {
+        BEAM_CUDA(cudaFuncSetAttribute(stream_gateup_kernel<__nv_bfloat16, __half>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_gu));
+        BEAM_CUDA(cudaFuncSetAttribute(stream_down_kernel<__half>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 65536));
+    } else {
+        BEAM_CUDA(cudaFuncSetAttribute(stream_gateup_kernel<float, float>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_gu));
+        BEAM_CUDA(cudaFuncSetAttribute(stream_down_kernel<float>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 65536));
+    }
+    BEAM_CUDA(cudaStreamSynchronize(st));
+    int bad = 0;
+    BEAM_CUDA(cudaMemcpy(&bad, h->range_flag, sizeof bad, cudaMemcpyDeviceToHost));
+    if (bad)
+        return fail(BEAM_ERR_UNSUPPORTED, "a down-projection weight has magnitude >= 65504, "
+                    "outside the fp16 range of the intermediate");
+    if (cfg->dtype == BEAM_DTYPE_BF16 && h->D % tc::BN == 0) BEAM_TRY(setup_tc(h));
+    return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- launch helper (PDL)
+// Every forward kernel goes through here: it is counted, launched with programmatic stream
+// serialisation, and (while profiling) bracketed by an event pair of its stage.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3 grid,
+                          dim3 block, size_t smem, cudaStream_t st, Args&&... args)
+{
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    if (h->prof && h->prof_pool.size() >= 2) {
+        ea = h->prof_pool.back(); h->prof_pool.pop_back();
+        eb = h->prof_pool.back(); h->prof_pool.pop_back();
+        cudaError_t e = cudaEventRecord(ea, st);
+        if (e != cudaSuccess) return e;
+    }
+    ++h->launches;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess && ea) {
+        e = cudaEventRecord(eb, st);
+        h->prof_recs.push_back({stage, ea, eb});
+    }
+    return e;
+}
+
+template <int EPL>
+static cudaError_t launch_select(beam_moe* h, int Tr, int T, int mask_off, cudaStream_t st)
+{
+    return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256), 0, st,
+                  (const float*)h->L, Tr, T, h->E, h->K, h->S, mask_off, h->topk_id, h->gate,
+                  h->mlogit, h->keep, h->ghat, h->nkeep_tok, h->lreg_tok);
+}
+
+template <typename T>
+static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uint32_t flags,
+                                  bool use_tc, cudaStream_t st)
+{
+    const int E = h->E, K = h->K, D = h->D;
+    const int S = h->S;
+    const int Tr = ceil_div(T_, S);
+    const int nch = ceil_div(T_, 32);
+    const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
+
+    // 1. router logits L = x [W_r | W_m]  (routed rows only: segment leaders when S > 1)
+    BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_logits_kernel<T>,
+                     dim3(ceil_div(h->n2E, 8 * kRouterColsPerWarp), ceil_div(Tr, kRouterRows)),
+                     dim3(256), 0, st, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->L));
+    // 2. Top-K, softmax, mask, per-token statistics
+    cudaError_t e;
+    switch ((E + 31) / 32) {
+        case 1: e = launch_select<1>(h, Tr, T_, mask_off, st); break;
+        case 2: e = launch_select<2>(h, Tr, T_, mask_off, st); break;
+        case 3: e = launch_select<3>(h, Tr, T_, mask_off, st); break;
+        case 4: e = launch_select<4>(h, Tr, T_, mask_off, st); break;
+        case 5: e = launch_select<5>(h, Tr, T_, mask_off, st); break;
+        case 6: e = launch_select<6>(h, Tr, T_, mask_off, st); break;
+        case 7: e = launch_select<7>(h, Tr, T_, mask_off, st); break;
+        default: e = launch_select<8>(h, Tr, T_, mask_off, st); break;
+    }
+    BEAM_CUDA(e);
+    // 3. compaction: bit planes, scan (+ statistics), scatter + activation gather
+    BEAM_CUDA(launch(h, ST_COMPACT_BITS, compact_bits_kernel, dim3(ceil_div(nch, 8)), dim3(256), 0, st,
+                     (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, E, nch, h->bits));
+    BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(1), dim3(1024), 0, st, (const uint32_t*)h->bits,
+                     nch, E, T_, (const int*)h->nkeep_tok, (const float*)h->lreg_tok, h->counts,
+                     h->offsets, h->chunk_base, h->groups, h->n_groups, h->dstats));
+    BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>, dim3(ceil_div((long long)T_ * K, 8)),
+                     dim3(256), 0, st, (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D,
+                     nch, (const uint32_t*)h->bits, (const int*)h->offsets,
+                     (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
+    // 4. experts (kept groups only) and shared experts
+    using TH = typename HType<T>::type;
+    if (use_tc) {
+        tc::TcParams& p1 = h->p1;
+        BEAM_TRY(encode_map(h, &p1.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
+                            (uint64_t)D, tc::BM));
+        p1.shared_rows = h->Fsh ? T_ : 0;
+        h->p2.shared_rows = h->Fsh ? T_ : 0;
+        BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1));
+        BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
+    } else {
+        StreamArgs a;
+        a.xperm = h->xperm; a.x = x; a.wgu = h->wgu; a.wsgu = h->wsgu; a.wd = h->wd; a.wsd = h->wsd;
+        a.h = h->hbuf; a.hsh = h->hsh; a.yperm = h->yperm; a.ysh = h->ysh;
+        a.groups = h->groups; a.n_groups = h->n_groups;
+        a.D = D; a.F = h->F; a.Fsh = h->Fsh; a.T = T_;
+        const int grid = h->num_sms * 2;
+        BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(grid), dim3(256),
+                         (size_t)kStreamMT * D * sizeof(T), st, a));
+        BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(grid), dim3(256),
+                         (size_t)65536, st, a));
+    }
+    // 5. fixed-order combine
+    BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel, dim3(T_), dim3(256), 0, st, (const float*)h->yperm,
+                     (const float*)(h->Fsh ? h->ysh : nullptr), (const int*)h->inv,
+                     (const float*)h->ghat, T_, K, D, y));
+    return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- C ABI
+extern "C" {
+
+beam_status_t beam_moe_create(const beam_moe_config_t* cfg, const beam_moe_weights_t* w,
+                              void* stream, beam_moe_t** out)
+{
+    g_err[0] = 0;
+    BEAM_TRY(validate(cfg));
+    if (!w || !out) return fail(BEAM_ERR_INVALID_ARG, "weights or out is NULL");
+    if (!w->w_router || !w->w_mask || !w->w_gate || !w->w_up || !w->w_down)
+        return fail(BEAM_ERR_INVALID_ARG, "a routed weight pointer is NULL");
+    if (cfg->n_shared > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down))
+        return fail(BEAM_ERR_INVALID_ARG, "a shared-expert weight pointer is NULL");
+    beam_moe* h = new (std::nothrow) beam_moe();
+    if (!h) return fail(BEAM_ERR_OOM, "host allocation failed");
+    beam_status_t s = create_impl(cfg, w, static_cast<cudaStream_t>(stream), h);
+    if (s != BEAM_OK) {
+        cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+        free_all(h);
+        delete h;
+        return s;
+    }
+    *out = h;
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y, uint32_t flags,
+                               void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
+    if (T > 0 && (!x || !y)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
+    if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
+    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR))
+        return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
+        return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core expert path needs a bf16 layer with "
+                    "d_model a multiple of 256");
+    if (T > 0 && (reinterpret_cast<uintptr_t>(x) & 15))
+        return fail(BEAM_ERR_INVALID_ARG, "x must be 16-byte aligned");
+    bool use_tc;
+    if (flags & BEAM_PATH_TENSOR) use_tc = true;
+    else if (flags & BEAM_PATH_STREAM) use_tc = false;
+    else use_tc = h->tc_ok && T > kStreamMaxTokens;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
+    if (h->prof) ++h->prof_forwards;
+    if (T > 0) {
+        if (h->cfg.dtype == BEAM_DTYPE_BF16)
+            BEAM_TRY(forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y,
+                                                 flags, use_tc, st));
+        else
+            BEAM_TRY(forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st));
+    }
+    h->last_T = T;
+    BEAM_CUDA(cudaEventRecord(h->done, st));
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T, float* y_host,
+                                    uint32_t flags, void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
+    if (T > 0 && (!x_host || !y_host)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t xb = (size_t)T * h->D * h->esz, yb = (size_t)T * h->D * sizeof(float);
+    if (T > 0) BEAM_CUDA(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st));
+    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, h->y_stage, flags, stream));
+    if (T > 0) BEAM_CUDA(cudaMemcpyAsync(y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, st));
+    BEAM_CUDA(cudaStreamSynchronize(st));
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_stats(beam_moe_t* h, beam_moe_stats_t* out, int32_t* counts_host)
+{
+    g_err[0] = 0;
+    if (!h || !out) return fail(BEAM_ERR_INVALID_ARG, "handle or out is NULL");
+    if (h->last_T < 0) return fail(BEAM_ERR_NO_FORWARD, "no forward has run on this handle");
+    BEAM_CUDA(cudaEventSynchronize(h->done));
+    memset(out, 0, sizeof *out);
+    if (h->last_T == 0) {
+        if (counts_host) memset(counts_host, 0, sizeof(int32_t) * h->E);
+        return BEAM_OK;
+    }
+    DevStats ds;
+    BEAM_CUDA(cudaMemcpy(&ds, h->dstats, sizeof ds, cudaMemcpyDeviceToHost));
+    if (ds.err) return fail(BEAM_ERR_TIMEOUT, "a bounded device wait ran out (code %d)", ds.err);
+    out->tokens = ds.tokens;
+    out->avg_k = ds.tokens ? (double)ds.keep_sum / ds.tokens : 0.0;
+    out->l_reg = ds.tokens ? ds.lreg_sum / ds.tokens : 0.0;
+    out->n_active_experts = ds.n_active;
+    out->n_tokens_all_masked = ds.n_all_masked;
+    out->n_kept = ds.n_kept;
+    if (counts_host)
+        BEAM_CUDA(cudaMemcpy(counts_host, h->counts, sizeof(int32_t) * h->E, cudaMemcpyDeviceToHost));
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_get_routing(beam_moe_t* h, int32_t* topk_id, float* gate, float* mask_logit,
+                                   uint8_t* keep, int32_t* offsets, int32_t* perm, int32_t* inv)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (h->last_T < 0) return fail(BEAM_ERR_NO_FORWARD, "no forward has run on this handle");
+    BEAM_CUDA(cudaEventSynchronize(h->done));
+    const size_t n = (size_t)h->last_T * h->K;
+    if (h->last_T == 0) {
+        if (offsets) memset(offsets, 0, sizeof(int32_t) * (h->E + 1));
+        return BEAM_OK;
+    }
+    if (topk_id) BEAM_CUDA(cudaMemcpy(topk_id, h->topk_id, n * 4, cudaMemcpyDeviceToHost));
+    if (gate) BEAM_CUDA(cudaMemcpy(gate, h->gate, n * 4, cudaMemcpyDeviceToHost));
+    if (mask_logit) BEAM_CUDA(cudaMemcpy(mask_logit, h->mlogit, n * 4, cudaMemcpyDeviceToHost));
+    if (keep) BEAM_CUDA(cudaMemcpy(keep, h->keep, n, cudaMemcpyDeviceToHost));
+    if (inv) BEAM_CUDA(cudaMemcpy(inv, h->inv, n * 4, cudaMemcpyDeviceToHost));
+    int nk = 0;
+    BEAM_CUDA(cudaMemcpy(&nk, h->offsets + h->E, sizeof nk, cudaMemcpyDeviceToHost));
+    if (offsets) BEAM_CUDA(cudaMemcpy(offsets, h->offsets, sizeof(int32_t) * (h->E + 1), cudaMemcpyDeviceToHost));
+    if (perm && nk > 0) BEAM_CUDA(cudaMemcpy(perm, h->perm, sizeof(int32_t) * nk, cudaMemcpyDeviceToHost));
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_profile_begin(beam_moe_t* h, int32_t max_forwards)
+{
+    g_err[0] = 0;
+    if (!h || max_forwards < 1 || max_forwards > 100000)
+        return fail(BEAM_ERR_INVALID_ARG, "handle NULL or max_forwards outside [1, 100000]");
+    prof_release(h);
+    const size_t n = (size_t)max_forwards * 2 * 16;  // <= 16 launches per forward
+    h->prof_pool.reserve(n);
+    for (size_t i = 0; i < n; ++i) {
+        cudaEvent_t e;
+        cudaError_t err = cudaEventCreate(&e);
+        if (err != cudaSuccess) {
+            prof_release(h);
+            return fail(BEAM_ERR_CUDA, "cudaEventCreate failed: %s", cudaGetErrorString(err));
+        }
+        h->prof_pool.push_back(e);
+    }
+    h->prof_recs.reserve(n / 2);
+    h->prof_max = max_forwards;
+    h->prof_forwards = 0;
+    h->prof = true;
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_profile_end(beam_moe_t* h, float* stage_ms, int32_t* stage_launches,
+                                   int32_t* n_forwards)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    float ms[ST_COUNT] = {0};
+    int32_t cnt[ST_COUNT] = {0};
+    for (auto& r : h->prof_recs) {
+        cudaError_t e = cudaEventSynchronize(r.b);
+        float t = 0.f;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+        if (e != cudaSuccess) {
+            prof_release(h);
+            return fail(BEAM_ERR_CUDA, "profiling events failed: %s", cudaGetErrorString(e));
+        }
+        ms[r.stage] += t;
+        cnt[r.stage] += 1;
+    }
+    if (stage_ms) memcpy(stage_ms, ms, sizeof ms);
+    if (stage_launches) memcpy(stage_launches, cnt, sizeof cnt);
+    if (n_forwards) *n_forwards = h->prof_forwards;
+    prof_release(h);
+    return BEAM_OK;
+}
+
+const char* beam_moe_stage_name(int32_t stage)
+{
+    return (stage >= 0 && stage < ST_COUNT) ? kStageNames[stage] : "";
+}
+
+int64_t beam_moe_launch_count(const beam_moe_t* h) { return h ? h->launches : 0; }
+
+void beam_moe_destroy(beam_moe_t* h)
+{
+    if (!h) return;
+    if (h->done) cudaEventSynchronize(h->done);
+    free_all(h);
+    delete h;
+}
+
+const char* beam_moe_last_error(void) { return g_err; }
+
+const char* beam_moe_version(void) { return "beam_moe 0.1 (sm_100a)"; }
+
+}  // extern "C"

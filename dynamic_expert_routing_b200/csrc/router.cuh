@@ -1,0 +1,156 @@
+// router.cuh -- fused router of the BEAM layer: logits of x [W_r | W_m], then per token the
+// Top-K (ties to the lower index), the K-way softmax, the mask test and the statistics.
+//
+// BEAM article on aitrends.kr ("BEAM: Dynamic MoE 라우팅을 위한 Binary Expert Activation
+// Masking"), four-step pipeline: Step 1 (Top-K of r = x W_r, softmax over the K kept logits),
+// Step 2 (m_hat = sigmoid(x W_m)), Step 3 (m_i = 1 iff m_hat_i >= 0.5, evaluated as mask logit
+// >= 0), the training paragraph (L_reg = (1/K) sum_{i in TK} m_hat_i, recorded per token) and
+// Stepped MoE's segment routing (core method: one decision per segment of S tokens, taken at
+// the segment's first token).
+#pragma once
+#include "common.cuh"
+
+namespace beam {
+
+// ---------------------------------------------------------------- logits, SIMT
+// L[i][j] = sum_d x[i*S][d] * Wrm[j][d] for routed rows i < Tr and columns j < n2E, where
+// Wrm = [W_r | W_m]^T ([2E][D], one contiguous row per output column).  fp32 accumulation.
+// CTA: 8 warps, 8 routed rows x 16 columns (2 per warp); x is staged in shared memory as
+// float in chunks of kRouterDC elements.
+constexpr int kRouterRows = 8;
+constexpr int kRouterColsPerWarp = 2;
+constexpr int kRouterDC = 1024;
+
+template <typename TW>
+__global__ void __launch_bounds__(256)
+router_logits_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
+                     const TW* __restrict__ wrm, int n2E, float* __restrict__ L)
+{
+    __shared__ __align__(16) float xs[kRouterRows][kRouterDC];
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row0 = blockIdx.y * kRouterRows;
+    const int col0 = (blockIdx.x * 8 + warp) * kRouterColsPerWarp;
+    const int S = seg > 1 ? seg : 1;
+    const int nrows = min(kRouterRows, Tr - row0);
+    constexpr int VN = Vec<TW>::N;
+    float acc[kRouterColsPerWarp][kRouterRows];
+#pragma unroll
+    for (int c = 0; c < kRouterColsPerWarp; ++c)
+#pragma unroll
+        for (int r = 0; r < kRouterRows; ++r) acc[c][r] = 0.f;
+
+    for (int d0 = 0; d0 < D; d0 += kRouterDC) {
+        const int dl = min(kRouterDC, D - d0);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < kRouterRows * dl; idx += blockDim.x) {
+            int r = idx / dl, d = idx - r * dl;
+            xs[r][d] = (r < nrows) ? to_float(x[(size_t)(row0 + r) * S * D + d0 + d]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < kRouterColsPerWarp; ++c) {
+            const int col = col0 + c;
+            if (col >= n2E) continue;
+            const TW* wrow = wrm + (size_t)col * D + d0;
+            for (int d = lane * VN; d < dl; d += 32 * VN) {
+                float w[VN];
+                Vec<TW>::widen(ldg_stream(wrow + d), w);
+#pragma unroll
+                for (int r = 0; r < kRouterRows; ++r) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int v = 0; v < VN; ++v) s = fmaf(w[v], xs[r][d + v], s);
+                    acc[c][r] += s;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < kRouterColsPerWarp; ++c) {
+        const int col = col0 + c;
+#pragma unroll
+        for (int r = 0; r < kRouterRows; ++r) {
+            float s = warp_sum(acc[c][r]);
+            if (lane == 0 && col < n2E && r < nrows) L[(size_t)(row0 + r) * n2E + col] = s;
+        }
+    }
+    pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------- Top-K, softmax, mask
+// One warp per routed row i.  Lane l holds logits of experts l, l+32, ... (EPL per lane).
+// K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
+// rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
+// L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
+// to every token of the routed row's segment (S = 1: the row's own token).
+template <int EPL>
+__global__ void __launch_bounds__(256)
+route_select_kernel(const float* __restrict__ L, int Tr, int T, int E, int K, int seg,
+                    int mask_off, int* __restrict__ topk_id, float* __restrict__ gate,
+                    float* __restrict__ mlogit, uint8_t* __restrict__ keep,
+                    float* __restrict__ ghat, int* __restrict__ nkeep_tok,
+                    float* __restrict__ lreg_tok)
+{
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x * 8 + warp;
+    if (i < Tr) {
+        const int n2E = 2 * E;
+        const float* Li = L + (size_t)i * n2E;
+        float v[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            int e = lane + 32 * j;
+            v[j] = (e < E) ? Li[e] : -INFINITY;
+        }
+        unsigned chosen = 0;
+        int my_id = 0;
+        float my_v = 0.f;
+        for (int k = 0; k < K; ++k) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                int e = lane + 32 * j;
+                bool ok = (e < E) && !((chosen >> j) & 1u);
+                if (ok && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if ((bi & 31) == lane) chosen |= 1u << (bi >> 5);
+            if (lane == k) { my_id = bi; my_v = bv; }
+        }
+        const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+        const bool active = lane < K;
+        float ex = active ? expf(my_v - vmax) : 0.f;
+        const float den = warp_sum(ex);
+        const float g = ex / den;
+        const float l = active ? Li[E + my_id] : 0.f;
+        const bool kp = active && (mask_off || l >= 0.f);
+        const float gh = kp ? g : 0.f;
+        const float sg = active ? sigmoid_f(l) : 0.f;
+        const int nk = __popc(__ballot_sync(0xffffffffu, kp));
+        const float lr = warp_sum(sg) / (float)K;
+        const int S = seg > 1 ? seg : 1;
+        const int t0 = i * S, t1 = min(T, t0 + S);
+        for (int t = t0; t < t1; ++t) {
+            if (active) {
+                size_t o = (size_t)t * K + lane;
+                topk_id[o] = my_id;
+                gate[o] = g;
+                mlogit[o] = l;
+                keep[o] = kp ? 1 : 0;
+                ghat[o] = gh;
+            }
+            if (lane == 0) { nkeep_tok[t] = nk; lreg_tok[t] = lr; }
+        }
+    }
+    pdl_launch_dependents();
+}
+
+}  // namespace beam

@@ -1,0 +1,424 @@
+// tc_experts.cuh -- grouped SwiGLU experts on the 5th-generation tensor cores (tcgen05) for
+// prefill-sized groups: step 4 of the BEAM pipeline (BEAM article on aitrends.kr, masked
+// aggregation) over the device-built list of kept groups, plus the always-on shared experts
+// (limitation (C)).  The expert FFN is a dense contraction, so it runs as two grouped GEMMs:
+//   GEMM1  acc[t][0:128 | 128:256] = X_g[t] . [W_g rows | W_u rows]^T  ->  H = silu(gate) * up
+//   GEMM2  Y_g[t][n] = H_g[t] . W_d[n]^T
+// Design (sm_100a):
+//   * one persistent CTA per SM walks a tile list derived on the device from the group table:
+//     tiles are (problem, group, n tile, m tile) with the m tile fastest, so CTAs running at
+//     the same time share a weight tile through L2; groups with no kept token have no tile,
+//     so their weights are never read;
+//   * tile 128 (tokens) x 256 x 64, TMA (cp.async.bulk.tensor, 128-byte swizzle, no cluster
+//     multicast) fills a 4-stage shared-memory ring guarded by mbarriers;
+//   * warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma (kind::f16, fp32
+//     accumulation in TMEM, double-buffered accumulators of 256 columns), warps 2..5 drain
+//     TMEM with tcgen05.ld and run the epilogue (SwiGLU -> fp16 H, or fp32 Y stores);
+//   * every mbarrier wait is bounded by a time limit; on expiry the CTA records an error code,
+//     drains the copies and MMAs it issued (again bounded), frees TMEM and returns.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+
+namespace beam {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int kThreads = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*alignment slack*/ + 256 /*barriers*/;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s: far above any tile
+constexpr int ERR_TC_TIMEOUT = 0x100;
+
+enum Epi { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
+
+struct TcParams {
+    CUtensorMap a_routed;   // activations of the routed groups (rows = kept pairs)
+    CUtensorMap b_routed;   // weights of the routed experts, [E * rows_per_expert][K]
+    CUtensorMap a_shared;   // activations of the shared group (rows = tokens)
+    CUtensorMap b_shared;   // shared-expert weights
+    const Group* groups;
+    const int* n_groups;
+    void* out_routed;       // EPI_SWIGLU: fp16 H [rows][F]; EPI_STORE_F32: f32 Y [rows][D]
+    void* out_shared;
+    int ld_routed;          // row length of out_routed
+    int ld_shared;
+    int b_rows_per_expert;  // 2F for GEMM1, D for GEMM2
+    int n_tiles_routed;     // N / 256
+    int n_tiles_shared;
+    int k_steps_routed;     // K / 64
+    int k_steps_shared;
+    int shared_rows;        // T, or 0 when there is no shared group
+    int* err;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait: false when the abort flag is raised or the time limit passes (the caller
+// then raises the flag itself).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 lanes x 32 consecutive fp32 columns of TMEM into 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), sm_100 version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;                 // leading byte offset (unused with swizzle): 16 B
+    d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: 1024 B
+    d |= (uint64_t)1 << 46;                 // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;                 // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, A/B of format `fmt` (0 = f16,
+// 1 = bf16), both K-major, N = 256, M = 128.
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- tile sequence
+struct Tile {
+    int shared;   // 1 = shared-expert problem
+    int row0;     // first activation / output row of the group
+    int m;        // rows in the group
+    int mt;       // m tile inside the group
+    int n;        // n tile
+    int brow;     // first weight row of the tile
+    int ksteps;
+};
+
+// Walks tiles blockIdx.x, blockIdx.x + gridDim.x, ... in order; every role of a CTA holds
+// its own copy and sees the same sequence.
+struct TileWalker {
+    const TcParams* p;
+    int ng;
+    int count_sh;      // tiles of the shared problem
+    int mts_sh;
+    long long next;    // next global tile index
+    int g;             // cursor: current group and the first tile index of it
+    long long g_base;
+
+    __device__ void init(const TcParams* p_, int ng_) {
+        p = p_;
+        ng = ng_;
+        mts_sh = p->shared_rows > 0 ? (p->shared_rows + BM - 1) / BM : 0;
+        count_sh = mts_sh * p->n_tiles_shared;
+        next = blockIdx.x;
+        g = 0;
+        g_base = count_sh;
+    }
+    __device__ bool get(Tile& t) {
+        const long long i = next;
+        next += gridDim.x;
+        if (i < count_sh) {
+            t.shared = 1;
+            t.n = (int)(i / mts_sh);
+            t.mt = (int)(i % mts_sh);
+            t.row0 = 0;
+            t.m = p->shared_rows;
+            t.brow = t.n * BN;
+            t.ksteps = p->k_steps_shared;
+            return true;
+        }
+        while (g < ng) {
+            const Group G = p->groups[g];
+            const int mts = (G.m + BM - 1) / BM;
+            const long long cnt = (long long)mts * p->n_tiles_routed;
+            if (i < g_base + cnt) {
+                const long long r = i - g_base;
+                t.shared = 0;
+                t.n = (int)(r / mts);
+                t.mt = (int)(r % mts);
+                t.row0 = G.row0;
+                t.m = G.m;
+                t.brow = G.expert * p->b_rows_per_expert + t.n * BN;
+                t.ksteps = p->k_steps_routed;
+                return true;
+            }
+            g_base += cnt;
+            ++g;
+        }
+        return false;
+    }
+};
+
+// ---------------------------------------------------------------- the kernel
+template <int EPI, int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    // layout: [stage s: A (16 KB) | B (32 KB)] x STAGES, then the barriers
+    const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&p.a_routed); tma_prefetch_desc(&p.b_routed);
+        tma_prefetch_desc(&p.a_shared); tma_prefetch_desc(&p.b_shared);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_wait();  // groups, counts and activations come from the previous kernels
+    const int ng = *p.n_groups;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        TileWalker w;
+        w.init(&p, ng);
+        Tile t;
+        int s = 0;
+        uint32_t ph = 0;
+        int pend_ph[STAGES];
+        bool pend[STAGES];
+        for (int i = 0; i < STAGES; ++i) { pend[i] = false; pend_ph[i] = 0; }
+        bool ok = true;
+        while (ok && w.get(t)) {
+            const CUtensorMap* am = t.shared ? &p.a_shared : &p.a_routed;
+            const CUtensorMap* bm = t.shared ? &p.b_shared : &p.b_routed;
+            const int arow = t.row0 + t.mt * BM;
+            for (int k = 0; k < t.ksteps; ++k) {
+                if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
+                mbar_expect_tx(full_bar(s), STAGE_BYTES);
+                const uint32_t sa = base + s * STAGE_BYTES;
+                tma_load_2d(sa, am, full_bar(s), k * BK, arow);
+                tma_load_2d(sa + A_BYTES, bm, full_bar(s), k * BK, t.brow);
+                pend[s] = true;
+                pend_ph[s] = (int)ph;
+                if (++s == STAGES) { s = 0; ph ^= 1u; }
+            }
+        }
+        if (!ok) {
+            // drain: let every copy this thread issued land before the CTA can exit
+            for (int i = 0; i < STAGES; ++i) {
+                if (!pend[i]) continue;
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(full_bar(i), (uint32_t)pend_ph[i]) &&
+                       globaltimer() - t0 < kWaitLimitNs) {}
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        TileWalker w;
+        w.init(&p, ng);
+        Tile t;
+        int s = 0, acc = 0;
+        uint32_t ph = 0, aph = 0;
+        bool ok = true, issued = false;
+        constexpr uint32_t idesc = make_idesc(FMT);
+        while (ok && w.get(t)) {
+            if (!mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+            for (int k = 0; k < t.ksteps; ++k) {
+                if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sa = base + s * STAGE_BYTES;
+                const uint64_t ad = sw128_desc(sa);
+                const uint64_t bd = sw128_desc(sa + A_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    tc_mma_f16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (k | kk) != 0);
+                issued = true;
+                tc_commit(empty_bar(s));
+                if (++s == STAGES) { s = 0; ph ^= 1u; }
+            }
+            if (!ok) break;
+            tc_commit(tfull_bar(acc));
+            if (++acc == 2) { acc = 0; aph ^= 1u; }
+        }
+        if (!ok && issued) {
+            tc_commit(drain_bar);  // completes when every MMA issued so far has finished
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(drain_bar, 0) && globaltimer() - t0 < kWaitLimitNs) {}
+        }
+    } else if (warp >= 2) {
+        // ------------------------------------------------ epilogue (TMEM -> registers -> global)
+        TileWalker w;
+        w.init(&p, ng);
+        Tile t;
+        int acc = 0;
+        uint32_t aph = 0;
+        const int lb = 32 * (warp & 3);  // TMEM lanes this warp may access
+        while (w.get(t)) {
+            if (!mbar_wait(tfull_bar(acc), aph, abort_flag)) break;
+            tc_fence_after();
+            const int r = t.mt * BM + lb + lane;  // row inside the group
+            const bool valid = r < t.m;
+            const uint32_t tbase = tmem_base + ((uint32_t)lb << 16) + (uint32_t)(acc * BN);
+            if (EPI == EPI_SWIGLU) {
+                __half* out = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed);
+                const int ld = t.shared ? p.ld_shared : p.ld_routed;
+                __half* orow = out + (size_t)(t.row0 + r) * ld + t.n * (BN / 2);
+#pragma unroll 1
+                for (int j = 0; j < BN / 2 / 32; ++j) {
+                    float g[32], u[32];
+                    tmem_ld32(tbase + 32 * j, g);
+                    tmem_ld32(tbase + BN / 2 + 32 * j, u);
+                    if (valid) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const __half2 hv = __floats2half2_rn(silu_f(g[2 * i]) * u[2 * i],
+                                                                 silu_f(g[2 * i + 1]) * u[2 * i + 1]);
+                            packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * j);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                }
+            } else {
+                float* out = static_cast<float*>(t.shared ? p.out_shared : p.out_routed);
+                const int ld = t.shared ? p.ld_shared : p.ld_routed;
+                float* orow = out + (size_t)(t.row0 + r) * ld + t.n * BN;
+#pragma unroll 1
+                for (int j = 0; j < BN / 32; ++j) {
+                    float v[32];
+                    tmem_ld32(tbase + 32 * j, v);
+                    if (valid) {
+                        float4* dst = reinterpret_cast<float4*>(orow + 32 * j);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (++acc == 2) { acc = 0; aph ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, ERR_TC_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    }
+    pdl_launch_dependents();
+}
+
+}  // namespace tc
+}  // namespace beam

@@ -1,0 +1,147 @@
+"""Python handle over the C ABI: torch tensors in, pointers to the CUDA library out.
+
+Every step of the layer runs in the library's kernels; this module only marshals arguments.
+PyTorch provides device memory and the current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import (BEAM_DTYPE_BF16, BEAM_DTYPE_F32, BEAM_MASK_OFF, BEAM_PATH_STREAM,
+                   BEAM_PATH_TENSOR, BeamConfig, BeamStats, BeamWeights, check)
+
+_DTYPES = {torch.float32: BEAM_DTYPE_F32, torch.bfloat16: BEAM_DTYPE_BF16}
+_PATHS = {None: 0, "auto": 0, "stream": BEAM_PATH_STREAM, "tensor": BEAM_PATH_TENSOR}
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class BeamMoE:
+    """A BEAM masked MoE layer held by the CUDA library.
+
+    weights: dict with w_router [D][E], w_mask [D][E], w_gate/w_up [E][F][D], w_down [E][D][F]
+    and, with shared experts, ws_gate/ws_up [S][Fs][D], ws_down [S][D][Fs]; CUDA tensors of one
+    storage type (float32 or bfloat16).  The library copies them at construction.
+    """
+
+    def __init__(self, weights: dict, top_k: int, max_tokens: int, segment_len: int = 0,
+                 stream=None):
+        lib = _lib.load()
+        wr = weights["w_router"]
+        dt = _DTYPES.get(wr.dtype)
+        if dt is None:
+            raise TypeError(f"unsupported storage dtype {wr.dtype}")
+        for k in ("w_router", "w_mask", "w_gate", "w_up", "w_down"):
+            t = weights[k]
+            if not (t.is_cuda and t.is_contiguous() and t.dtype == wr.dtype):
+                raise ValueError(f"{k} must be a contiguous CUDA tensor of dtype {wr.dtype}")
+        D, E = wr.shape
+        F = weights["w_gate"].shape[1]
+        wsg = weights.get("ws_gate")
+        S = 0 if wsg is None else wsg.shape[0]
+        Fs = 0 if wsg is None else wsg.shape[1]
+        self.cfg = BeamConfig(D, E, top_k, F, S, Fs, dt, segment_len, max_tokens)
+        w = BeamWeights(*[_ptr(weights.get(k)) for k in ("w_router", "w_mask", "w_gate", "w_up",
+                                                         "w_down", "ws_gate", "ws_up", "ws_down")])
+        h = ctypes.c_void_p()
+        check(lib.beam_moe_create(ctypes.byref(self.cfg), ctypes.byref(w),
+                                  ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(h)))
+        self._h = h
+        self.dtype = wr.dtype
+        self.d_model, self.n_experts, self.top_k = D, E, top_k
+        self.max_tokens = max_tokens
+
+    # -------------------------------------------------------------- forward
+    @staticmethod
+    def flags(mask_off: bool = False, path: str | None = None) -> int:
+        return (BEAM_MASK_OFF if mask_off else 0) | _PATHS[path]
+
+    def forward(self, x: torch.Tensor, mask_off: bool = False, path: str | None = None,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """y [T][D] float32 of x [T][D] (storage dtype, CUDA), enqueued on the current stream."""
+        if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype):
+            raise ValueError("x must be a contiguous CUDA tensor of the layer's storage dtype")
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
+        check(_lib.load().beam_moe_forward(self._h, _ptr(x), T, _ptr(out),
+                                           self.flags(mask_off, path),
+                                           ctypes.c_void_p(_stream_handle(stream))))
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, mask_off: bool = False,
+                     path: str | None = None, stream=None) -> torch.Tensor:
+        """Host-buffer variant: copies x in, runs the layer, copies y out, synchronises."""
+        T = x_host.shape[0]
+        check(_lib.load().beam_moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host),
+                                                self.flags(mask_off, path),
+                                                ctypes.c_void_p(_stream_handle(stream))))
+        return y_host
+
+    # -------------------------------------------------------------- inspection
+    def stats(self) -> dict:
+        s = BeamStats()
+        counts = np.zeros(self.n_experts, np.int32)
+        check(_lib.load().beam_moe_stats(self._h, ctypes.byref(s),
+                                         counts.ctypes.data_as(ctypes.c_void_p)))
+        return dict(avg_k=s.avg_k, l_reg=s.l_reg, n_active_experts=s.n_active_experts,
+                    n_tokens_all_masked=s.n_tokens_all_masked, tokens=s.tokens,
+                    n_kept=s.n_kept, counts=counts)
+
+    def routing(self, T: int) -> dict:
+        """Routing of the last forward (T must be that forward's token count)."""
+        K, E = self.top_k, self.n_experts
+        out = dict(topk_id=np.zeros((T, K), np.int32), gate=np.zeros((T, K), np.float32),
+                   mask_logit=np.zeros((T, K), np.float32), keep=np.zeros((T, K), np.uint8),
+                   offsets=np.zeros(E + 1, np.int32), perm=np.zeros(max(1, T * K), np.int32),
+                   inv=np.zeros((T, K), np.int32))
+        p = {k: v.ctypes.data_as(ctypes.c_void_p) for k, v in out.items()}
+        check(_lib.load().beam_moe_get_routing(self._h, p["topk_id"], p["gate"], p["mask_logit"],
+                                               p["keep"], p["offsets"], p["perm"], p["inv"]))
+        out["perm"] = out["perm"][: int(out["offsets"][E])].copy()
+        return out
+
+    def profile_begin(self, max_forwards: int) -> None:
+        """Time every kernel of the next `max_forwards` forwards with CUDA events."""
+        check(_lib.load().beam_moe_profile_begin(self._h, int(max_forwards)))
+
+    def profile_end(self) -> dict:
+        """{stage name: (total ms, launches)} over the profiled forwards, plus 'forwards'."""
+        n = _lib.BEAM_N_STAGES
+        ms = (ctypes.c_float * n)()
+        cnt = (ctypes.c_int32 * n)()
+        nf = ctypes.c_int32()
+        lib = _lib.load()
+        check(lib.beam_moe_profile_end(self._h, ms, cnt, ctypes.byref(nf)))
+        out = {lib.beam_moe_stage_name(i).decode(): (float(ms[i]), int(cnt[i]))
+               for i in range(n) if cnt[i] > 0}
+        out["forwards"] = int(nf.value)
+        return out
+
+    def launch_count(self) -> int:
+        """Kernels launched by this layer's forwards so far."""
+        return int(_lib.load().beam_moe_launch_count(self._h))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.load().beam_moe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,174 @@
+/*
+ * beam_moe.h -- C ABI of the B200 (sm_100a) BEAM masked MoE-layer forward.
+ *
+ * The layer (BEAM article on aitrends.kr, "BEAM: Dynamic MoE 라우팅을 위한 Binary Expert
+ * Activation Masking", four-step pipeline paragraph), per token x:
+ *   Step 1  r = x W_r; keep the Top-K logits (set TK) and take a softmax over those K: g.
+ *   Step 2  raw mask m_hat = sigmoid(x W_m).
+ *   Step 3  m_i = 1 if m_hat_i >= 0.5 else 0, on the Top-K set only (evaluated as the mask
+ *           logit (x W_m)_i >= 0, which is the same test in exact arithmetic).
+ *   Step 4  g_hat = g (.) m, no renormalisation; y = sum_{i in TK, m_i = 1} g_hat_i E_i(x),
+ *           plus the always-on shared experts (limitation (C) of the same article).
+ * Experts whose mask is 0 are skipped: their weights are not read and none of their FLOPs
+ * are spent (ai-feeds.com summary "BEAM: 用于 MoE 动态路由的二进制专家激活掩码", Method,
+ * output and inference acceleration).  E_i is a SwiGLU FFN without biases:
+ *   E(x) = W_d (silu(W_g x) * (W_u x)).
+ * Optional segment routing ("Stepped MoE: Segment-Level Routing with Configurable Inference
+ * Complexity", core method): with segment_len = S > 1, token t uses the Top-K set, gates and
+ * mask of token S*floor(t/S); the experts still see x[t].
+ *
+ * Conventions for every call:
+ *   - Pointers named *_dev are CUDA device pointers; *_host are host pointers.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Calls return a beam_status_t; nothing throws.  beam_moe_last_error() gives a message for
+ *     the last failing call on the calling thread.
+ *   - A handle is not thread-safe: calls on one handle must not overlap.
+ *   - Ties in the Top-K go to the lower expert index; Top-K outputs are in rank order.
+ */
+#ifndef BEAM_MOE_H
+#define BEAM_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BEAM_OK = 0,
+    BEAM_ERR_INVALID_ARG = 1,  /* a NULL pointer, a size out of range, an unsupported shape */
+    BEAM_ERR_OOM = 2,          /* device allocation failed in beam_moe_create */
+    BEAM_ERR_CUDA = 3,         /* a CUDA runtime error; the message has the CUDA error string */
+    BEAM_ERR_UNSUPPORTED = 4,  /* valid request this build cannot serve (e.g. tensor path in fp32) */
+    BEAM_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out; outputs are not valid */
+    BEAM_ERR_NO_FORWARD = 6    /* beam_moe_stats / get_routing before any forward */
+} beam_status_t;
+
+enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
+
+/* forward flags */
+#define BEAM_MASK_OFF     0x1u  /* plain Top-K: every Top-K slot kept (the W_m = 0 behaviour) */
+#define BEAM_PATH_STREAM  0x2u  /* force the weight-streaming (GEMV) expert path */
+#define BEAM_PATH_TENSOR  0x4u  /* force the tcgen05 tensor-core expert path (bf16 only) */
+
+typedef struct {
+    int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
+    int32_t n_experts;    /* E routed experts, 1..256 */
+    int32_t top_k;        /* K, 1..min(E, 32) */
+    int32_t d_ff;         /* F, SwiGLU intermediate size per routed expert; multiple of 128 */
+    int32_t n_shared;     /* S_sh always-on shared experts, 0..16 */
+    int32_t d_ff_shared;  /* intermediate size per shared expert; multiple of 128 (0 if none) */
+    int32_t dtype;        /* BEAM_DTYPE_F32 or BEAM_DTYPE_BF16: storage of x and all weights */
+    int32_t segment_len;  /* 0 or 1: per-token routing; S > 1: segment routing */
+    int32_t max_tokens;   /* largest T any forward will pass, 1..65536 */
+} beam_moe_config_t;
+
+/*
+ * Layer weights, device pointers in the storage type, row-major:
+ *   w_router [D][E]   r = x W_r            w_mask [D][E]   mask logits = x W_m
+ *   w_gate   [E][F][D]  w_up [E][F][D]     w_down [E][D][F]
+ *   ws_gate  [S][Fs][D] ws_up [S][Fs][D]   ws_down [S][D][Fs]  (NULL when n_shared == 0)
+ * Borrowed only during beam_moe_create, which copies them into handle-owned layouts; the
+ * caller may free its copies afterwards.
+ */
+typedef struct {
+    const void *w_router, *w_mask;
+    const void *w_gate, *w_up, *w_down;
+    const void *ws_gate, *ws_up, *ws_down;
+} beam_moe_weights_t;
+
+/* Statistics of the last forward (BEAM article on aitrends.kr: Avg-K in the results
+ * paragraph, L_reg = (1/K) sum_{i in TK} m_hat_i in the training paragraph, as means over
+ * tokens). */
+typedef struct {
+    double avg_k;                /* mean number of kept experts per token */
+    double l_reg;                /* mean over tokens of (1/K) sum_{i in TK} sigmoid(mask logit) */
+    int32_t n_active_experts;    /* routed experts with at least one kept slot */
+    int32_t n_tokens_all_masked; /* tokens whose Top-K slots were all masked */
+    int32_t tokens;              /* T of the last forward */
+    int32_t n_kept;              /* kept (token, slot) pairs = sum of per-expert counts */
+} beam_moe_stats_t;
+
+typedef struct beam_moe beam_moe_t;
+
+/*
+ * Build a layer handle: validates cfg, allocates every device buffer for up to
+ * cfg->max_tokens tokens, and repacks the weights on `stream` (then synchronises it).
+ * Returns BEAM_ERR_INVALID_ARG for a bad cfg/pointer, BEAM_ERR_OOM if allocation fails
+ * (nothing is leaked), BEAM_ERR_CUDA otherwise on a CUDA error.  *out is set only on success.
+ */
+beam_status_t beam_moe_create(const beam_moe_config_t *cfg, const beam_moe_weights_t *w_dev,
+                              void *stream, beam_moe_t **out);
+
+/*
+ * The hot path: y_dev[T][D] (float32) = BEAM layer of x_dev[T][D] (storage type), enqueued on
+ * `stream` without any host synchronisation (per-expert token counts stay on the device).
+ * Runs the fused router (x [W_r | W_m], Top-K, K-way softmax, mask, statistics), the
+ * expert-grouping compaction, the grouped SwiGLU experts (kept experts only), the shared
+ * experts and the fixed-order combine.  Deterministic: the same inputs give the same bits.
+ * T = 0 is a no-op.  T > max_tokens or NULL pointers -> BEAM_ERR_INVALID_ARG.
+ * flags: BEAM_MASK_OFF, and at most one of BEAM_PATH_STREAM / BEAM_PATH_TENSOR (by default the
+ * path is chosen from T).  x_dev and y_dev must stay valid until the stream reaches the end
+ * of the call's work.
+ */
+beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, float *y_dev,
+                               uint32_t flags, void *stream);
+
+/*
+ * beam_moe_forward with host buffers: copies x_host (T*D elements of the storage type) to a
+ * handle-owned device buffer, runs the forward and copies y back to y_host (T*D float32),
+ * then synchronises `stream`.  Pinned host memory gives full-bandwidth copies.
+ */
+beam_status_t beam_moe_forward_host(beam_moe_t *h, const void *x_host, int32_t T, float *y_host,
+                                    uint32_t flags, void *stream);
+
+/*
+ * Statistics of the last forward; waits for it to finish.  counts_host, if not NULL,
+ * receives the per-expert kept-slot counts (E int32).  Returns BEAM_ERR_TIMEOUT if a
+ * bounded device wait of that forward ran out.
+ */
+beam_status_t beam_moe_stats(beam_moe_t *h, beam_moe_stats_t *out, int32_t *counts_host);
+
+/*
+ * Routing of the last forward, copied to host arrays (any may be NULL); waits for it:
+ *   topk_id [T][K] int32 (rank order), gate [T][K] float32 (softmax over the K),
+ *   mask_logit [T][K] float32, keep [T][K] uint8, offsets [E+1] int32 (exclusive prefix sum
+ *   of per-expert counts), perm [n_kept] int32 (t*K+k of the kept pairs, by expert then
+ *   token), inv [T][K] int32 (position in perm, or -1 for a masked slot).
+ * A test and debugging hook; not needed by the forward.
+ */
+beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
+                                   float *mask_logit, uint8_t *keep, int32_t *offsets,
+                                   int32_t *perm, int32_t *inv);
+
+/*
+ * Per-stage timing for roofline reports.  beam_moe_profile_begin(h, n) makes the next (up to)
+ * n forwards record a CUDA event pair around every kernel they launch (this disables the
+ * launch overlap between kernels while it is on).  beam_moe_profile_end waits for them, adds
+ * up the event times per stage into stage_ms[BEAM_N_STAGES] and the launches per stage into
+ * stage_launches[BEAM_N_STAGES] (either may be NULL), sets *n_forwards, and switches timing
+ * off.  beam_moe_stage_name(i) names stage i ("" when out of range).
+ */
+#define BEAM_N_STAGES 12
+beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
+beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
+                                   int32_t *n_forwards);
+const char *beam_moe_stage_name(int32_t stage);
+
+/* Number of kernels the handle has launched since it was created (repacking excluded). */
+int64_t beam_moe_launch_count(const beam_moe_t *h);
+
+/* Free every device buffer of the handle (waits for its pending work).  NULL is ignored. */
+void beam_moe_destroy(beam_moe_t *h);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char *beam_moe_last_error(void);
+
+/* Library version string. */
+const char *beam_moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_H */

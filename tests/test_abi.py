@@ -1,0 +1,76 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every declared entry point,
+and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "beam_moe.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(beam_moe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dynamic_expert_routing_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_named_calls():
+    names = _declared_functions()
+    for n in ("beam_moe_create", "beam_moe_forward", "beam_moe_stats"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in _declared_functions():
+        assert hasattr(lib, n), f"{n} not exported"
+
+
+def test_invalid_config_is_rejected_without_cuda(lib):
+    from dynamic_expert_routing_b200._lib import BeamConfig, BeamWeights, BEAM_ERR_INVALID_ARG
+    w = BeamWeights(*([ctypes.c_void_p(16)] * 5 + [None] * 3))
+    h = ctypes.c_void_p()
+    bad = [
+        BeamConfig(100, 8, 2, 512, 0, 0, 1, 0, 64),     # d_model not a multiple of 64 (bf16)
+        BeamConfig(256, 0, 2, 512, 0, 0, 1, 0, 64),     # no experts
+        BeamConfig(256, 8, 9, 512, 0, 0, 1, 0, 64),     # K > E
+        BeamConfig(256, 8, 2, 500, 0, 0, 1, 0, 64),     # F not a multiple of 128
+        BeamConfig(256, 8, 2, 512, 1, 0, 1, 0, 64),     # shared expert without a size
+        BeamConfig(256, 8, 2, 512, 0, 0, 7, 0, 64),     # unknown dtype
+        BeamConfig(256, 8, 2, 512, 0, 0, 1, 0, 0),      # max_tokens 0
+        BeamConfig(256, 300, 2, 512, 0, 0, 1, 0, 64),   # too many experts
+    ]
+    for cfg in bad:
+        st = lib.beam_moe_create(ctypes.byref(cfg), ctypes.byref(w), None, ctypes.byref(h))
+        assert st == BEAM_ERR_INVALID_ARG
+        assert lib.beam_moe_last_error()
+        assert not h.value
+
+
+def test_null_handle_calls(lib):
+    from dynamic_expert_routing_b200._lib import BeamStats, BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_forward(None, None, 1, None, 0, None) == BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_forward_host(None, None, 1, None, 0, None) == BEAM_ERR_INVALID_ARG
+    s = BeamStats()
+    assert lib.beam_moe_stats(None, ctypes.byref(s), None) == BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_get_routing(None, None, None, None, None, None, None, None) == BEAM_ERR_INVALID_ARG
+    lib.beam_moe_destroy(None)
+    assert b"sm_100a" in lib.beam_moe_version()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from dynamic_expert_routing_b200 import _lib
+    with pytest.raises(RuntimeError):
+        _lib._lib = None
+        try:
+            _lib.load(str(tmp_path / "nope.so"))
+        finally:
+            _lib._lib = None

@@ -1,0 +1,175 @@
+"""CUDA library vs the fp64 oracle, element by element on the same seeded inputs.
+
+Shapes span several tiles and ragged tails of every kernel (token chunks of 32, row blocks of
+16/128, 8-token passes), the edge cases of the method (W_m = 0, every slot masked, K = E,
+segment routing with a partial last segment, T = 0, T = max_tokens) and the layer shapes the
+BEAM pages name (Mixtral-like, DeepSeekV2-Lite-like, Qwen-MoE-like, fine-grained 212 experts).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import parity
+from tests.gpu_util import run_case, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(**kw):
+    return synth.LayerSpec("small", 512, 16, 4, 256, storage="bf16").with_(**kw)
+
+
+# ------------------------------------------------------------------ the tiny fp32 layer
+def test_tiny_fp32_parity():
+    spec = synth.SPECS["tiny"]
+    info = run_case(spec, 64)
+    assert info["rel_l2"] <= parity.TOL_F32_REL
+    assert 0 < info["stats"]["n_kept"] < 64 * 2
+
+
+def test_tiny_zero_mask_router_is_plain_topk():
+    spec = synth.SPECS["tiny"]
+    info = run_case(spec, 64, zero_mask=True)
+    assert info["routing"]["keep"].all()
+    assert info["stats"]["l_reg"] == 0.5
+    assert info["stats"]["avg_k"] == 2.0
+    # the mask-off flag on the masked layer reproduces the W_m = 0 layer bit for bit
+    w = synth.make_layer(spec, keep_rate=0.5)
+    w0 = dict(w, w_mask=torch.zeros_like(w["w_mask"]))
+    a = run_case(spec, 64, weights=w, mask_off=True)
+    b = run_case(spec, 64, weights=w0)
+    assert torch.equal(a["y"], b["y"])
+    np.testing.assert_array_equal(a["routing"]["perm"], b["routing"]["perm"])
+
+
+# ------------------------------------------------------------------ bf16, ragged shapes
+@pytest.mark.parametrize("T", [1, 5, 8, 33, 100])
+def test_small_bf16_stream_path(T):
+    run_case(_small(n_shared=1, d_ff_shared=128), T, seed=T, path="stream")
+
+
+@pytest.mark.parametrize("E,K", [(212, 16), (60, 4), (64, 6), (8, 2), (32, 32)])
+def test_expert_counts_and_topk_widths(E, K):
+    spec = _small(n_experts=E, top_k=K, d_ff=128)
+    run_case(spec, 70, seed=E + K)
+
+
+def test_all_slots_masked_gives_shared_only():
+    spec = _small(n_shared=2, d_ff_shared=128)
+    info = run_case(spec, 40, mask_bias=-1.0e4)
+    st = info["stats"]
+    assert st["n_kept"] == 0 and st["n_active_experts"] == 0 and st["n_tokens_all_masked"] == 40
+    # no shared experts and nothing kept: y is exactly zero
+    spec0 = _small()
+    info0 = run_case(spec0, 40, mask_bias=-1.0e4)
+    assert torch.count_nonzero(info0["y"]) == 0
+
+
+def test_segment_routing_partial_last_segment():
+    spec = _small(segment_len=16, n_shared=1, d_ff_shared=128)
+    info = run_case(spec, 16 * 5 + 7)
+    ids = info["routing"]["topk_id"]
+    for t in range(ids.shape[0]):
+        np.testing.assert_array_equal(ids[t], ids[(t // 16) * 16])
+
+
+def test_zero_tokens_and_max_tokens():
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small()
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=48)
+    x0 = torch.empty((0, spec.d_model), dtype=torch.bfloat16, device="cuda")
+    y0 = layer.forward(x0)
+    assert y0.shape == (0, spec.d_model)
+    assert layer.stats()["tokens"] == 0
+    run_case(spec, 48, weights=w, layer=layer)
+    with pytest.raises(Exception):
+        layer.forward(synth.make_tokens(spec, 49).cuda())
+
+
+def test_deterministic_bits():
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=200)
+    x = synth.make_tokens(spec, 200).cuda()
+    y1 = layer.forward(x).clone()
+    r1 = layer.routing(200)
+    y2 = layer.forward(x).clone()
+    r2 = layer.routing(200)
+    assert torch.equal(y1, y2)
+    for k in r1:
+        np.testing.assert_array_equal(r1[k], r2[k])
+
+
+def test_host_buffer_entry_point():
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=64)
+    x = synth.make_tokens(spec, 64)
+    y_dev = layer.forward(x.cuda()).cpu()
+    y_host = torch.empty((64, spec.d_model), dtype=torch.float32).pin_memory()
+    layer.forward_host(x.pin_memory(), y_host)
+    assert torch.equal(y_dev, y_host)
+
+
+# ------------------------------------------------------------------ tensor-core path
+@pytest.mark.parametrize("T", [1, 17, 128, 129, 700])
+def test_small_bf16_tensor_path(T):
+    run_case(_small(n_shared=1, d_ff_shared=128), T, seed=100 + T, path="tensor")
+
+
+@pytest.mark.parametrize("E,K,T", [(212, 16, 300), (60, 4, 1000), (8, 2, 2000)])
+def test_tensor_path_group_shapes(E, K, T):
+    spec = _small(n_experts=E, top_k=K, d_ff=384, n_shared=2, d_ff_shared=256)
+    run_case(spec, T, seed=E, path="tensor")
+
+
+def test_tensor_and_stream_paths_agree():
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=64)
+    x = synth.make_tokens(spec, 64).cuda()
+    ys = layer.forward(x, path="stream").cpu().double().numpy()
+    r1 = layer.routing(64)
+    yt = layer.forward(x, path="tensor").cpu().double().numpy()
+    r2 = layer.routing(64)
+    for k in r1:
+        np.testing.assert_array_equal(r1[k], r2[k])
+    assert parity.rel_l2(yt, ys) < 1e-3
+
+
+def test_tensor_path_segment_and_mask_off():
+    spec = _small(segment_len=16, n_shared=1, d_ff_shared=128)
+    run_case(spec, 16 * 20 + 3, path="tensor")
+    run_case(_small(), 200, path="tensor", mask_off=True)
+
+
+# ------------------------------------------------------------------ the pages' layer shapes
+@pytest.mark.parametrize("name,T,keep", [
+    ("mixtral", 1, 0.5), ("mixtral", 8, 0.25), ("dsv2lite", 1, 0.07), ("dsv2lite", 64, 0.45),
+    ("qwenmoe", 8, 0.14), ("fine", 32, 0.5),
+])
+def test_model_shapes_decode(name, T, keep):
+    spec = synth.SPECS[name]
+    run_case(spec, T, keep_rate=keep)
+
+
+@pytest.mark.parametrize("name,T,keep,mask_off", [
+    ("mixtral", 4096, 0.5, False), ("mixtral", 4096, 0.25, False), ("mixtral", 64, 0.5, False),
+    ("dsv2lite", 8192, 0.45, False), ("dsv2lite", 8192, 0.07, False),
+    ("qwenmoe", 16384, 0.14, False), ("fine", 8192, 0.25, False), ("fine", 8192, 0.5, True),
+    ("fine_seg16", 8192, 0.5, False),
+])
+def test_model_shapes_prefill(name, T, keep, mask_off):
+    """Full-size prefill on the path the bench times: routing on every token, y on a sample of
+    tokens spread over the batch (every 97th, plus the last)."""
+    spec = synth.SPECS[name]
+    sample = np.unique(np.concatenate([np.arange(0, T, 97), [T - 1]]))
+    info = run_case(spec, T, keep_rate=keep, mask_off=mask_off, y_tokens=sample)
+    # with segment routing an unclean leader makes its whole segment unclean
+    assert info["unclean"] <= 0.05 * T * max(1, spec.segment_len)
