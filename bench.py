@@ -27,8 +27,12 @@ sys.path.insert(0, ROOT)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# name -> (layer spec, tokens, keep rate; None = mask off / plain Top-K)
+# name -> (layer spec, tokens, keep rate; None = mask off / plain Top-K[, spec overrides])
 WORKLOADS = {
+    # reduced copy of the Mixtral-like layer (4 experts, 1024 tokens, about 1.5 GB on the
+    # device) for ncu captures of the same kernels
+    "profile-prefill": ("mixtral", 1024, 0.5, {"n_experts": 4}),
+    "profile-decode": ("mixtral", 1, 0.5, {"n_experts": 4}),
     "mixtral-prefill": ("mixtral", 4096, 0.5),
     "mixtral-prefill-high": ("mixtral", 4096, 0.25),
     "mixtral-decode1": ("mixtral", 1, 0.5),
@@ -184,7 +188,11 @@ TENSOR_STAGES = {"tc_gateup", "tc_down", "tc_router"}
 
 
 def roofline_for(stage, work, ms_per_launch, peaks, workload):
-    if stage in TENSOR_STAGES:
+    """Roofline of one kernel against its binding resource: tensor peak for a tensor-core
+    kernel whose FLOPs take longer than its bytes at HBM speed, HBM bandwidth otherwise."""
+    t_bytes = work["bytes"] / (peaks["hbm"] * 1e9)
+    t_flops = work["flops"] / (peaks["tc_sustained"] * 1e12)
+    if stage in TENSOR_STAGES and t_flops >= t_bytes:
         achieved = work["flops"] / (ms_per_launch * 1e-3) / 1e12
         peak = peaks["tc_sustained"]
         out = dict(bound="tensor", achieved=round(achieved, 2), peak=peak, unit="TFLOP/s")
@@ -198,16 +206,25 @@ def roofline_for(stage, work, ms_per_launch, peaks, workload):
     out["ms_per_launch"] = round(ms_per_launch, 5)
     out["algorithmic_bytes"] = int(work["bytes"])
     out["algorithmic_flops"] = int(work["flops"])
-    out["peak_source"] = peaks["source"] + (" (sustained bf16)" if stage in TENSOR_STAGES else "")
+    out["peak_source"] = peaks["source"] + (" (sustained bf16)" if out["bound"] == "tensor" else "")
     return out
 
 
 # ------------------------------------------------------------------ our arm
+def workload_spec(name):
+    import synth
+    entry = WORKLOADS[name]
+    spec_name, T, keep = entry[:3]
+    spec = synth.SPECS[spec_name]
+    if len(entry) > 3:
+        spec = spec.with_(**entry[3])
+    return spec, T, keep
+
+
 def build_layer(torch, name, device, seed=0):
     import synth
     from dynamic_expert_routing_b200 import BeamMoE
-    spec_name, T, keep = WORKLOADS[name]
-    spec = synth.SPECS[spec_name]
+    spec, T, keep = workload_spec(name)
     w = synth.make_layer(spec, seed=seed, keep_rate=keep if keep else 0.5, device=device)
     wd = {k: v for k, v in w.items() if isinstance(v, torch.Tensor)}
     layer = BeamMoE(wd, spec.top_k, max_tokens=T, segment_len=spec.segment_len)
@@ -262,7 +279,9 @@ def point(torch, dist, name, steps, warmup, world, device, peaks, mask_off=False
     return dict(workload=name, tokens=T, keep_rate=keep, mask="off" if mo else "on",
                 value=round(T * world / (ms * 1e-3), 2), ms_per_step=round(ms, 5),
                 avg_k=round(st["avg_k"], 4), n_active_experts=st["n_active_experts"],
-                layer_roofline_frac=round(t_roof / (ms * 1e-3), 4), roofline=rl)
+                layer_roofline_frac=round(t_roof / (ms * 1e-3), 4), roofline=rl,
+                stage_ms_per_forward={k: round(v[0] / prof["forwards"], 5)
+                                      for k, v in prof.items() if k != "forwards"})
 
 
 def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_steps=None):
@@ -426,8 +445,7 @@ def run_reference(args):
     import torch
     import oracle
     import synth
-    spec_name, T, keep = WORKLOADS[args.workload]
-    spec = synth.SPECS[spec_name]
+    spec, T, keep = workload_spec(args.workload)
     oracle.build()
     w = synth.make_layer(spec, seed=0, keep_rate=keep if keep else 0.5,
                          device="cuda" if torch.cuda.is_available() else "cpu")
