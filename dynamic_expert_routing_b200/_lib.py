@@ -23,6 +23,7 @@ BEAM_PATH_STREAM = 0x2
 BEAM_PATH_TENSOR = 0x4
 
 BEAM_N_STAGES = 12
+BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 STATUS_NAMES = {0: "BEAM_OK", 1: "BEAM_ERR_INVALID_ARG", 2: "BEAM_ERR_OOM", 3: "BEAM_ERR_CUDA",
                 4: "BEAM_ERR_UNSUPPORTED", 5: "BEAM_ERR_TIMEOUT", 6: "BEAM_ERR_NO_FORWARD"}
@@ -72,6 +73,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.beam_moe_forward_host.argtypes = [P, P, I, P, U, P]
     lib.beam_moe_stats.argtypes = [P, ctypes.POINTER(BeamStats), P]
     lib.beam_moe_get_routing.argtypes = [P, P, P, P, P, P, P, P]
+    lib.beam_moe_route_noalloc.argtypes = [P, P, I, P, P, P, P, P, U, P]
+    lib.beam_moe_route_noalloc.restype = ctypes.c_int
     lib.beam_moe_profile_begin.argtypes = [P, I]
     lib.beam_moe_profile_end.argtypes = [P, P, P, P]
     lib.beam_moe_stage_name.argtypes = [I]

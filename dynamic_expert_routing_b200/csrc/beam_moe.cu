@@ -13,6 +13,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -522,8 +523,111 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     return BEAM_OK;
 }
 
+// ---------------------------------------------------------------- routing without allocation
+// Scratch of beam_moe_route_noalloc: a fixed array in the library's own device memory, so the
+// call needs no cudaMalloc.  Every GPU that loads the library holds it until the process
+// exits.  Layout per call: logits [Tr][2E] f32 (256-byte aligned), then per-token kept counts
+// [T] i32 and L_reg terms [T] f32.  Nothing in it has to start at zero: each element the
+// kernels read is written earlier in the same call.  Calls share it, so calls whose work
+// overlaps on the GPU (other streams, other threads) race on it.
+static __device__ __align__(256) unsigned char g_route_scratch[BEAM_ROUTE_NOALLOC_SCRATCH_BYTES];
+
+static std::mutex g_route_scratch_mu;
+static void* g_route_scratch_dev[256] = {};  // device address of the array, per device
+
+// Device address of the scratch array on the current device, looked up once per device (the
+// host-side name of a __device__ array is not a device address).
+static beam_status_t route_scratch_address(void** out)
+{
+    int dev = -1;
+    BEAM_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 256) return fail(BEAM_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+    if (!g_route_scratch_dev[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(BEAM_ERR_CUDA, "cudaGetSymbolAddress of the routing scratch failed: %s",
+                        cudaGetErrorString(e));
+        g_route_scratch_dev[dev] = p;
+    }
+    *out = g_route_scratch_dev[dev];
+    return BEAM_OK;
+}
+
+template <int EPL>
+static cudaError_t launch_select_into(beam_moe* h, const float* L, int Tr, int T, int mask_off,
+                                      int* topk_id, float* gate, float* mlogit, uint8_t* keep,
+                                      float* ghat, int* nkeep_tok, float* lreg_tok,
+                                      cudaStream_t st)
+{
+    return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256),
+                  0, st, L, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate, mlogit, keep, ghat,
+                  nkeep_tok, lreg_tok);
+}
+
+template <typename T>
+static beam_status_t route_noalloc_impl(beam_moe* h, const T* x, int T_, int32_t* topk_id,
+                                        float* gate, float* mlogit, uint8_t* keep, float* ghat,
+                                        int mask_off, unsigned char* scratch, cudaStream_t st)
+{
+    const int S = h->S;
+    const int Tr = ceil_div(T_, S);
+    const size_t l_bytes = ((size_t)Tr * h->n2E * sizeof(float) + 255) & ~(size_t)255;
+    float* L = reinterpret_cast<float*>(scratch);
+    int* nkeep = reinterpret_cast<int*>(scratch + l_bytes);
+    float* lreg = reinterpret_cast<float*>(scratch + l_bytes + (size_t)T_ * sizeof(int));
+    BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_logits_kernel<T>,
+                     dim3(ceil_div(h->n2E, 8 * kRouterColsPerWarp), ceil_div(Tr, kRouterRows)),
+                     dim3(256), 0, st, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, L));
+    cudaError_t e;
+    switch ((h->E + 31) / 32) {
+        case 1: e = launch_select_into<1>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        case 2: e = launch_select_into<2>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        case 3: e = launch_select_into<3>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        case 4: e = launch_select_into<4>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        case 5: e = launch_select_into<5>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        case 6: e = launch_select_into<6>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        case 7: e = launch_select_into<7>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+        default: e = launch_select_into<8>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+    }
+    BEAM_CUDA(e);
+    return BEAM_OK;
+}
+
 // ---------------------------------------------------------------- C ABI
 extern "C" {
+
+beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, int32_t* topk_id,
+                                     float* gate, float* mask_logit, uint8_t* keep, float* ghat,
+                                     uint32_t flags, void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0) return fail(BEAM_ERR_INVALID_ARG, "T=%d is negative", T);
+    if (flags & ~BEAM_MASK_OFF)
+        return fail(BEAM_ERR_INVALID_ARG, "only BEAM_MASK_OFF is accepted, got flags 0x%x", flags);
+    if (T == 0) return BEAM_OK;
+    if (!x || !topk_id || !gate || !mask_logit || !keep || !ghat)
+        return fail(BEAM_ERR_INVALID_ARG, "x and every output pointer must be non-NULL");
+    const long long Tr = (T + h->S - 1) / h->S;
+    const long long need = ((Tr * h->n2E * 4 + 255) & ~255LL) + 8LL * T;
+    if (need > (long long)BEAM_ROUTE_NOALLOC_SCRATCH_BYTES)
+        return fail(BEAM_ERR_INVALID_ARG,
+                    "T=%d needs %lld bytes of routing scratch; the static buffer holds %u bytes",
+                    T, need, (unsigned)BEAM_ROUTE_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    BEAM_TRY(route_scratch_address(&scratch));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
+    unsigned char* sc = static_cast<unsigned char*>(scratch);
+    if (h->cfg.dtype == BEAM_DTYPE_BF16)
+        return route_noalloc_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T,
+                                                 topk_id, gate, mask_logit, keep, ghat, mask_off,
+                                                 sc, st);
+    return route_noalloc_impl<float>(h, static_cast<const float*>(x), T, topk_id, gate,
+                                     mask_logit, keep, ghat, mask_off, sc, st);
+}
 
 beam_status_t beam_moe_create(const beam_moe_config_t* cfg, const beam_moe_weights_t* w,
                               void* stream, beam_moe_t** out)

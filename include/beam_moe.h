@@ -158,6 +158,28 @@ const char *beam_moe_stage_name(int32_t stage);
 /* Number of kernels the handle has launched since it was created (repacking excluded). */
 int64_t beam_moe_launch_count(const beam_moe_t *h);
 
+/*
+ * Routing only, without allocating: Steps 1-3 (Top-K, K-way softmax, mask) for x_dev[T][D]
+ * into caller-provided device arrays topk_id[T][K] int32, gate[T][K] f32, mask_logit[T][K]
+ * f32, keep[T][K] uint8 and ghat[T][K] f32 (same values and layout as beam_moe_forward
+ * produces), enqueued on `stream`.  The BEAM pages have no counterpart to this call; it exists
+ * for callers that cannot allocate device memory when they route, e.g. a serving engine that
+ * reserves all free device memory for its own pools up front, so any later cudaMalloc fails.
+ * The call allocates nothing: its only scratch (the router logits and per-token statistics)
+ * is a fixed array of BEAM_ROUTE_NOALLOC_SCRATCH_BYTES compiled into the library, which every
+ * GPU that loads the library holds until the process exits.  It needs
+ * ceil(ceil(T/S)*2E*4 / 256)*256 + 8*T bytes (S = segment length, 1 when off); a larger T is
+ * rejected with BEAM_ERR_INVALID_ARG and a message giving both sizes.  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress) and caches it; make
+ * that first call before any stream capture.  All calls share the array, so calls whose GPU
+ * work overlaps (different streams or threads) race on it and must be serialised by the
+ * caller.  flags: 0 or BEAM_MASK_OFF.  The handle's own buffers and statistics are untouched.
+ */
+#define BEAM_ROUTE_NOALLOC_SCRATCH_BYTES (2u << 20)
+beam_status_t beam_moe_route_noalloc(beam_moe_t *h, const void *x_dev, int32_t T,
+                                     int32_t *topk_id, float *gate, float *mask_logit,
+                                     uint8_t *keep, float *ghat, uint32_t flags, void *stream);
+
 /* Free every device buffer of the handle (waits for its pending work).  NULL is ignored. */
 void beam_moe_destroy(beam_moe_t *h);
 

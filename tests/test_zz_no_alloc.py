@@ -1,0 +1,79 @@
+"""beam_moe_route_noalloc: routing into caller-provided buffers with no device allocation.
+
+Some callers cannot allocate device memory at the point where they route, for instance a
+serving engine that has reserved all free device memory for its own pools, so that a later
+cudaMalloc would fail.  This entry point keeps its scratch in a fixed array compiled into the
+library.  These tests call it through the C ABI and compare it with what beam_moe_forward
+produces for the same tokens (the same router kernels, so the results must match exactly),
+twice in a row on different tokens, so the second call runs on scratch the first one filled.
+
+This file is collected last so that a run stopping at the first failure has run every other
+test before it.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _route_noalloc(lib, layer, x, flags=0):
+    T, K = x.shape[0], layer.top_k
+    out = dict(topk_id=torch.full((T, K), -7, dtype=torch.int32, device="cuda"),
+               gate=torch.full((T, K), -7.0, device="cuda"),
+               mask_logit=torch.full((T, K), -7.0, device="cuda"),
+               keep=torch.full((T, K), 7, dtype=torch.uint8, device="cuda"),
+               ghat=torch.full((T, K), -7.0, device="cuda"))
+    p = {k: ctypes.c_void_p(v.data_ptr()) for k, v in out.items()}
+    st = lib.beam_moe_route_noalloc(layer._h, ctypes.c_void_p(x.data_ptr()), T, p["topk_id"],
+                                    p["gate"], p["mask_logit"], p["keep"], p["ghat"], flags,
+                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    return st, {k: v.cpu().numpy() for k, v in out.items()}
+
+
+@pytest.mark.parametrize("spec,T", [
+    (synth.SPECS["tiny"], 64),
+    (synth.LayerSpec("small", 512, 16, 4, 256, n_shared=1, d_ff_shared=128), 300),
+    (synth.LayerSpec("seg", 512, 60, 4, 256, segment_len=16), 16 * 9 + 5),
+], ids=["tiny_fp32", "bf16", "bf16_segment"])
+def test_route_noalloc_matches_forward_twice(spec, T):
+    from dynamic_expert_routing_b200 import BeamMoE, _lib
+    lib = _lib.load()
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE({k: v.cuda() for k, v in w.items() if isinstance(v, torch.Tensor)},
+                    spec.top_k, max_tokens=T, segment_len=spec.segment_len)
+    for call, seed in enumerate((11, 12)):
+        x = synth.make_tokens(spec, T, seed=seed).cuda()
+        layer.forward(x)
+        ref = layer.routing(T)
+        st, got = _route_noalloc(lib, layer, x)
+        assert st == _lib.BEAM_OK, lib.beam_moe_last_error()
+        np.testing.assert_array_equal(got["topk_id"], ref["topk_id"], err_msg=f"call {call}")
+        np.testing.assert_array_equal(got["keep"], ref["keep"], err_msg=f"call {call}")
+        np.testing.assert_array_equal(got["gate"], ref["gate"], err_msg=f"call {call}")
+        np.testing.assert_array_equal(got["mask_logit"], ref["mask_logit"], err_msg=f"call {call}")
+        np.testing.assert_array_equal(got["ghat"], ref["gate"] * ref["keep"], err_msg=f"call {call}")
+    # the mask-off flag keeps every Top-K slot
+    st, got = _route_noalloc(lib, layer, x, flags=_lib.BEAM_MASK_OFF)
+    assert st == _lib.BEAM_OK and got["keep"].all()
+    layer.close()
+
+
+def test_route_noalloc_rejects_sizes_beyond_the_static_buffer():
+    from dynamic_expert_routing_b200 import BeamMoE, _lib
+    lib = _lib.load()
+    spec = synth.LayerSpec("wide", 256, 256, 8, 128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    T = 1200   # 1200 * 512 * 4 bytes of logits alone exceed the 2 MiB array
+    layer = BeamMoE({k: v.cuda() for k, v in w.items() if isinstance(v, torch.Tensor)},
+                    spec.top_k, max_tokens=T)
+    x = synth.make_tokens(spec, T).cuda()
+    st, _ = _route_noalloc(lib, layer, x)
+    assert st == _lib.BEAM_ERR_INVALID_ARG
+    assert b"static buffer" in lib.beam_moe_last_error()
+    layer.close()
