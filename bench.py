@@ -32,7 +32,7 @@ WORKLOADS = {
     # reduced copy of the Mixtral-like layer (4 experts, 1024 tokens, about 1.5 GB on the
     # device) for ncu captures of the same kernels
     "profile-prefill": ("mixtral", 1024, 0.5, {"n_experts": 4}),
-    "profile-decode": ("mixtral", 1, 0.5, {"n_experts": 4}),
+    "profile-decode": ("mixtral", 2, None, {"n_experts": 4}),
     "mixtral-prefill": ("mixtral", 4096, 0.5),
     "mixtral-prefill-high": ("mixtral", 4096, 0.25),
     "mixtral-decode1": ("mixtral", 1, 0.5),

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -109,7 +110,8 @@ __global__ void repack_down_kernel(const TI* __restrict__ w, long long n, int S,
 struct beam_moe {
     beam_moe_config_t cfg;
     int E, K, D, F, Fsh, Tmax, S;
-    int n2E;
+    int n2E;             // 2E: router + mask logit columns
+    int ldL;             // leading dimension of the logits and rows of the repacked router
     size_t esz;
     int num_sms;
     int max_nch;
@@ -136,7 +138,15 @@ struct beam_moe {
     size_t hsz;          // bytes per element of H and of the stored down projections
     bool tc_ok = false;  // tensor-core expert path available (bf16, D % 256 == 0)
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    tc::TcParams p0;      // router GEMM (one dense problem; its x map is set per forward)
     tc::TcParams p1, p2;  // GEMM1 / GEMM2 parameters (the x map of GEMM1 is set per forward)
+    tc::TcParams p1s;     // GEMM1 in split-K mode: f32 partials into g1part
+    int split_rows = 0;   // token rows (routed: x K) the split-K workspaces hold
+    float* g1part = nullptr;     // [kMaxSplits][split_rows*K][2F]
+    float* g1part_sh = nullptr;  // [kMaxSplits][split_rows][2Fsh]
+    float* ypart = nullptr;      // [kMaxSplits][split_rows*K][D]
+    float* ysh_part = nullptr;   // [kMaxSplits][split_rows][D]
+    int* zero_int = nullptr;
     int* range_flag = nullptr;
     cudaEvent_t done = nullptr;
     int last_T = -1;
@@ -229,9 +239,46 @@ static beam_status_t validate(const beam_moe_config_t* c)
 
 static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
-// Automatic path choice: up to this many tokens per forward the experts run as
-// weight-streaming GEMVs, above it on the tensor cores.
-constexpr int kStreamMaxTokens = 16;
+// Automatic path choice for bf16 layers: from this many tokens up the experts run on the
+// tensor cores (measured on B200 to stream weights faster than the CUDA-core GEMV from one
+// token up, once small batches split K); the GEMV path serves fp32 layers and the
+// BEAM_PATH_STREAM flag.
+constexpr int kTcMinTokens = 1;
+// Router logits run on the tensor cores from this many routed rows up (bf16 layers).
+constexpr int kTcRouterMinRows = 64;
+// Split-K for small batches on the tensor-core path: up to kMaxSplits K slices per tile, for
+// forwards of at most kSplitMaxTokens tokens (the partial-sum workspaces are sized for that).
+constexpr int kMaxSplits = 8;
+constexpr int kSplitMaxTokens = 64;
+constexpr int kMinStepsPerSplit = 4;
+
+// K-split factor that spreads `tiles` output tiles over the SMs, keeping at least
+// kMinStepsPerSplit k steps per slice and no empty slice.
+// Split count s in [1, kMaxSplits] that minimises the wave makespan of `tiles` tiles split
+// s ways on num_sms SMs, ceil(tiles*s/num_sms)/s (in units of one unsplit tile), plus a small
+// charge per extra split for the partial sums it writes and adds back.
+static int choose_splits(int num_sms, long long tiles)
+{
+    if (tiles <= 0) return 1;
+    int best = 1;
+    double best_cost = 1e30;
+    for (int s = 1; s <= kMaxSplits; ++s) {
+        const double waves = (double)((tiles * s + num_sms - 1) / num_sms);
+        const double cost = waves / s + 0.03 * (s - 1);
+        if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
+    }
+    return best;
+}
+
+// The split count actually used for a problem with `ksteps` k steps: at least
+// kMinStepsPerSplit steps per slice, and slices of equal length except the last, which is
+// never empty (every slice writes its partial sums).
+static int normalise_splits(int s, int ksteps)
+{
+    s = std::max(1, std::min(s, std::max(1, ksteps / kMinStepsPerSplit)));
+    const int per = (ksteps + s - 1) / s;
+    return (ksteps + per - 1) / per;
+}
 
 template <typename T>
 static beam_status_t repack(beam_moe* h, const beam_moe_weights_t* w, cudaStream_t st)
@@ -239,7 +286,7 @@ static beam_status_t repack(beam_moe* h, const beam_moe_weights_t* w, cudaStream
     using TH = typename HType<T>::type;
     const int D = h->D, E = h->E, F = h->F;
     repack_router_kernel<T><<<1024, 256, 0, st>>>(static_cast<const T*>(w->w_router),
-                                                  static_cast<const T*>(w->w_mask), D, E, h->n2E,
+                                                  static_cast<const T*>(w->w_mask), D, E, h->ldL,
                                                   static_cast<T*>(h->wrm));
     BEAM_CUDA(cudaGetLastError());
     repack_gateup_kernel<T><<<(unsigned)((long long)E * 2 * F), 128, 0, st>>>(
@@ -265,10 +312,11 @@ static beam_status_t repack(beam_moe* h, const beam_moe_weights_t* w, cudaStream
 
 // ---------------------------------------------------------------- tensor-core path set-up
 static beam_status_t encode_map(beam_moe* h, CUtensorMap* m, CUtensorMapDataType dt,
-                                const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows)
+                                const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                                uint64_t row_stride_elems = 0)
 {
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
+    cuuint64_t strides[1] = {(row_stride_elems ? row_stride_elems : cols) * 2};
     cuuint32_t box[2] = {(cuuint32_t)tc::BK, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = h->encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -326,6 +374,42 @@ static beam_status_t setup_tc(beam_moe* h)
     b.k_steps_routed = (int)(F / tc::BK);
     b.k_steps_shared = (int)(Fsh / tc::BK);
     a.err = b.err = &h->dstats->err;
+    a.k_splits_routed = a.k_splits_shared = 1;
+    b.k_splits_routed = b.k_splits_shared = 1;
+    // split-K variant of GEMM1: raw f32 gate/up accumulators, one slice per K split
+    {
+        const size_t sr = (size_t)std::min(h->Tmax, kSplitMaxTokens);
+        h->split_rows = (int)sr;
+        BEAM_TRY(dalloc(h, &h->g1part, kMaxSplits * sr * h->K * 2 * F * sizeof(float)));
+        BEAM_TRY(dalloc(h, &h->ypart, kMaxSplits * sr * h->K * D * sizeof(float)));
+        if (Fsh) {
+            BEAM_TRY(dalloc(h, &h->g1part_sh, kMaxSplits * sr * 2 * Fsh * sizeof(float)));
+            BEAM_TRY(dalloc(h, &h->ysh_part, kMaxSplits * sr * D * sizeof(float)));
+        }
+        tc::TcParams& c = h->p1s;
+        c = a;
+        c.out_routed = h->g1part; c.ld_routed = (int)(2 * F);
+        c.out_shared = h->g1part_sh; c.ld_shared = (int)(2 * Fsh);
+        c.split_stride_routed = (long long)sr * h->K * 2 * F;
+        c.split_stride_shared = (long long)sr * 2 * Fsh;
+    }
+    // router: logits L [Tr][ldL] = x_rows [Tr][D] . Wrm [ldL][D]^T as one dense problem
+    tc::TcParams& r = h->p0;
+    memset(&r, 0, sizeof r);
+    BEAM_TRY(encode_map(h, &r.b_shared, BF, h->wrm, (uint64_t)h->ldL, D, tc::BN));
+    r.b_routed = r.b_shared;
+    r.a_routed = r.a_shared = a.a_routed;  // the x map is set in every forward
+    r.groups = h->groups;
+    r.n_groups = h->zero_int;              // no routed groups
+    r.out_routed = r.out_shared = h->L;
+    r.ld_routed = r.ld_shared = h->ldL;
+    r.b_rows_per_expert = 0;
+    r.n_tiles_routed = r.n_tiles_shared = h->ldL / tc::BN;
+    r.k_steps_routed = r.k_steps_shared = (int)(D / tc::BK);
+    r.k_splits_routed = r.k_splits_shared = 1;
+    r.err = &h->dstats->err;
+    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
     BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
     BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
@@ -343,6 +427,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     h->Tmax = cfg->max_tokens;
     h->S = cfg->segment_len > 1 ? cfg->segment_len : 1;
     h->n2E = 2 * h->E;
+    // bf16 layers pad the router rows to the tensor-core tile width (extra rows are zero)
+    h->ldL = (cfg->dtype == BEAM_DTYPE_BF16) ? ((h->n2E + tc::BN - 1) / tc::BN) * tc::BN : h->n2E;
     h->esz = cfg->dtype == BEAM_DTYPE_BF16 ? 2 : 4;
     h->hsz = cfg->dtype == BEAM_DTYPE_BF16 ? 2 : 4;
     h->max_nch = ceil_div(h->Tmax, 32);
@@ -353,7 +439,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     const size_t D = h->D, E = h->E, K = h->K, F = h->F, Fsh = h->Fsh, Tm = h->Tmax;
     const size_t es = h->esz, hs = h->hsz;
     const size_t rows = Tm * K;  // upper bound on kept pairs
-    BEAM_TRY(dalloc(h, &h->wrm, (size_t)h->n2E * D * es));
+    BEAM_TRY(dalloc(h, &h->wrm, (size_t)h->ldL * D * es));
+    BEAM_TRY(dalloc(h, &h->zero_int, sizeof(int)));
     BEAM_TRY(dalloc(h, &h->wgu, E * 2 * F * D * es));
     BEAM_TRY(dalloc(h, &h->wd, E * D * F * hs));
     BEAM_TRY(dalloc(h, &h->range_flag, sizeof(int)));
@@ -363,7 +450,7 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
         BEAM_TRY(dalloc(h, &h->hsh, Tm * Fsh * hs));
         BEAM_TRY(dalloc(h, &h->ysh, Tm * D * sizeof(float)));
     }
-    BEAM_TRY(dalloc(h, &h->L, Tm * h->n2E * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->L, Tm * h->ldL * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->topk_id, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->gate, rows * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->mlogit, rows * sizeof(float)));
@@ -387,22 +474,26 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
     BEAM_CUDA(cudaMemsetAsync(h->dstats, 0, sizeof(DevStats), st));
     BEAM_CUDA(cudaMemsetAsync(h->range_flag, 0, sizeof(int), st));
+    BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, sizeof(int), st));
     BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
 
     if (cfg->dtype == BEAM_DTYPE_BF16) BEAM_TRY(repack<__nv_bfloat16>(h, w, st));
     else BEAM_TRY(repack<float>(h, w, st));
 
-    const int smem_gu = kStreamMT * h->D * (int)h->esz;
     if (cfg->dtype == BEAM_DTYPE_BF16) {
         BEAM_CUDA(cudaFuncSetAttribute(stream_gateup_kernel<__nv_bfloat16, __half>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_gu));
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       stream_gateup_smem()));
         BEAM_CUDA(cudaFuncSetAttribute(stream_down_kernel<__half>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 65536));
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       stream_down_smem()));
     } else {
         BEAM_CUDA(cudaFuncSetAttribute(stream_gateup_kernel<float, float>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem_gu));
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       stream_gateup_smem()));
         BEAM_CUDA(cudaFuncSetAttribute(stream_down_kernel<float>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 65536));
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       stream_down_smem()));
     }
     BEAM_CUDA(cudaStreamSynchronize(st));
     int bad = 0;
@@ -451,7 +542,7 @@ template <int EPL>
 static cudaError_t launch_select(beam_moe* h, int Tr, int T, int mask_off, cudaStream_t st)
 {
     return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256), 0, st,
-                  (const float*)h->L, Tr, T, h->E, h->K, h->S, mask_off, h->topk_id, h->gate,
+                  (const float*)h->L, h->ldL, Tr, T, h->E, h->K, h->S, mask_off, h->topk_id, h->gate,
                   h->mlogit, h->keep, h->ghat, h->nkeep_tok, h->lreg_tok);
 }
 
@@ -466,9 +557,20 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
 
     // 1. router logits L = x [W_r | W_m]  (routed rows only: segment leaders when S > 1)
-    BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_logits_kernel<T>,
-                     dim3(ceil_div(h->n2E, 8 * kRouterColsPerWarp), ceil_div(Tr, kRouterRows)),
-                     dim3(256), 0, st, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->L));
+    if (h->tc_ok && Tr >= kTcRouterMinRows) {
+        tc::TcParams& p0 = h->p0;
+        BEAM_TRY(encode_map(h, &p0.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)Tr,
+                            (uint64_t)D, tc::BM, (uint64_t)S * D));
+        p0.a_routed = p0.a_shared;
+        p0.shared_rows = Tr;
+        BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
+                         dim3(std::min(h->num_sms, ceil_div(Tr, tc::BM) * p0.n_tiles_shared)),
+                         dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
+    } else {
+        BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
+                         dim3(h->n2E, ceil_div(Tr, kGemvRows)),
+                         dim3(256), 0, st, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->ldL, h->L));
+    }
     // 2. Top-K, softmax, mask, per-token statistics
     cudaError_t e;
     switch ((E + 31) / 32) {
@@ -494,31 +596,81 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                      (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     // 4. experts (kept groups only) and shared experts
     using TH = typename HType<T>::type;
+    const float* ybase = h->yperm;
+    const float* yshbase = h->Fsh ? h->ysh : nullptr;
+    int ysplits = 1, yshsplits = 1;
+    long long ystride = 0, yshstride = 0;
     if (use_tc) {
-        tc::TcParams& p1 = h->p1;
-        BEAM_TRY(encode_map(h, &p1.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
-                            (uint64_t)D, tc::BM));
-        p1.shared_rows = h->Fsh ? T_ : 0;
-        h->p2.shared_rows = h->Fsh ? T_ : 0;
-        BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
-                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1));
+        const int Fsh = h->Fsh, F = h->F;
+        int s1 = 1, s2 = 1;
+        if (T_ <= kSplitMaxTokens) {
+            // a small batch has few kept groups: split K so their tiles cover every SM
+            const long long groups = std::min<long long>(E, std::max(1LL, ((long long)T_ * K + 1) / 2));
+            const long long mts = ceil_div(T_, tc::BM);
+            s1 = choose_splits(h->num_sms, mts * ((Fsh ? 2LL * Fsh / tc::BN : 0) + groups * (2LL * F / tc::BN)));
+            s2 = choose_splits(h->num_sms, mts * ((Fsh ? (long long)D / tc::BN : 0) + groups * (D / tc::BN)));
+        }
+        const int s1r = normalise_splits(s1, D / tc::BK);          // GEMM1: K = D for both problems
+        const int s2r = normalise_splits(s2, F / tc::BK);          // GEMM2 routed: K = F
+        const int s2s = Fsh ? normalise_splits(s2, Fsh / tc::BK) : 1;  // GEMM2 shared: K = Fsh
+        s1 = s1r;
+        if (s1 > 1) {
+            tc::TcParams& p = h->p1s;
+            BEAM_TRY(encode_map(h, &p.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
+                                (uint64_t)D, tc::BM));
+            p.shared_rows = Fsh ? T_ : 0;
+            p.k_splits_routed = p.k_splits_shared = s1;
+            BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1s));
+            const long long work = ((long long)T_ * K * F + (long long)T_ * Fsh);
+            BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::swiglu_finish_kernel,
+                             dim3((unsigned)std::min<long long>(h->num_sms * 4, ceil_div(work, 256))),
+                             dim3(256), 0, st, (const float*)h->g1part, s1, p.split_stride_routed,
+                             (const int*)(h->offsets + E), F, (__half*)h->hbuf,
+                             (const float*)h->g1part_sh, s1, p.split_stride_shared,
+                             Fsh ? T_ : 0, Fsh, (__half*)h->hsh));
+        } else {
+            tc::TcParams& p1 = h->p1;
+            BEAM_TRY(encode_map(h, &p1.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
+                                (uint64_t)D, tc::BM));
+            p1.shared_rows = Fsh ? T_ : 0;
+            BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1));
+        }
+        tc::TcParams& p2 = h->p2;
+        p2.shared_rows = Fsh ? T_ : 0;
+        if (s2r > 1 || s2s > 1) {
+            p2.k_splits_routed = s2r;
+            p2.k_splits_shared = s2s;
+            p2.out_routed = h->ypart;
+            p2.split_stride_routed = (long long)h->split_rows * K * D;
+            p2.out_shared = h->ysh_part;
+            p2.split_stride_shared = (long long)h->split_rows * D;
+            ybase = h->ypart; ysplits = s2r; ystride = p2.split_stride_routed;
+            if (Fsh) { yshbase = h->ysh_part; yshsplits = s2s; yshstride = p2.split_stride_shared; }
+        } else {
+            p2.k_splits_routed = p2.k_splits_shared = 1;
+            p2.out_routed = h->yperm;
+            p2.out_shared = h->ysh;
+            p2.split_stride_routed = p2.split_stride_shared = 0;
+        }
         BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
     } else {
         StreamArgs a;
         a.xperm = h->xperm; a.x = x; a.wgu = h->wgu; a.wsgu = h->wsgu; a.wd = h->wd; a.wsd = h->wsd;
         a.h = h->hbuf; a.hsh = h->hsh; a.yperm = h->yperm; a.ysh = h->ysh;
-        a.groups = h->groups; a.n_groups = h->n_groups;
+        a.groups = h->groups; a.n_groups = h->n_groups; a.err = &h->dstats->err;
         a.D = D; a.F = h->F; a.Fsh = h->Fsh; a.T = T_;
-        const int grid = h->num_sms * 2;
+        const int grid = h->num_sms;  // one 256-thread CTA per SM (shared-memory rings)
         BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(grid), dim3(256),
-                         (size_t)kStreamMT * D * sizeof(T), st, a));
+                         (size_t)stream_gateup_smem(), st, a));
         BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(grid), dim3(256),
-                         (size_t)65536, st, a));
+                         (size_t)stream_down_smem(), st, a));
     }
     // 5. fixed-order combine
-    BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel, dim3(T_), dim3(256), 0, st, (const float*)h->yperm,
-                     (const float*)(h->Fsh ? h->ysh : nullptr), (const int*)h->inv,
+    BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel, dim3(T_), dim3(256), 0, st, ybase, ysplits,
+                     ystride, yshbase, yshsplits, yshstride, (const int*)h->inv,
                      (const float*)h->ghat, T_, K, D, y));
     return BEAM_OK;
 }
@@ -562,8 +714,8 @@ static cudaError_t launch_select_into(beam_moe* h, const float* L, int Tr, int T
                                       cudaStream_t st)
 {
     return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256),
-                  0, st, L, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate, mlogit, keep, ghat,
-                  nkeep_tok, lreg_tok);
+                  0, st, L, h->n2E, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate, mlogit, keep,
+                  ghat, nkeep_tok, lreg_tok);
 }
 
 template <typename T>
@@ -577,9 +729,9 @@ static beam_status_t route_noalloc_impl(beam_moe* h, const T* x, int T_, int32_t
     float* L = reinterpret_cast<float*>(scratch);
     int* nkeep = reinterpret_cast<int*>(scratch + l_bytes);
     float* lreg = reinterpret_cast<float*>(scratch + l_bytes + (size_t)T_ * sizeof(int));
-    BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_logits_kernel<T>,
-                     dim3(ceil_div(h->n2E, 8 * kRouterColsPerWarp), ceil_div(Tr, kRouterRows)),
-                     dim3(256), 0, st, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, L));
+    BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
+                     dim3(h->n2E, ceil_div(Tr, kGemvRows)),
+                     dim3(256), 0, st, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, h->n2E, L));
     cudaError_t e;
     switch ((h->E + 31) / 32) {
         case 1: e = launch_select_into<1>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
@@ -671,7 +823,7 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
     bool use_tc;
     if (flags & BEAM_PATH_TENSOR) use_tc = true;
     else if (flags & BEAM_PATH_STREAM) use_tc = false;
-    else use_tc = h->tc_ok && T > kStreamMaxTokens;
+    else use_tc = h->tc_ok && T >= kTcMinTokens;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
     if (h->prof) ++h->prof_forwards;

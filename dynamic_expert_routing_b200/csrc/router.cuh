@@ -14,79 +14,75 @@ namespace beam {
 
 // ---------------------------------------------------------------- logits, SIMT
 // L[i][j] = sum_d x[i*S][d] * Wrm[j][d] for routed rows i < Tr and columns j < n2E, where
-// Wrm = [W_r | W_m]^T ([2E][D], one contiguous row per output column).  fp32 accumulation.
-// CTA: 8 warps, 8 routed rows x 16 columns (2 per warp); x is staged in shared memory as
-// float in chunks of kRouterDC elements.
-constexpr int kRouterRows = 8;
-constexpr int kRouterColsPerWarp = 2;
-constexpr int kRouterDC = 1024;
+// Wrm = [W_r | W_m]^T (one contiguous row of D per output column).  fp32 accumulation; L has
+// leading dimension ldL >= n2E.  Used for decode-sized batches and fp32 layers; large bf16
+// batches run the same product on the tensor cores (tc_experts.cuh, f32-store epilogue).
+// One CTA per (column j, block of kGemvRows routed rows): its 256 threads split the D-long
+// weight row with 16-byte loads, each thread keeps one partial per row, and the partials are
+// reduced in a fixed order (warp butterfly, then the 8 warps in index order).
+constexpr int kGemvRows = 16;
 
 template <typename TW>
 __global__ void __launch_bounds__(256)
-router_logits_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
-                     const TW* __restrict__ wrm, int n2E, float* __restrict__ L)
+router_gemv_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
+                   const TW* __restrict__ wrm, int n2E, int ldL, float* __restrict__ L)
 {
-    __shared__ __align__(16) float xs[kRouterRows][kRouterDC];
+    __shared__ float red[8][kGemvRows];
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row0 = blockIdx.y * kRouterRows;
-    const int col0 = (blockIdx.x * 8 + warp) * kRouterColsPerWarp;
-    const int S = seg > 1 ? seg : 1;
-    const int nrows = min(kRouterRows, Tr - row0);
+    const int j = blockIdx.x;
+    const int row0 = blockIdx.y * kGemvRows;
+    const int nrows = min(kGemvRows, Tr - row0);
+    const size_t xstride = (size_t)(seg > 1 ? seg : 1) * D;
     constexpr int VN = Vec<TW>::N;
-    float acc[kRouterColsPerWarp][kRouterRows];
+    float acc[kGemvRows];
 #pragma unroll
-    for (int c = 0; c < kRouterColsPerWarp; ++c)
+    for (int r = 0; r < kGemvRows; ++r) acc[r] = 0.f;
+    const TW* wrow = wrm + (size_t)j * D;
+    const TW* x0 = x + (size_t)row0 * xstride;
+    for (int d = threadIdx.x * VN; d < D; d += 256 * VN) {
+        float w[VN];
+        Vec<TW>::widen(ldg_stream(wrow + d), w);
 #pragma unroll
-        for (int r = 0; r < kRouterRows; ++r) acc[c][r] = 0.f;
-
-    for (int d0 = 0; d0 < D; d0 += kRouterDC) {
-        const int dl = min(kRouterDC, D - d0);
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < kRouterRows * dl; idx += blockDim.x) {
-            int r = idx / dl, d = idx - r * dl;
-            xs[r][d] = (r < nrows) ? to_float(x[(size_t)(row0 + r) * S * D + d0 + d]) : 0.f;
-        }
-        __syncthreads();
+        for (int r = 0; r < kGemvRows; ++r) {
+            if (r < nrows) {
+                float xv[VN];
+                Vec<TW>::widen(__ldg(reinterpret_cast<const uint4*>(x0 + r * xstride + d)), xv);
+                float s = 0.f;
 #pragma unroll
-        for (int c = 0; c < kRouterColsPerWarp; ++c) {
-            const int col = col0 + c;
-            if (col >= n2E) continue;
-            const TW* wrow = wrm + (size_t)col * D + d0;
-            for (int d = lane * VN; d < dl; d += 32 * VN) {
-                float w[VN];
-                Vec<TW>::widen(ldg_stream(wrow + d), w);
-#pragma unroll
-                for (int r = 0; r < kRouterRows; ++r) {
-                    float s = 0.f;
-#pragma unroll
-                    for (int v = 0; v < VN; ++v) s = fmaf(w[v], xs[r][d + v], s);
-                    acc[c][r] += s;
-                }
+                for (int v = 0; v < VN; ++v) s = fmaf(w[v], xv[v], s);
+                acc[r] += s;
             }
         }
     }
 #pragma unroll
-    for (int c = 0; c < kRouterColsPerWarp; ++c) {
-        const int col = col0 + c;
-#pragma unroll
-        for (int r = 0; r < kRouterRows; ++r) {
-            float s = warp_sum(acc[c][r]);
-            if (lane == 0 && col < n2E && r < nrows) L[(size_t)(row0 + r) * n2E + col] = s;
+    for (int r = 0; r < kGemvRows; ++r) {
+        if (r < nrows) {
+            const float s = warp_sum(acc[r]);
+            if (lane == 0) red[warp][r] = s;
         }
     }
+    __syncthreads();
+    if (threadIdx.x < nrows) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
+        L[(size_t)(row0 + threadIdx.x) * ldL + j] = s;
+    }
+    (void)n2E;
     pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------- Top-K, softmax, mask
-// One warp per routed row i.  Lane l holds logits of experts l, l+32, ... (EPL per lane).
+// One warp per routed row i (row i of L, leading dimension ldL: router logits in columns
+// [0, E), mask logits in [E, 2E)).  Lane l holds logits of experts l, l+32, ... (EPL per lane).
 // K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
 // rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
 // L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
 // to every token of the routed row's segment (S = 1: the row's own token).
 template <int EPL>
 __global__ void __launch_bounds__(256)
-route_select_kernel(const float* __restrict__ L, int Tr, int T, int E, int K, int seg,
+route_select_kernel(const float* __restrict__ L, int ldL, int Tr, int T, int E, int K, int seg,
                     int mask_off, int* __restrict__ topk_id, float* __restrict__ gate,
                     float* __restrict__ mlogit, uint8_t* __restrict__ keep,
                     float* __restrict__ ghat, int* __restrict__ nkeep_tok,
@@ -96,8 +92,7 @@ route_select_kernel(const float* __restrict__ L, int Tr, int T, int E, int K, in
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * 8 + warp;
     if (i < Tr) {
-        const int n2E = 2 * E;
-        const float* Li = L + (size_t)i * n2E;
+        const float* Li = L + (size_t)i * ldL;
         float v[EPL];
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {

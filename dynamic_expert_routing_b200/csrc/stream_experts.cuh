@@ -34,6 +34,7 @@ struct StreamArgs {
     float* ysh;          // shared Y [T][D]
     const Group* groups;
     const int* n_groups;
+    int* err;            // error word of the forward's statistics
     int D, F, Fsh, T;
 };
 
@@ -68,31 +69,193 @@ __device__ __forceinline__ ItemView stream_item(const StreamArgs& a, long item, 
     return v;
 }
 
-// H[i][f] = silu(sum_d Wg[f][d] x_i[d]) * (sum_d Wu[f][d] x_i[d]) for the group's tokens i.
-// T: storage type of x and the gate/up weights; TH: type of H.
+// ---------------------------------------------------------------- warp-private TMA ring
+// Each warp streams its weight rows through its own ring of kRingNS shared-memory stages,
+// filled by 1-D bulk copies (cp.async.bulk, no multicast) that lane 0 issues kRingNS segments
+// ahead of the computation; an mbarrier per stage signals arrival (transaction bytes).  A
+// stage is refilled once every lane of the warp has read it (__syncwarp + proxy fence).
+// This keeps kRingNS x (segment bytes) x (rows) in flight per warp independently of
+// register pressure.  Segment k of a warp's stream always lands in stage k % kRingNS and its
+// wait parity is (k / kRingNS) & 1.  Every wait is bounded in time.
+constexpr int kRingNS = 4;
+constexpr unsigned long long kRingWaitNs = 2000000000ull;
+constexpr int ERR_STREAM_TIMEOUT = 0x200;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void ring_bar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar));
+}
+__device__ __forceinline__ void ring_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void ring_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ bool ring_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait; false (and the CTA-wide abort flag raised) on expiry or on an abort elsewhere.
+__device__ __forceinline__ bool ring_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (ring_try(bar, parity)) return true;
+    const unsigned long long t0 = gtimer();
+    while (!ring_try(bar, parity)) {
+        if (*abort_flag) return false;
+        if (gtimer() - t0 > kRingWaitNs) { *abort_flag = 1; return false; }
+    }
+    return true;
+}
+__device__ __forceinline__ void ring_release() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Issue segment c (elements [c*SEG, c*SEG + len)) of NQ rows into stage k % kRingNS.
+template <typename T, int NQ>
+__device__ __forceinline__ void ring_issue(uint32_t ring, uint32_t bars, int stage_bytes,
+                                           int seg_bytes, long long k, const T* const* rows,
+                                           int c, int SEG, int len)
+{
+    const int s = (int)(k % kRingNS);
+    const uint32_t bar = bars + 8u * s;
+    const uint32_t bytes = (uint32_t)(len * (int)sizeof(T));
+    ring_expect(bar, bytes * NQ);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+        ring_copy(ring + (uint32_t)(s * stage_bytes + q * seg_bytes), rows[q] + (size_t)c * SEG, bytes, bar);
+}
+
+// After an abort: let every copy a warp issued land before the CTA can exit.
+__device__ __forceinline__ void ring_drain(uint32_t bars, long long issued, long long consumed) {
+    for (long long k = consumed; k < issued; ++k) {
+        const uint32_t bar = bars + 8u * (uint32_t)(k % kRingNS);
+        const unsigned long long t0 = gtimer();
+        while (!ring_try(bar, (uint32_t)((k / kRingNS) & 1)) && gtimer() - t0 < kRingWaitNs) {}
+    }
+}
+
+constexpr int kGuSegBytes = 1024;    // bytes per row segment, gate/up kernel (4 rows per stage)
+constexpr int kDnSegBytes = 2048;    // bytes per row segment, down kernel (2 rows per stage)
+constexpr int kXTileBytes = 65536;   // activation tile of the gate/up kernel
+constexpr int kHTileBytes = 81920;   // H tile of the down kernel
+
+__host__ __device__ constexpr int stream_gateup_smem() {
+    return kXTileBytes + 8 * kRingNS * 4 * kGuSegBytes + 8 * kRingNS * 8 + 16;
+}
+__host__ __device__ constexpr int stream_down_smem() {
+    return kHTileBytes + 8 * kRingNS * 2 * kDnSegBytes + 8 * kRingNS * 8 + 16;
+}
+
+// Producer cursor of the gate/up kernel: position (item, pass p0, segment c) in the warp's
+// segment stream, with the item's four weight rows.  The consumer walks the same sequence,
+// so the producer can run kRingNS segments ahead across item and pass boundaries.
+template <typename T>
+struct GuCursor {
+    long item;
+    int p0, c, m;
+    const T* rows[4];
+    bool valid;
+};
+
 template <typename T, typename TH>
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void gu_rows(const StreamArgs& a, const ItemView& v, int warp,
+                                        const T** rows)
+{
+    const T* wbase = v.expert < 0 ? static_cast<const T*>(a.wsgu)
+                                  : static_cast<const T*>(a.wgu) + (size_t)v.expert * 2 * a.F * a.D;
+    const int f0 = v.rb * kStreamR + warp * kStreamNR;
+#pragma unroll
+    for (int q = 0; q < kStreamNR; ++q) {
+        const int f = f0 + q;
+        rows[2 * q] = wbase + ((size_t)(f >> 7) * 256 + (f & 127)) * a.D;
+        rows[2 * q + 1] = rows[2 * q] + (size_t)128 * a.D;
+    }
+}
+
+// H[i][f] = silu(sum_d Wg[f][d] x_i[d]) * (sum_d Wu[f][d] x_i[d]) for the group's tokens i.
+// T: storage type of x and the gate/up weights; TH: type of H.  Each warp owns two
+// intermediate rows of an item (four weight streams: gate f, up f, gate f+1, up f+1).
+template <typename T, typename TH>
+__global__ void __launch_bounds__(256, 1)
 stream_gateup_kernel(StreamArgs a)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    T* xs = reinterpret_cast<T*>(smem_raw);  // [kStreamMT][D]
-    pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = a.D;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     constexpr int VN = Vec<T>::N;
+    constexpr int SEG = kGuSegBytes / (int)sizeof(T);
+    constexpr int STAGE = 4 * kGuSegBytes;
+    T* xs = reinterpret_cast<T*>(smem_raw);
+    unsigned char* ring_p = smem_raw + kXTileBytes;
+    uint64_t* bars_p = reinterpret_cast<uint64_t*>(ring_p + 8 * kRingNS * STAGE);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_p + 8 * kRingNS);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ring = smem_addr(ring_p) + (uint32_t)(warp * kRingNS * STAGE);
+    const uint32_t bars = smem_addr(bars_p) + (uint32_t)(warp * kRingNS * 8);
+    const unsigned char* ring_g = ring_p + warp * kRingNS * STAGE;
+    if (lane == 0)
+        for (int s = 0; s < kRingNS; ++s) ring_bar_init(bars + 8u * s);
+    if (threadIdx.x == 0) *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    pdl_wait();
+
+    const int D = a.D;
+    const int MTX = min(kStreamMT, kXTileBytes / (D * (int)sizeof(T)));
     const int ng = *a.n_groups;
     const int rb_routed = a.F / kStreamR;
     const int rb_shared = a.Fsh / kStreamR;
     const long total = (long)rb_shared + (long)ng * rb_routed;
+    const int nseg = (D + SEG - 1) / SEG;
     const void* cached = nullptr;
     int cached_rows = 0;
+    // ok turns false (warp-uniformly) when a wait gives up; the warp then keeps walking the
+    // same loops, so every __syncthreads is still reached, but issues and computes nothing.
+    bool ok = true;
 
+    // ---- producer (lane 0 issues; every lane keeps the cursor so the state stays uniform)
+    GuCursor<T> pc;
+    auto load = [&]() {
+        pc.valid = pc.item < total;
+        if (pc.valid) {
+            const ItemView v = stream_item<T, TH>(a, pc.item, rb_shared, rb_routed, ng);
+            pc.m = v.m;
+            gu_rows<T, TH>(a, v, warp, pc.rows);
+        }
+    };
+    pc.item = blockIdx.x; pc.p0 = 0; pc.c = 0;
+    load();
+    long long k_issue = 0, k_cons = 0;
+    auto produce = [&]() {
+        if (!ok || !pc.valid) return;
+        if (lane == 0) {
+            ring_release();
+            ring_issue<T, 4>(ring, bars, STAGE, kGuSegBytes, k_issue, pc.rows, pc.c, SEG,
+                             min(SEG, D - pc.c * SEG));
+        }
+        ++k_issue;
+        if (++pc.c == nseg) {
+            pc.c = 0;
+            pc.p0 += MTX;
+            if (pc.p0 >= pc.m) { pc.p0 = 0; pc.item += gridDim.x; load(); }
+        }
+    };
+    for (int i = 0; i < kRingNS; ++i) produce();
+
+    // ---- consumer
     for (long item = blockIdx.x; item < total; item += gridDim.x) {
-        ItemView v = stream_item<T, TH>(a, item, rb_shared, rb_routed, ng);
-        const T* wbase = v.expert < 0 ? static_cast<const T*>(a.wsgu)
-                                      : static_cast<const T*>(a.wgu) + (size_t)v.expert * 2 * a.F * D;
-        for (int p0 = 0; p0 < v.m; p0 += kStreamMT) {
-            const int mp = min(kStreamMT, v.m - p0);
+        const ItemView v = stream_item<T, TH>(a, item, rb_shared, rb_routed, ng);
+        const int f0 = v.rb * kStreamR + warp * kStreamNR;
+        for (int p0 = 0; p0 < v.m; p0 += MTX) {
+            const int mp = min(MTX, v.m - p0);
             const T* src = static_cast<const T*>(v.act) + (size_t)p0 * D;
             if (src != cached || mp != cached_rows) {
                 __syncthreads();
@@ -104,52 +267,51 @@ stream_gateup_kernel(StreamArgs a)
                 cached = src;
                 cached_rows = mp;
             }
-            const int f0 = v.rb * kStreamR + warp * kStreamNR;
-            const T* wg[kStreamNR];
-            const T* wu[kStreamNR];
+            float acc[4][kStreamMT];
 #pragma unroll
-            for (int q = 0; q < kStreamNR; ++q) {
-                const int f = f0 + q;
-                wg[q] = wbase + ((size_t)(f >> 7) * 256 + (f & 127)) * D;
-                wu[q] = wg[q] + (size_t)128 * D;
-            }
-            float ag[kStreamNR][kStreamMT], au[kStreamNR][kStreamMT];
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int q = 0; q < kStreamNR; ++q)
+                for (int i = 0; i < kStreamMT; ++i) acc[q][i] = 0.f;
+            for (int c = 0; c < nseg && ok; ++c) {
+                const long long k = k_cons;
+                ok = __all_sync(0xffffffffu, ring_wait(bars + 8u * (uint32_t)(k % kRingNS),
+                                                       (uint32_t)((k / kRingNS) & 1), abort_flag));
+                if (!ok) break;
+                const unsigned char* st = ring_g + (k % kRingNS) * STAGE;
+                const int len = min(SEG, D - c * SEG);
+                for (int e = lane * VN; e < len; e += 32 * VN) {
+                    float w[4][VN];
 #pragma unroll
-                for (int i = 0; i < kStreamMT; ++i) { ag[q][i] = 0.f; au[q][i] = 0.f; }
-
-            for (int d = lane * VN; d < D; d += 32 * VN) {
-                uint4 rg[kStreamNR], ru[kStreamNR];
+                    for (int q = 0; q < 4; ++q)
+                        Vec<T>::widen(*reinterpret_cast<const uint4*>(st + q * kGuSegBytes + e * sizeof(T)), w[q]);
 #pragma unroll
-                for (int q = 0; q < kStreamNR; ++q) { rg[q] = ldg_stream(wg[q] + d); ru[q] = ldg_stream(wu[q] + d); }
+                    for (int i = 0; i < kStreamMT; ++i) {
+                        if (i < mp) {
+                            float xv[VN];
+                            Vec<T>::widen(*reinterpret_cast<const uint4*>(xs + (size_t)i * D + c * SEG + e), xv);
 #pragma unroll
-                for (int i = 0; i < kStreamMT; ++i) {
-                    if (i < mp) {
-                        float xv[VN];
-                        Vec<T>::widen(*reinterpret_cast<const uint4*>(xs + (size_t)i * D + d), xv);
+                            for (int q = 0; q < 4; ++q) {
+                                float sacc = 0.f;
 #pragma unroll
-                        for (int q = 0; q < kStreamNR; ++q) {
-                            float wgv[VN], wuv[VN];
-                            Vec<T>::widen(rg[q], wgv);
-                            Vec<T>::widen(ru[q], wuv);
-                            float sg = 0.f, su = 0.f;
-#pragma unroll
-                            for (int j = 0; j < VN; ++j) { sg = fmaf(wgv[j], xv[j], sg); su = fmaf(wuv[j], xv[j], su); }
-                            ag[q][i] += sg;
-                            au[q][i] += su;
+                                for (int j = 0; j < VN; ++j) sacc = fmaf(w[q][j], xv[j], sacc);
+                                acc[q][i] += sacc;
+                            }
                         }
                     }
                 }
+                ++k_cons;
+                __syncwarp();
+                produce();
             }
+            if (!ok) continue;
             TH* hout = static_cast<TH*>(v.hrow);
 #pragma unroll
             for (int q = 0; q < kStreamNR; ++q) {
 #pragma unroll
                 for (int i = 0; i < kStreamMT; ++i) {
                     if (i < mp) {
-                        const float g = warp_sum(ag[q][i]);
-                        const float u = warp_sum(au[q][i]);
+                        const float g = warp_sum(acc[2 * q][i]);
+                        const float u = warp_sum(acc[2 * q + 1][i]);
                         if (lane == 0)
                             hout[(size_t)(p0 + i) * v.FF + f0 + q] = from_float<TH>(silu_f(g) * u);
                     }
@@ -157,97 +319,188 @@ stream_gateup_kernel(StreamArgs a)
             }
         }
     }
+    if (!ok && lane == 0) {
+        ring_drain(bars, k_issue, k_cons);
+        atomicOr(a.err, ERR_STREAM_TIMEOUT);
+    }
     pdl_launch_dependents();
 }
 
-// Y[i][j] = sum_f Wd[j][f] H[i][f] for the group's tokens i; H is staged in shared memory in
-// chunks of kFC elements and every warp keeps its two output rows' partial sums in registers.
+// Largest H chunk (a whole number of segments) that fits the H tile for mp token rows.
+template <typename T>
+__device__ __forceinline__ int down_chunk(int mp, int SEG) {
+    return max(SEG, (kHTileBytes / (mp * (int)sizeof(T))) / SEG * SEG);
+}
+
+// Y[i][j] = sum_f Wd[j][f] H[i][f] for the group's tokens i.  Each warp owns two output rows
+// of an item (two weight streams).  H is staged in shared memory in chunks of up to
+// kHTileBytes; the producer cursor runs across chunk, pass and item boundaries, so the next
+// weight segments are already in flight while a chunk of H is being staged.
 // T: type of H and of the down weights.
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
 stream_down_kernel(StreamArgs a)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    constexpr int kFC = 65536 / (kStreamMT * (int)sizeof(T));  // 64 KB of H per stage
-    T* hs = reinterpret_cast<T*>(smem_raw);                    // [kStreamMT][kFC]
-    pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = a.D;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     constexpr int VN = Vec<T>::N;
+    constexpr int SEG = kDnSegBytes / (int)sizeof(T);
+    constexpr int STAGE = 2 * kDnSegBytes;
+    T* hs = reinterpret_cast<T*>(smem_raw);
+    unsigned char* ring_p = smem_raw + kHTileBytes;
+    uint64_t* bars_p = reinterpret_cast<uint64_t*>(ring_p + 8 * kRingNS * STAGE);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_p + 8 * kRingNS);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ring = smem_addr(ring_p) + (uint32_t)(warp * kRingNS * STAGE);
+    const uint32_t bars = smem_addr(bars_p) + (uint32_t)(warp * kRingNS * 8);
+    const unsigned char* ring_g = ring_p + warp * kRingNS * STAGE;
+    if (lane == 0)
+        for (int s = 0; s < kRingNS; ++s) ring_bar_init(bars + 8u * s);
+    if (threadIdx.x == 0) *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    pdl_wait();
+
+    const int D = a.D;
     const int ng = *a.n_groups;
     const int rb_routed = D / kStreamR;
     const int rb_shared = a.Fsh > 0 ? D / kStreamR : 0;
     const long total = (long)rb_shared + (long)ng * rb_routed;
+    bool ok = true;  // as in the gate/up kernel: a warp that gave up still reaches every barrier
 
+    // ---- producer cursor: (item, pass p0, chunk start c0, segment c)
+    struct {
+        long item;
+        int p0, c0, c, m, FF, cap;
+        const T* rows[2];
+        bool valid;
+    } pc;
+    auto load = [&]() {
+        pc.valid = pc.item < total;
+        if (pc.valid) {
+            const ItemView v = stream_item<T, T>(a, pc.item, rb_shared, rb_routed, ng);
+            const T* wbase = v.expert < 0 ? static_cast<const T*>(a.wsd)
+                                          : static_cast<const T*>(a.wd) + (size_t)v.expert * D * a.F;
+            const int j0 = v.rb * kStreamR + warp * kStreamNR;
+            pc.m = v.m;
+            pc.FF = v.FF;
+            pc.rows[0] = wbase + (size_t)j0 * v.FF;
+            pc.rows[1] = wbase + (size_t)(j0 + 1) * v.FF;
+            pc.p0 = 0; pc.c0 = 0; pc.c = 0;
+            pc.cap = down_chunk<T>(min(kStreamMT, pc.m), SEG);
+        }
+    };
+    pc.item = blockIdx.x;
+    load();
+    long long k_issue = 0, k_cons = 0;
+    auto produce = [&]() {
+        if (!ok || !pc.valid) return;
+        const int fl = min(pc.cap, pc.FF - pc.c0);
+        const int nseg = (fl + SEG - 1) / SEG;
+        if (lane == 0) {
+            const T* crow[2] = {pc.rows[0] + pc.c0, pc.rows[1] + pc.c0};
+            ring_release();
+            ring_issue<T, 2>(ring, bars, STAGE, kDnSegBytes, k_issue, crow, pc.c, SEG,
+                             min(SEG, fl - pc.c * SEG));
+        }
+        ++k_issue;
+        if (++pc.c == nseg) {
+            pc.c = 0;
+            pc.c0 += pc.cap;
+            if (pc.c0 >= pc.FF) {
+                pc.c0 = 0;
+                pc.p0 += kStreamMT;
+                if (pc.p0 >= pc.m) { pc.item += gridDim.x; load(); }
+                else pc.cap = down_chunk<T>(min(kStreamMT, pc.m - pc.p0), SEG);
+            }
+        }
+    };
+    for (int i = 0; i < kRingNS; ++i) produce();
+
+    // ---- consumer
     for (long item = blockIdx.x; item < total; item += gridDim.x) {
-        ItemView v = stream_item<T, T>(a, item, rb_shared, rb_routed, ng);
-        const T* wbase = v.expert < 0 ? static_cast<const T*>(a.wsd)
-                                      : static_cast<const T*>(a.wd) + (size_t)v.expert * D * a.F;
+        const ItemView v = stream_item<T, T>(a, item, rb_shared, rb_routed, ng);
         const int FF = v.FF;
         const int j0 = v.rb * kStreamR + warp * kStreamNR;
         for (int p0 = 0; p0 < v.m; p0 += kStreamMT) {
             const int mp = min(kStreamMT, v.m - p0);
+            const int cap = down_chunk<T>(mp, SEG);
             const T* hsrc = static_cast<const T*>(v.hrow) + (size_t)p0 * FF;
-            float acc[kStreamNR][kStreamMT];
+            float acc[2][kStreamMT];
 #pragma unroll
-            for (int q = 0; q < kStreamNR; ++q)
+            for (int q = 0; q < 2; ++q)
 #pragma unroll
                 for (int i = 0; i < kStreamMT; ++i) acc[q][i] = 0.f;
-            for (int c0 = 0; c0 < FF; c0 += kFC) {
-                const int fl = min(kFC, FF - c0);
+            for (int c0 = 0; c0 < FF; c0 += cap) {
+                const int fl = min(cap, FF - c0);
+                const int nseg = (fl + SEG - 1) / SEG;
                 __syncthreads();
                 const int vpr = fl / VN;
                 for (int q = threadIdx.x; q < mp * vpr; q += blockDim.x) {
-                    const int i = q / vpr, c = q - i * vpr;
-                    reinterpret_cast<uint4*>(hs + (size_t)i * kFC)[c] =
-                        reinterpret_cast<const uint4*>(hsrc + (size_t)i * FF + c0)[c];
+                    const int i = q / vpr, cc = q - i * vpr;
+                    reinterpret_cast<uint4*>(hs + (size_t)i * cap)[cc] =
+                        reinterpret_cast<const uint4*>(hsrc + (size_t)i * FF + c0)[cc];
                 }
                 __syncthreads();
-                const T* wr[kStreamNR];
+                for (int c = 0; c < nseg && ok; ++c) {
+                    const long long k = k_cons;
+                    ok = __all_sync(0xffffffffu, ring_wait(bars + 8u * (uint32_t)(k % kRingNS),
+                                                           (uint32_t)((k / kRingNS) & 1), abort_flag));
+                    if (!ok) break;
+                    const unsigned char* st = ring_g + (k % kRingNS) * STAGE;
+                    const int len = min(SEG, fl - c * SEG);
+                    for (int e = lane * VN; e < len; e += 32 * VN) {
+                        float w[2][VN];
 #pragma unroll
-                for (int q = 0; q < kStreamNR; ++q) wr[q] = wbase + (size_t)(j0 + q) * FF + c0;
-                for (int f = lane * VN; f < fl; f += 32 * VN) {
-                    uint4 rw[kStreamNR];
+                        for (int q = 0; q < 2; ++q)
+                            Vec<T>::widen(*reinterpret_cast<const uint4*>(st + q * kDnSegBytes + e * sizeof(T)), w[q]);
 #pragma unroll
-                    for (int q = 0; q < kStreamNR; ++q) rw[q] = ldg_stream(wr[q] + f);
+                        for (int i = 0; i < kStreamMT; ++i) {
+                            if (i < mp) {
+                                float hv[VN];
+                                Vec<T>::widen(*reinterpret_cast<const uint4*>(hs + (size_t)i * cap + c * SEG + e), hv);
 #pragma unroll
-                    for (int i = 0; i < kStreamMT; ++i) {
-                        if (i < mp) {
-                            float hv[VN];
-                            Vec<T>::widen(*reinterpret_cast<const uint4*>(hs + (size_t)i * kFC + f), hv);
+                                for (int q = 0; q < 2; ++q) {
+                                    float sacc = 0.f;
 #pragma unroll
-                            for (int q = 0; q < kStreamNR; ++q) {
-                                float wv[VN];
-                                Vec<T>::widen(rw[q], wv);
-                                float s = 0.f;
-#pragma unroll
-                                for (int j = 0; j < VN; ++j) s = fmaf(wv[j], hv[j], s);
-                                acc[q][i] += s;
+                                    for (int j = 0; j < VN; ++j) sacc = fmaf(w[q][j], hv[j], sacc);
+                                    acc[q][i] += sacc;
+                                }
                             }
                         }
                     }
+                    ++k_cons;
+                    __syncwarp();
+                    produce();
                 }
             }
+            if (!ok) continue;
 #pragma unroll
-            for (int q = 0; q < kStreamNR; ++q) {
+            for (int q = 0; q < 2; ++q) {
 #pragma unroll
                 for (int i = 0; i < kStreamMT; ++i) {
                     if (i < mp) {
-                        const float s = warp_sum(acc[q][i]);
-                        if (lane == 0) v.yrow[(size_t)(p0 + i) * D + j0 + q] = s;
+                        const float sum = warp_sum(acc[q][i]);
+                        if (lane == 0) v.yrow[(size_t)(p0 + i) * D + j0 + q] = sum;
                     }
                 }
             }
         }
+    }
+    if (!ok && lane == 0) {
+        ring_drain(bars, k_issue, k_cons);
+        atomicOr(a.err, ERR_STREAM_TIMEOUT);
     }
     pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------- combine
 // y[t] = sum over slots k in rank order with keep = 1 of g_hat[t][k] * Y_perm[inv[t][k]],
-// plus the shared-expert output; a fixed order, so the result is bit-reproducible.
+// plus the shared-expert output; a fixed order, so the result is bit-reproducible.  When the
+// down projection ran split-K, Y_perm / Y_sh hold `splits` partial slices `stride` floats
+// apart, added in slice order before the gate is applied.
 __global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ yperm, const float* __restrict__ ysh,
+combine_kernel(const float* __restrict__ yperm, int splits, long long stride,
+               const float* __restrict__ ysh, int splits_sh, long long stride_sh,
                const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K, int D,
                float* __restrict__ y)
 {
@@ -256,20 +509,28 @@ combine_kernel(const float* __restrict__ yperm, const float* __restrict__ ysh,
     if (t < T) {
         const int D4 = D >> 2;
         const float4* Y = reinterpret_cast<const float4*>(yperm);
+        const long long s4 = stride >> 2, ssh4 = stride_sh >> 2;
         for (int c = threadIdx.x; c < D4; c += blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int k = 0; k < K; ++k) {
                 const int p = inv[(size_t)t * K + k];
                 if (p >= 0) {
                     const float g = ghat[(size_t)t * K + k];
-                    const float4 v = Y[(size_t)p * D4 + c];
+                    float4 v = Y[(size_t)p * D4 + c];
+                    for (int s = 1; s < splits; ++s) {
+                        const float4 w = Y[s * s4 + (size_t)p * D4 + c];
+                        v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                    }
                     acc.x = fmaf(g, v.x, acc.x); acc.y = fmaf(g, v.y, acc.y);
                     acc.z = fmaf(g, v.z, acc.z); acc.w = fmaf(g, v.w, acc.w);
                 }
             }
             if (ysh) {
-                const float4 s = reinterpret_cast<const float4*>(ysh)[(size_t)t * D4 + c];
-                acc.x += s.x; acc.y += s.y; acc.z += s.z; acc.w += s.w;
+                const float4* S = reinterpret_cast<const float4*>(ysh);
+                for (int s = 0; s < splits_sh; ++s) {
+                    const float4 w = S[s * ssh4 + (size_t)t * D4 + c];
+                    acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
+                }
             }
             reinterpret_cast<float4*>(y)[(size_t)t * D4 + c] = acc;
         }

@@ -6,9 +6,12 @@
 //   GEMM2  Y_g[t][n] = H_g[t] . W_d[n]^T
 // Design (sm_100a):
 //   * one persistent CTA per SM walks a tile list derived on the device from the group table:
-//     tiles are (problem, group, n tile, m tile) with the m tile fastest, so CTAs running at
-//     the same time share a weight tile through L2; groups with no kept token have no tile,
-//     so their weights are never read;
+//     tiles are (problem, group, n tile, K split, m tile) with the m tile fastest, so CTAs
+//     running at the same time share a weight tile through L2; groups with no kept token have
+//     no tile, so their weights are never read;
+//   * small batches split K across tiles so that a handful of kept groups still spreads over
+//     every SM: the f32-store epilogue then writes per-split partial sums, which the next step
+//     adds in a fixed order (the SwiGLU finishing kernel for gate/up, the combine for down);
 //   * tile 128 (tokens) x 256 x 64, TMA (cp.async.bulk.tensor, 128-byte swizzle, no cluster
 //     multicast) fills a 4-stage shared-memory ring guarded by mbarriers;
 //   * warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma (kind::f16, fp32
@@ -54,6 +57,10 @@ struct TcParams {
     int n_tiles_shared;
     int k_steps_routed;     // K / 64
     int k_steps_shared;
+    int k_splits_routed;    // split-K factor (1 = whole K per tile)
+    int k_splits_shared;
+    long long split_stride_routed;  // elements between the outputs of consecutive K splits
+    long long split_stride_shared;
     int shared_rows;        // T, or 0 when there is no shared group
     int* err;
 };
@@ -175,8 +182,15 @@ struct Tile {
     int mt;       // m tile inside the group
     int n;        // n tile
     int brow;     // first weight row of the tile
-    int ksteps;
+    int k0, k1;   // k steps [k0, k1) of this tile (its K split)
+    int ks;       // K split index (selects the output slice)
 };
+
+__device__ __forceinline__ void split_range(int ksteps, int splits, int ks, int& k0, int& k1) {
+    const int per = (ksteps + splits - 1) / splits;
+    k0 = min(ksteps, ks * per);
+    k1 = min(ksteps, k0 + per);
+}
 
 // Walks tiles blockIdx.x, blockIdx.x + gridDim.x, ... in order; every role of a CTA holds
 // its own copy and sees the same sequence.
@@ -193,37 +207,44 @@ struct TileWalker {
         p = p_;
         ng = ng_;
         mts_sh = p->shared_rows > 0 ? (p->shared_rows + BM - 1) / BM : 0;
-        count_sh = mts_sh * p->n_tiles_shared;
+        count_sh = mts_sh * p->n_tiles_shared * p->k_splits_shared;
         next = blockIdx.x;
         g = 0;
         g_base = count_sh;
     }
+    // tile index order inside a problem: m tile fastest, then K split, then n tile
     __device__ bool get(Tile& t) {
         const long long i = next;
         next += gridDim.x;
         if (i < count_sh) {
+            const int per_n = mts_sh * p->k_splits_shared;
             t.shared = 1;
-            t.n = (int)(i / mts_sh);
-            t.mt = (int)(i % mts_sh);
+            t.n = (int)(i / per_n);
+            const int r = (int)(i % per_n);
+            t.ks = r / mts_sh;
+            t.mt = r % mts_sh;
             t.row0 = 0;
             t.m = p->shared_rows;
             t.brow = t.n * BN;
-            t.ksteps = p->k_steps_shared;
+            split_range(p->k_steps_shared, p->k_splits_shared, t.ks, t.k0, t.k1);
             return true;
         }
         while (g < ng) {
             const Group G = p->groups[g];
             const int mts = (G.m + BM - 1) / BM;
-            const long long cnt = (long long)mts * p->n_tiles_routed;
+            const long long cnt = (long long)mts * p->n_tiles_routed * p->k_splits_routed;
             if (i < g_base + cnt) {
                 const long long r = i - g_base;
+                const int per_n = mts * p->k_splits_routed;
                 t.shared = 0;
-                t.n = (int)(r / mts);
-                t.mt = (int)(r % mts);
+                t.n = (int)(r / per_n);
+                const int rr = (int)(r % per_n);
+                t.ks = rr / mts;
+                t.mt = rr % mts;
                 t.row0 = G.row0;
                 t.m = G.m;
                 t.brow = G.expert * p->b_rows_per_expert + t.n * BN;
-                t.ksteps = p->k_steps_routed;
+                split_range(p->k_steps_routed, p->k_splits_routed, t.ks, t.k0, t.k1);
                 return true;
             }
             g_base += cnt;
@@ -293,7 +314,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             const CUtensorMap* am = t.shared ? &p.a_shared : &p.a_routed;
             const CUtensorMap* bm = t.shared ? &p.b_shared : &p.b_routed;
             const int arow = t.row0 + t.mt * BM;
-            for (int k = 0; k < t.ksteps; ++k) {
+            for (int k = t.k0; k < t.k1; ++k) {
                 if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
                 mbar_expect_tx(full_bar(s), STAGE_BYTES);
                 const uint32_t sa = base + s * STAGE_BYTES;
@@ -326,7 +347,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             if (!mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-            for (int k = 0; k < t.ksteps; ++k) {
+            for (int k = t.k0; k < t.k1; ++k) {
                 if (!mbar_wait(full_bar(s), ph, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = base + s * STAGE_BYTES;
@@ -334,7 +355,8 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                 const uint64_t bd = sw128_desc(sa + A_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
-                    tc_mma_f16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (k | kk) != 0);
+                    tc_mma_f16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc,
+                               (k != t.k0 || kk != 0) ? 1u : 0u);
                 issued = true;
                 tc_commit(empty_bar(s));
                 if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -388,7 +410,8 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             } else {
                 float* out = static_cast<float*>(t.shared ? p.out_shared : p.out_routed);
                 const int ld = t.shared ? p.ld_shared : p.ld_routed;
-                float* orow = out + (size_t)(t.row0 + r) * ld + t.n * BN;
+                const long long sstride = t.shared ? p.split_stride_shared : p.split_stride_routed;
+                float* orow = out + (size_t)t.ks * sstride + (size_t)(t.row0 + r) * ld + t.n * BN;
 #pragma unroll 1
                 for (int j = 0; j < BN / 32; ++j) {
                     float v[32];
@@ -416,6 +439,40 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                      ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    }
+    pdl_launch_dependents();
+}
+
+// Finishing step of a split-K gate/up GEMM: H[r][f] = silu(sum_s G[s][r][gate f]) *
+// (sum_s G[s][r][up f]), with the per-split partials G [splits][rows][2F] laid out like the
+// gate/up weight rows (128 gate columns, then the same 128 up columns).  Splits are added in
+// index order.  Routed rows: n_rows = offsets[E] read on the device; shared rows: T.
+__global__ void __launch_bounds__(256)
+swiglu_finish_kernel(const float* __restrict__ g, int splits, long long stride,
+                     const int* __restrict__ n_rows_ptr, int F, __half* __restrict__ h,
+                     const float* __restrict__ gsh, int splits_sh, long long stride_sh,
+                     int rows_sh, int Fsh, __half* __restrict__ hsh)
+{
+    pdl_wait();
+    const long long nr = (long long)(*n_rows_ptr) * F;
+    const long long ns = (long long)rows_sh * Fsh;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nr + ns;
+         i += (long long)gridDim.x * blockDim.x) {
+        const bool shared = i >= nr;
+        const long long j = shared ? i - nr : i;
+        const int FF = shared ? Fsh : F;
+        const long long r = j / FF;
+        const int f = (int)(j % FF);
+        const long long base = r * 2 * FF + (long long)(f >> 7) * 256 + (f & 127);
+        const float* src = shared ? gsh : g;
+        const int ns_ = shared ? splits_sh : splits;
+        const long long st = shared ? stride_sh : stride;
+        float gate = 0.f, up = 0.f;
+        for (int s = 0; s < ns_; ++s) {
+            gate += src[s * st + base];
+            up += src[s * st + base + 128];
+        }
+        (shared ? hsh : h)[r * FF + f] = __float2half_rn(silu_f(gate) * up);
     }
     pdl_launch_dependents();
 }

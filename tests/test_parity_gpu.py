@@ -128,6 +128,14 @@ def test_tensor_path_group_shapes(E, K, T):
     run_case(spec, T, seed=E, path="tensor")
 
 
+@pytest.mark.parametrize("T", [1, 2, 3, 9, 64])
+def test_tensor_path_split_k(T):
+    """Small batches split K: gate/up partials finished by the SwiGLU kernel, down partials
+    added by the combine; the shared group (smaller K) gets its own split count."""
+    spec = _small(d_ff=1024, n_shared=1, d_ff_shared=512)
+    run_case(spec, T, seed=200 + T, path="tensor")
+
+
 def test_tensor_and_stream_paths_agree():
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=128)

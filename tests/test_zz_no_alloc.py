@@ -4,8 +4,11 @@ Some callers cannot allocate device memory at the point where they route, for in
 serving engine that has reserved all free device memory for its own pools, so that a later
 cudaMalloc would fail.  This entry point keeps its scratch in a fixed array compiled into the
 library.  These tests call it through the C ABI and compare it with what beam_moe_forward
-produces for the same tokens (the same router kernels, so the results must match exactly),
-twice in a row on different tokens, so the second call runs on scratch the first one filled.
+produces for the same tokens, twice in a row on different tokens, so the second call runs on
+scratch the first one filled.  The two may compute the logits with a different fp32
+summation order (large bf16 batches use the tensor cores in the forward), so the comparison
+uses the routing tolerance of the parity tests: Top-K ids and keep bits equal wherever the
+decision margin exceeds 1e-3, gates and mask logits within 1e-4.
 
 This file is collected last so that a run stopping at the first failure has run every other
 test before it.
@@ -36,6 +39,21 @@ def _route_noalloc(lib, layer, x, flags=0):
     return st, {k: v.cpu().numpy() for k, v in out.items()}
 
 
+def _compare(got, ref, msg, margin=1e-3):
+    same_ids = (got["topk_id"] == ref["topk_id"]).all(axis=1)
+    # a differing Top-K row is only acceptable at a near-tie of two gates
+    for t in np.nonzero(~same_ids)[0]:
+        g = np.sort(ref["gate"][t])
+        assert np.min(np.diff(g)) < margin, f"{msg}: Top-K differs at token {t} without a tie"
+    assert same_ids.mean() >= 0.99, msg
+    sel = same_ids[:, None] & (np.abs(ref["mask_logit"]) > margin)
+    np.testing.assert_array_equal(got["keep"][sel], ref["keep"][sel], err_msg=msg)
+    np.testing.assert_allclose(got["gate"][same_ids], ref["gate"][same_ids], atol=1e-4, err_msg=msg)
+    np.testing.assert_allclose(got["mask_logit"][same_ids], ref["mask_logit"][same_ids], atol=1e-4,
+                               err_msg=msg)
+    np.testing.assert_array_equal(got["ghat"], got["gate"] * got["keep"], err_msg=msg)
+
+
 @pytest.mark.parametrize("spec,T", [
     (synth.SPECS["tiny"], 64),
     (synth.LayerSpec("small", 512, 16, 4, 256, n_shared=1, d_ff_shared=128), 300),
@@ -53,11 +71,7 @@ def test_route_noalloc_matches_forward_twice(spec, T):
         ref = layer.routing(T)
         st, got = _route_noalloc(lib, layer, x)
         assert st == _lib.BEAM_OK, lib.beam_moe_last_error()
-        np.testing.assert_array_equal(got["topk_id"], ref["topk_id"], err_msg=f"call {call}")
-        np.testing.assert_array_equal(got["keep"], ref["keep"], err_msg=f"call {call}")
-        np.testing.assert_array_equal(got["gate"], ref["gate"], err_msg=f"call {call}")
-        np.testing.assert_array_equal(got["mask_logit"], ref["mask_logit"], err_msg=f"call {call}")
-        np.testing.assert_array_equal(got["ghat"], ref["gate"] * ref["keep"], err_msg=f"call {call}")
+        _compare(got, ref, f"call {call}")
     # the mask-off flag keeps every Top-K slot
     st, got = _route_noalloc(lib, layer, x, flags=_lib.BEAM_MASK_OFF)
     assert st == _lib.BEAM_OK and got["keep"].all()
