@@ -45,10 +45,30 @@ WORKLOADS = {
     "fine-prefill": ("fine", 8192, 0.25),
     "fine-decode32": ("fine", 32, 0.5),
     "tiny": ("tiny", 64, 0.5),
+    # keep-rate sweep of the fine-grained layer (layer time vs Avg-K), plus the plain Top-K
+    "fine-prefill-k100": ("fine", 8192, None),
+    "fine-prefill-k50": ("fine", 8192, 0.5),
+    "fine-prefill-k25": ("fine", 8192, 0.25),
+    "fine-prefill-k10": ("fine", 8192, 0.1),
+    "fine-seg16-prefill": ("fine_seg16", 8192, 0.5),
+    "mixtral-prefill-plain": ("mixtral", 4096, None),
+    "dsv2lite-prefill-high": ("dsv2lite", 8192, 0.07),
+    "dsv2lite-decode1-mid": ("dsv2lite", 1, 0.45),
+    "dsv2lite-decode64-high": ("dsv2lite", 64, 0.07),
+    "qwenmoe-prefill-high": ("qwenmoe", 16384, 0.14),
+    "mixtral-decode1-high": ("mixtral", 1, 0.25),
 }
 DEFAULT_WORKLOAD = "mixtral-prefill"
 # supplementary points measured after the headline in the default run
-EXTRA_POINTS = ["mixtral-decode1", "mixtral-decode8", "mixtral-decode64"]
+EXTRA_POINTS = ["mixtral-decode1", "mixtral-decode8", "mixtral-decode64", "dsv2lite-decode1",
+                "fine-decode32"]
+# every workload, one JSON line each (--sweep)
+SWEEP = ["mixtral-prefill", "mixtral-prefill-high", "mixtral-prefill-plain", "mixtral-decode1",
+         "mixtral-decode1-high", "mixtral-decode8", "mixtral-decode64", "dsv2lite-prefill",
+         "dsv2lite-prefill-high", "dsv2lite-decode1", "dsv2lite-decode1-mid", "dsv2lite-decode64",
+         "dsv2lite-decode64-high", "qwenmoe-prefill", "qwenmoe-prefill-high", "fine-prefill-k100",
+         "fine-prefill-k50", "fine-prefill-k25", "fine-prefill-k10", "fine-seg16-prefill",
+         "fine-decode32", "tiny"]
 
 
 # ------------------------------------------------------------------ environment helpers
@@ -179,6 +199,7 @@ def layer_work(spec, T, st):
     w["combine"] = dict(bytes=nk * D * 4 + (T * D * 4 if Fsh else 0) + T * D * 4 + T * K * 8,
                         flops=2 * nk * D)
     w["scatter_gather"] = dict(bytes=2 * nk * D * es + T * K * 12, flops=0)
+    w["swiglu_finish"] = dict(bytes=(nk * F + T * Fsh) * 2, flops=0)
     total_bytes = (na * 3 * F * D + 3 * Fsh * D + 2 * E * D) * es + T * D * es + T * D * 4
     total_flops = 2 * (nk * 3 * F * D + T * 3 * Fsh * D + Tr * D * 2 * E)
     return w, dict(bytes=total_bytes, flops=total_flops)
@@ -234,6 +255,20 @@ def build_layer(torch, name, device, seed=0):
     return spec, T, keep, layer, x
 
 
+def max_over_ranks(torch, dist, value: float, world: int, device) -> float:
+    """The largest `value` over all ranks (the job time of N replicas); identity for N = 1."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s of N weak-scaled replicas timed by the slowest rank."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
+
+
 def time_steps(torch, dist, layer, x, y, steps, warmup, mask_off, world):
     for _ in range(warmup):
         layer.forward(x, mask_off=mask_off, out=y)
@@ -253,10 +288,7 @@ def time_steps(torch, dist, layer, x, y, steps, warmup, mask_off, world):
     ms = a.elapsed_time(b) / steps
     if world > 1:
         dist.barrier()
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms, launches
+    return max_over_ranks(torch, dist, ms, world, x.device), launches
 
 
 def point(torch, dist, name, steps, warmup, world, device, peaks, mask_off=False):
@@ -277,7 +309,7 @@ def point(torch, dist, name, steps, warmup, world, device, peaks, mask_off=False
     t_roof = max(total["bytes"] / (peaks["hbm"] * 1e9), total["flops"] / (peaks["tc"] * 1e12))
     layer.close()
     return dict(workload=name, tokens=T, keep_rate=keep, mask="off" if mo else "on",
-                value=round(T * world / (ms * 1e-3), 2), ms_per_step=round(ms, 5),
+                value=round(job_throughput(T, world, ms), 2), ms_per_step=round(ms, 5),
                 avg_k=round(st["avg_k"], 4), n_active_experts=st["n_active_experts"],
                 layer_roofline_frac=round(t_roof / (ms * 1e-3), 4), roofline=rl,
                 stage_ms_per_forward={k: round(v[0] / prof["forwards"], 5)
@@ -364,11 +396,7 @@ def run_ours(args):
         layer.forward_host(xh, yh, mask_off=mask_off)
     b.record()
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(torch, dist, a.elapsed_time(b) / e2e_steps, world, device)
 
     # mask off through the same library at the headline shape: the layer speedup from skipping
     y.zero_()
@@ -394,7 +422,7 @@ def run_ours(args):
     if rank == 0:
         line = {
             "metric": "masked MoE-layer tokens/s",
-            "value": round(T * world / (ms * 1e-3), 2),
+            "value": round(job_throughput(T, world, ms), 2),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -417,11 +445,11 @@ def run_ours(args):
             },
             "roofline": rl,
             "layer_roofline_frac": round(t_roof / (ms * 1e-3), 4),
-            "mask_off": {"value": round(T * world / (ms_off * 1e-3), 2),
+            "mask_off": {"value": round(job_throughput(T, world, ms_off), 2),
                          "ms_per_step": round(ms_off, 5),
                          "layer_speedup_from_mask": round(ms_off / ms, 4)},
             "stage_ms_per_forward": {k: round(v[0] / prof["forwards"], 5) for k, v in stages.items()},
-            "e2e": {"value": round(T * world / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+            "e2e": {"value": round(job_throughput(T, world, e2e_ms), 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * spec.d_model * es,
                     "d2h_bytes_per_step": T * spec.d_model * 4},
             "gpu_launches": launches,
@@ -434,6 +462,24 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_sweep(args):
+    """One JSON line per workload on one GPU: tokens/s, the layer roofline fraction, the
+    dominant kernel against its roofline, and the plain Top-K (mask off) time at the shape."""
+    import torch
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    for name in SWEEP:
+        r = point(torch, None, name, args.steps, args.warmup, 1, device, peaks)
+        if r["mask"] == "on":
+            off = point(torch, None, name, args.steps, args.warmup, 1, device, peaks, mask_off=True)
+            r["mask_off_ms_per_step"] = off["ms_per_step"]
+            r["layer_speedup_from_mask"] = round(off["ms_per_step"] / r["ms_per_step"], 4)
+        r["metric"] = "masked MoE-layer tokens/s"
+        r["unit"] = "tokens/s"
+        print(json.dumps(r), flush=True)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
@@ -504,11 +550,15 @@ def main():
     ap.add_argument("--no-points", action="store_true", help="skip the supplementary points")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
+    ap.add_argument("--sweep", action="store_true",
+                    help="measure every workload (one JSON line each) instead of the headline")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

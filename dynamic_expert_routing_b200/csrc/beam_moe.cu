@@ -163,12 +163,13 @@ struct beam_moe {
 enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
-    ST_RESERVED, ST_COUNT
+    ST_SWIGLU_FINISH, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
-    "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router", "reserved"};
+    "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
+    "swiglu_finish"};
 
 static void prof_release(beam_moe* h)
 {
@@ -255,8 +256,8 @@ constexpr int kMinStepsPerSplit = 4;
 // K-split factor that spreads `tiles` output tiles over the SMs, keeping at least
 // kMinStepsPerSplit k steps per slice and no empty slice.
 // Split count s in [1, kMaxSplits] that minimises the wave makespan of `tiles` tiles split
-// s ways on num_sms SMs, ceil(tiles*s/num_sms)/s (in units of one unsplit tile), plus a small
-// charge per extra split for the partial sums it writes and adds back.
+// s ways on num_sms SMs, ceil(tiles*s/num_sms)/s (in units of one unsplit tile), inflated by
+// 4 % per extra split for the per-tile fixed costs and the partial sums written and re-read.
 static int choose_splits(int num_sms, long long tiles)
 {
     if (tiles <= 0) return 1;
@@ -264,7 +265,7 @@ static int choose_splits(int num_sms, long long tiles)
     double best_cost = 1e30;
     for (int s = 1; s <= kMaxSplits; ++s) {
         const double waves = (double)((tiles * s + num_sms - 1) / num_sms);
-        const double cost = waves / s + 0.03 * (s - 1);
+        const double cost = waves / s * (1.0 + 0.04 * (s - 1));
         if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
     }
     return best;
@@ -623,7 +624,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
             BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
                              dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1s));
             const long long work = ((long long)T_ * K * F + (long long)T_ * Fsh);
-            BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::swiglu_finish_kernel,
+            BEAM_CUDA(launch(h, ST_SWIGLU_FINISH, tc::swiglu_finish_kernel,
                              dim3((unsigned)std::min<long long>(h->num_sms * 4, ceil_div(work, 256))),
                              dim3(256), 0, st, (const float*)h->g1part, s1, p.split_stride_routed,
                              (const int*)(h->offsets + E), F, (__half*)h->hbuf,
