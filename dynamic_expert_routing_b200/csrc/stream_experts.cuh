@@ -223,6 +223,7 @@ stream_gateup_kernel(StreamArgs a)
 
     // ---- producer (lane 0 issues; every lane keeps the cursor so the state stays uniform)
     GuCursor<T> pc;
+    pc.item = blockIdx.x; pc.p0 = 0; pc.c = 0; pc.m = 0; pc.valid = false;
     auto load = [&]() {
         pc.valid = pc.item < total;
         if (pc.valid) {
@@ -231,7 +232,6 @@ stream_gateup_kernel(StreamArgs a)
             gu_rows<T, TH>(a, v, warp, pc.rows);
         }
     };
-    pc.item = blockIdx.x; pc.p0 = 0; pc.c = 0;
     load();
     long long k_issue = 0, k_cons = 0;
     auto produce = [&]() {
@@ -374,6 +374,8 @@ stream_down_kernel(StreamArgs a)
         const T* rows[2];
         bool valid;
     } pc;
+    pc.item = blockIdx.x; pc.p0 = 0; pc.c0 = 0; pc.c = 0; pc.m = 0; pc.FF = 0; pc.cap = SEG;
+    pc.valid = false;
     auto load = [&]() {
         pc.valid = pc.item < total;
         if (pc.valid) {
@@ -389,7 +391,6 @@ stream_down_kernel(StreamArgs a)
             pc.cap = down_chunk<T>(min(kStreamMT, pc.m), SEG);
         }
     };
-    pc.item = blockIdx.x;
     load();
     long long k_issue = 0, k_cons = 0;
     auto produce = [&]() {
