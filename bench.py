@@ -33,6 +33,8 @@ WORKLOADS = {
     # device) for ncu captures of the same kernels
     "profile-prefill": ("mixtral", 1024, 0.5, {"n_experts": 4}),
     "profile-decode": ("mixtral", 2, None, {"n_experts": 4}),
+    # reduced fine-grained prefill (2048 tokens) for ncu captures of the small-K down GEMM
+    "profile-fine": ("fine", 2048, 0.5),
     "mixtral-prefill": ("mixtral", 4096, 0.5),
     "mixtral-prefill-high": ("mixtral", 4096, 0.25),
     "mixtral-decode1": ("mixtral", 1, 0.5),

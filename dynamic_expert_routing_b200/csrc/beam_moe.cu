@@ -415,6 +415,8 @@ static beam_status_t setup_tc(beam_moe* h)
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
     BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
     h->tc_ok = true;
     return BEAM_OK;
 }
@@ -597,10 +599,11 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                      (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     // 4. experts (kept groups only) and shared experts
     using TH = typename HType<T>::type;
-    const float* ybase = h->yperm;
-    const float* yshbase = h->Fsh ? h->ysh : nullptr;
+    const void* ybase = h->yperm;
+    const void* yshbase = h->Fsh ? h->ysh : nullptr;
     int ysplits = 1, yshsplits = 1;
     long long ystride = 0, yshstride = 0;
+    bool y_f16 = false;  // unsplit tensor-core outputs are stored in fp16
     if (use_tc) {
         const int Fsh = h->Fsh, F = h->F;
         int s1 = 1, s2 = 1;
@@ -649,14 +652,17 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
             p2.split_stride_shared = (long long)h->split_rows * D;
             ybase = h->ypart; ysplits = s2r; ystride = p2.split_stride_routed;
             if (Fsh) { yshbase = h->ysh_part; yshsplits = s2s; yshstride = p2.split_stride_shared; }
+            BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
         } else {
             p2.k_splits_routed = p2.k_splits_shared = 1;
             p2.out_routed = h->yperm;
             p2.out_shared = h->ysh;
             p2.split_stride_routed = p2.split_stride_shared = 0;
+            y_f16 = true;
+            BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
         }
-        BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
-                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
     } else {
         StreamArgs a;
         a.xperm = h->xperm; a.x = x; a.wgu = h->wgu; a.wsgu = h->wsgu; a.wd = h->wd; a.wsd = h->wsd;
@@ -670,9 +676,14 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          (size_t)stream_down_smem(), st, a));
     }
     // 5. fixed-order combine
-    BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel, dim3(T_), dim3(256), 0, st, ybase, ysplits,
-                     ystride, yshbase, yshsplits, yshstride, (const int*)h->inv,
-                     (const float*)h->ghat, T_, K, D, y));
+    if (y_f16)
+        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<__half>, dim3(T_), dim3(256), 0, st,
+                         (const __half*)ybase, ysplits, ystride, (const __half*)yshbase, yshsplits,
+                         yshstride, (const int*)h->inv, (const float*)h->ghat, T_, K, D, y));
+    else
+        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<float>, dim3(T_), dim3(256), 0, st,
+                         (const float*)ybase, ysplits, ystride, (const float*)yshbase, yshsplits,
+                         yshstride, (const int*)h->inv, (const float*)h->ghat, T_, K, D, y));
     return BEAM_OK;
 }
 

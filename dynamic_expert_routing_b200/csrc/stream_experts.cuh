@@ -497,11 +497,23 @@ stream_down_kernel(StreamArgs a)
 // ---------------------------------------------------------------- combine
 // y[t] = sum over slots k in rank order with keep = 1 of g_hat[t][k] * Y_perm[inv[t][k]],
 // plus the shared-expert output; a fixed order, so the result is bit-reproducible.  When the
-// down projection ran split-K, Y_perm / Y_sh hold `splits` partial slices `stride` floats
-// apart, added in slice order before the gate is applied.
+// down projection ran split-K, Y_perm / Y_sh hold `splits` partial slices `stride` elements
+// apart (fp32), added in slice order before the gate is applied.  TY is the element type of
+// Y_perm / Y_sh: fp16 for unsplit tensor-core outputs of bf16 layers, fp32 otherwise.
+__device__ __forceinline__ float4 load4(const float* p, size_t i) {
+    return reinterpret_cast<const float4*>(p)[i];
+}
+__device__ __forceinline__ float4 load4(const __half* p, size_t i) {
+    const uint2 u = reinterpret_cast<const uint2*>(p)[i];
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <typename TY>
 __global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ yperm, int splits, long long stride,
-               const float* __restrict__ ysh, int splits_sh, long long stride_sh,
+combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
+               const TY* __restrict__ ysh, int splits_sh, long long stride_sh,
                const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K, int D,
                float* __restrict__ y)
 {
@@ -509,7 +521,6 @@ combine_kernel(const float* __restrict__ yperm, int splits, long long stride,
     const int t = blockIdx.x;
     if (t < T) {
         const int D4 = D >> 2;
-        const float4* Y = reinterpret_cast<const float4*>(yperm);
         const long long s4 = stride >> 2, ssh4 = stride_sh >> 2;
         for (int c = threadIdx.x; c < D4; c += blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -517,9 +528,9 @@ combine_kernel(const float* __restrict__ yperm, int splits, long long stride,
                 const int p = inv[(size_t)t * K + k];
                 if (p >= 0) {
                     const float g = ghat[(size_t)t * K + k];
-                    float4 v = Y[(size_t)p * D4 + c];
+                    float4 v = load4(yperm, (size_t)p * D4 + c);
                     for (int s = 1; s < splits; ++s) {
-                        const float4 w = Y[s * s4 + (size_t)p * D4 + c];
+                        const float4 w = load4(yperm, s * s4 + (size_t)p * D4 + c);
                         v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
                     }
                     acc.x = fmaf(g, v.x, acc.x); acc.y = fmaf(g, v.y, acc.y);
@@ -527,9 +538,8 @@ combine_kernel(const float* __restrict__ yperm, int splits, long long stride,
                 }
             }
             if (ysh) {
-                const float4* S = reinterpret_cast<const float4*>(ysh);
                 for (int s = 0; s < splits_sh; ++s) {
-                    const float4 w = S[s * ssh4 + (size_t)t * D4 + c];
+                    const float4 w = load4(ysh, s * ssh4 + (size_t)t * D4 + c);
                     acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
                 }
             }

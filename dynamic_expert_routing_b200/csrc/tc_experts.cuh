@@ -35,11 +35,18 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int kThreads = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*alignment slack*/ + 256 /*barriers*/;
+// Epilogue staging: each of the 4 epilogue warps transposes 32x32 fp32 sub-tiles through its
+// own padded shared-memory buffer (row stride 33 words: conflict-free both ways).
+constexpr int EPI_PITCH = 33;
+constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH * 4;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES + 1024 /*alignment slack*/ +
+                           256 /*barriers*/;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s: far above any tile
 constexpr int ERR_TC_TIMEOUT = 0x100;
 
-enum Epi { EPI_SWIGLU = 0, EPI_STORE_F32 = 1 };
+// Epilogues: SwiGLU -> fp16 H; f32 stores (router logits, split-K partials); f16 stores
+// (unsplit expert outputs Y_perm / Y_sh of bf16 layers).
+enum Epi { EPI_SWIGLU = 0, EPI_STORE_F32 = 1, EPI_STORE_F16 = 2 };
 
 struct TcParams {
     CUtensorMap a_routed;   // activations of the routed groups (rows = kept pairs)
@@ -263,14 +270,16 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
-    // layout: [stage s: A (16 KB) | B (32 KB)] x STAGES, then the barriers
-    const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+    // layout: [stage s: A (16 KB) | B (32 KB)] x STAGES, epilogue buffers, then the barriers
+    float* epi_buf = reinterpret_cast<float*>(gbase + STAGES * STAGE_BYTES);
+    const uint32_t bar0 = base + STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES +
+                                                      8 * (2 * STAGES + 5));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -378,50 +387,54 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         int acc = 0;
         uint32_t aph = 0;
         const int lb = 32 * (warp & 3);  // TMEM lanes this warp may access
+        const int warp_e = warp - 2;     // index of this epilogue warp (its staging buffer)
         while (w.get(t)) {
             if (!mbar_wait(tfull_bar(acc), aph, abort_flag)) break;
             tc_fence_after();
-            const int r = t.mt * BM + lb + lane;  // row inside the group
-            const bool valid = r < t.m;
+            // rows lb .. lb+31 of the tile belong to this warp; row_ok(i) = row i of them is
+            // a row of the group.  Each 32-column chunk goes TMEM -> registers (thread = row)
+            // -> padded shared memory -> registers (thread = column) -> one coalesced store per
+            // row, so every store instruction writes one contiguous row segment.
+            const int r0 = t.mt * BM + lb;                 // first row of this warp, in the group
+            const int nrows = max(0, min(32, t.m - r0));   // valid rows of this warp
             const uint32_t tbase = tmem_base + ((uint32_t)lb << 16) + (uint32_t)(acc * BN);
+            float* buf = epi_buf + warp_e * (32 * EPI_PITCH);
+            const int ld = t.shared ? p.ld_shared : p.ld_routed;
+            const size_t row_base = (size_t)(t.row0 + r0);
             if (EPI == EPI_SWIGLU) {
                 __half* out = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed);
-                const int ld = t.shared ? p.ld_shared : p.ld_routed;
-                __half* orow = out + (size_t)(t.row0 + r) * ld + t.n * (BN / 2);
 #pragma unroll 1
                 for (int j = 0; j < BN / 2 / 32; ++j) {
                     float g[32], u[32];
                     tmem_ld32(tbase + 32 * j, g);
                     tmem_ld32(tbase + BN / 2 + 32 * j, u);
-                    if (valid) {
-                        uint32_t packed[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const __half2 hv = __floats2half2_rn(silu_f(g[2 * i]) * u[2 * i],
-                                                                 silu_f(g[2 * i + 1]) * u[2 * i + 1]);
-                            packed[i] = *reinterpret_cast<const uint32_t*>(&hv);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * j);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-                    }
+                    for (int c = 0; c < 32; ++c) buf[lane * EPI_PITCH + c] = silu_f(g[c]) * u[c];
+                    __syncwarp();
+                    __half* col = out + row_base * ld + (size_t)t.n * (BN / 2) + 32 * j + lane;
+                    for (int i = 0; i < nrows; ++i)
+                        col[(size_t)i * ld] = __float2half_rn(buf[i * EPI_PITCH + lane]);
+                    __syncwarp();
                 }
             } else {
-                float* out = static_cast<float*>(t.shared ? p.out_shared : p.out_routed);
-                const int ld = t.shared ? p.ld_shared : p.ld_routed;
                 const long long sstride = t.shared ? p.split_stride_shared : p.split_stride_routed;
-                float* orow = out + (size_t)t.ks * sstride + (size_t)(t.row0 + r) * ld + t.n * BN;
 #pragma unroll 1
                 for (int j = 0; j < BN / 32; ++j) {
                     float v[32];
                     tmem_ld32(tbase + 32 * j, v);
-                    if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(orow + 32 * j);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    for (int c = 0; c < 32; ++c) buf[lane * EPI_PITCH + c] = v[c];
+                    __syncwarp();
+                    const size_t off = (size_t)t.ks * sstride + row_base * ld + (size_t)t.n * BN + 32 * j + lane;
+                    if (EPI == EPI_STORE_F16) {
+                        __half* col = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed) + off;
+                        for (int i = 0; i < nrows; ++i)
+                            col[(size_t)i * ld] = __float2half_rn(buf[i * EPI_PITCH + lane]);
+                    } else {
+                        float* col = static_cast<float*>(t.shared ? p.out_shared : p.out_routed) + off;
+                        for (int i = 0; i < nrows; ++i) col[(size_t)i * ld] = buf[i * EPI_PITCH + lane];
                     }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
