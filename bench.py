@@ -295,6 +295,11 @@ def time_steps(torch, dist, layer, x, y, steps, warmup, mask_off, world):
 
 def point(torch, dist, name, steps, warmup, world, device, peaks, mask_off=False):
     """Measure one supplementary point (tokens/s, roofline of its dominant kernel)."""
+    with torch.cuda.stream(torch.cuda.Stream(device)):
+        return _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off)
+
+
+def _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off):
     spec, T, keep, layer, x = build_layer(torch, name, device)
     y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
     mo = mask_off or keep is None
@@ -345,6 +350,14 @@ def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_ste
 
 
 def run_ours(args):
+    """Headline run.  Work is issued on a dedicated (non-default) stream, so the library can
+    replay each forward as a captured CUDA graph, as a serving engine would."""
+    import torch
+    with torch.cuda.stream(torch.cuda.Stream()):
+        _run_ours(args)
+
+
+def _run_ours(args):
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -21,6 +21,7 @@ BEAM_DTYPE_BF16 = 1
 BEAM_MASK_OFF = 0x1
 BEAM_PATH_STREAM = 0x2
 BEAM_PATH_TENSOR = 0x4
+BEAM_NO_GRAPH = 0x8
 
 BEAM_N_STAGES = 12
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
@@ -75,6 +76,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.beam_moe_get_routing.argtypes = [P, P, P, P, P, P, P, P]
     lib.beam_moe_route_noalloc.argtypes = [P, P, I, P, P, P, P, P, U, P]
     lib.beam_moe_route_noalloc.restype = ctypes.c_int
+    lib.beam_moe_wait_selftest.argtypes = [I, P]
+    lib.beam_moe_wait_selftest.restype = ctypes.c_int
     lib.beam_moe_profile_begin.argtypes = [P, I]
     lib.beam_moe_profile_end.argtypes = [P, P, P, P]
     lib.beam_moe_stage_name.argtypes = [I]

@@ -151,6 +151,14 @@ struct beam_moe {
     cudaEvent_t done = nullptr;
     int last_T = -1;
     std::vector<void*> allocs;
+    // replay cache: the last forward captured as a CUDA graph, keyed by its arguments
+    cudaGraphExec_t graph_exec = nullptr;
+    const void* g_x = nullptr;
+    float* g_y = nullptr;
+    int g_T = -1;
+    uint32_t g_flags = 0;
+    bool g_tc = false;
+    int g_kernels = 0;   // kernels in the captured graph
     // launch accounting and optional per-stage timing
     long long launches = 0;
     bool prof = false;
@@ -180,8 +188,16 @@ static void prof_release(beam_moe* h)
     h->prof = false;
 }
 
+static void drop_graph(beam_moe* h)
+{
+    if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+    h->graph_exec = nullptr;
+    h->g_T = -1;
+}
+
 static void free_all(beam_moe* h)
 {
+    drop_graph(h);
     prof_release(h);
     for (void* p : h->allocs) cudaFree(p);
     h->allocs.clear();
@@ -825,7 +841,7 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
     if (T > 0 && (!x || !y)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
         return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
-    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR))
+    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH))
         return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
     if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
         return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core expert path needs a bf16 layer with "
@@ -840,11 +856,60 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
     if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
     if (h->prof) ++h->prof_forwards;
     if (T > 0) {
-        if (h->cfg.dtype == BEAM_DTYPE_BF16)
-            BEAM_TRY(forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y,
-                                                 flags, use_tc, st));
-        else
-            BEAM_TRY(forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st));
+        // Replay: the whole forward (8-10 kernels, their tensor maps and split choices) was
+        // captured as a CUDA graph for these exact arguments; one launch replays it.  Not
+        // used while profiling, on the legacy default stream, or with BEAM_NO_GRAPH.
+        const bool graphable = !(flags & BEAM_NO_GRAPH) && !h->prof && st != nullptr;
+        const uint32_t key_flags = flags & ~BEAM_NO_GRAPH;
+        if (graphable && h->graph_exec && h->g_x == x && h->g_y == y && h->g_T == T &&
+            h->g_flags == key_flags && h->g_tc == use_tc) {
+            BEAM_CUDA(cudaGraphLaunch(h->graph_exec, st));
+            h->launches += h->g_kernels;
+        } else {
+            bool captured = false;
+            if (graphable) {
+                cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+                if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone &&
+                    cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
+                    const long long n0 = h->launches;
+                    beam_status_t s1 = (h->cfg.dtype == BEAM_DTYPE_BF16)
+                        ? forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y, flags, use_tc, st)
+                        : forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st);
+                    cudaGraph_t g = nullptr;
+                    cudaError_t e1 = cudaStreamEndCapture(st, &g);
+                    h->launches = n0;  // counted again when the graph runs
+                    if (s1 != BEAM_OK) {
+                        if (g) cudaGraphDestroy(g);
+                        return s1;
+                    }
+                    cudaGraphExec_t ex = nullptr;
+                    if (e1 == cudaSuccess && g && cudaGraphInstantiate(&ex, g, 0) == cudaSuccess) {
+                        size_t nn = 0;
+                        cudaGraphGetNodes(g, nullptr, &nn);
+                        drop_graph(h);
+                        h->graph_exec = ex;
+                        h->g_x = x; h->g_y = y; h->g_T = T; h->g_flags = key_flags; h->g_tc = use_tc;
+                        h->g_kernels = (int)nn;
+                        captured = true;
+                    }
+                    if (g) cudaGraphDestroy(g);
+                    cudaGetLastError();
+                    if (captured) {
+                        BEAM_CUDA(cudaGraphLaunch(h->graph_exec, st));
+                        h->launches += h->g_kernels;
+                    }
+                } else {
+                    cudaGetLastError();
+                }
+            }
+            if (!captured) {
+                if (h->cfg.dtype == BEAM_DTYPE_BF16)
+                    BEAM_TRY(forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y,
+                                                         flags, use_tc, st));
+                else
+                    BEAM_TRY(forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st));
+            }
+        }
     }
     h->last_T = T;
     BEAM_CUDA(cudaEventRecord(h->done, st));
@@ -971,6 +1036,27 @@ const char* beam_moe_stage_name(int32_t stage)
 }
 
 int64_t beam_moe_launch_count(const beam_moe_t* h) { return h ? h->launches : 0; }
+
+static __device__ int g_wait_selftest_result;
+
+beam_status_t beam_moe_wait_selftest(int32_t timeout_us, void* stream)
+{
+    g_err[0] = 0;
+    if (timeout_us < 1 || timeout_us > 2000000)
+        return fail(BEAM_ERR_INVALID_ARG, "timeout_us=%d outside [1, 2000000]", timeout_us);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* res = nullptr;
+    BEAM_CUDA(cudaGetSymbolAddress((void**)&res, g_wait_selftest_result));
+    const int minus_one = -1;
+    BEAM_CUDA(cudaMemcpyAsync(res, &minus_one, sizeof(int), cudaMemcpyHostToDevice, st));
+    tc::wait_selftest_kernel<<<1, 32, 0, st>>>((unsigned long long)timeout_us * 1000ull, res);
+    BEAM_CUDA(cudaGetLastError());
+    int out = -1;
+    BEAM_CUDA(cudaMemcpyAsync(&out, res, sizeof(int), cudaMemcpyDeviceToHost, st));
+    BEAM_CUDA(cudaStreamSynchronize(st));
+    if (out == 2) return fail(BEAM_ERR_TIMEOUT, "the bounded wait expired after %d us, as designed", timeout_us);
+    return fail(BEAM_ERR_CUDA, "the self-test wait did not expire (result %d)", out);
+}
 
 void beam_moe_destroy(beam_moe_t* h)
 {

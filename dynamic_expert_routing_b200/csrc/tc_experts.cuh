@@ -100,18 +100,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait: false when the abort flag is raised or the time limit passes (the caller
-// then raises the flag itself).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait: false when the abort flag is raised elsewhere or the time limit passes (then
+// this thread raises the flag itself).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             return false;
         }
+    }
+}
+
+// Self-test of the bounded wait: one thread waits on an mbarrier whose phase nothing
+// completes (its only expected arrival never comes), with a limit of limit_ns; the wait gives
+// up, raises the abort flag, and the kernel records the outcome (2 = expired as designed,
+// 0 = the phase completed, which cannot happen) and returns normally.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns, int* result)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+        *result = ok ? 0 : (abort_flag ? 2 : 1);
     }
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,

@@ -50,6 +50,7 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_MASK_OFF     0x1u  /* plain Top-K: every Top-K slot kept (the W_m = 0 behaviour) */
 #define BEAM_PATH_STREAM  0x2u  /* force the weight-streaming (GEMV) expert path */
 #define BEAM_PATH_TENSOR  0x4u  /* force the tcgen05 tensor-core expert path (bf16 only) */
+#define BEAM_NO_GRAPH     0x8u  /* launch the kernels directly instead of replaying a graph */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
@@ -108,8 +109,14 @@ beam_status_t beam_moe_create(const beam_moe_config_t *cfg, const beam_moe_weigh
  * experts and the fixed-order combine.  Deterministic: the same inputs give the same bits.
  * T = 0 is a no-op.  T > max_tokens or NULL pointers -> BEAM_ERR_INVALID_ARG.
  * flags: BEAM_MASK_OFF, and at most one of BEAM_PATH_STREAM / BEAM_PATH_TENSOR (by default the
- * path is chosen from T).  x_dev and y_dev must stay valid until the stream reaches the end
- * of the call's work.
+ * path is chosen from T), BEAM_NO_GRAPH.  x_dev and y_dev must stay valid until the stream
+ * reaches the end of the call's work.
+ * Replay: on a non-default stream that is not being captured, the first forward with a given
+ * (x_dev, y_dev, T, flags) is captured into a CUDA graph owned by the handle, and later calls
+ * with the same arguments replay it with one launch (one graph is kept; new arguments replace
+ * it).  The contents of x_dev may change between calls; the pointers may not, for a replay.
+ * BEAM_NO_GRAPH, the legacy default stream, an already-capturing stream and profiling all use
+ * direct kernel launches.
  */
 beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, float *y_dev,
                                uint32_t flags, void *stream);
@@ -179,6 +186,17 @@ int64_t beam_moe_launch_count(const beam_moe_t *h);
 beam_status_t beam_moe_route_noalloc(beam_moe_t *h, const void *x_dev, int32_t T,
                                      int32_t *topk_id, float *gate, float *mask_logit,
                                      uint8_t *keep, float *ghat, uint32_t flags, void *stream);
+
+/*
+ * Self-test of the library's bounded device waits (no counterpart on the BEAM pages): runs one
+ * tiny kernel whose thread waits on an mbarrier that nothing completes, giving up after
+ * timeout_us microseconds (1..2,000,000).  The kernel then records the expiry and returns
+ * normally, so the context stays usable.  Returns BEAM_ERR_TIMEOUT when the wait expired as
+ * designed (the expected outcome); BEAM_ERR_INVALID_ARG for a bad timeout; BEAM_ERR_CUDA
+ * otherwise.  Synchronises `stream`.  Every wait in the forward's kernels uses the same
+ * primitive, with a limit of 2 s.
+ */
+beam_status_t beam_moe_wait_selftest(int32_t timeout_us, void *stream);
 
 /* Free every device buffer of the handle (waits for its pending work).  NULL is ignored. */
 void beam_moe_destroy(beam_moe_t *h);

@@ -63,6 +63,7 @@ def test_null_handle_calls(lib):
     assert lib.beam_moe_stats(None, ctypes.byref(s), None) == BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_get_routing(None, None, None, None, None, None, None, None) == BEAM_ERR_INVALID_ARG
     lib.beam_moe_destroy(None)
+    assert lib.beam_moe_wait_selftest(0, None) == BEAM_ERR_INVALID_ARG
     assert b"sm_100a" in lib.beam_moe_version()
 
 

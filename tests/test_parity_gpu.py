@@ -104,6 +104,48 @@ def test_deterministic_bits():
         np.testing.assert_array_equal(r1[k], r2[k])
 
 
+def test_graph_replay_matches_direct_launches():
+    """On a non-default stream the forward is captured once and replayed; replays must give
+    the same bits as direct launches, also after x's contents change under the same pointer."""
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=96)
+        for T, path in ((96, None), (3, None), (96, "stream")):
+            x = synth.make_tokens(spec, T, seed=1).cuda()
+            y = torch.empty((T, spec.d_model), device="cuda")
+            ref = layer.forward(x, path=path, graph=False).clone()
+            n0 = layer.launch_count()
+            layer.forward(x, path=path, out=y)          # capture + first replay
+            layer.forward(x, path=path, out=y)          # replay
+            assert layer.launch_count() > n0
+            torch.cuda.synchronize()
+            assert torch.equal(y, ref)
+            x.copy_(synth.make_tokens(spec, T, seed=2).cuda())
+            layer.forward(x, path=path, out=y)
+            ref2 = layer.forward(x, path=path, graph=False)
+            torch.cuda.synchronize()
+            assert torch.equal(y, ref2)
+            assert not torch.equal(ref, ref2)
+
+
+def test_bounded_wait_expires_and_the_context_survives():
+    """A wait on an mbarrier nothing completes gives up after its limit and reports
+    BEAM_ERR_TIMEOUT; the GPU context stays usable (a forward afterwards is still correct)."""
+    import time
+    from dynamic_expert_routing_b200 import _lib
+    lib = _lib.load()
+    t0 = time.perf_counter()
+    st = lib.beam_moe_wait_selftest(20000, None)
+    dt = time.perf_counter() - t0
+    assert st == _lib.BEAM_ERR_TIMEOUT, lib.beam_moe_last_error()
+    assert b"as designed" in lib.beam_moe_last_error()
+    assert 0.015 < dt < 5.0
+    run_case(_small(), 40, seed=9)
+
+
 def test_host_buffer_entry_point():
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=128)
