@@ -263,6 +263,8 @@ static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 constexpr int kTcMinTokens = 1;
 // Router logits run on the tensor cores from this many routed rows up (bf16 layers).
 constexpr int kTcRouterMinRows = 64;
+// Small batches gather their kept rows inside the fused routing kernel up to this many bytes.
+constexpr long long kInlineGatherBytes = 256 * 1024;
 // Split-K for small batches on the tensor-core path: up to kMaxSplits K slices per tile, for
 // forwards of at most kSplitMaxTokens tokens (the partial-sum workspaces are sized for that).
 constexpr int kMaxSplits = 8;
@@ -469,7 +471,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
         BEAM_TRY(dalloc(h, &h->hsh, Tm * Fsh * hs));
         BEAM_TRY(dalloc(h, &h->ysh, Tm * D * sizeof(float)));
     }
-    BEAM_TRY(dalloc(h, &h->L, Tm * h->ldL * sizeof(float)));
+    // logits; bf16 layers keep room for K-split slices of the tensor-core router
+    BEAM_TRY(dalloc(h, &h->L, (cfg->dtype == BEAM_DTYPE_BF16 ? kMaxSplits : 1) * Tm * h->ldL * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->topk_id, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->gate, rows * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->mlogit, rows * sizeof(float)));
@@ -558,11 +561,24 @@ static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3
 }
 
 template <int EPL>
-static cudaError_t launch_select(beam_moe* h, int Tr, int T, int mask_off, cudaStream_t st)
+static cudaError_t launch_select(beam_moe* h, int Tr, int T, int mask_off, int splits,
+                                 long long split_stride, cudaStream_t st)
 {
     return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256), 0, st,
-                  (const float*)h->L, h->ldL, Tr, T, h->E, h->K, h->S, mask_off, h->topk_id, h->gate,
-                  h->mlogit, h->keep, h->ghat, h->nkeep_tok, h->lreg_tok);
+                  (const float*)h->L, h->ldL, splits, split_stride, Tr, T, h->E, h->K, h->S,
+                  mask_off, h->topk_id, h->gate, h->mlogit, h->keep, h->ghat, h->nkeep_tok,
+                  h->lreg_tok);
+}
+
+template <int EPL, typename T>
+static cudaError_t launch_small(beam_moe* h, const T* x, int Tr, int T_, int mask_off, int splits,
+                                long long split_stride, int gather, cudaStream_t st)
+{
+    return launch(h, ST_ROUTE_SELECT, route_compact_small_kernel<EPL, T>, dim3(1), dim3(1024), 0, st,
+                  (const float*)h->L, h->ldL, splits, split_stride, Tr, T_, h->E, h->K, h->S,
+                  mask_off, h->topk_id, h->gate, h->mlogit, h->keep, h->ghat, h->nkeep_tok,
+                  h->lreg_tok, h->counts, h->offsets, h->groups, h->n_groups, h->dstats, h->perm,
+                  h->inv, x, (T*)h->xperm, h->D, gather);
 }
 
 template <typename T>
@@ -576,43 +592,72 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
 
     // 1. router logits L = x [W_r | W_m]  (routed rows only: segment leaders when S > 1)
+    int lsplits = 1;
+    long long lstride = 0;
     if (h->tc_ok && Tr >= kTcRouterMinRows) {
         tc::TcParams& p0 = h->p0;
         BEAM_TRY(encode_map(h, &p0.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)Tr,
                             (uint64_t)D, tc::BM, (uint64_t)S * D));
         p0.a_routed = p0.a_shared;
         p0.shared_rows = Tr;
+        // few M tiles: split K so the router covers the SMs; route_select adds the slices
+        const long long tiles = (long long)ceil_div(Tr, tc::BM) * p0.n_tiles_shared;
+        lsplits = normalise_splits(choose_splits(h->num_sms, tiles), D / tc::BK);
+        lstride = (long long)Tr * h->ldL;
+        p0.k_splits_routed = p0.k_splits_shared = lsplits;
+        p0.split_stride_routed = p0.split_stride_shared = lstride;
         BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
-                         dim3(std::min(h->num_sms, ceil_div(Tr, tc::BM) * p0.n_tiles_shared)),
+                         dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
     } else {
         BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
                          dim3(h->n2E, ceil_div(Tr, kGemvRows)),
                          dim3(256), 0, st, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->ldL, h->L));
     }
-    // 2. Top-K, softmax, mask, per-token statistics
+    // 2-3. routing decision and compaction.  Small batches (one 32-token chunk) run them as one
+    // single-CTA kernel; larger ones as select -> bit planes -> scan -> scatter + gather.
     cudaError_t e;
-    switch ((E + 31) / 32) {
-        case 1: e = launch_select<1>(h, Tr, T_, mask_off, st); break;
-        case 2: e = launch_select<2>(h, Tr, T_, mask_off, st); break;
-        case 3: e = launch_select<3>(h, Tr, T_, mask_off, st); break;
-        case 4: e = launch_select<4>(h, Tr, T_, mask_off, st); break;
-        case 5: e = launch_select<5>(h, Tr, T_, mask_off, st); break;
-        case 6: e = launch_select<6>(h, Tr, T_, mask_off, st); break;
-        case 7: e = launch_select<7>(h, Tr, T_, mask_off, st); break;
-        default: e = launch_select<8>(h, Tr, T_, mask_off, st); break;
+    if (T_ <= kSmallT) {
+        const int gather_inline = (long long)T_ * K * D * (long long)sizeof(T) <= kInlineGatherBytes;
+        switch ((E + 31) / 32) {
+            case 1: e = launch_small<1>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            case 2: e = launch_small<2>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            case 3: e = launch_small<3>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            case 4: e = launch_small<4>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            case 5: e = launch_small<5>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            case 6: e = launch_small<6>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            case 7: e = launch_small<7>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+            default: e = launch_small<8>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
+        }
+        BEAM_CUDA(e);
+        if (!gather_inline)
+            BEAM_CUDA(launch(h, ST_SCATTER_GATHER, gather_rows_kernel<T>, dim3(h->num_sms * 2),
+                             dim3(256), 0, st, (const int*)h->perm, (const int*)(h->offsets + E),
+                             K, D, x, (T*)h->xperm));
+    } else {
+        switch ((E + 31) / 32) {
+            case 1: e = launch_select<1>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            case 2: e = launch_select<2>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            case 3: e = launch_select<3>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            case 4: e = launch_select<4>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            case 5: e = launch_select<5>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            case 6: e = launch_select<6>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            case 7: e = launch_select<7>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            default: e = launch_select<8>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+        }
+        BEAM_CUDA(e);
+        BEAM_CUDA(launch(h, ST_COMPACT_BITS, compact_bits_kernel, dim3(ceil_div(nch, 8)), dim3(256), 0, st,
+                         (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, E, nch, h->bits));
+        BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(1), dim3(1024), 0, st,
+                         (const uint32_t*)h->bits, nch, E, T_, (const int*)h->nkeep_tok,
+                         (const float*)h->lreg_tok, h->counts, h->offsets, h->chunk_base, h->groups,
+                         h->n_groups, h->dstats));
+        BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>,
+                         dim3(ceil_div((long long)T_ * K, 8)), dim3(256), 0, st,
+                         (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D, nch,
+                         (const uint32_t*)h->bits, (const int*)h->offsets,
+                         (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     }
-    BEAM_CUDA(e);
-    // 3. compaction: bit planes, scan (+ statistics), scatter + activation gather
-    BEAM_CUDA(launch(h, ST_COMPACT_BITS, compact_bits_kernel, dim3(ceil_div(nch, 8)), dim3(256), 0, st,
-                     (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, E, nch, h->bits));
-    BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(1), dim3(1024), 0, st, (const uint32_t*)h->bits,
-                     nch, E, T_, (const int*)h->nkeep_tok, (const float*)h->lreg_tok, h->counts,
-                     h->offsets, h->chunk_base, h->groups, h->n_groups, h->dstats));
-    BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>, dim3(ceil_div((long long)T_ * K, 8)),
-                     dim3(256), 0, st, (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D,
-                     nch, (const uint32_t*)h->bits, (const int*)h->offsets,
-                     (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     // 4. experts (kept groups only) and shared experts
     using TH = typename HType<T>::type;
     const void* ybase = h->yperm;
@@ -692,12 +737,14 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          (size_t)stream_down_smem(), st, a));
     }
     // 5. fixed-order combine
+    // few tokens: split each token's columns over several CTAs so the combine spans the SMs
+    const dim3 cgrid(T_, T_ < h->num_sms ? ceil_div(D / 4, 256) : 1);
     if (y_f16)
-        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<__half>, dim3(T_), dim3(256), 0, st,
+        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<__half>, cgrid, dim3(256), 0, st,
                          (const __half*)ybase, ysplits, ystride, (const __half*)yshbase, yshsplits,
                          yshstride, (const int*)h->inv, (const float*)h->ghat, T_, K, D, y));
     else
-        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<float>, dim3(T_), dim3(256), 0, st,
+        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<float>, cgrid, dim3(256), 0, st,
                          (const float*)ybase, ysplits, ystride, (const float*)yshbase, yshsplits,
                          yshstride, (const int*)h->inv, (const float*)h->ghat, T_, K, D, y));
     return BEAM_OK;
@@ -742,8 +789,8 @@ static cudaError_t launch_select_into(beam_moe* h, const float* L, int Tr, int T
                                       cudaStream_t st)
 {
     return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256),
-                  0, st, L, h->n2E, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate, mlogit, keep,
-                  ghat, nkeep_tok, lreg_tok);
+                  0, st, L, h->n2E, 1, 0LL, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate,
+                  mlogit, keep, ghat, nkeep_tok, lreg_tok);
 }
 
 template <typename T>

@@ -13,6 +13,7 @@
 //      perm / inv and copies x[t] into row pos of X_perm.
 #pragma once
 #include "common.cuh"
+#include "router.cuh"
 
 namespace beam {
 
@@ -204,6 +205,188 @@ compact_scatter_gather_kernel(const int* __restrict__ topk_id, const uint8_t* __
             const int nv = D * (int)sizeof(TW) / 16;
             for (int v = lane; v < nv; v += 32) dst[v] = src[v];
         }
+    }
+    pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------- small batches, one kernel
+// For T <= 32 tokens (one 32-token chunk) a single 1024-thread CTA does what route_select,
+// compact_bits, compact_scan and compact_scatter_gather do for larger batches, saving three
+// dependent launches on the decode path:
+//   1. warp w < Tr selects routed row w (select_row) and writes the routing of its segment;
+//   2. warp w builds, for experts e = w, w+32, ..., the ballot word of tokens keeping e;
+//   3. warp 0 scans the per-expert counts into offsets, the active-group list and the
+//      statistics (fixed reduction order);
+//   4. every thread places one (token, slot) pair: pos = offsets[e] + popc(word[e] & below(t));
+//   5. optionally, the warps copy the kept tokens' rows into X_perm (small batches only).
+// The results are bit-identical to the multi-kernel path.
+constexpr int kSmallT = 32;
+
+template <int EPL, typename TW>
+__global__ void __launch_bounds__(1024)
+route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, long long split_stride,
+                           int Tr, int T, int E, int K, int seg, int mask_off,
+                           int* __restrict__ topk_id, float* __restrict__ gate,
+                           float* __restrict__ mlogit, uint8_t* __restrict__ keep,
+                           float* __restrict__ ghat, int* __restrict__ nkeep_tok,
+                           float* __restrict__ lreg_tok, int* __restrict__ counts,
+                           int* __restrict__ offsets, Group* __restrict__ groups,
+                           int* __restrict__ n_groups, DevStats* __restrict__ stats,
+                           int* __restrict__ perm, int* __restrict__ inv,
+                           const TW* __restrict__ x, TW* __restrict__ xperm, int D, int gather)
+{
+    __shared__ int s_id[kSmallT][32];
+    __shared__ uint8_t s_keep[kSmallT][32];
+    __shared__ uint32_t s_mask[kSmallT][kMaxE / 32 + 1];  // kept experts of each token (padded row)
+    __shared__ int s_nk[kSmallT];
+    __shared__ float s_lr[kSmallT];
+    __shared__ uint32_t s_word[kMaxE];
+    __shared__ int s_cnt[kMaxE];
+    __shared__ int s_off[kMaxE + 1];
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kSmallT * (kMaxE / 32 + 1); i += blockDim.x)
+        (&s_mask[0][0])[i] = 0u;
+    __syncthreads();
+
+    // 1. selection
+    if (warp < Tr) {
+        const RowDecision d = select_row<EPL>(L + (size_t)warp * ldL, splits, split_stride, E, K,
+                                              mask_off, lane);
+        const int S = seg > 1 ? seg : 1;
+        const int t0 = warp * S, t1 = min(T, t0 + S);
+        for (int t = t0; t < t1; ++t) {
+            if (lane < K) {
+                const size_t o = (size_t)t * K + lane;
+                topk_id[o] = d.id;
+                gate[o] = d.g;
+                mlogit[o] = d.l;
+                keep[o] = d.keep ? 1 : 0;
+                ghat[o] = d.ghat;
+                s_id[t][lane] = d.id;
+                s_keep[t][lane] = d.keep ? 1 : 0;
+                if (d.keep) atomicOr(&s_mask[t][d.id >> 5], 1u << (d.id & 31));  // order-free OR
+            }
+            if (lane == 0) {
+                nkeep_tok[t] = d.nkeep;
+                lreg_tok[t] = d.lreg;
+                s_nk[t] = d.nkeep;
+                s_lr[t] = d.lreg;
+            }
+        }
+    }
+    __syncthreads();
+
+    // 2. one ballot word per expert (lane = token)
+    for (int e = warp; e < E; e += 32) {
+        const bool has = lane < T && ((s_mask[lane][e >> 5] >> (e & 31)) & 1u);
+        const uint32_t word = __ballot_sync(0xffffffffu, has);
+        if (lane == 0) { s_word[e] = word; s_cnt[e] = __popc(word); counts[e] = __popc(word); }
+    }
+    __syncthreads();
+
+    // 3. offsets, active groups, statistics
+    if (warp == 0) {
+        int loc[8], act[8];
+        int sum = 0, nact = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            loc[j] = (e < E) ? s_cnt[e] : 0;
+            act[j] = loc[j] > 0;
+            sum += loc[j];
+            nact += act[j];
+        }
+        int incl = sum, inca = nact;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            const int na = __shfl_up_sync(0xffffffffu, inca, o);
+            if (lane >= o) { incl += n; inca += na; }
+        }
+        int run = incl - sum, runa = inca - nact;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            if (e < E) {
+                offsets[e] = run;
+                s_off[e] = run;
+                if (act[j]) {
+                    Group g;
+                    g.row0 = run; g.m = loc[j]; g.expert = e; g.pad = 0;
+                    groups[runa] = g;
+                    ++runa;
+                }
+            }
+            run += loc[j];
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        const int tact = __shfl_sync(0xffffffffu, inca, 31);
+        long long ks = lane < T ? s_nk[lane] : 0;
+        double ls = lane < T ? (double)s_lr[lane] : 0.0;
+        int nz = (lane < T && s_nk[lane] == 0) ? 1 : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ks += __shfl_xor_sync(0xffffffffu, ks, o);
+            ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            nz += __shfl_xor_sync(0xffffffffu, nz, o);
+        }
+        if (lane == 0) {
+            offsets[E] = total;
+            s_off[E] = total;
+            *n_groups = tact;
+            stats->n_kept = total;
+            stats->n_active = tact;
+            stats->keep_sum = ks;
+            stats->lreg_sum = ls;
+            stats->n_all_masked = nz;
+            stats->tokens = T;
+            stats->err = 0;
+        }
+    }
+    __syncthreads();
+
+    // 4. placement of every (token, slot) pair
+    for (int i = threadIdx.x; i < T * K; i += blockDim.x) {
+        const int t = i / K, k = i - t * K;
+        int pos = -1;
+        if (s_keep[t][k]) {
+            const int e = s_id[t][k];
+            pos = s_off[e] + __popc(s_word[e] & ((1u << t) - 1u));
+            perm[pos] = i;
+        }
+        inv[i] = pos;
+    }
+    if (gather) {
+        __syncthreads();
+        const int nk = s_off[E];
+        const int nv = D * (int)sizeof(TW) / 16;
+        for (int pos = warp; pos < nk; pos += 32) {
+            const int t = perm[pos] / K;
+            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
+            uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
+            for (int v = lane; v < nv; v += 32) dst[v] = src[v];
+        }
+    }
+    pdl_launch_dependents();
+}
+
+// X_perm[pos] = x[perm[pos] / K] for every kept pair (one warp per row, grid-stride).
+template <typename TW>
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const int* __restrict__ perm, const int* __restrict__ n_kept_ptr, int K, int D,
+                   const TW* __restrict__ x, TW* __restrict__ xperm)
+{
+    pdl_wait();
+    const int nk = *n_kept_ptr;
+    const int nv = D * (int)sizeof(TW) / 16;
+    const int lane = threadIdx.x & 31;
+    for (int pos = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; pos < nk;
+         pos += (gridDim.x * blockDim.x) >> 5) {
+        const int t = perm[pos] / K;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
+        uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
+        for (int v = lane; v < nv; v += 32) dst[v] = src[v];
     }
     pdl_launch_dependents();
 }

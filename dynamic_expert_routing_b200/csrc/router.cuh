@@ -75,14 +75,89 @@ router_gemv_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
 
 // ---------------------------------------------------------------- Top-K, softmax, mask
 // One warp per routed row i (row i of L, leading dimension ldL: router logits in columns
-// [0, E), mask logits in [E, 2E)).  Lane l holds logits of experts l, l+32, ... (EPL per lane).
+// [0, E), mask logits in [E, 2E); `splits` K-split slices split_stride floats apart, added in
+// slice order).  Lane l holds logits of experts l, l+32, ... (EPL per lane).
+// K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
+// rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
+// L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
+// to every token of the routed row's segment (S = 1: the row's own token).
+// Decision for one routed row, computed by one warp (all lanes return the same values except
+// the per-slot ones, which lane k < K holds for slot k).
+struct RowDecision {
+    int id;        // lane k: expert of slot k
+    float g;       // lane k: softmax gate of slot k
+    float l;       // lane k: mask logit of slot k
+    bool keep;     // lane k: slot kept
+    float ghat;    // lane k: g * keep
+    int nkeep;     // all lanes: kept slots of the row
+    float lreg;    // all lanes: (1/K) sum_k sigmoid(l_k)
+};
+
+template <int EPL>
+__device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, int splits,
+                                                  long long split_stride, int E, int K,
+                                                  int mask_off, int lane)
+{
+    // the logits may arrive as split-K slices: add them in slice order
+    auto logit = [&](int col) {
+        float a = Li[col];
+        for (int s = 1; s < splits; ++s) a += Li[s * split_stride + col];
+        return a;
+    };
+    float v[EPL];
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+        int e = lane + 32 * j;
+        v[j] = (e < E) ? logit(e) : -INFINITY;
+    }
+    unsigned chosen = 0;
+    int my_id = 0;
+    float my_v = 0.f;
+    for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            int e = lane + 32 * j;
+            bool ok = (e < E) && !((chosen >> j) & 1u);
+            if (ok && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if ((bi & 31) == lane) chosen |= 1u << (bi >> 5);
+        if (lane == k) { my_id = bi; my_v = bv; }
+    }
+    RowDecision d;
+    const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const bool active = lane < K;
+    float ex = active ? expf(my_v - vmax) : 0.f;
+    const float den = warp_sum(ex);
+    d.id = my_id;
+    d.g = ex / den;
+    d.l = active ? logit(E + my_id) : 0.f;
+    d.keep = active && (mask_off || d.l >= 0.f);
+    d.ghat = d.keep ? d.g : 0.f;
+    const float sg = active ? sigmoid_f(d.l) : 0.f;
+    d.nkeep = __popc(__ballot_sync(0xffffffffu, d.keep));
+    d.lreg = warp_sum(sg) / (float)K;
+    return d;
+}
+
+// One warp per routed row i (row i of L, leading dimension ldL: router logits in columns
+// [0, E), mask logits in [E, 2E); `splits` K-split slices split_stride floats apart, added in
+// slice order).  Lane l holds logits of experts l, l+32, ... (EPL per lane).
 // K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
 // rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
 // L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
 // to every token of the routed row's segment (S = 1: the row's own token).
 template <int EPL>
 __global__ void __launch_bounds__(256)
-route_select_kernel(const float* __restrict__ L, int ldL, int Tr, int T, int E, int K, int seg,
+route_select_kernel(const float* __restrict__ L, int ldL, int splits, long long split_stride,
+                    int Tr, int T, int E, int K, int seg,
                     int mask_off, int* __restrict__ topk_id, float* __restrict__ gate,
                     float* __restrict__ mlogit, uint8_t* __restrict__ keep,
                     float* __restrict__ ghat, int* __restrict__ nkeep_tok,
@@ -92,57 +167,20 @@ route_select_kernel(const float* __restrict__ L, int ldL, int Tr, int T, int E, 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * 8 + warp;
     if (i < Tr) {
-        const float* Li = L + (size_t)i * ldL;
-        float v[EPL];
-#pragma unroll
-        for (int j = 0; j < EPL; ++j) {
-            int e = lane + 32 * j;
-            v[j] = (e < E) ? Li[e] : -INFINITY;
-        }
-        unsigned chosen = 0;
-        int my_id = 0;
-        float my_v = 0.f;
-        for (int k = 0; k < K; ++k) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < EPL; ++j) {
-                int e = lane + 32 * j;
-                bool ok = (e < E) && !((chosen >> j) & 1u);
-                if (ok && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-            }
-            if ((bi & 31) == lane) chosen |= 1u << (bi >> 5);
-            if (lane == k) { my_id = bi; my_v = bv; }
-        }
-        const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-        const bool active = lane < K;
-        float ex = active ? expf(my_v - vmax) : 0.f;
-        const float den = warp_sum(ex);
-        const float g = ex / den;
-        const float l = active ? Li[E + my_id] : 0.f;
-        const bool kp = active && (mask_off || l >= 0.f);
-        const float gh = kp ? g : 0.f;
-        const float sg = active ? sigmoid_f(l) : 0.f;
-        const int nk = __popc(__ballot_sync(0xffffffffu, kp));
-        const float lr = warp_sum(sg) / (float)K;
+        const RowDecision d = select_row<EPL>(L + (size_t)i * ldL, splits, split_stride, E, K,
+                                              mask_off, lane);
         const int S = seg > 1 ? seg : 1;
         const int t0 = i * S, t1 = min(T, t0 + S);
         for (int t = t0; t < t1; ++t) {
-            if (active) {
+            if (lane < K) {
                 size_t o = (size_t)t * K + lane;
-                topk_id[o] = my_id;
-                gate[o] = g;
-                mlogit[o] = l;
-                keep[o] = kp ? 1 : 0;
-                ghat[o] = gh;
+                topk_id[o] = d.id;
+                gate[o] = d.g;
+                mlogit[o] = d.l;
+                keep[o] = d.keep ? 1 : 0;
+                ghat[o] = d.ghat;
             }
-            if (lane == 0) { nkeep_tok[t] = nk; lreg_tok[t] = lr; }
+            if (lane == 0) { nkeep_tok[t] = d.nkeep; lreg_tok[t] = d.lreg; }
         }
     }
     pdl_launch_dependents();

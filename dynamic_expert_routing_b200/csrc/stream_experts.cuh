@@ -517,34 +517,44 @@ combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
                const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K, int D,
                float* __restrict__ y)
 {
+    __shared__ int s_inv[32];
+    __shared__ float s_g[32];
     pdl_wait();
-    const int t = blockIdx.x;
-    if (t < T) {
-        const int D4 = D >> 2;
-        const long long s4 = stride >> 2, ssh4 = stride_sh >> 2;
-        for (int c = threadIdx.x; c < D4; c += blockDim.x) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k < K; ++k) {
-                const int p = inv[(size_t)t * K + k];
-                if (p >= 0) {
-                    const float g = ghat[(size_t)t * K + k];
-                    float4 v = load4(yperm, (size_t)p * D4 + c);
-                    for (int s = 1; s < splits; ++s) {
-                        const float4 w = load4(yperm, s * s4 + (size_t)p * D4 + c);
-                        v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-                    }
-                    acc.x = fmaf(g, v.x, acc.x); acc.y = fmaf(g, v.y, acc.y);
-                    acc.z = fmaf(g, v.z, acc.z); acc.w = fmaf(g, v.w, acc.w);
+    const int t = blockIdx.x;   // token; blockIdx.y picks a slice of the columns
+    if (t >= T) return;
+    if (threadIdx.x < K) {
+        s_inv[threadIdx.x] = inv[(size_t)t * K + threadIdx.x];
+        s_g[threadIdx.x] = ghat[(size_t)t * K + threadIdx.x];
+    }
+    __syncthreads();
+    const int D4 = D >> 2;
+    const long long s4 = stride >> 2, ssh4 = stride_sh >> 2;
+    const int chunk = (D4 + gridDim.y - 1) / gridDim.y;   // columns of this CTA: one slice
+    const int c_end = min(D4, (int)(blockIdx.y + 1) * chunk);
+    for (int c = blockIdx.y * chunk + threadIdx.x; c < c_end; c += blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        // independent loads of up to 4 slots in flight before they are accumulated in order
+#pragma unroll 4
+        for (int k = 0; k < K; ++k) {
+            const int p = s_inv[k];
+            if (p >= 0) {
+                float4 v = load4(yperm, (size_t)p * D4 + c);
+                for (int s = 1; s < splits; ++s) {
+                    const float4 w = load4(yperm, s * s4 + (size_t)p * D4 + c);
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
                 }
+                const float g = s_g[k];
+                acc.x = fmaf(g, v.x, acc.x); acc.y = fmaf(g, v.y, acc.y);
+                acc.z = fmaf(g, v.z, acc.z); acc.w = fmaf(g, v.w, acc.w);
             }
-            if (ysh) {
-                for (int s = 0; s < splits_sh; ++s) {
-                    const float4 w = load4(ysh, s * ssh4 + (size_t)t * D4 + c);
-                    acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
-                }
-            }
-            reinterpret_cast<float4*>(y)[(size_t)t * D4 + c] = acc;
         }
+        if (ysh) {
+            for (int s = 0; s < splits_sh; ++s) {
+                const float4 w = load4(ysh, s * ssh4 + (size_t)t * D4 + c);
+                acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
+            }
+        }
+        __stcs(reinterpret_cast<float4*>(y) + (size_t)t * D4 + c, acc);
     }
     pdl_launch_dependents();
 }
