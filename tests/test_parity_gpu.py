@@ -223,3 +223,23 @@ def test_model_shapes_prefill(name, T, keep, mask_off):
     info = run_case(spec, T, keep_rate=keep, mask_off=mask_off, y_tokens=sample)
     # with segment routing an unclean leader makes its whole segment unclean
     assert info["unclean"] <= 0.05 * T * max(1, spec.segment_len)
+
+
+# ------------------------------------------------------------------ configuration limits
+@pytest.mark.parametrize("spec,T", [
+    (synth.LayerSpec("wide_d", 8192, 8, 2, 256, n_shared=1, d_ff_shared=128), 40),      # D = 8192
+    (synth.LayerSpec("e256", 512, 256, 32, 128), 33),                                    # E = 256, K = 32
+    (synth.LayerSpec("k1", 256, 4, 1, 128), 70),                                         # K = 1
+    (synth.LayerSpec("fp32_shared_seg", 256, 8, 3, 256, n_shared=2, d_ff_shared=128,
+                     storage="fp32", segment_len=8), 61),                                # fp32 path
+], ids=["d8192", "e256_k32", "k1", "fp32_shared_segment"])
+def test_configuration_limits(spec, T):
+    run_case(spec, T, seed=77)
+
+
+def test_large_max_tokens_small_forward():
+    """A handle sized for a long prefill serves a one-token decode (split-K workspaces are
+    sized independently of max_tokens)."""
+    spec = _small(n_shared=1, d_ff_shared=128)
+    run_case(spec, 1, seed=5, max_tokens=20000)
+    run_case(spec, 3000, seed=6, max_tokens=20000)
