@@ -12,6 +12,7 @@
 
 #include <algorithm>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -149,6 +150,9 @@ struct beam_moe {
     int* zero_int = nullptr;
     int* range_flag = nullptr;
     cudaEvent_t done = nullptr;
+    // side stream for the shared experts (they depend on x only, so they overlap routing)
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     int last_T = -1;
     std::vector<void*> allocs;
     // replay cache: the last forward captured as a CUDA graph, keyed by its arguments
@@ -203,6 +207,19 @@ static void free_all(beam_moe* h)
     h->allocs.clear();
     if (h->done) cudaEventDestroy(h->done);
     h->done = nullptr;
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->side) cudaStreamDestroy(h->side);
+    h->ev_fork = h->ev_join = nullptr;
+    h->side = nullptr;
+}
+
+// Test hook: BEAM_TEST_FAIL_ALLOC=n makes the n-th device allocation of a create fail as if
+// the device were out of memory (n = 1 is the first), so the error path can be exercised.
+static int fail_alloc_at()
+{
+    const char* v = getenv("BEAM_TEST_FAIL_ALLOC");
+    return v ? atoi(v) : 0;
 }
 
 template <typename P>
@@ -210,6 +227,9 @@ static beam_status_t dalloc(beam_moe* h, P** out, size_t bytes)
 {
     void* p = nullptr;
     if (bytes == 0) bytes = 16;
+    const int fail_at = fail_alloc_at();
+    if (fail_at > 0 && (int)h->allocs.size() + 1 == fail_at)
+        return fail(BEAM_ERR_OOM, "device allocation %d failed (BEAM_TEST_FAIL_ALLOC)", fail_at);
     cudaError_t e = cudaMalloc(&p, bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -267,7 +287,7 @@ constexpr int kTcRouterMinRows = 64;
 constexpr long long kInlineGatherBytes = 256 * 1024;
 // Split-K for small batches on the tensor-core path: up to kMaxSplits K slices per tile, for
 // forwards of at most kSplitMaxTokens tokens (the partial-sum workspaces are sized for that).
-constexpr int kMaxSplits = 8;
+constexpr int kMaxSplits = 16;
 constexpr int kSplitMaxTokens = 64;
 constexpr int kMinStepsPerSplit = 4;
 
@@ -498,6 +518,11 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_CUDA(cudaMemsetAsync(h->range_flag, 0, sizeof(int), st));
     BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, sizeof(int), st));
     BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
+    if (h->Fsh > 0) {
+        BEAM_CUDA(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
+    }
 
     if (cfg->dtype == BEAM_DTYPE_BF16) BEAM_TRY(repack<__nv_bfloat16>(h, w, st));
     else BEAM_TRY(repack<float>(h, w, st));
@@ -581,6 +606,101 @@ static cudaError_t launch_small(beam_moe* h, const T* x, int Tr, int T_, int mas
                   h->inv, x, (T*)h->xperm, h->D, gather);
 }
 
+// Output of one expert problem for the combine: `splits` slices `stride` elements apart,
+// fp16 (unsplit tensor-core output) or fp32 (split-K partials, GEMV path).
+struct YOut {
+    const void* base = nullptr;
+    int splits = 1;
+    long long stride = 0;
+    bool f16 = false;
+};
+
+// GEMM1 (+ SwiGLU finish when split) and GEMM2 of one problem on the tensor cores: the routed
+// groups (shared = false) or the always-on shared group (shared = true), on stream `st`.
+template <typename T>
+static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cudaStream_t st,
+                                YOut& out)
+{
+    const int D = h->D, F = h->F, Fsh = h->Fsh, K = h->K, E = h->E;
+    int s1 = 1, s2 = 1;
+    if (T_ <= kSplitMaxTokens) {
+        // a small batch has few tiles: split K so they cover every SM
+        const long long mts = ceil_div(T_, tc::BM);
+        const long long groups = std::min<long long>(E, std::max(1LL, ((long long)T_ * K + 1) / 2));
+        const long long t1 = shared ? mts * (2LL * Fsh / tc::BN) : mts * groups * (2LL * F / tc::BN);
+        const long long t2 = shared ? mts * ((long long)D / tc::BN) : mts * groups * (D / tc::BN);
+        s1 = choose_splits(h->num_sms, t1);
+        s2 = choose_splits(h->num_sms, t2);
+    }
+    s1 = normalise_splits(s1, D / tc::BK);
+    s2 = normalise_splits(s2, (shared ? Fsh : F) / tc::BK);
+    const int rows_sh = shared ? T_ : 0;
+    const int* ngroups = shared ? h->zero_int : h->n_groups;
+
+    // GEMM1: gate/up, SwiGLU in the epilogue, or f32 partials + the finishing kernel
+    tc::TcParams p = (s1 > 1) ? h->p1s : h->p1;
+    if (shared)
+        BEAM_TRY(encode_map(h, &p.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
+                            (uint64_t)D, tc::BM));
+    p.n_groups = ngroups;
+    p.shared_rows = rows_sh;
+    p.k_splits_routed = p.k_splits_shared = s1;
+    if (s1 > 1) {
+        BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
+        const long long work = shared ? (long long)T_ * Fsh : (long long)T_ * K * F;
+        BEAM_CUDA(launch(h, ST_SWIGLU_FINISH, tc::swiglu_finish_kernel,
+                         dim3((unsigned)std::max<long long>(1, std::min<long long>(h->num_sms * 4, ceil_div(work, 256)))),
+                         dim3(256), 0, st, (const float*)h->g1part, s1, p.split_stride_routed,
+                         (const int*)(shared ? h->zero_int : h->offsets + E), F, (__half*)h->hbuf,
+                         (const float*)h->g1part_sh, s1, p.split_stride_shared, rows_sh, Fsh,
+                         (__half*)h->hsh));
+    } else {
+        BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
+    }
+
+    // GEMM2: down projection, fp16 output, or f32 partials added by the combine
+    tc::TcParams q = h->p2;
+    q.n_groups = ngroups;
+    q.shared_rows = rows_sh;
+    q.k_splits_routed = q.k_splits_shared = s2;
+    if (s2 > 1) {
+        q.out_routed = h->ypart;
+        q.split_stride_routed = (long long)h->split_rows * K * D;
+        q.out_shared = h->ysh_part;
+        q.split_stride_shared = (long long)h->split_rows * D;
+        out.base = shared ? (const void*)h->ysh_part : (const void*)h->ypart;
+        out.splits = s2;
+        out.stride = shared ? q.split_stride_shared : q.split_stride_routed;
+        out.f16 = false;
+        BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
+    } else {
+        q.out_routed = h->yperm;
+        q.out_shared = h->ysh;
+        q.split_stride_routed = q.split_stride_shared = 0;
+        out.base = shared ? (const void*)h->ysh : (const void*)h->yperm;
+        out.splits = 1;
+        out.stride = 0;
+        out.f16 = true;
+        BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
+    }
+    return BEAM_OK;
+}
+
+template <typename TR, typename TS>
+static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, int T_, float* y,
+                                  cudaStream_t st)
+{
+    // few tokens: split each token's columns over several CTAs so the combine spans the SMs
+    const dim3 cgrid(T_, T_ < h->num_sms ? ceil_div(h->D / 4, 256) : 1);
+    return launch(h, ST_COMBINE, combine_kernel<TR, TS>, cgrid, dim3(256), 0, st,
+                  (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
+                  (const int*)h->inv, (const float*)h->ghat, T_, h->K, h->D, y);
+}
+
 template <typename T>
 static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uint32_t flags,
                                   bool use_tc, cudaStream_t st)
@@ -590,6 +710,18 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     const int Tr = ceil_div(T_, S);
     const int nch = ceil_div(T_, 32);
     const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
+
+    // 0. shared experts: they need only x, so on the tensor path they run on a side stream,
+    // concurrently with the router and the compaction, and join before the combine
+    BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, sizeof(int), st));
+    YOut ysh_out;
+    const bool fork = use_tc && h->Fsh > 0;
+    if (fork) {
+        BEAM_CUDA(cudaEventRecord(h->ev_fork, st));
+        BEAM_CUDA(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+        BEAM_TRY(tc_problem(h, x, T_, true, h->side, ysh_out));
+        BEAM_CUDA(cudaEventRecord(h->ev_join, h->side));
+    }
 
     // 1. router logits L = x [W_r | W_m]  (routed rows only: segment leaders when S > 1)
     int lsplits = 1;
@@ -658,72 +790,11 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          (const uint32_t*)h->bits, (const int*)h->offsets,
                          (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     }
-    // 4. experts (kept groups only) and shared experts
+    // 4. experts: kept groups only (the shared group is already running on the side stream)
     using TH = typename HType<T>::type;
-    const void* ybase = h->yperm;
-    const void* yshbase = h->Fsh ? h->ysh : nullptr;
-    int ysplits = 1, yshsplits = 1;
-    long long ystride = 0, yshstride = 0;
-    bool y_f16 = false;  // unsplit tensor-core outputs are stored in fp16
+    YOut yr;
     if (use_tc) {
-        const int Fsh = h->Fsh, F = h->F;
-        int s1 = 1, s2 = 1;
-        if (T_ <= kSplitMaxTokens) {
-            // a small batch has few kept groups: split K so their tiles cover every SM
-            const long long groups = std::min<long long>(E, std::max(1LL, ((long long)T_ * K + 1) / 2));
-            const long long mts = ceil_div(T_, tc::BM);
-            s1 = choose_splits(h->num_sms, mts * ((Fsh ? 2LL * Fsh / tc::BN : 0) + groups * (2LL * F / tc::BN)));
-            s2 = choose_splits(h->num_sms, mts * ((Fsh ? (long long)D / tc::BN : 0) + groups * (D / tc::BN)));
-        }
-        const int s1r = normalise_splits(s1, D / tc::BK);          // GEMM1: K = D for both problems
-        const int s2r = normalise_splits(s2, F / tc::BK);          // GEMM2 routed: K = F
-        const int s2s = Fsh ? normalise_splits(s2, Fsh / tc::BK) : 1;  // GEMM2 shared: K = Fsh
-        s1 = s1r;
-        if (s1 > 1) {
-            tc::TcParams& p = h->p1s;
-            BEAM_TRY(encode_map(h, &p.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
-                                (uint64_t)D, tc::BM));
-            p.shared_rows = Fsh ? T_ : 0;
-            p.k_splits_routed = p.k_splits_shared = s1;
-            BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
-                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1s));
-            const long long work = ((long long)T_ * K * F + (long long)T_ * Fsh);
-            BEAM_CUDA(launch(h, ST_SWIGLU_FINISH, tc::swiglu_finish_kernel,
-                             dim3((unsigned)std::min<long long>(h->num_sms * 4, ceil_div(work, 256))),
-                             dim3(256), 0, st, (const float*)h->g1part, s1, p.split_stride_routed,
-                             (const int*)(h->offsets + E), F, (__half*)h->hbuf,
-                             (const float*)h->g1part_sh, s1, p.split_stride_shared,
-                             Fsh ? T_ : 0, Fsh, (__half*)h->hsh));
-        } else {
-            tc::TcParams& p1 = h->p1;
-            BEAM_TRY(encode_map(h, &p1.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
-                                (uint64_t)D, tc::BM));
-            p1.shared_rows = Fsh ? T_ : 0;
-            BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
-                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p1));
-        }
-        tc::TcParams& p2 = h->p2;
-        p2.shared_rows = Fsh ? T_ : 0;
-        if (s2r > 1 || s2s > 1) {
-            p2.k_splits_routed = s2r;
-            p2.k_splits_shared = s2s;
-            p2.out_routed = h->ypart;
-            p2.split_stride_routed = (long long)h->split_rows * K * D;
-            p2.out_shared = h->ysh_part;
-            p2.split_stride_shared = (long long)h->split_rows * D;
-            ybase = h->ypart; ysplits = s2r; ystride = p2.split_stride_routed;
-            if (Fsh) { yshbase = h->ysh_part; yshsplits = s2s; yshstride = p2.split_stride_shared; }
-            BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
-                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
-        } else {
-            p2.k_splits_routed = p2.k_splits_shared = 1;
-            p2.out_routed = h->yperm;
-            p2.out_shared = h->ysh;
-            p2.split_stride_routed = p2.split_stride_shared = 0;
-            y_f16 = true;
-            BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0>,
-                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p2));
-        }
+        BEAM_TRY(tc_problem(h, x, T_, false, st, yr));
     } else {
         StreamArgs a;
         a.xperm = h->xperm; a.x = x; a.wgu = h->wgu; a.wsgu = h->wsgu; a.wd = h->wd; a.wsd = h->wsd;
@@ -735,18 +806,18 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          (size_t)stream_gateup_smem(), st, a));
         BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(grid), dim3(256),
                          (size_t)stream_down_smem(), st, a));
+        yr.base = h->yperm; yr.f16 = false;
+        if (h->Fsh) { ysh_out.base = h->ysh; ysh_out.f16 = false; }
     }
-    // 5. fixed-order combine
-    // few tokens: split each token's columns over several CTAs so the combine spans the SMs
-    const dim3 cgrid(T_, T_ < h->num_sms ? ceil_div(D / 4, 256) : 1);
-    if (y_f16)
-        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<__half>, cgrid, dim3(256), 0, st,
-                         (const __half*)ybase, ysplits, ystride, (const __half*)yshbase, yshsplits,
-                         yshstride, (const int*)h->inv, (const float*)h->ghat, T_, K, D, y));
-    else
-        BEAM_CUDA(launch(h, ST_COMBINE, combine_kernel<float>, cgrid, dim3(256), 0, st,
-                         (const float*)ybase, ysplits, ystride, (const float*)yshbase, yshsplits,
-                         yshstride, (const int*)h->inv, (const float*)h->ghat, T_, K, D, y));
+    // 5. fixed-order combine (after the side stream joins)
+    if (fork) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_join, 0));
+    if (!h->Fsh) ysh_out.f16 = yr.f16;  // no shared term: only its (unused) type must match
+    cudaError_t ce;
+    if (yr.f16 && ysh_out.f16) ce = launch_combine<__half, __half>(h, yr, ysh_out, T_, y, st);
+    else if (yr.f16) ce = launch_combine<__half, float>(h, yr, ysh_out, T_, y, st);
+    else if (ysh_out.f16) ce = launch_combine<float, __half>(h, yr, ysh_out, T_, y, st);
+    else ce = launch_combine<float, float>(h, yr, ysh_out, T_, y, st);
+    BEAM_CUDA(ce);
     return BEAM_OK;
 }
 

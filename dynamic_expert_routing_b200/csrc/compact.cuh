@@ -167,7 +167,6 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
             stats->lreg_sum = ls;
             stats->n_all_masked = nz;
             stats->tokens = T;
-            stats->err = 0;
         }
     }
     pdl_launch_dependents();
@@ -341,7 +340,6 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
             stats->lreg_sum = ls;
             stats->n_all_masked = nz;
             stats->tokens = T;
-            stats->err = 0;
         }
     }
     __syncthreads();

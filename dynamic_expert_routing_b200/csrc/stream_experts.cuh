@@ -498,8 +498,8 @@ stream_down_kernel(StreamArgs a)
 // y[t] = sum over slots k in rank order with keep = 1 of g_hat[t][k] * Y_perm[inv[t][k]],
 // plus the shared-expert output; a fixed order, so the result is bit-reproducible.  When the
 // down projection ran split-K, Y_perm / Y_sh hold `splits` partial slices `stride` elements
-// apart (fp32), added in slice order before the gate is applied.  TY is the element type of
-// Y_perm / Y_sh: fp16 for unsplit tensor-core outputs of bf16 layers, fp32 otherwise.
+// apart (fp32), added in slice order before the gate is applied.  TY / TS are the element
+// types of Y_perm / Y_sh: fp16 for unsplit tensor-core outputs of bf16 layers, fp32 otherwise.
 __device__ __forceinline__ float4 load4(const float* p, size_t i) {
     return reinterpret_cast<const float4*>(p)[i];
 }
@@ -510,10 +510,10 @@ __device__ __forceinline__ float4 load4(const __half* p, size_t i) {
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
-template <typename TY>
+template <typename TY, typename TS>
 __global__ void __launch_bounds__(256)
 combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
-               const TY* __restrict__ ysh, int splits_sh, long long stride_sh,
+               const TS* __restrict__ ysh, int splits_sh, long long stride_sh,
                const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K, int D,
                float* __restrict__ y)
 {

@@ -146,6 +146,27 @@ def test_bounded_wait_expires_and_the_context_survives():
     run_case(_small(), 40, seed=9)
 
 
+def test_allocation_failure_frees_everything(monkeypatch):
+    """An allocation failing part-way through create returns BEAM_ERR_OOM, releases what was
+    already allocated, and leaves the library usable."""
+    from dynamic_expert_routing_b200 import BeamMoE, BeamError, _lib
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = to_dev(synth.make_layer(spec, keep_rate=0.5))
+    wd = {k: v for k, v in w.items() if isinstance(v, torch.Tensor)}
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for n in (1, 7, 20):
+        monkeypatch.setenv("BEAM_TEST_FAIL_ALLOC", str(n))
+        with pytest.raises(BeamError) as ei:
+            BeamMoE(wd, spec.top_k, max_tokens=4096)
+        assert ei.value.status == _lib.BEAM_ERR_OOM
+    monkeypatch.delenv("BEAM_TEST_FAIL_ALLOC")
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert abs(free0 - free1) < 64 << 20      # nothing of the failed creates is left behind
+    run_case(spec, 50, seed=4)
+
+
 def test_host_buffer_entry_point():
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=128)
