@@ -15,8 +15,9 @@
 //   * tile 128 (tokens) x 256 x 64, TMA (cp.async.bulk.tensor, 128-byte swizzle, no cluster
 //     multicast) fills a 4-stage shared-memory ring guarded by mbarriers;
 //   * warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma (kind::f16, fp32
-//     accumulation in TMEM, double-buffered accumulators of 256 columns), warps 2..5 drain
-//     TMEM with tcgen05.ld and run the epilogue (SwiGLU -> fp16 H, or fp32 Y stores);
+//     accumulation in TMEM, double-buffered accumulators of 256 columns), warps 2..9 drain
+//     TMEM with tcgen05.ld (two warps per lane quadrant, each half the columns) and run the
+//     epilogue (SwiGLU -> fp16 H, or f32 / f16 stores);
 //   * every mbarrier wait is bounded by a time limit; on expiry the CTA records an error code,
 //     drains the copies and MMAs it issued (again bounded), frees TMEM and returns.
 #pragma once
@@ -34,12 +35,13 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quadrant, each half the columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer warp, MMA warp, epilogue warps
 // Epilogue staging: each of the 4 epilogue warps transposes 32x32 fp32 sub-tiles through its
 // own padded shared-memory buffer (row stride 33 words: conflict-free both ways).
 constexpr int EPI_PITCH = 33;
 constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH * 4;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES + 1024 /*alignment slack*/ +
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES + 1024 /*alignment slack*/ +
                            256 /*barriers*/;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s: far above any tile
 constexpr int ERR_TC_TIMEOUT = 0x100;
@@ -293,20 +295,20 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     uint8_t* gbase = smem_raw + (base - raw);
     // layout: [stage s: A (16 KB) | B (32 KB)] x STAGES, epilogue buffers, then the barriers
     float* epi_buf = reinterpret_cast<float*>(gbase + STAGES * STAGE_BYTES);
-    const uint32_t bar0 = base + STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES;
+    const uint32_t bar0 = base + STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 4 * EPI_WARP_BYTES +
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES +
                                                       8 * (2 * STAGES + 5));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), kEpiWarps); }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -409,6 +411,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         uint32_t aph = 0;
         const int lb = 32 * (warp & 3);  // TMEM lanes this warp may access
         const int warp_e = warp - 2;     // index of this epilogue warp (its staging buffer)
+        const int half = warp_e / 4;     // which half of the tile's columns this warp drains
         while (w.get(t)) {
             if (!mbar_wait(tfull_bar(acc), aph, abort_flag)) break;
             tc_fence_after();
@@ -425,7 +428,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             if (EPI == EPI_SWIGLU) {
                 __half* out = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed);
 #pragma unroll 1
-                for (int j = 0; j < BN / 2 / 32; ++j) {
+                for (int j = half * (BN / 2 / 64); j < (half + 1) * (BN / 2 / 64); ++j) {
                     float g[32], u[32];
                     tmem_ld32(tbase + 32 * j, g);
                     tmem_ld32(tbase + BN / 2 + 32 * j, u);
@@ -440,7 +443,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             } else {
                 const long long sstride = t.shared ? p.split_stride_shared : p.split_stride_routed;
 #pragma unroll 1
-                for (int j = 0; j < BN / 32; ++j) {
+                for (int j = half * (BN / 64); j < (half + 1) * (BN / 64); ++j) {
                     float v[32];
                     tmem_ld32(tbase + 32 * j, v);
 #pragma unroll
