@@ -179,35 +179,43 @@ def gpu_uuid(torch, dev):
 
 
 # ------------------------------------------------------------------ algorithmic work
-def layer_work(spec, T, st):
-    """Algorithmic bytes and FLOPs of one forward (what the method must move / compute)."""
+def layer_work(spec, T, st, tc_path=True):
+    """Algorithmic bytes and FLOPs of one forward (what the method must move / compute), per
+    stage.  The intermediates are counted at the precision the path keeps them in: H in fp16
+    for bf16 layers (fp32 for fp32 layers); expert output rows in fp16 on the tensor-core
+    path, fp32 on the streaming path.  On the tensor-core path the shared experts are a
+    problem of their own (tc_shared_* stages); the streaming kernels do both in one launch."""
     D, E, K, F = spec.d_model, spec.n_experts, spec.top_k, spec.d_ff
     es = 4 if spec.storage == "fp32" else 2
+    hs = 4 if spec.storage == "fp32" else 2
+    ys = 2 if tc_path else 4
     Fsh = spec.n_shared * spec.d_ff_shared
+    Tsh = T if Fsh else 0
     na, nk = st["n_active_experts"], st["n_kept"]
     Tr = math.ceil(T / spec.segment_len) if spec.segment_len > 1 else T
     w = {}
     w["router_logits"] = dict(bytes=2 * E * D * es + Tr * D * es + Tr * 2 * E * 4,
                               flops=2 * Tr * D * 2 * E)
-    gu_bytes = (na * 2 * F * D + 2 * Fsh * D) * es + (nk + (T if Fsh else 0)) * D * es \
-        + (nk * F + T * Fsh) * es
-    gu_flops = 2 * (nk * 2 * F * D + T * 2 * Fsh * D)
-    dn_bytes = (na * D * F + D * Fsh) * es + (nk * F + T * Fsh) * es + (nk + (T if Fsh else 0)) * D * 4
-    dn_flops = 2 * (nk * F * D + T * Fsh * D)
-    for s in ("stream_gateup", "tc_gateup"):
-        w[s] = dict(bytes=gu_bytes, flops=gu_flops)
-    for s in ("stream_down", "tc_down"):
-        w[s] = dict(bytes=dn_bytes, flops=dn_flops)
-    w["combine"] = dict(bytes=nk * D * 4 + (T * D * 4 if Fsh else 0) + T * D * 4 + T * K * 8,
+    w["tc_router"] = w["router_logits"]
+    gu_r = dict(bytes=na * 2 * F * D * es + nk * D * es + nk * F * hs, flops=4 * nk * F * D)
+    gu_s = dict(bytes=2 * Fsh * D * es + Tsh * D * es + Tsh * Fsh * hs, flops=4 * Tsh * Fsh * D)
+    dn_r = dict(bytes=na * D * F * es + nk * F * hs + nk * D * ys, flops=2 * nk * F * D)
+    dn_s = dict(bytes=D * Fsh * es + Tsh * Fsh * hs + Tsh * D * ys, flops=2 * Tsh * Fsh * D)
+    both = lambda a, b: {k: a[k] + b[k] for k in a}
+    w["stream_gateup"], w["stream_down"] = both(gu_r, gu_s), both(dn_r, dn_s)
+    w["tc_gateup"], w["tc_down"] = gu_r, dn_r
+    w["tc_shared_gateup"], w["tc_shared_down"] = gu_s, dn_s
+    w["combine"] = dict(bytes=nk * D * ys + Tsh * D * ys + T * D * 4 + T * K * 8,
                         flops=2 * nk * D)
     w["scatter_gather"] = dict(bytes=2 * nk * D * es + T * K * 12, flops=0)
-    w["swiglu_finish"] = dict(bytes=(nk * F + T * Fsh) * 2, flops=0)
+    w["swiglu_finish"] = dict(bytes=nk * F * hs, flops=0)
+    w["shared_swiglu_finish"] = dict(bytes=Tsh * Fsh * hs, flops=0)
     total_bytes = (na * 3 * F * D + 3 * Fsh * D + 2 * E * D) * es + T * D * es + T * D * 4
     total_flops = 2 * (nk * 3 * F * D + T * 3 * Fsh * D + Tr * D * 2 * E)
     return w, dict(bytes=total_bytes, flops=total_flops)
 
 
-TENSOR_STAGES = {"tc_gateup", "tc_down", "tc_router"}
+TENSOR_STAGES = {"tc_gateup", "tc_down", "tc_router", "tc_shared_gateup", "tc_shared_down"}
 
 
 def roofline_for(stage, work, ms_per_launch, peaks, workload):
@@ -309,7 +317,7 @@ def _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off):
     for _ in range(steps):
         layer.forward(x, mask_off=mo, out=y)
     prof = layer.profile_end()
-    work, total = layer_work(spec, T, st)
+    work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof)
     stage = max((k for k in prof if k != "forwards"), key=lambda k: prof[k][0])
     rl = roofline_for(stage, work.get(stage, dict(bytes=0, flops=0)),
                       prof[stage][0] / prof[stage][1], peaks, name)
@@ -386,7 +394,7 @@ def _run_ours(args):
     for _ in range(args.steps):
         layer.forward(x, mask_off=mask_off, out=y)
     prof = layer.profile_end()
-    work, total = layer_work(spec, T, st)
+    work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof)
     stages = {k: v for k, v in prof.items() if k != "forwards"}
     tot_ms = sum(v[0] for v in stages.values())
     dom = max(stages, key=lambda k: stages[k][0])

@@ -128,7 +128,7 @@ struct beam_moe {
     uint32_t* bits = nullptr;
     int *chunk_base = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
     Group* groups = nullptr;
-    int* n_groups = nullptr;
+    int* n_groups = nullptr;     // [0]: kept groups, [1]: their 128-row tiles
     DevStats* dstats = nullptr;
     // expert workspace
     void *xperm = nullptr, *hbuf = nullptr, *hsh = nullptr;
@@ -147,7 +147,11 @@ struct beam_moe {
     float* g1part_sh = nullptr;  // [kMaxSplits][split_rows][2Fsh]
     float* ypart = nullptr;      // [kMaxSplits][split_rows*K][D]
     float* ysh_part = nullptr;   // [kMaxSplits][split_rows][D]
-    int* zero_int = nullptr;
+    // tail split of the routed problem's whole-K launches: partial workspace and arrival
+    // counters (cleared by the compaction scan of every forward)
+    float* tail_ws = nullptr;
+    int* tail_cnt = nullptr;     // [kTailCntRegions][num_sms][kEpiWarps]
+    int* zero_int = nullptr;     // two zeros: an empty group table
     int* range_flag = nullptr;
     cudaEvent_t done = nullptr;
     // side stream for the shared experts (they depend on x only, so they overlap routing)
@@ -175,13 +179,13 @@ struct beam_moe {
 enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
-    ST_SWIGLU_FINISH, ST_COUNT
+    ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
-    "swiglu_finish"};
+    "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish"};
 
 static void prof_release(beam_moe* h)
 {
@@ -283,6 +287,11 @@ static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 constexpr int kTcMinTokens = 1;
 // Router logits run on the tensor cores from this many routed rows up (bf16 layers).
 constexpr int kTcRouterMinRows = 64;
+// Counter regions of the tail split: routed gate/up, routed down.  (The shared problem runs
+// concurrently with the routing on a second stream, so its last wave has no idle SMs to fill.)
+constexpr int kTailCntRegions = 2;
+static int tail_cnt_ints(int num_sms) { return kTailCntRegions * num_sms * tc::kEpiWarps; }
+
 // Small batches gather their kept rows inside the fused routing kernel up to this many bytes.
 constexpr long long kInlineGatherBytes = 256 * 1024;
 // Split-K for small batches on the tensor-core path: up to kMaxSplits K slices per tile, for
@@ -432,6 +441,11 @@ static beam_status_t setup_tc(beam_moe* h)
         c.split_stride_routed = (long long)sr * h->K * 2 * F;
         c.split_stride_shared = (long long)sr * 2 * Fsh;
     }
+    // tail split: at most kTailMaxSubWaves * num_sms piece slots per launch
+    {
+        const size_t slots = (size_t)tc::kTailMaxSubWaves * h->num_sms * tc::kEpiWarps;
+        BEAM_TRY(dalloc(h, &h->tail_ws, slots * tc::kTailSlotFloats * sizeof(float)));
+    }
     // router: logits L [Tr][ldL] = x_rows [Tr][D] . Wrm [ldL][D]^T as one dense problem
     tc::TcParams& r = h->p0;
     memset(&r, 0, sizeof r);
@@ -447,14 +461,17 @@ static beam_status_t setup_tc(beam_moe* h)
     r.k_steps_routed = r.k_steps_shared = (int)(D / tc::BK);
     r.k_splits_routed = r.k_splits_shared = 1;
     r.err = &h->dstats->err;
-    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
-    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
-    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
-    BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+    {
+        const void* kernels[] = {
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, false>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, false>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, true>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, false>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, false>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, true>};
+        for (const void* k : kernels)
+            BEAM_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+    }
     h->tc_ok = true;
     return BEAM_OK;
 }
@@ -481,7 +498,7 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     const size_t es = h->esz, hs = h->hsz;
     const size_t rows = Tm * K;  // upper bound on kept pairs
     BEAM_TRY(dalloc(h, &h->wrm, (size_t)h->ldL * D * es));
-    BEAM_TRY(dalloc(h, &h->zero_int, sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->zero_int, 2 * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->wgu, E * 2 * F * D * es));
     BEAM_TRY(dalloc(h, &h->wd, E * D * F * hs));
     BEAM_TRY(dalloc(h, &h->range_flag, sizeof(int)));
@@ -507,16 +524,18 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->perm, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->inv, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->groups, E * sizeof(Group)));
-    BEAM_TRY(dalloc(h, &h->n_groups, sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->n_groups, 2 * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->dstats, sizeof(DevStats)));
+    BEAM_TRY(dalloc(h, &h->tail_cnt, tail_cnt_ints(h->num_sms) * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->xperm, rows * D * es));
     BEAM_TRY(dalloc(h, &h->hbuf, rows * F * hs));
     BEAM_TRY(dalloc(h, &h->yperm, rows * D * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->x_stage, Tm * D * es));
     BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
     BEAM_CUDA(cudaMemsetAsync(h->dstats, 0, sizeof(DevStats), st));
+    BEAM_CUDA(cudaMemsetAsync(h->tail_cnt, 0, tail_cnt_ints(h->num_sms) * sizeof(int), st));
     BEAM_CUDA(cudaMemsetAsync(h->range_flag, 0, sizeof(int), st));
-    BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, sizeof(int), st));
+    BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, 2 * sizeof(int), st));
     BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
     if (h->Fsh > 0) {
         BEAM_CUDA(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
@@ -603,7 +622,7 @@ static cudaError_t launch_small(beam_moe* h, const T* x, int Tr, int T_, int mas
                   (const float*)h->L, h->ldL, splits, split_stride, Tr, T_, h->E, h->K, h->S,
                   mask_off, h->topk_id, h->gate, h->mlogit, h->keep, h->ghat, h->nkeep_tok,
                   h->lreg_tok, h->counts, h->offsets, h->groups, h->n_groups, h->dstats, h->perm,
-                  h->inv, x, (T*)h->xperm, h->D, gather);
+                  h->inv, x, (T*)h->xperm, h->D, gather, h->tail_cnt, tail_cnt_ints(h->num_sms));
 }
 
 // Output of one expert problem for the combine: `splits` slices `stride` elements apart,
@@ -635,6 +654,10 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
     s1 = normalise_splits(s1, D / tc::BK);
     s2 = normalise_splits(s2, (shared ? Fsh : F) / tc::BK);
     const int rows_sh = shared ? T_ : 0;
+    // the shared problem runs as launches of its own, timed under stages of its own
+    const int st_gu = shared ? ST_TC_SH_GATEUP : ST_TC_GATEUP;
+    const int st_dn = shared ? ST_TC_SH_DOWN : ST_TC_DOWN;
+    const int st_fin = shared ? ST_SH_SWIGLU_FINISH : ST_SWIGLU_FINISH;
     const int* ngroups = shared ? h->zero_int : h->n_groups;
 
     // GEMM1: gate/up, SwiGLU in the epilogue, or f32 partials + the finishing kernel
@@ -645,18 +668,28 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
     p.n_groups = ngroups;
     p.shared_rows = rows_sh;
     p.k_splits_routed = p.k_splits_shared = s1;
+    // routed whole-K launches deep enough in K may cut the tiles of their last, partial wave
+    // into K pieces (the kernel variant with the tail path; the cut is decided on the device)
+    const size_t creg = (size_t)h->num_sms * tc::kEpiWarps;
+    const bool tail1 = !shared && s1 == 1 && D / tc::BK >= tc::kTailMinKSteps;
+    const bool tail2 = !shared && s2 == 1 && F / tc::BK >= tc::kTailMinKSteps;
+    p.tail_cnt = tail1 ? h->tail_cnt : nullptr;
+    p.tail_ws = tail1 ? h->tail_ws : nullptr;
     if (s1 > 1) {
-        BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, false>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
         const long long work = shared ? (long long)T_ * Fsh : (long long)T_ * K * F;
-        BEAM_CUDA(launch(h, ST_SWIGLU_FINISH, tc::swiglu_finish_kernel,
+        BEAM_CUDA(launch(h, st_fin, tc::swiglu_finish_kernel,
                          dim3((unsigned)std::max<long long>(1, std::min<long long>(h->num_sms * 4, ceil_div(work, 256)))),
                          dim3(256), 0, st, (const float*)h->g1part, s1, p.split_stride_routed,
                          (const int*)(shared ? h->zero_int : h->offsets + E), F, (__half*)h->hbuf,
                          (const float*)h->g1part_sh, s1, p.split_stride_shared, rows_sh, Fsh,
                          (__half*)h->hsh));
+    } else if (tail1) {
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, true>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
     } else {
-        BEAM_CUDA(launch(h, ST_TC_GATEUP, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1>,
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, false>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
     }
 
@@ -665,6 +698,8 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
     q.n_groups = ngroups;
     q.shared_rows = rows_sh;
     q.k_splits_routed = q.k_splits_shared = s2;
+    q.tail_cnt = tail2 ? h->tail_cnt + creg : nullptr;
+    q.tail_ws = tail2 ? h->tail_ws : nullptr;
     if (s2 > 1) {
         q.out_routed = h->ypart;
         q.split_stride_routed = (long long)h->split_rows * K * D;
@@ -674,7 +709,7 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
         out.splits = s2;
         out.stride = shared ? q.split_stride_shared : q.split_stride_routed;
         out.f16 = false;
-        BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0>,
+        BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, false>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
     } else {
         q.out_routed = h->yperm;
@@ -684,8 +719,12 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
         out.splits = 1;
         out.stride = 0;
         out.f16 = true;
-        BEAM_CUDA(launch(h, ST_TC_DOWN, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0>,
-                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
+        if (tail2)
+            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, true>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
+        else
+            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, false>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
     }
     return BEAM_OK;
 }
@@ -738,7 +777,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         lstride = (long long)Tr * h->ldL;
         p0.k_splits_routed = p0.k_splits_shared = lsplits;
         p0.split_stride_routed = p0.split_stride_shared = lstride;
-        BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1>,
+        BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, false>,
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
     } else {
@@ -783,7 +822,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(1), dim3(1024), 0, st,
                          (const uint32_t*)h->bits, nch, E, T_, (const int*)h->nkeep_tok,
                          (const float*)h->lreg_tok, h->counts, h->offsets, h->chunk_base, h->groups,
-                         h->n_groups, h->dstats));
+                         h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms)));
         BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>,
                          dim3(ceil_div((long long)T_ * K, 8)), dim3(256), 0, st,
                          (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D, nch,

@@ -20,6 +20,10 @@ struct Group {
 };
 
 // Device-side statistics of one forward, reduced in a fixed order.
+// Row-tile height of the tensor-core grouped GEMMs.  The compaction records, next to the
+// number of groups, how many tiles of this height the groups take (the GEMMs' tile count).
+constexpr int kGroupTileRows = 128;
+
 struct DevStats {
     long long keep_sum;   // sum over tokens of kept slots
     double lreg_sum;      // sum over tokens of (1/K) sum_{TK} sigmoid(mask logit)

@@ -61,7 +61,8 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                     const int* __restrict__ nkeep_tok, const float* __restrict__ lreg_tok,
                     int* __restrict__ counts, int* __restrict__ offsets,
                     int* __restrict__ chunk_base, Group* __restrict__ groups,
-                    int* __restrict__ n_groups, DevStats* __restrict__ stats)
+                    int* __restrict__ n_groups, DevStats* __restrict__ stats,
+                    int* __restrict__ tail_cnt, int n_tail_cnt)
 {
     __shared__ int s_counts[kMaxE];
     __shared__ long long s_keep[32];
@@ -70,6 +71,8 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
+    // the arrival counters of the grouped GEMMs' tail split start every forward at zero
+    for (int i = threadIdx.x; i < n_tail_cnt; i += blockDim.x) tail_cnt[i] = 0;
 
     // 1. per-expert chunk prefix sums
     for (int e = warp; e < E; e += nwarps) {
@@ -126,9 +129,15 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
         }
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         const int tact = __shfl_sync(0xffffffffu, inca, 31);
+        int mt = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mt += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mt += __shfl_xor_sync(0xffffffffu, mt, o);
         if (lane == 0) {
             offsets[E] = total;
-            *n_groups = tact;
+            n_groups[0] = tact;
+            n_groups[1] = mt;
             stats->n_kept = total;
             stats->n_active = tact;
         }
@@ -232,7 +241,8 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
                            int* __restrict__ offsets, Group* __restrict__ groups,
                            int* __restrict__ n_groups, DevStats* __restrict__ stats,
                            int* __restrict__ perm, int* __restrict__ inv,
-                           const TW* __restrict__ x, TW* __restrict__ xperm, int D, int gather)
+                           const TW* __restrict__ x, TW* __restrict__ xperm, int D, int gather,
+                           int* __restrict__ tail_cnt, int n_tail_cnt)
 {
     __shared__ int s_id[kSmallT][32];
     __shared__ uint8_t s_keep[kSmallT][32];
@@ -246,6 +256,8 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kSmallT * (kMaxE / 32 + 1); i += blockDim.x)
         (&s_mask[0][0])[i] = 0u;
+    // the arrival counters of the grouped GEMMs' tail split start every forward at zero
+    for (int i = threadIdx.x; i < n_tail_cnt; i += blockDim.x) tail_cnt[i] = 0;
     __syncthreads();
 
     // 1. selection
@@ -321,6 +333,11 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
         }
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         const int tact = __shfl_sync(0xffffffffu, inca, 31);
+        int mt = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mt += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mt += __shfl_xor_sync(0xffffffffu, mt, o);
         long long ks = lane < T ? s_nk[lane] : 0;
         double ls = lane < T ? (double)s_lr[lane] : 0.0;
         int nz = (lane < T && s_nk[lane] == 0) ? 1 : 0;
@@ -333,7 +350,8 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
         if (lane == 0) {
             offsets[E] = total;
             s_off[E] = total;
-            *n_groups = tact;
+            n_groups[0] = tact;
+            n_groups[1] = mt;
             stats->n_kept = total;
             stats->n_active = tact;
             stats->keep_sum = ks;

@@ -12,6 +12,10 @@
 //   * small batches split K across tiles so that a handful of kept groups still spreads over
 //     every SM: the f32-store epilogue then writes per-split partial sums, which the next step
 //     adds in a fixed order (the SwiGLU finishing kernel for gate/up, the combine for down);
+//   * larger batches keep whole-K tiles, except for the last, partial wave: its tiles may be cut
+//     into K pieces run on otherwise idle SMs.  Each piece stores an f32 partial; the epilogue
+//     warp that arrives last at a sub-block (an atomic counter decides who, never the order)
+//     adds the pieces' partials in piece order and runs the normal epilogue on the sum;
 //   * tile 128 (tokens) x 256 x 64, TMA (cp.async.bulk.tensor, 128-byte swizzle, no cluster
 //     multicast) fills a 4-stage shared-memory ring guarded by mbarriers;
 //   * warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma (kind::f16, fp32
@@ -27,7 +31,7 @@
 namespace beam {
 namespace tc {
 
-constexpr int BM = 128;
+constexpr int BM = kGroupTileRows;
 constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
@@ -44,6 +48,17 @@ constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH * 4;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES + 1024 /*alignment slack*/ +
                            256 /*barriers*/;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s: far above any tile
+// Tail split: at most kTailMaxPieces K pieces per tile, each at least kTailMinSteps k steps,
+// spread over at most two sub-waves of the grid.  One piece's partial is one epilogue warp's
+// 32 x 128 f32 sub-block per warp: kTailSlotFloats floats per (piece, warp).
+constexpr int kTailMaxPieces = 8;
+constexpr int kTailMinSteps = 8;
+constexpr int kTailMaxSubWaves = 2;
+constexpr int kTailSlotFloats = 4 * 32 * 32;
+// Launches of fewer k steps use the kernel without the tail path: below 32 tail_pieces never
+// splits (pieces of at least 8 steps that cut the tail by a quarter), and from 32 to 39 it
+// splits only tails of at most a third of a wave, saving less than the heavier epilogue costs.
+constexpr int kTailMinKSteps = 40;
 constexpr int ERR_TC_TIMEOUT = 0x100;
 
 // Epilogues: SwiGLU -> fp16 H; f32 stores (router logits, split-K partials); f16 stores
@@ -56,7 +71,7 @@ struct TcParams {
     CUtensorMap a_shared;   // activations of the shared group (rows = tokens)
     CUtensorMap b_shared;   // shared-expert weights
     const Group* groups;
-    const int* n_groups;
+    const int* n_groups;    // [0]: groups, [1]: their m tiles (tiles of BM rows)
     void* out_routed;       // EPI_SWIGLU: fp16 H [rows][F]; EPI_STORE_F32: f32 Y [rows][D]
     void* out_shared;
     int ld_routed;          // row length of out_routed
@@ -72,7 +87,33 @@ struct TcParams {
     long long split_stride_shared;
     int shared_rows;        // T, or 0 when there is no shared group
     int* err;
+    // Tail split (whole-K launches of one problem only; null = off): arrival counters
+    // [grid][kEpiWarps], zero on entry, and the partial workspace
+    // [kTailMaxSubWaves * grid slots][kEpiWarps][kTailSlotFloats].
+    int* tail_cnt;
+    float* tail_ws;
 };
+
+// Number of K pieces for the tail wave: rem whole-K tiles of ksteps k steps are left over after
+// the full waves of a grid of G CTAs.  The estimated tail makespan, in k steps, is ksteps
+// unsplit, and sub_waves * (ceil(ksteps / s) + 4 + 3 s) with s pieces (the constant covers the
+// partial store and the fences, the 3 s the reading of s partials by the warp that finishes
+// the sub-block).  A split must cut the estimate by at least a quarter; ties keep the smaller
+// s.  Every thread of the grid evaluates this on the same integers.
+__host__ __device__ inline int tail_pieces(long long rem, int ksteps, int G)
+{
+    if (rem <= 0) return 1;
+    int best = 1;
+    long long best_cost = ksteps;
+    for (int s = 2; s <= kTailMaxPieces; ++s) {
+        if (ksteps < kTailMinSteps * s) break;
+        const long long sub = (rem * s + G - 1) / G;
+        if (sub > kTailMaxSubWaves) break;
+        const long long cost = sub * ((ksteps + s - 1) / s + 4 + 3 * s);
+        if (cost < best_cost) { best_cost = cost; best = s; }
+    }
+    return 4 * best_cost <= 3LL * ksteps ? best : 1;
+}
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -214,6 +255,9 @@ struct Tile {
     int brow;     // first weight row of the tile
     int k0, k1;   // k steps [k0, k1) of this tile (its K split)
     int ks;       // K split index (selects the output slice)
+    int pieces;   // tail split: K pieces of this tile (1 = a whole tile)
+    int tail;     // tail split: index of the tile among the split ones
+    int slot;     // tail split: workspace slot of this piece (tail * pieces + piece)
 };
 
 __device__ __forceinline__ void split_range(int ksteps, int splits, int ks, int& k0, int& k1) {
@@ -222,18 +266,26 @@ __device__ __forceinline__ void split_range(int ksteps, int splits, int ks, int&
     k1 = min(ksteps, k0 + per);
 }
 
-// Walks tiles blockIdx.x, blockIdx.x + gridDim.x, ... in order; every role of a CTA holds
-// its own copy and sees the same sequence.
+// Walks work units blockIdx.x, blockIdx.x + gridDim.x, ... in order; every role of a CTA
+// holds its own copy and sees the same sequence.  Without a tail split a unit is a tile.  With
+// one, units [0, whole_end) are the whole tiles of the full waves and the units after them the
+// K pieces of the remaining tiles, tile-major (so tile indices never decrease along a walk).
+// TAIL = false compiles the plain walk only.
+template <bool TAIL>
 struct TileWalker {
     const TcParams* p;
     int ng;
     int count_sh;      // tiles of the shared problem
     int mts_sh;
-    long long next;    // next global tile index
+    long long next;    // next unit index
+    int whole_end;     // units below this are whole tiles
+    int n_units;       // units of the launch
+    int pieces;
     int g;             // cursor: current group and the first tile index of it
     long long g_base;
 
-    __device__ void init(const TcParams* p_, int ng_) {
+    // n_tiles: tiles of the launch (needed only with a tail split, else ignored)
+    __device__ void init(const TcParams* p_, int ng_, long long n_tiles = 0) {
         p = p_;
         ng = ng_;
         mts_sh = p->shared_rows > 0 ? (p->shared_rows + BM - 1) / BM : 0;
@@ -241,11 +293,40 @@ struct TileWalker {
         next = blockIdx.x;
         g = 0;
         g_base = count_sh;
+        pieces = 1;
+        whole_end = n_units = 0x7fffffff;
+        if (TAIL && p->tail_cnt != nullptr) {
+            const int ksteps = p->shared_rows > 0 ? p->k_steps_shared : p->k_steps_routed;
+            const int rem = (int)(n_tiles % gridDim.x);
+            pieces = tail_pieces(rem, ksteps, gridDim.x);
+            if (pieces > 1) {
+                whole_end = (int)(n_tiles - rem);
+                n_units = whole_end + rem * pieces;
+            }
+        }
     }
     // tile index order inside a problem: m tile fastest, then K split, then n tile
     __device__ bool get(Tile& t) {
-        const long long i = next;
+        const long long u = next;
         next += gridDim.x;
+        long long i = u;
+        int piece = 0;
+        t.pieces = 1;
+        t.tail = t.slot = 0;
+        if (TAIL && u >= n_units) return false;
+        if (TAIL && u >= whole_end) {
+            const int local = (int)(u - whole_end);
+            t.tail = local / pieces;
+            piece = local % pieces;
+            t.slot = local;
+            t.pieces = pieces;
+            i = whole_end + t.tail;
+        }
+        if (!locate(i, t)) return false;
+        if (TAIL && t.pieces > 1) split_range(t.k1 - t.k0, t.pieces, piece, t.k0, t.k1);
+        return true;
+    }
+    __device__ bool locate(long long i, Tile& t) {
         if (i < count_sh) {
             const int per_n = mts_sh * p->k_splits_shared;
             t.shared = 1;
@@ -285,7 +366,9 @@ struct TileWalker {
 };
 
 // ---------------------------------------------------------------- the kernel
-template <int EPI, int FMT>
+// TAIL: the launch may cut its last wave into K pieces (p.tail_cnt, p.tail_ws set); the
+// kernel without it has no piece path at all.
+template <int EPI, int FMT, bool TAIL>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
 {
@@ -330,11 +413,17 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
 
     pdl_wait();  // groups, counts and activations come from the previous kernels
     const int ng = *p.n_groups;
+    // tiles of the launch (used by the tail split): n_groups[1] holds the groups' m tiles
+    long long n_tiles = 0;
+    if (TAIL && p.tail_cnt != nullptr) {
+        const long long mts_sh = p.shared_rows > 0 ? (p.shared_rows + BM - 1) / BM : 0;
+        n_tiles = (long long)p.n_groups[1] * p.n_tiles_routed + mts_sh * p.n_tiles_shared;
+    }
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer
-        TileWalker w;
-        w.init(&p, ng);
+        TileWalker<TAIL> w;
+        w.init(&p, ng, n_tiles);
         Tile t;
         int s = 0;
         uint32_t ph = 0;
@@ -368,8 +457,8 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
-        TileWalker w;
-        w.init(&p, ng);
+        TileWalker<TAIL> w;
+        w.init(&p, ng, n_tiles);
         Tile t;
         int s = 0, acc = 0;
         uint32_t ph = 0, aph = 0;
@@ -404,36 +493,95 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue (TMEM -> registers -> global)
-        TileWalker w;
-        w.init(&p, ng);
+        TileWalker<TAIL> w;
+        w.init(&p, ng, n_tiles);
         Tile t;
         int acc = 0;
         uint32_t aph = 0;
         const int lb = 32 * (warp & 3);  // TMEM lanes this warp may access
         const int warp_e = warp - 2;     // index of this epilogue warp (its staging buffer)
         const int half = warp_e / 4;     // which half of the tile's columns this warp drains
+        // TMEM column of chunk c (0..3) of this warp's sub-block: 32-column chunks of its half
+        // of the tile; for SwiGLU the even chunks are gate columns, the odd ones the matching
+        // up columns.
+        auto chunk_col = [&](int c) {
+            return EPI == EPI_SWIGLU ? (c & 1) * (BN / 2) + 32 * (half * 2 + (c >> 1))
+                                     : 32 * (half * 4 + c);
+        };
         while (w.get(t)) {
             if (!mbar_wait(tfull_bar(acc), aph, abort_flag)) break;
             tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)lb << 16) + (uint32_t)(acc * BN);
             // rows lb .. lb+31 of the tile belong to this warp; row_ok(i) = row i of them is
             // a row of the group.  Each 32-column chunk goes TMEM -> registers (thread = row)
             // -> padded shared memory -> registers (thread = column) -> one coalesced store per
             // row, so every store instruction writes one contiguous row segment.
             const int r0 = t.mt * BM + lb;                 // first row of this warp, in the group
             const int nrows = max(0, min(32, t.m - r0));   // valid rows of this warp
-            const uint32_t tbase = tmem_base + ((uint32_t)lb << 16) + (uint32_t)(acc * BN);
             float* buf = epi_buf + warp_e * (32 * EPI_PITCH);
             const int ld = t.shared ? p.ld_shared : p.ld_routed;
             const size_t row_base = (size_t)(t.row0 + r0);
+            // A K piece of a tail tile stores this warp's partial sub-block, frees the TMEM
+            // buffer and counts the arrival; the warp that completes the count adds the
+            // pieces' partials in piece order (red != null) and runs the epilogue on the sum.
+            // Partial layout per (piece, warp): [chunk c][column i][row lane], so that a warp
+            // writes and reads 32 consecutive floats per column.
+            const float* red = nullptr;
+            if (TAIL && t.pieces > 1) {
+                float* mine = p.tail_ws + ((size_t)t.slot * kEpiWarps + warp_e) * kTailSlotFloats;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tbase + chunk_col(c), v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) __stcg(mine + (c * 32 + i) * 32 + lane, v[i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(acc));
+                if (++acc == 2) { acc = 0; aph ^= 1u; }
+                __threadfence();
+                __syncwarp();
+                int prev = 0;
+                if (lane == 0) prev = atomicAdd(p.tail_cnt + t.tail * kEpiWarps + warp_e, 1);
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev != t.pieces - 1) continue;
+                __syncwarp();
+                __threadfence();   // the other pieces' partials are visible past this point
+                red = p.tail_ws + ((size_t)t.tail * t.pieces * kEpiWarps + warp_e) * kTailSlotFloats;
+            }
+            // chunk c of this warp's rows (thread = row) summed over the pieces, in piece order
+            auto reduce = [&](int c, float* v) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                const float* src = red + c * 32 * 32 + lane;
+#pragma unroll 1
+                for (int q = 0; q < t.pieces; ++q, src += (size_t)kEpiWarps * kTailSlotFloats) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] += __ldcg(src + i * 32);
+                }
+            };
             if (EPI == EPI_SWIGLU) {
                 __half* out = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed);
 #pragma unroll 1
                 for (int j = half * (BN / 2 / 64); j < (half + 1) * (BN / 2 / 64); ++j) {
-                    float g[32], u[32];
-                    tmem_ld32(tbase + 32 * j, g);
-                    tmem_ld32(tbase + BN / 2 + 32 * j, u);
+                    if (!TAIL || red == nullptr) {
+                        float g[32], u[32];
+                        tmem_ld32(tbase + 32 * j, g);
+                        tmem_ld32(tbase + BN / 2 + 32 * j, u);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) buf[lane * EPI_PITCH + c] = silu_f(g[c]) * u[c];
+                        for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] = silu_f(g[i]) * u[i];
+                    } else {
+                        // two passes keep 32 sums live: silu(gate) into the buffer, then * up
+                        const int c = 2 * (j - half * (BN / 2 / 64));
+                        float v[32];
+                        reduce(c, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] = silu_f(v[i]);
+                        reduce(c + 1, v);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] *= v[i];
+                    }
                     __syncwarp();
                     __half* col = out + row_base * ld + (size_t)t.n * (BN / 2) + 32 * j + lane;
                     for (int i = 0; i < nrows; ++i)
@@ -445,9 +593,10 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
 #pragma unroll 1
                 for (int j = half * (BN / 64); j < (half + 1) * (BN / 64); ++j) {
                     float v[32];
-                    tmem_ld32(tbase + 32 * j, v);
+                    if (!TAIL || red == nullptr) tmem_ld32(tbase + 32 * j, v);
+                    else reduce(j - half * (BN / 64), v);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) buf[lane * EPI_PITCH + c] = v[c];
+                    for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] = v[i];
                     __syncwarp();
                     const size_t off = (size_t)t.ks * sstride + row_base * ld + (size_t)t.n * BN + 32 * j + lane;
                     if (EPI == EPI_STORE_F16) {
@@ -461,10 +610,12 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                     __syncwarp();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
-            if (++acc == 2) { acc = 0; aph ^= 1u; }
+            if (!TAIL || red == nullptr) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(acc));
+                if (++acc == 2) { acc = 0; aph ^= 1u; }
+            }
         }
     }
 

@@ -154,9 +154,12 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * launch overlap between kernels while it is on).  beam_moe_profile_end waits for them, adds
  * up the event times per stage into stage_ms[BEAM_N_STAGES] and the launches per stage into
  * stage_launches[BEAM_N_STAGES] (either may be NULL), sets *n_forwards, and switches timing
- * off.  beam_moe_stage_name(i) names stage i ("" when out of range).
+ * off.  beam_moe_stage_name(i) names stage i ("" when out of range).  On the tensor-core path
+ * the shared experts' GEMMs run on a second stream, overlapping the routing; they are timed
+ * under stages of their own (tc_shared_gateup, tc_shared_down, shared_swiglu_finish), so that
+ * each stage's time covers the work of one problem.
  */
-#define BEAM_N_STAGES 12
+#define BEAM_N_STAGES 15
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);

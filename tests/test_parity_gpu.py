@@ -264,3 +264,117 @@ def test_large_max_tokens_small_forward():
     spec = _small(n_shared=1, d_ff_shared=128)
     run_case(spec, 1, seed=5, max_tokens=20000)
     run_case(spec, 3000, seed=6, max_tokens=20000)
+
+
+@pytest.mark.parametrize("T", [4, 300])
+def test_profiling_stages_count_every_launch(T):
+    """Per-stage timing: the shared experts' GEMMs are timed under stages of their own, each
+    tensor-core stage launches once per forward, and the launches per stage add up to the
+    handle's launch counter (so a roofline that divides a stage's time by its launches and
+    its work by one problem is consistent).  T = 4 takes the split-K variants, T = 300 not."""
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=256)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=T)
+    x = synth.make_tokens(spec, T, seed=5).cuda()
+    y = torch.empty((T, spec.d_model), device="cuda")
+    layer.forward(x, path="tensor", out=y)
+    n = 3
+    n0 = layer.launch_count()
+    layer.profile_begin(n)
+    for _ in range(n):
+        layer.forward(x, path="tensor", out=y)
+    prof = layer.profile_end()
+    assert prof["forwards"] == n
+    stages = {k: v for k, v in prof.items() if k != "forwards"}
+    assert sum(c for _, c in stages.values()) == layer.launch_count() - n0
+    for s in ("tc_gateup", "tc_down", "tc_shared_gateup", "tc_shared_down"):
+        assert stages[s][1] == n, (s, stages[s])
+        assert stages[s][0] > 0
+    split = "swiglu_finish" in stages
+    assert split == (T <= 64)
+    if split:
+        assert stages["shared_swiglu_finish"][1] == n
+    layer.close()
+
+
+# ------------------------------------------------------------------ tail-wave K pieces
+def _tail_pieces(rem, ksteps, G):
+    """K pieces per tile of the last, partial wave, as the grouped GEMM chooses them: at most
+    8 pieces of at least 8 k steps each in at most two sub-waves, minimising the estimated
+    tail makespan sub_waves * (ceil(ksteps / s) + 4 + 3 s), and only when that is at most
+    three quarters of ksteps (the unsplit tail)."""
+    if rem <= 0:
+        return 1
+    best, best_cost = 1, ksteps
+    for s in range(2, 9):
+        if ksteps < 8 * s:
+            break
+        sub = -(-rem * s // G)
+        if sub > 2:
+            break
+        cost = sub * (-(-ksteps // s) + 4 + 3 * s)
+        if cost < best_cost:
+            best, best_cost = s, cost
+    return best if 4 * best_cost <= 3 * ksteps else 1
+
+
+def _k_splits(G, tiles, ksteps):
+    """Split-K factor of a forward of at most 64 tokens (the host's makespan rule: 4 % per
+    extra split, at least 4 k steps per slice, no empty slice)."""
+    best, best_cost = 1, float("inf")
+    for s in range(1, 17):
+        cost = (-(-tiles * s // G)) / s * (1.0 + 0.04 * (s - 1))
+        if cost < best_cost - 1e-9:
+            best, best_cost = s, cost
+    s = max(1, min(best, max(1, ksteps // 4)))
+    per = -(-ksteps // s)
+    return -(-ksteps // per)
+
+
+def _routed_tail_pieces(spec, T, counts):
+    """K pieces of the tail tiles of the routed gate/up and down launches of a forward with
+    these kept rows per expert (1 = no tail split: also whenever the launch splits K, and for
+    launches of fewer than 40 k steps, which run the kernel without the tail path)."""
+    G = torch.cuda.get_device_properties(0).multi_processor_count
+    D, F, K, E = spec.d_model, spec.d_ff, spec.top_k, spec.n_experts
+    M = int(sum(-(-int(c) // 128) for c in counts))
+    out = {}
+    for name, nt, ks in (("gateup", 2 * F // 256, D // 64), ("down", D // 256, F // 64)):
+        if T <= 64:
+            groups = min(E, max(1, (T * K + 1) // 2))
+            if _k_splits(G, -(-T // 128) * groups * nt, ks) > 1:
+                out[name] = 1
+                continue
+        out[name] = _tail_pieces(M * nt % G, ks, G) if ks >= 40 else 1
+    return out
+
+
+@pytest.mark.parametrize("spec,T,expect", [
+    (synth.LayerSpec("tail_a", 4096, 2, 1, 4096), 128, ("gateup", "down")),
+    (synth.LayerSpec("tail_b", 4096, 4, 1, 512), 300, ("gateup",)),
+    (synth.LayerSpec("tail_c", 1024, 4, 1, 4096), 256, ("down",)),
+    (synth.LayerSpec("tail_d", 4096, 8, 2, 512), 4400, ("gateup",)),
+    (synth.LayerSpec("tail_e", 3072, 2, 1, 3072, n_shared=1, d_ff_shared=512), 256, ("gateup", "down")),
+    (synth.LayerSpec("tail_f", 4096, 160, 16, 256), 18, ("gateup",)),
+], ids=["both_gemms", "deep_k_gateup", "deep_k_down", "full_wave_then_pieces",
+        "with_shared_problem", "fused_small_routing"])
+def test_tail_wave_k_pieces(spec, T, expect):
+    """Whole-K launches of the routed problem cut the tiles of their last, partial wave into K
+    pieces whose f32 partials the last-arriving epilogue warp adds in piece order.  These
+    shapes make the launches named in `expect` take that path (checked from the routing the
+    GPU produced); the last one routes through the fused small-batch kernel, which also clears
+    the arrival counters.  y is compared with the oracle on every token (or a spread sample
+    for the larger layers); run_case runs two forwards (the second on counters the first
+    used), and a direct launch gives the same bits as the graph replay."""
+    big = spec.d_model * spec.d_ff * T > 2_000_000_000 or spec.d_ff_shared * spec.d_model * T > 1_000_000_000
+    sample = np.unique(np.concatenate([np.arange(0, T, 13), [T - 1]])) if big else None
+    info = run_case(spec, T, seed=31, y_tokens=sample)
+    pieces = _routed_tail_pieces(spec, T, info["stats"]["counts"])
+    for name in expect:
+        assert pieces[name] > 1, (name, pieces)
+    layer = info["layer"]
+    y2 = layer.forward(info["x"].cuda(), graph=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, info["y"])
+    layer.close()
