@@ -563,6 +563,54 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+_BYTE_UNITS = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12,
+               "KB": 1e3, "MB": 1e6, "GB": 1e9, "B": 1}
+
+
+def record_traffic(args):
+    """Write the per-launch DRAM bytes of one kernel, read from an ncu CSV log of
+    dram__bytes_read.sum and dram__bytes_write.sum, into profiles/traffic.json under
+    (workload, stage), stamped with the hash of the kernel sources it was measured on (a later
+    source change makes the bench report null until it is captured again)."""
+    import csv
+    import re
+    pat = re.compile(args.traffic_kernel)
+    per_launch = {}
+    with open(args.record_traffic, newline="") as f:
+        rows = [r for r in csv.reader(f) if r]
+    head = next(i for i, r in enumerate(rows) if "Metric Name" in r)
+    cols = {name: j for j, name in enumerate(rows[head])}
+    for r in rows[head + 1:]:
+        if len(r) < len(cols) or not pat.search(r[cols["Kernel Name"]]):
+            continue
+        name = r[cols["Metric Name"]]
+        if name not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        v = float(r[cols["Metric Value"]].replace(",", "")) * _BYTE_UNITS[r[cols["Metric Unit"]]]
+        per_launch.setdefault(r[cols["ID"]], {})[name] = v
+    totals = [d["dram__bytes_read.sum"] + d["dram__bytes_write.sum"] for d in per_launch.values()
+              if len(d) == 2]
+    if not totals:
+        raise SystemExit(f"no launch of /{args.traffic_kernel}/ with both DRAM metrics")
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except FileNotFoundError:
+        d = {}
+    d.setdefault(args.workload, {})[args.traffic_stage] = {
+        "dram_bytes_per_launch": int(round(sum(totals) / len(totals))),
+        "launches": len(totals),
+        "kernel": args.traffic_kernel,
+        "source_hash": kernel_source_hash(),
+        "command": args.traffic_command,
+    }
+    with open(path, "w") as f:
+        json.dump(d, f, indent=1, sort_keys=True)
+        f.write("\n")
+    print(json.dumps(d[args.workload][args.traffic_stage]))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -575,7 +623,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
     ap.add_argument("--sweep", action="store_true",
                     help="measure every workload (one JSON line each) instead of the headline")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="store a kernel's DRAM bytes per launch from an ncu CSV log (no GPU work)")
+    ap.add_argument("--traffic-kernel", default=r"tc_grouped_gemm_kernel<(\(int\))?0,",
+                    help="regex of the kernel name in the CSV (gate/up: EPI 0, down: EPI 2)")
+    ap.add_argument("--traffic-stage", default="tc_gateup", help="bench stage of that kernel")
+    ap.add_argument("--traffic-command", default="", help="the ncu command that wrote the CSV")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
