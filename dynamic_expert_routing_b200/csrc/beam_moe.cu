@@ -460,6 +460,7 @@ static beam_status_t setup_tc(beam_moe* h)
     r.n_tiles_routed = r.n_tiles_shared = h->ldL / tc::BN;
     r.k_steps_routed = r.k_steps_shared = (int)(D / tc::BK);
     r.k_splits_routed = r.k_splits_shared = 1;
+    r.store_cols = 2 * E;                  // columns past 2E are padding nobody reads
     r.err = &h->dstats->err;
     {
         const void* kernels[] = {

@@ -86,6 +86,7 @@ struct TcParams {
     long long split_stride_routed;  // elements between the outputs of consecutive K splits
     long long split_stride_shared;
     int shared_rows;        // T, or 0 when there is no shared group
+    int store_cols;         // f32 store epilogue: columns [0, store_cols) are stored (0 = all)
     int* err;
     // Tail split (whole-K launches of one problem only; null = off): arrival counters
     // [grid][kEpiWarps], zero on entry, and the partial workspace
@@ -592,6 +593,10 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                 const long long sstride = t.shared ? p.split_stride_shared : p.split_stride_routed;
 #pragma unroll 1
                 for (int j = half * (BN / 64); j < (half + 1) * (BN / 64); ++j) {
+                    // the router's logit rows are padded to the tile width: only the chunks
+                    // holding the 2E real columns are read back
+                    if (EPI == EPI_STORE_F32 && p.store_cols > 0 && t.n * BN + 32 * j >= p.store_cols)
+                        continue;
                     float v[32];
                     if (!TAIL || red == nullptr) tmem_ld32(tbase + 32 * j, v);
                     else reduce(j - half * (BN / 64), v);
