@@ -397,6 +397,9 @@ static beam_status_t setup_tc(beam_moe* h)
     // GEMM2: H [rows][F] x W_d [E*D][F] -> Y_perm (f32) [rows][D]
     BEAM_TRY(encode_map(h, &b.a_routed, HF, h->hbuf, rows, F, tc::BM));
     BEAM_TRY(encode_map(h, &b.b_routed, HF, h->wd, E * D, F, tc::BN));
+    // the same activations in boxes of kSwapBox rows, for the swapped small groups
+    BEAM_TRY(encode_map(h, &a.a_routed_tail, BF, h->xperm, rows, D, tc::kSwapBox));
+    BEAM_TRY(encode_map(h, &b.a_routed_tail, HF, h->hbuf, rows, F, tc::kSwapBox));
     if (Fsh) {
         BEAM_TRY(encode_map(h, &a.b_shared, BF, h->wsgu, 2 * Fsh, D, tc::BN));
         BEAM_TRY(encode_map(h, &b.a_shared, HF, h->hsh, Tm, Fsh, tc::BM));
@@ -464,12 +467,14 @@ static beam_status_t setup_tc(beam_moe* h)
     r.err = &h->dstats->err;
     {
         const void* kernels[] = {
-            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, false>,
-            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, false>,
-            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, true>,
-            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, false>,
-            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, false>,
-            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, true>};
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_PLAIN>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_TAIL>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_SWAP>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, tc::MODE_PLAIN>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_PLAIN>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_TAIL>,
+            (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_SWAP>};
         for (const void* k : kernels)
             BEAM_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
     }
@@ -669,15 +674,20 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
     p.n_groups = ngroups;
     p.shared_rows = rows_sh;
     p.k_splits_routed = p.k_splits_shared = s1;
-    // routed whole-K launches deep enough in K may cut the tiles of their last, partial wave
-    // into K pieces (the kernel variant with the tail path; the cut is decided on the device)
+    // Kernel form of a routed whole-K launch.  Groups averaging at most 2 * kSwapBox rows
+    // (T*K <= 64 E): the swap form, which runs groups of <= 64 rows with the weights as the M
+    // operand.  Otherwise, deep enough in K: the tail form, which may cut the tiles of the
+    // last, partial wave into K pieces (the cut is decided on the device).
     const size_t creg = (size_t)h->num_sms * tc::kEpiWarps;
-    const bool tail1 = !shared && s1 == 1 && D / tc::BK >= tc::kTailMinKSteps;
-    const bool tail2 = !shared && s2 == 1 && F / tc::BK >= tc::kTailMinKSteps;
+    const bool small_groups = !shared && (long long)T_ * K <= 2LL * tc::kSwapBox * E;
+    const bool swap1 = small_groups && s1 == 1;
+    const bool swap2 = small_groups && s2 == 1;
+    const bool tail1 = !shared && !small_groups && s1 == 1 && D / tc::BK >= tc::kTailMinKSteps;
+    const bool tail2 = !shared && !small_groups && s2 == 1 && F / tc::BK >= tc::kTailMinKSteps;
     p.tail_cnt = tail1 ? h->tail_cnt : nullptr;
     p.tail_ws = tail1 ? h->tail_ws : nullptr;
     if (s1 > 1) {
-        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, false>,
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
         const long long work = shared ? (long long)T_ * Fsh : (long long)T_ * K * F;
         BEAM_CUDA(launch(h, st_fin, tc::swiglu_finish_kernel,
@@ -686,11 +696,14 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
                          (const int*)(shared ? h->zero_int : h->offsets + E), F, (__half*)h->hbuf,
                          (const float*)h->g1part_sh, s1, p.split_stride_shared, rows_sh, Fsh,
                          (__half*)h->hsh));
+    } else if (swap1) {
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_SWAP>,
+                         dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
     } else if (tail1) {
-        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, true>,
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_TAIL>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
     } else {
-        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, false>,
+        BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
     }
 
@@ -710,7 +723,7 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
         out.splits = s2;
         out.stride = shared ? q.split_stride_shared : q.split_stride_routed;
         out.f16 = false;
-        BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, false>,
+        BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
     } else {
         q.out_routed = h->yperm;
@@ -720,11 +733,14 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
         out.splits = 1;
         out.stride = 0;
         out.f16 = true;
-        if (tail2)
-            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, true>,
+        if (swap2)
+            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_SWAP>,
+                             dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
+        else if (tail2)
+            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_TAIL>,
                              dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
         else
-            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, false>,
+            BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_PLAIN>,
                              dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
     }
     return BEAM_OK;
@@ -778,7 +794,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         lstride = (long long)Tr * h->ldL;
         p0.k_splits_routed = p0.k_splits_shared = lsplits;
         p0.split_stride_routed = p0.split_stride_shared = lstride;
-        BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, false>,
+        BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
     } else {

@@ -12,6 +12,11 @@
 //   * small batches split K across tiles so that a handful of kept groups still spreads over
 //     every SM: the f32-store epilogue then writes per-split partial sums, which the next step
 //     adds in a fixed order (the SwiGLU finishing kernel for gate/up, the combine for down);
+//   * a group of at most 64 rows runs swapped (weights as the M = 128 operand, the group's rows
+//     as N = 32 or 64, loaded as 32-row boxes): such a tile streams its weights alone, and the
+//     swap cuts the activation copies from 16 to 4-8 KB per k-step.  (The short last tile of a
+//     larger group keeps the normal form: there the tensor pipe is the bound, and N <= 64
+//     instructions take longer per row than the full-width tile.);
 //   * larger batches keep whole-K tiles, except for the last, partial wave: its tiles may be cut
 //     into K pieces run on otherwise idle SMs.  Each piece stores an f32 partial; the epilogue
 //     warp that arrives last at a sub-block (an atomic counter decides who, never the order)
@@ -48,6 +53,9 @@ constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH * 4;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES + 1024 /*alignment slack*/ +
                            256 /*barriers*/;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s: far above any tile
+// Swapped small groups: rows come in boxes of kSwapBox; groups of at most 2 boxes swap.
+constexpr int kSwapBox = 32;
+constexpr int SWAP_BOX_BYTES = kSwapBox * BK * 2;
 // Tail split: at most kTailMaxPieces K pieces per tile, each at least kTailMinSteps k steps,
 // spread over at most two sub-waves of the grid.  One piece's partial is one epilogue warp's
 // 32 x 128 f32 sub-block per warp: kTailSlotFloats floats per (piece, warp).
@@ -70,6 +78,7 @@ struct TcParams {
     CUtensorMap b_routed;   // weights of the routed experts, [E * rows_per_expert][K]
     CUtensorMap a_shared;   // activations of the shared group (rows = tokens)
     CUtensorMap b_shared;   // shared-expert weights
+    CUtensorMap a_routed_tail;  // a_routed with a kSwapBox-row box (swapped small groups)
     const Group* groups;
     const int* n_groups;    // [0]: groups, [1]: their m tiles (tiles of BM rows)
     void* out_routed;       // EPI_SWIGLU: fp16 H [rows][F]; EPI_STORE_F32: f32 Y [rows][D]
@@ -241,8 +250,8 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 // Instruction descriptor, kind::f16: fp32 accumulator, A/B of format `fmt` (0 = f16,
 // 1 = bf16), both K-major, N = 256, M = 128.
-__host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt) {
-    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BN >> 3) << 17) |
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t n = BN) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((n >> 3) << 17) |
            ((uint32_t)(BM >> 4) << 24);
 }
 
@@ -256,6 +265,7 @@ struct Tile {
     int brow;     // first weight row of the tile
     int k0, k1;   // k steps [k0, k1) of this tile (its K split)
     int ks;       // K split index (selects the output slice)
+    int swap;     // 0, or N (32 / 64): a swapped tail tile (weights = M operand, rows = N)
     int pieces;   // tail split: K pieces of this tile (1 = a whole tile)
     int tail;     // tail split: index of the tile among the split ones
     int slot;     // tail split: workspace slot of this piece (tail * pieces + piece)
@@ -271,8 +281,8 @@ __device__ __forceinline__ void split_range(int ksteps, int splits, int ks, int&
 // holds its own copy and sees the same sequence.  Without a tail split a unit is a tile.  With
 // one, units [0, whole_end) are the whole tiles of the full waves and the units after them the
 // K pieces of the remaining tiles, tile-major (so tile indices never decrease along a walk).
-// TAIL = false compiles the plain walk only.
-template <bool TAIL>
+// TAIL = false compiles the plain walk only; SWAP marks the groups of at most 64 rows.
+template <bool TAIL, bool SWAP>
 struct TileWalker {
     const TcParams* p;
     int ng;
@@ -338,6 +348,7 @@ struct TileWalker {
             t.row0 = 0;
             t.m = p->shared_rows;
             t.brow = t.n * BN;
+            t.swap = 0;
             split_range(p->k_steps_shared, p->k_splits_shared, t.ks, t.k0, t.k1);
             return true;
         }
@@ -356,6 +367,7 @@ struct TileWalker {
                 t.row0 = G.row0;
                 t.m = G.m;
                 t.brow = G.expert * p->b_rows_per_expert + t.n * BN;
+                t.swap = (SWAP && G.m <= 2 * kSwapBox) ? (G.m <= kSwapBox ? kSwapBox : 2 * kSwapBox) : 0;
                 split_range(p->k_steps_routed, p->k_splits_routed, t.ks, t.k0, t.k1);
                 return true;
             }
@@ -367,12 +379,17 @@ struct TileWalker {
 };
 
 // ---------------------------------------------------------------- the kernel
-// TAIL: the launch may cut its last wave into K pieces (p.tail_cnt, p.tail_ws set); the
-// kernel without it has no piece path at all.
-template <int EPI, int FMT, bool TAIL>
+// Kernel forms.  MODE_TAIL: the launch may cut its last wave into K pieces (p.tail_cnt and
+// p.tail_ws set).  MODE_SWAP: groups of at most 64 rows run swapped (p.a_routed_tail set).
+// MODE_PLAIN has neither path compiled in.
+enum Mode { MODE_PLAIN = 0, MODE_TAIL = 1, MODE_SWAP = 2 };
+
+template <int EPI, int FMT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
 {
+    constexpr bool TAIL = MODE == MODE_TAIL;
+    constexpr bool SWAP = MODE == MODE_SWAP && EPI != EPI_STORE_F32;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -401,6 +418,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&p.a_routed); tma_prefetch_desc(&p.b_routed);
         tma_prefetch_desc(&p.a_shared); tma_prefetch_desc(&p.b_shared);
+        if (SWAP) tma_prefetch_desc(&p.a_routed_tail);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -423,7 +441,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer
-        TileWalker<TAIL> w;
+        TileWalker<TAIL, SWAP> w;
         w.init(&p, ng, n_tiles);
         Tile t;
         int s = 0;
@@ -436,11 +454,19 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             const CUtensorMap* am = t.shared ? &p.a_shared : &p.a_routed;
             const CUtensorMap* bm = t.shared ? &p.b_shared : &p.b_routed;
             const int arow = t.row0 + t.mt * BM;
+            const int nbox = t.swap / kSwapBox;  // swapped tile: 1 or 2 boxes of rows
             for (int k = t.k0; k < t.k1; ++k) {
                 if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) { ok = false; break; }
-                mbar_expect_tx(full_bar(s), STAGE_BYTES);
                 const uint32_t sa = base + s * STAGE_BYTES;
-                tma_load_2d(sa, am, full_bar(s), k * BK, arow);
+                if (SWAP && t.swap) {
+                    mbar_expect_tx(full_bar(s), B_BYTES + nbox * SWAP_BOX_BYTES);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(sa + b * SWAP_BOX_BYTES, &p.a_routed_tail, full_bar(s), k * BK,
+                                    arow + b * kSwapBox);
+                } else {
+                    mbar_expect_tx(full_bar(s), STAGE_BYTES);
+                    tma_load_2d(sa, am, full_bar(s), k * BK, arow);
+                }
                 tma_load_2d(sa + A_BYTES, bm, full_bar(s), k * BK, t.brow);
                 pend[s] = true;
                 pend_ph[s] = (int)ph;
@@ -458,7 +484,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
-        TileWalker<TAIL> w;
+        TileWalker<TAIL, SWAP> w;
         w.init(&p, ng, n_tiles);
         Tile t;
         int s = 0, acc = 0;
@@ -475,10 +501,23 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                 const uint32_t sa = base + s * STAGE_BYTES;
                 const uint64_t ad = sw128_desc(sa);
                 const uint64_t bd = sw128_desc(sa + A_BYTES);
+                if (SWAP && t.swap) {
+                    // D[weight row][token]: each 128-row half of the weight tile is an M = 128
+                    // operand; the tokens are the N operand; half h accumulates at column h*N
+                    const uint32_t idesc_s = make_idesc(FMT, (uint32_t)t.swap);
+                    const uint64_t wd1 = sw128_desc(sa + A_BYTES + BM * 128);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    tc_mma_f16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc,
-                               (k != t.k0 || kk != 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t accum = (k != t.k0 || kk != 0) ? 1u : 0u;
+                        tc_mma_f16(d_tmem, bd + 2ull * kk, ad + 2ull * kk, idesc_s, accum);
+                        tc_mma_f16(d_tmem + (uint32_t)t.swap, wd1 + 2ull * kk, ad + 2ull * kk, idesc_s, accum);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma_f16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc,
+                                   (k != t.k0 || kk != 0) ? 1u : 0u);
+                }
                 issued = true;
                 tc_commit(empty_bar(s));
                 if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -494,7 +533,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         }
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue (TMEM -> registers -> global)
-        TileWalker<TAIL> w;
+        TileWalker<TAIL, SWAP> w;
         w.init(&p, ng, n_tiles);
         Tile t;
         int acc = 0;
@@ -522,6 +561,50 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             float* buf = epi_buf + warp_e * (32 * EPI_PITCH);
             const int ld = t.shared ? p.ld_shared : p.ld_routed;
             const size_t row_base = (size_t)(t.row0 + r0);
+            // Swapped tile (a small group): TMEM lane = weight row (feature), column = token.  Gate/up:
+            // gate of the 128 features at columns [0, N), up at [N, 2N); warp half h takes the
+            // tokens [32h, 32h + 32).  Down: features 128h + lane at columns [hN, hN + N).  Every
+            // store writes 32 consecutive features of one token row.
+            if (SWAP && t.swap) {
+                const int N = t.swap;
+                const int r_first = t.mt * BM;   // first row of the tile, in the group
+                const uint32_t tb = tmem_base + ((uint32_t)lb << 16) + (uint32_t)(acc * BN);
+                __half* out = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed);
+                if (EPI == EPI_SWIGLU) {
+                    if (32 * half < N) {
+                        float g[32], u[32];
+                        tmem_ld32(tb + 32 * half, g);
+                        tmem_ld32(tb + N + 32 * half, u);
+                        const int r0h = r_first + 32 * half;
+                        const int nr = max(0, min(32, t.m - r0h));
+                        __half* col = out + (size_t)(t.row0 + r0h) * ld + (size_t)t.n * (BN / 2) + lb + lane;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            if (i < nr) *col = __float2half_rn(silu_f(g[i]) * u[i]);
+                            col += ld;
+                        }
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < N; c += 32) {
+                        float v[32];
+                        tmem_ld32(tb + half * N + c, v);
+                        const int nr = max(0, min(32, t.m - r_first - c));
+                        __half* col = out + (size_t)(t.row0 + r_first + c) * ld + (size_t)t.n * BN +
+                                      half * BM + lb + lane;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            if (i < nr) *col = __float2half_rn(v[i]);
+                            col += ld;
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(acc));
+                if (++acc == 2) { acc = 0; aph ^= 1u; }
+                continue;
+            }
             // A K piece of a tail tile stores this warp's partial sub-block, frees the TMEM
             // buffer and counts the arrival; the warp that completes the count adds the
             // pieces' partials in piece order (red != null) and runs the epilogue on the sum.

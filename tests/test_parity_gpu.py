@@ -334,10 +334,13 @@ def _k_splits(G, tiles, ksteps):
 
 def _routed_tail_pieces(spec, T, counts):
     """K pieces of the tail tiles of the routed gate/up and down launches of a forward with
-    these kept rows per expert (1 = no tail split: also whenever the launch splits K, and for
-    launches of fewer than 40 k steps, which run the kernel without the tail path)."""
+    these kept rows per expert (1 = no tail split: also whenever the launch splits K, for
+    launches of fewer than 40 k steps, and for forwards with T*K <= 64 E, which run the
+    swapped form for small groups instead)."""
     G = torch.cuda.get_device_properties(0).multi_processor_count
     D, F, K, E = spec.d_model, spec.d_ff, spec.top_k, spec.n_experts
+    if T * K <= 64 * E:
+        return {"gateup": 1, "down": 1}
     M = int(sum(-(-int(c) // 128) for c in counts))
     out = {}
     for name, nt, ks in (("gateup", 2 * F // 256, D // 64), ("down", D // 256, F // 64)):
@@ -351,22 +354,20 @@ def _routed_tail_pieces(spec, T, counts):
 
 
 @pytest.mark.parametrize("spec,T,expect", [
-    (synth.LayerSpec("tail_a", 4096, 2, 1, 4096), 128, ("gateup", "down")),
+    (synth.LayerSpec("tail_a", 4096, 2, 1, 4096), 130, ("gateup", "down")),
     (synth.LayerSpec("tail_b", 4096, 4, 1, 512), 300, ("gateup",)),
-    (synth.LayerSpec("tail_c", 1024, 4, 1, 4096), 256, ("down",)),
+    (synth.LayerSpec("tail_c", 1024, 4, 1, 4096), 300, ("down",)),
     (synth.LayerSpec("tail_d", 4096, 8, 2, 512), 4400, ("gateup",)),
     (synth.LayerSpec("tail_e", 3072, 2, 1, 3072, n_shared=1, d_ff_shared=512), 256, ("gateup", "down")),
-    (synth.LayerSpec("tail_f", 4096, 160, 16, 256), 18, ("gateup",)),
 ], ids=["both_gemms", "deep_k_gateup", "deep_k_down", "full_wave_then_pieces",
-        "with_shared_problem", "fused_small_routing"])
+        "with_shared_problem"])
 def test_tail_wave_k_pieces(spec, T, expect):
     """Whole-K launches of the routed problem cut the tiles of their last, partial wave into K
     pieces whose f32 partials the last-arriving epilogue warp adds in piece order.  These
     shapes make the launches named in `expect` take that path (checked from the routing the
-    GPU produced); the last one routes through the fused small-batch kernel, which also clears
-    the arrival counters.  y is compared with the oracle on every token (or a spread sample
-    for the larger layers); run_case runs two forwards (the second on counters the first
-    used), and a direct launch gives the same bits as the graph replay."""
+    GPU produced).  y is compared with the oracle on every token (or a spread sample for the
+    larger layers); run_case runs two forwards (the second on counters the first used, which
+    the compaction clears), and a direct launch gives the same bits as the graph replay."""
     big = spec.d_model * spec.d_ff * T > 2_000_000_000 or spec.d_ff_shared * spec.d_model * T > 1_000_000_000
     sample = np.unique(np.concatenate([np.arange(0, T, 13), [T - 1]])) if big else None
     info = run_case(spec, T, seed=31, y_tokens=sample)
@@ -375,6 +376,44 @@ def test_tail_wave_k_pieces(spec, T, expect):
         assert pieces[name] > 1, (name, pieces)
     layer = info["layer"]
     y2 = layer.forward(info["x"].cuda(), graph=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, info["y"])
+    layer.close()
+
+
+# ------------------------------------------------------------------ swapped small groups
+@pytest.mark.parametrize("spec,T", [
+    (synth.LayerSpec("swap", 4096, 8, 8, 2048), 16),      # groups of 16 rows: N = 32
+    (synth.LayerSpec("swap", 4096, 8, 8, 2048), 32),      # 32 rows: N = 32
+    (synth.LayerSpec("swap", 4096, 8, 8, 2048), 33),      # 33 rows: N = 64
+    (synth.LayerSpec("swap", 4096, 8, 8, 2048), 64),      # 64 rows: N = 64
+], ids=["rows16", "rows32", "rows33", "rows64"])
+def test_swapped_small_groups(spec, T):
+    """A group of at most 64 rows in a whole-K launch runs with the weights as the M operand
+    and its rows as N = 32 or 64.  With K = E and the mask off every expert gets exactly T rows
+    (these sizes keep K unsplit: 128 gate/up and 128 down tiles).  T <= 32 routes through the
+    fused small-batch kernel, T = 33 and 64 through the multi-kernel path."""
+    sample = np.unique(np.concatenate([np.arange(0, T, 4), [T - 1]]))
+    info = run_case(spec, T, seed=41, mask_off=True, y_tokens=sample)
+    np.testing.assert_array_equal(info["stats"]["counts"], np.full(spec.n_experts, T))
+    layer = info["layer"]
+    y2 = layer.forward(info["x"].cuda(), mask_off=True, graph=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, info["y"])
+    layer.close()
+
+
+def test_swapped_many_small_groups():
+    """Many small groups (64 experts, K = 2, 1000 tokens: 15 to 44 rows each, T*K <= 64 E) in
+    whole-K launches with several waves of tiles: every group runs swapped."""
+    spec = synth.LayerSpec("swap_many", 4096, 64, 2, 1280)
+    T = 1000
+    sample = np.unique(np.concatenate([np.arange(0, T, 16), [T - 1]]))
+    info = run_case(spec, T, seed=43, mask_off=True, y_tokens=sample)
+    counts = info["stats"]["counts"]
+    assert (counts <= 64).all() and (counts > 0).all()
+    layer = info["layer"]
+    y2 = layer.forward(info["x"].cuda(), mask_off=True, graph=False)
     torch.cuda.synchronize()
     assert torch.equal(y2, info["y"])
     layer.close()
