@@ -129,6 +129,7 @@ struct beam_moe {
     int *chunk_base = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
     Group* groups = nullptr;
     int* n_groups = nullptr;     // [0]: kept groups, [1]: their 128-row tiles
+    Group* tile_group = nullptr; // 128-row tile (numbered across the groups) -> its group
     DevStats* dstats = nullptr;
     // expert workspace
     void *xperm = nullptr, *hbuf = nullptr, *hsh = nullptr;
@@ -412,6 +413,7 @@ static beam_status_t setup_tc(beam_moe* h)
     a.a_shared = a.a_routed;  // replaced by the map of x in every forward
     a.groups = b.groups = h->groups;
     a.n_groups = b.n_groups = h->n_groups;
+    a.tile_group = b.tile_group = h->tile_group;
     a.out_routed = h->hbuf; a.ld_routed = (int)F;
     a.out_shared = h->hsh;  a.ld_shared = (int)Fsh;
     b.out_routed = h->yperm; b.ld_routed = (int)D;
@@ -531,6 +533,7 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->inv, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->groups, E * sizeof(Group)));
     BEAM_TRY(dalloc(h, &h->n_groups, 2 * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->tile_group, (ceil_div((long long)rows, kGroupTileRows) + E) * sizeof(Group)));
     BEAM_TRY(dalloc(h, &h->dstats, sizeof(DevStats)));
     BEAM_TRY(dalloc(h, &h->tail_cnt, tail_cnt_ints(h->num_sms) * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->xperm, rows * D * es));
@@ -628,7 +631,8 @@ static cudaError_t launch_small(beam_moe* h, const T* x, int Tr, int T_, int mas
                   (const float*)h->L, h->ldL, splits, split_stride, Tr, T_, h->E, h->K, h->S,
                   mask_off, h->topk_id, h->gate, h->mlogit, h->keep, h->ghat, h->nkeep_tok,
                   h->lreg_tok, h->counts, h->offsets, h->groups, h->n_groups, h->dstats, h->perm,
-                  h->inv, x, (T*)h->xperm, h->D, gather, h->tail_cnt, tail_cnt_ints(h->num_sms));
+                  h->inv, x, (T*)h->xperm, h->D, gather, h->tail_cnt, tail_cnt_ints(h->num_sms),
+                  h->tile_group);
 }
 
 // Output of one expert problem for the combine: `splits` slices `stride` elements apart,
@@ -839,7 +843,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(1), dim3(1024), 0, st,
                          (const uint32_t*)h->bits, nch, E, T_, (const int*)h->nkeep_tok,
                          (const float*)h->lreg_tok, h->counts, h->offsets, h->chunk_base, h->groups,
-                         h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms)));
+                         h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms), h->tile_group));
         BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>,
                          dim3(ceil_div((long long)T_ * K, 8)), dim3(256), 0, st,
                          (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D, nch,

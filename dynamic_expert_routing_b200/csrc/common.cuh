@@ -12,12 +12,14 @@ constexpr int kWarp = 32;
 
 // One routed group = the kept (token, slot) pairs of one expert, contiguous in the permuted
 // activation matrix: rows [row0, row0 + m) of X_perm / H / Y_perm belong to expert `expert`.
-struct Group {
+// Its tiles of kGroupTileRows rows are numbered mt0, mt0 + 1, ... across all groups in order.
+struct __align__(16) Group {
     int row0;
     int m;
     int expert;
-    int pad;
+    int mt0;
 };
+static_assert(sizeof(Group) == 16, "Group is read as one 16-byte vector");
 
 // Device-side statistics of one forward, reduced in a fixed order.
 // Row-tile height of the tensor-core grouped GEMMs.  The compaction records, next to the

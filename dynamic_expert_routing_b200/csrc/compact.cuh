@@ -56,13 +56,30 @@ compact_bits_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__
     pdl_launch_dependents();
 }
 
+// tile_group[q] = the group that owns tile q (tiles of kGroupTileRows rows, numbered across
+// the groups in order), so that the grouped GEMMs find a tile's group with one 16-byte load.
+// Called by every warp of the block after the group table is written and the block has
+// synchronised.  The table was written by this block, so it is read through L2
+// (ld.global.cg), never through the non-coherent path.
+__device__ __forceinline__ void fill_tile_groups(const Group* groups, const int* n_groups,
+                                                 Group* __restrict__ tile_group, int warp, int lane,
+                                                 int nwarps)
+{
+    const int ng = __ldcg(n_groups);
+    for (int g = warp; g < ng; g += nwarps) {
+        const int4 G = __ldcg(reinterpret_cast<const int4*>(groups + g));  // row0, m, expert, mt0
+        const int mts = (G.y + kGroupTileRows - 1) / kGroupTileRows;
+        for (int q = lane; q < mts; q += 32) reinterpret_cast<int4*>(tile_group)[G.w + q] = G;
+    }
+}
+
 __global__ void __launch_bounds__(1024)
 compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                     const int* __restrict__ nkeep_tok, const float* __restrict__ lreg_tok,
                     int* __restrict__ counts, int* __restrict__ offsets,
                     int* __restrict__ chunk_base, Group* __restrict__ groups,
                     int* __restrict__ n_groups, DevStats* __restrict__ stats,
-                    int* __restrict__ tail_cnt, int n_tail_cnt)
+                    int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group)
 {
     __shared__ int s_counts[kMaxE];
     __shared__ long long s_keep[32];
@@ -112,7 +129,17 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
             int na = __shfl_up_sync(0xffffffffu, inca, o);
             if (lane >= o) { incl += n; inca += na; }
         }
-        int run = incl - sum, runa = inca - nact;
+        // tiles of kGroupTileRows rows: this lane's experts, then an exclusive scan over lanes
+        int mtl = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mtl += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
+        int inclm = mtl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, inclm, o);
+            if (lane >= o) inclm += n;
+        }
+        int run = incl - sum, runa = inca - nact, runm = inclm - mtl;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             int e = lane * 8 + j;
@@ -120,20 +147,17 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                 offsets[e] = run;
                 if (act[j]) {
                     Group g;
-                    g.row0 = run; g.m = loc[j]; g.expert = e; g.pad = 0;
+                    g.row0 = run; g.m = loc[j]; g.expert = e; g.mt0 = runm;
                     groups[runa] = g;
                     ++runa;
+                    runm += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
                 }
             }
             run += loc[j];
         }
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         const int tact = __shfl_sync(0xffffffffu, inca, 31);
-        int mt = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mt += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mt += __shfl_xor_sync(0xffffffffu, mt, o);
+        const int mt = __shfl_sync(0xffffffffu, inclm, 31);
         if (lane == 0) {
             offsets[E] = total;
             n_groups[0] = tact;
@@ -161,6 +185,7 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
     }
     if (lane == 0) { s_keep[warp] = ks; s_lreg[warp] = ls; s_zero[warp] = nz; }
     __syncthreads();
+    fill_tile_groups(groups, n_groups, tile_group, warp, lane, nwarps);
     if (warp == 0) {
         ks = lane < nwarps ? s_keep[lane] : 0;
         ls = lane < nwarps ? s_lreg[lane] : 0.0;
@@ -242,7 +267,7 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
                            int* __restrict__ n_groups, DevStats* __restrict__ stats,
                            int* __restrict__ perm, int* __restrict__ inv,
                            const TW* __restrict__ x, TW* __restrict__ xperm, int D, int gather,
-                           int* __restrict__ tail_cnt, int n_tail_cnt)
+                           int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group)
 {
     __shared__ int s_id[kSmallT][32];
     __shared__ uint8_t s_keep[kSmallT][32];
@@ -315,7 +340,17 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
             const int na = __shfl_up_sync(0xffffffffu, inca, o);
             if (lane >= o) { incl += n; inca += na; }
         }
-        int run = incl - sum, runa = inca - nact;
+        // tiles of kGroupTileRows rows: this lane's experts, then an exclusive scan over lanes
+        int mtl = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mtl += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
+        int inclm = mtl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, inclm, o);
+            if (lane >= o) inclm += n;
+        }
+        int run = incl - sum, runa = inca - nact, runm = inclm - mtl;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
@@ -324,20 +359,20 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
                 s_off[e] = run;
                 if (act[j]) {
                     Group g;
-                    g.row0 = run; g.m = loc[j]; g.expert = e; g.pad = 0;
+                    g.row0 = run; g.m = loc[j]; g.expert = e; g.mt0 = runm;
                     groups[runa] = g;
                     ++runa;
+                    // at most 32 tokens: a group has at most 8 tiles, written here directly
+                    const int mts = (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
+                    for (int q = 0; q < mts; ++q) tile_group[runm + q] = g;
+                    runm += mts;
                 }
             }
             run += loc[j];
         }
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         const int tact = __shfl_sync(0xffffffffu, inca, 31);
-        int mt = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mt += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mt += __shfl_xor_sync(0xffffffffu, mt, o);
+        const int mt = __shfl_sync(0xffffffffu, inclm, 31);
         long long ks = lane < T ? s_nk[lane] : 0;
         double ls = lane < T ? (double)s_lr[lane] : 0.0;
         int nz = (lane < T && s_nk[lane] == 0) ? 1 : 0;

@@ -80,7 +80,8 @@ struct TcParams {
     CUtensorMap b_shared;   // shared-expert weights
     CUtensorMap a_routed_tail;  // a_routed with a kSwapBox-row box (swapped small groups)
     const Group* groups;
-    const int* n_groups;    // [0]: groups, [1]: their m tiles (tiles of BM rows)
+    const int* n_groups;    // [0]: groups, [1]: their tiles of BM rows
+    const Group* tile_group;  // tile of BM rows (numbered across the groups) -> its group    // [0]: groups, [1]: their m tiles (tiles of BM rows)
     void* out_routed;       // EPI_SWIGLU: fp16 H [rows][F]; EPI_STORE_F32: f32 Y [rows][D]
     void* out_shared;
     int ld_routed;          // row length of out_routed
@@ -285,25 +286,25 @@ __device__ __forceinline__ void split_range(int ksteps, int splits, int ks, int&
 template <bool TAIL, bool SWAP>
 struct TileWalker {
     const TcParams* p;
-    int ng;
+    int total_mt;      // tiles of BM rows of the routed groups
     int count_sh;      // tiles of the shared problem
     int mts_sh;
     long long next;    // next unit index
     int whole_end;     // units below this are whole tiles
     int n_units;       // units of the launch
     int pieces;
-    int g;             // cursor: current group and the first tile index of it
-    long long g_base;
+    Group cg;          // the group of the last routed tile (most consecutive tiles share it)
+    int cg_mts;
 
     // n_tiles: tiles of the launch (needed only with a tail split, else ignored)
-    __device__ void init(const TcParams* p_, int ng_, long long n_tiles = 0) {
+    __device__ void init(const TcParams* p_, int total_mt_, long long n_tiles = 0) {
         p = p_;
-        ng = ng_;
+        total_mt = total_mt_;
         mts_sh = p->shared_rows > 0 ? (p->shared_rows + BM - 1) / BM : 0;
         count_sh = mts_sh * p->n_tiles_shared * p->k_splits_shared;
         next = blockIdx.x;
-        g = 0;
-        g_base = count_sh;
+        cg.mt0 = 0;
+        cg_mts = 0;
         pieces = 1;
         whole_end = n_units = 0x7fffffff;
         if (TAIL && p->tail_cnt != nullptr) {
@@ -352,29 +353,29 @@ struct TileWalker {
             split_range(p->k_steps_shared, p->k_splits_shared, t.ks, t.k0, t.k1);
             return true;
         }
-        while (g < ng) {
-            const Group G = p->groups[g];
-            const int mts = (G.m + BM - 1) / BM;
-            const long long cnt = (long long)mts * p->n_tiles_routed * p->k_splits_routed;
-            if (i < g_base + cnt) {
-                const long long r = i - g_base;
-                const int per_n = mts * p->k_splits_routed;
-                t.shared = 0;
-                t.n = (int)(r / per_n);
-                const int rr = (int)(r % per_n);
-                t.ks = rr / mts;
-                t.mt = rr % mts;
-                t.row0 = G.row0;
-                t.m = G.m;
-                t.brow = G.expert * p->b_rows_per_expert + t.n * BN;
-                t.swap = (SWAP && G.m <= 2 * kSwapBox) ? (G.m <= kSwapBox ? kSwapBox : 2 * kSwapBox) : 0;
-                split_range(p->k_steps_routed, p->k_splits_routed, t.ks, t.k0, t.k1);
-                return true;
-            }
-            g_base += cnt;
-            ++g;
+        // routed tiles: per group (n tile, K split, m tile), m fastest; a group's tiles start
+        // at mt0 * tiles_per_mt, so tile i belongs to the group of m-tile i / tiles_per_mt
+        const long long r = i - count_sh;
+        const long long per_mt = (long long)p->n_tiles_routed * p->k_splits_routed;
+        const long long q = r / per_mt;
+        if (q >= total_mt) return false;
+        if (q < cg.mt0 || q >= cg.mt0 + cg_mts) {
+            cg = p->tile_group[q];
+            cg_mts = (cg.m + BM - 1) / BM;
         }
-        return false;
+        const long long rl = r - (long long)cg.mt0 * per_mt;
+        const int per_n = cg_mts * p->k_splits_routed;
+        t.shared = 0;
+        t.n = (int)(rl / per_n);
+        const int rr = (int)(rl % per_n);
+        t.ks = rr / cg_mts;
+        t.mt = rr % cg_mts;
+        t.row0 = cg.row0;
+        t.m = cg.m;
+        t.brow = cg.expert * p->b_rows_per_expert + t.n * BN;
+        t.swap = (SWAP && cg.m <= 2 * kSwapBox) ? (cg.m <= kSwapBox ? kSwapBox : 2 * kSwapBox) : 0;
+        split_range(p->k_steps_routed, p->k_splits_routed, t.ks, t.k0, t.k1);
+        return true;
     }
 };
 
@@ -431,18 +432,18 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     const uint32_t tmem_base = *tmem_slot;
 
     pdl_wait();  // groups, counts and activations come from the previous kernels
-    const int ng = *p.n_groups;
+    const int total_mt = p.n_groups[1];
     // tiles of the launch (used by the tail split): n_groups[1] holds the groups' m tiles
     long long n_tiles = 0;
     if (TAIL && p.tail_cnt != nullptr) {
         const long long mts_sh = p.shared_rows > 0 ? (p.shared_rows + BM - 1) / BM : 0;
-        n_tiles = (long long)p.n_groups[1] * p.n_tiles_routed + mts_sh * p.n_tiles_shared;
+        n_tiles = (long long)total_mt * p.n_tiles_routed + mts_sh * p.n_tiles_shared;
     }
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer
         TileWalker<TAIL, SWAP> w;
-        w.init(&p, ng, n_tiles);
+        w.init(&p, total_mt, n_tiles);
         Tile t;
         int s = 0;
         uint32_t ph = 0;
@@ -485,7 +486,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
         TileWalker<TAIL, SWAP> w;
-        w.init(&p, ng, n_tiles);
+        w.init(&p, total_mt, n_tiles);
         Tile t;
         int s = 0, acc = 0;
         uint32_t ph = 0, aph = 0;
@@ -534,7 +535,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue (TMEM -> registers -> global)
         TileWalker<TAIL, SWAP> w;
-        w.init(&p, ng, n_tiles);
+        w.init(&p, total_mt, n_tiles);
         Tile t;
         int acc = 0;
         uint32_t aph = 0;
