@@ -179,12 +179,14 @@ def gpu_uuid(torch, dev):
 
 
 # ------------------------------------------------------------------ algorithmic work
-def layer_work(spec, T, st, tc_path=True):
+def layer_work(spec, T, st, tc_path=True, joint=False):
     """Algorithmic bytes and FLOPs of one forward (what the method must move / compute), per
     stage.  The intermediates are counted at the precision the path keeps them in: H in fp16
     for bf16 layers (fp32 for fp32 layers); expert output rows in fp16 on the tensor-core
     path, fp32 on the streaming path.  On the tensor-core path the shared experts are a
-    problem of their own (tc_shared_* stages); the streaming kernels do both in one launch."""
+    problem of their own (tc_shared_* stages) for larger batches; with joint=True (small
+    batches) they run inside the routed launches, whose stages then carry both problems, as
+    the streaming kernels always do."""
     D, E, K, F = spec.d_model, spec.n_experts, spec.top_k, spec.d_ff
     es = 4 if spec.storage == "fp32" else 2
     hs = 4 if spec.storage == "fp32" else 2
@@ -203,12 +205,12 @@ def layer_work(spec, T, st, tc_path=True):
     dn_s = dict(bytes=D * Fsh * es + Tsh * Fsh * hs + Tsh * D * ys, flops=2 * Tsh * Fsh * D)
     both = lambda a, b: {k: a[k] + b[k] for k in a}
     w["stream_gateup"], w["stream_down"] = both(gu_r, gu_s), both(dn_r, dn_s)
-    w["tc_gateup"], w["tc_down"] = gu_r, dn_r
+    w["tc_gateup"], w["tc_down"] = (both(gu_r, gu_s), both(dn_r, dn_s)) if joint else (gu_r, dn_r)
     w["tc_shared_gateup"], w["tc_shared_down"] = gu_s, dn_s
     w["combine"] = dict(bytes=nk * D * ys + Tsh * D * ys + T * D * 4 + T * K * 8,
                         flops=2 * nk * D)
     w["scatter_gather"] = dict(bytes=2 * nk * D * es + T * K * 12, flops=0)
-    w["swiglu_finish"] = dict(bytes=nk * F * hs, flops=0)
+    w["swiglu_finish"] = dict(bytes=(nk * F + (Tsh * Fsh if joint else 0)) * hs, flops=0)
     w["shared_swiglu_finish"] = dict(bytes=Tsh * Fsh * hs, flops=0)
     total_bytes = (na * 3 * F * D + 3 * Fsh * D + 2 * E * D) * es + T * D * es + T * D * 4
     total_flops = 2 * (nk * 3 * F * D + T * 3 * Fsh * D + Tr * D * 2 * E)
@@ -317,7 +319,9 @@ def _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off):
     for _ in range(steps):
         layer.forward(x, mask_off=mo, out=y)
     prof = layer.profile_end()
-    work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof)
+    work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof,
+                             joint=spec.n_shared > 0 and "tc_gateup" in prof
+                             and "tc_shared_gateup" not in prof)
     stage = max((k for k in prof if k != "forwards"), key=lambda k: prof[k][0])
     rl = roofline_for(stage, work.get(stage, dict(bytes=0, flops=0)),
                       prof[stage][0] / prof[stage][1], peaks, name)
@@ -394,7 +398,9 @@ def _run_ours(args):
     for _ in range(args.steps):
         layer.forward(x, mask_off=mask_off, out=y)
     prof = layer.profile_end()
-    work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof)
+    work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof,
+                             joint=spec.n_shared > 0 and "tc_gateup" in prof
+                             and "tc_shared_gateup" not in prof)
     stages = {k: v for k, v in prof.items() if k != "forwards"}
     tot_ms = sum(v[0] for v in stages.values())
     dom = max(stages, key=lambda k: stages[k][0])

@@ -644,61 +644,73 @@ struct YOut {
     bool f16 = false;
 };
 
-// GEMM1 (+ SwiGLU finish when split) and GEMM2 of one problem on the tensor cores: the routed
-// groups (shared = false) or the always-on shared group (shared = true), on stream `st`.
+// GEMM1 (+ SwiGLU finish when split) and GEMM2 on the tensor cores, on stream `st`, for the
+// routed groups (PROB_ROUTED), the always-on shared group (PROB_SHARED), or both in the same
+// launches (PROB_BOTH: the shared tiles first, then the routed ones; used for small batches,
+// where one set of launches costs less than two overlapping ones).
+enum { PROB_ROUTED = 1, PROB_SHARED = 2, PROB_BOTH = 3 };
+
 template <typename T>
-static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cudaStream_t st,
-                                YOut& out)
+static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cudaStream_t st,
+                                YOut& out_r, YOut& out_s)
 {
     const int D = h->D, F = h->F, Fsh = h->Fsh, K = h->K, E = h->E;
+    const bool routed = (which & PROB_ROUTED) != 0, shared = (which & PROB_SHARED) != 0;
     int s1 = 1, s2 = 1;
     if (T_ <= kSplitMaxTokens) {
-        // a small batch has few tiles: split K so they cover every SM
+        // a small batch has few tiles: split K so the launch covers every SM
         const long long mts = ceil_div(T_, tc::BM);
         const long long groups = std::min<long long>(E, std::max(1LL, ((long long)T_ * K + 1) / 2));
-        const long long t1 = shared ? mts * (2LL * Fsh / tc::BN) : mts * groups * (2LL * F / tc::BN);
-        const long long t2 = shared ? mts * ((long long)D / tc::BN) : mts * groups * (D / tc::BN);
+        const long long t1 = (routed ? mts * groups * (2LL * F / tc::BN) : 0) +
+                             (shared ? mts * (2LL * Fsh / tc::BN) : 0);
+        const long long t2 = (routed ? mts * groups * (D / tc::BN) : 0) +
+                             (shared ? mts * ((long long)D / tc::BN) : 0);
         s1 = choose_splits(h->num_sms, t1);
         s2 = choose_splits(h->num_sms, t2);
     }
-    s1 = normalise_splits(s1, D / tc::BK);
-    s2 = normalise_splits(s2, (shared ? Fsh : F) / tc::BK);
+    // per-problem split counts (gate/up: both K = D; down: K = F routed, Fsh shared)
+    const int s1n = normalise_splits(s1, D / tc::BK);
+    const int s2r = normalise_splits(s2, F / tc::BK);
+    const int s2s = shared ? normalise_splits(s2, Fsh / tc::BK) : 1;
+    const bool split1 = s1n > 1;
+    const bool split2 = (routed && s2r > 1) || (shared && s2s > 1);
     const int rows_sh = shared ? T_ : 0;
-    // the shared problem runs as launches of its own, timed under stages of its own
-    const int st_gu = shared ? ST_TC_SH_GATEUP : ST_TC_GATEUP;
-    const int st_dn = shared ? ST_TC_SH_DOWN : ST_TC_DOWN;
-    const int st_fin = shared ? ST_SH_SWIGLU_FINISH : ST_SWIGLU_FINISH;
-    const int* ngroups = shared ? h->zero_int : h->n_groups;
+    // a shared-only launch is timed under stages of its own
+    const bool sh_only = which == PROB_SHARED;
+    const int st_gu = sh_only ? ST_TC_SH_GATEUP : ST_TC_GATEUP;
+    const int st_dn = sh_only ? ST_TC_SH_DOWN : ST_TC_DOWN;
+    const int st_fin = sh_only ? ST_SH_SWIGLU_FINISH : ST_SWIGLU_FINISH;
+    const int* ngroups = routed ? h->n_groups : h->zero_int;
 
     // GEMM1: gate/up, SwiGLU in the epilogue, or f32 partials + the finishing kernel
-    tc::TcParams p = (s1 > 1) ? h->p1s : h->p1;
+    tc::TcParams p = split1 ? h->p1s : h->p1;
     if (shared)
         BEAM_TRY(encode_map(h, &p.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
                             (uint64_t)D, tc::BM));
     p.n_groups = ngroups;
     p.shared_rows = rows_sh;
-    p.k_splits_routed = p.k_splits_shared = s1;
-    // Kernel form of a routed whole-K launch.  Groups averaging at most 2 * kSwapBox rows
+    p.k_splits_routed = p.k_splits_shared = s1n;
+    // Kernel form of a whole-K launch.  Routed groups averaging at most 2 * kSwapBox rows
     // (T*K <= 64 E): the swap form, which runs groups of <= 64 rows with the weights as the M
-    // operand.  Otherwise, deep enough in K: the tail form, which may cut the tiles of the
-    // last, partial wave into K pieces (the cut is decided on the device).
+    // operand.  Otherwise, for the routed problem alone and deep enough in K: the tail form,
+    // which may cut the tiles of the last, partial wave into K pieces (decided on the device).
     const size_t creg = (size_t)h->num_sms * tc::kEpiWarps;
-    const bool small_groups = !shared && (long long)T_ * K <= 2LL * tc::kSwapBox * E;
-    const bool swap1 = small_groups && s1 == 1;
-    const bool swap2 = small_groups && s2 == 1;
-    const bool tail1 = !shared && !small_groups && s1 == 1 && D / tc::BK >= tc::kTailMinKSteps;
-    const bool tail2 = !shared && !small_groups && s2 == 1 && F / tc::BK >= tc::kTailMinKSteps;
+    const bool small_groups = routed && (long long)T_ * K <= 2LL * tc::kSwapBox * E;
+    const bool swap1 = small_groups && !split1;
+    const bool swap2 = small_groups && !split2;
+    const bool tail1 = which == PROB_ROUTED && !small_groups && !split1 && D / tc::BK >= tc::kTailMinKSteps;
+    const bool tail2 = which == PROB_ROUTED && !small_groups && !split2 && F / tc::BK >= tc::kTailMinKSteps;
     p.tail_cnt = tail1 ? h->tail_cnt : nullptr;
     p.tail_ws = tail1 ? h->tail_ws : nullptr;
-    if (s1 > 1) {
+    if (split1) {
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
-        const long long work = shared ? (long long)T_ * Fsh : (long long)T_ * K * F;
+        const long long work = (routed ? (long long)T_ * K * F : 0) + (shared ? (long long)T_ * Fsh : 0);
         BEAM_CUDA(launch(h, st_fin, tc::swiglu_finish_kernel,
                          dim3((unsigned)std::max<long long>(1, std::min<long long>(h->num_sms * 4, ceil_div(work, 256)))),
-                         dim3(256), 0, st, (const float*)h->g1part, s1, p.split_stride_routed,
-                         (const int*)(shared ? h->zero_int : h->offsets + E), F, (__half*)h->hbuf,
-                         (const float*)h->g1part_sh, s1, p.split_stride_shared, rows_sh, Fsh,
+                         dim3(256), 0, st, (const float*)h->g1part, s1n, p.split_stride_routed,
+                         (const int*)(routed ? h->offsets + E : h->zero_int), F, (__half*)h->hbuf,
+                         (const float*)h->g1part_sh, s1n, p.split_stride_shared, rows_sh, Fsh,
                          (__half*)h->hsh));
     } else if (swap1) {
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_SWAP>,
@@ -715,28 +727,25 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, bool shared, cu
     tc::TcParams q = h->p2;
     q.n_groups = ngroups;
     q.shared_rows = rows_sh;
-    q.k_splits_routed = q.k_splits_shared = s2;
+    q.k_splits_routed = s2r;
+    q.k_splits_shared = s2s;
     q.tail_cnt = tail2 ? h->tail_cnt + creg : nullptr;
     q.tail_ws = tail2 ? h->tail_ws : nullptr;
-    if (s2 > 1) {
+    if (split2) {
         q.out_routed = h->ypart;
         q.split_stride_routed = (long long)h->split_rows * K * D;
         q.out_shared = h->ysh_part;
         q.split_stride_shared = (long long)h->split_rows * D;
-        out.base = shared ? (const void*)h->ysh_part : (const void*)h->ypart;
-        out.splits = s2;
-        out.stride = shared ? q.split_stride_shared : q.split_stride_routed;
-        out.f16 = false;
+        if (routed) { out_r.base = h->ypart; out_r.splits = s2r; out_r.stride = q.split_stride_routed; out_r.f16 = false; }
+        if (shared) { out_s.base = h->ysh_part; out_s.splits = s2s; out_s.stride = q.split_stride_shared; out_s.f16 = false; }
         BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 0, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
     } else {
         q.out_routed = h->yperm;
         q.out_shared = h->ysh;
         q.split_stride_routed = q.split_stride_shared = 0;
-        out.base = shared ? (const void*)h->ysh : (const void*)h->yperm;
-        out.splits = 1;
-        out.stride = 0;
-        out.f16 = true;
+        if (routed) { out_r.base = h->yperm; out_r.splits = 1; out_r.stride = 0; out_r.f16 = true; }
+        if (shared) { out_s.base = h->ysh; out_s.splits = 1; out_s.stride = 0; out_s.f16 = true; }
         if (swap2)
             BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_SWAP>,
                              dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
@@ -771,15 +780,19 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     const int nch = ceil_div(T_, 32);
     const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
 
-    // 0. shared experts: they need only x, so on the tensor path they run on a side stream,
-    // concurrently with the router and the compaction, and join before the combine
+    // 0. shared experts: they need only x, so for larger batches on the tensor path they run on
+    // a side stream, concurrently with the router and the compaction, and join before the
+    // combine.  Small batches (split K) run them in the routed launches instead: their GEMMs
+    // are short, and two streams of them would only add launches that wait for each other.
     BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, sizeof(int), st));
     YOut ysh_out;
-    const bool fork = use_tc && h->Fsh > 0;
+    const bool fork = use_tc && h->Fsh > 0 && T_ > kSplitMaxTokens;
+    const bool joint = use_tc && h->Fsh > 0 && !fork;
     if (fork) {
+        YOut unused;
         BEAM_CUDA(cudaEventRecord(h->ev_fork, st));
         BEAM_CUDA(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-        BEAM_TRY(tc_problem(h, x, T_, true, h->side, ysh_out));
+        BEAM_TRY(tc_problem(h, x, T_, PROB_SHARED, h->side, unused, ysh_out));
         BEAM_CUDA(cudaEventRecord(h->ev_join, h->side));
     }
 
@@ -850,11 +863,11 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          (const uint32_t*)h->bits, (const int*)h->offsets,
                          (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     }
-    // 4. experts: kept groups only (the shared group is already running on the side stream)
+    // 4. experts: kept groups only (plus the shared group when it is not on the side stream)
     using TH = typename HType<T>::type;
     YOut yr;
     if (use_tc) {
-        BEAM_TRY(tc_problem(h, x, T_, false, st, yr));
+        BEAM_TRY(tc_problem(h, x, T_, joint ? PROB_BOTH : PROB_ROUTED, st, yr, ysh_out));
     } else {
         StreamArgs a;
         a.xperm = h->xperm; a.x = x; a.wgu = h->wgu; a.wsgu = h->wsgu; a.wd = h->wd; a.wsd = h->wsd;

@@ -38,6 +38,18 @@ def test_layer_work_splits_routed_and_shared_problems():
     assert w_tc["tc_shared_gateup"]["flops"] == 2 * T * 2 * Fsh * D
 
 
+def test_layer_work_joint_launches_carry_both_problems():
+    """Small batches run the shared experts inside the routed launches: those stages then carry
+    the work of both problems, like the streaming kernels."""
+    spec = synth.LayerSpec("w", 1024, 64, 6, 512, n_shared=2, d_ff_shared=256)
+    T = 16
+    sep, _ = bench.layer_work(spec, T, STATS, tc_path=True)
+    jnt, _ = bench.layer_work(spec, T, STATS, tc_path=True, joint=True)
+    for s in ("gateup", "down"):
+        assert jnt["tc_" + s] == _sum(sep["tc_" + s], sep["tc_shared_" + s])
+    assert jnt["swiglu_finish"]["bytes"] == sep["swiglu_finish"]["bytes"] + sep["shared_swiglu_finish"]["bytes"]
+
+
 def test_layer_work_without_shared_experts_has_empty_shared_problem():
     spec = synth.LayerSpec("w", 1024, 8, 2, 512)
     w, _ = bench.layer_work(spec, 64, STATS)

@@ -268,10 +268,10 @@ def test_large_max_tokens_small_forward():
 
 @pytest.mark.parametrize("T", [4, 300])
 def test_profiling_stages_count_every_launch(T):
-    """Per-stage timing: the shared experts' GEMMs are timed under stages of their own, each
-    tensor-core stage launches once per forward, and the launches per stage add up to the
-    handle's launch counter (so a roofline that divides a stage's time by its launches and
-    its work by one problem is consistent).  T = 4 takes the split-K variants, T = 300 not."""
+    """Per-stage timing: every stage launches once per forward and the launches per stage add
+    up to the handle's launch counter (so a roofline that divides a stage's time by its
+    launches is consistent).  T = 300 runs the shared experts on the second stream, timed
+    under stages of their own; T = 4 splits K and runs them inside the routed launches."""
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=256)
     w = synth.make_layer(spec, keep_rate=0.5)
@@ -288,13 +288,14 @@ def test_profiling_stages_count_every_launch(T):
     assert prof["forwards"] == n
     stages = {k: v for k, v in prof.items() if k != "forwards"}
     assert sum(c for _, c in stages.values()) == layer.launch_count() - n0
-    for s in ("tc_gateup", "tc_down", "tc_shared_gateup", "tc_shared_down"):
-        assert stages[s][1] == n, (s, stages[s])
-        assert stages[s][0] > 0
-    split = "swiglu_finish" in stages
-    assert split == (T <= 64)
-    if split:
-        assert stages["shared_swiglu_finish"][1] == n
+    split = T <= 64
+    expect = ["tc_gateup", "tc_down"] + (["swiglu_finish"] if split else ["tc_shared_gateup", "tc_shared_down"])
+    for s_ in expect:
+        assert stages[s_][1] == n, (s_, stages[s_])
+        assert stages[s_][0] > 0
+    absent = ["tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish"] if split else ["swiglu_finish"]
+    for s_ in absent:
+        assert s_ not in stages, (s_, stages)
     layer.close()
 
 
