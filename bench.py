@@ -335,6 +335,13 @@ def _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off):
                                       for k, v in prof.items() if k != "forwards"})
 
 
+def spread_sample(T: int, n: int):
+    """n token indices of a T-token batch spread evenly over it (all of them when n >= T)."""
+    import numpy as np
+    n = max(1, min(T, n))
+    return np.unique(np.linspace(0, T - 1, n).round().astype(np.int64))
+
+
 def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_steps=None):
     """Time the fp64 oracle on a bounded sample of the workload (tokens/s on host cores)."""
     import numpy as np
@@ -349,16 +356,14 @@ def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_ste
     oracle.layer(x[:1], w, r1)
     per_tok = max(time.perf_counter() - t0, 1e-4)
     threads = oracle.num_threads()
-    n = int(max(1, min(T, budget_s * threads / per_tok)))
-    stride = max(1, T // n)
-    sel = np.arange(0, T, stride, dtype=np.int32)[:n]
+    sel = spread_sample(T, int(budget_s * threads / per_tok))
     t0 = time.perf_counter()
     xs = x[torch.from_numpy(sel).long()]
     r = oracle.route(xs, w["w_router"], w["w_mask"], spec.top_k, mask_off=keep is None)
     oracle.layer(xs, w, r)
     dt = time.perf_counter() - t0
     return dict(value=round(len(sel) / dt, 4), unit="tokens/s", cores=threads, kind="oracle",
-                sample=f"{len(sel)} of {T} tokens (every {stride}th), routing + experts, fp64")
+                sample=f"{len(sel)} of {T} tokens spread evenly over the batch, routing + experts, fp64")
 
 
 def run_ours(args):
@@ -533,9 +538,7 @@ def run_reference(args):
     oracle.layer(x[:1], w, r1)
     per_tok = max(time.perf_counter() - t0, 1e-4) / threads
     budget = 150.0 / (args.steps + args.warmup)
-    n = int(max(1, min(T, budget / per_tok)))
-    stride = max(1, T // n)
-    sel = torch.from_numpy(np.arange(0, T, stride)[:n]).long()
+    sel = torch.from_numpy(spread_sample(T, int(budget / per_tok))).long()
     xs = x[sel]
 
     def step():
@@ -561,8 +564,8 @@ def run_reference(args):
                    "d_model": spec.d_model, "n_experts": spec.n_experts, "top_k": spec.top_k,
                    "d_ff": spec.d_ff, "tokens_per_gpu": T, "keep_rate": keep},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{len(sel)} of {T} tokens per step (every {stride}th), "
-                                   "routing + experts, fp64"},
+                         "sample": f"{len(sel)} of {T} tokens per step, spread evenly over the "
+                                   "batch, routing + experts, fp64"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -97,3 +97,11 @@ def test_record_traffic_reads_ncu_csv(tmp_path, monkeypatch):
     assert bench.recorded_traffic("tc_down", "mixtral-prefill") is None
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "changed")
     assert bench.recorded_traffic("tc_gateup", "mixtral-prefill") is None
+
+
+def test_spread_sample_covers_the_batch():
+    s = bench.spread_sample(4096, 2331)
+    assert len(s) == 2331 and s[0] == 0 and s[-1] == 4095
+    assert (s[1:] > s[:-1]).all()
+    assert list(bench.spread_sample(5, 100)) == [0, 1, 2, 3, 4]
+    assert list(bench.spread_sample(64, 1)) == [0]
