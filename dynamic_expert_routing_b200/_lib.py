@@ -22,8 +22,9 @@ BEAM_MASK_OFF = 0x1
 BEAM_PATH_STREAM = 0x2
 BEAM_PATH_TENSOR = 0x4
 BEAM_NO_GRAPH = 0x8
+BEAM_FUSED_DECODE = 0x10
 
-BEAM_N_STAGES = 15
+BEAM_N_STAGES = 16
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 STATUS_NAMES = {0: "BEAM_OK", 1: "BEAM_ERR_INVALID_ARG", 2: "BEAM_ERR_OOM", 3: "BEAM_ERR_CUDA",

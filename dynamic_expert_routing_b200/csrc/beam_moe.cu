@@ -25,6 +25,7 @@
 #include "compact.cuh"
 #include "stream_experts.cuh"
 #include "tc_experts.cuh"
+#include "decode_fused.cuh"
 
 using namespace beam;
 
@@ -139,6 +140,7 @@ struct beam_moe {
     float* y_stage = nullptr;
     size_t hsz;          // bytes per element of H and of the stored down projections
     bool tc_ok = false;  // tensor-core expert path available (bf16, D % 256 == 0)
+    bool fused_ok = false;  // fused decode launch available (tc_ok and cooperative launches)
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     tc::TcParams p0;      // router GEMM (one dense problem; its x map is set per forward)
     tc::TcParams p1, p2;  // GEMM1 / GEMM2 parameters (the x map of GEMM1 is set per forward)
@@ -180,13 +182,14 @@ struct beam_moe {
 enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
-    ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_COUNT
+    ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
-    "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish"};
+    "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish",
+    "fused_decode"};
 
 static void prof_release(beam_moe* h)
 {
@@ -480,6 +483,21 @@ static beam_status_t setup_tc(beam_moe* h)
         for (const void* k : kernels)
             BEAM_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
     }
+    // the fused decode kernel: one resident block per SM is required for its grid barriers
+    {
+        const void* fk[] = {(const void*)fused_decode_kernel<1>, (const void*)fused_decode_kernel<2>,
+                            (const void*)fused_decode_kernel<3>, (const void*)fused_decode_kernel<4>,
+                            (const void*)fused_decode_kernel<5>, (const void*)fused_decode_kernel<6>,
+                            (const void*)fused_decode_kernel<7>, (const void*)fused_decode_kernel<8>};
+        for (const void* k : fk)
+            BEAM_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+        int dev = 0, coop = 0, per_sm = 0;
+        BEAM_CUDA(cudaGetDevice(&dev));
+        BEAM_CUDA(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+        BEAM_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_decode_kernel<8>,
+                                                                tc::kThreads, tc::SMEM_BYTES));
+        h->fused_ok = coop != 0 && per_sm >= 1;
+    }
     h->tc_ok = true;
     return BEAM_OK;
 }
@@ -584,8 +602,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
 // Every forward kernel goes through here: it is counted, launched with programmatic stream
 // serialisation, and (while profiling) bracketed by an event pair of its stage.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3 grid,
-                          dim3 block, size_t smem, cudaStream_t st, Args&&... args)
+static cudaError_t launch_ex(beam_moe* h, int stage, bool coop, void (*kernel)(KArgs...), dim3 grid,
+                             dim3 block, size_t smem, cudaStream_t st, Args&&... args)
 {
     cudaEvent_t ea = nullptr, eb = nullptr;
     if (h->prof && h->prof_pool.size() >= 2) {
@@ -601,8 +619,14 @@ static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3
     lc.dynamicSmemBytes = smem;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (coop) {
+        // a cooperative launch: every block resident at once (the kernel has grid barriers)
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
     lc.attrs = attr;
     lc.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
@@ -611,6 +635,13 @@ static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3
         h->prof_recs.push_back({stage, ea, eb});
     }
     return e;
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3 grid,
+                          dim3 block, size_t smem, cudaStream_t st, Args&&... args)
+{
+    return launch_ex(h, stage, false, kernel, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 template <int EPL>
@@ -784,7 +815,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     // a side stream, concurrently with the router and the compaction, and join before the
     // combine.  Small batches (split K) run them in the routed launches instead: their GEMMs
     // are short, and two streams of them would only add launches that wait for each other.
-    BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, sizeof(int), st));
+    BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, 2 * sizeof(int), st));  // err, grid_bar
     YOut ysh_out;
     const bool fork = use_tc && h->Fsh > 0 && T_ > kSplitMaxTokens;
     const bool joint = use_tc && h->Fsh > 0 && !fork;
@@ -891,6 +922,88 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     else if (ysh_out.f16) ce = launch_combine<float, __half>(h, yr, ysh_out, T_, y, st);
     else ce = launch_combine<float, float>(h, yr, ysh_out, T_, y, st);
     BEAM_CUDA(ce);
+    return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- fused decode
+// Whether a forward runs as the single fused decode launch.
+static bool fused_eligible(const beam_moe* h, int T, uint32_t flags, bool use_tc)
+{
+    return h->fused_ok && use_tc && T >= 1 && T <= kSmallT && (flags & BEAM_FUSED_DECODE) &&
+           h->cfg.dtype == BEAM_DTYPE_BF16;
+}
+
+// The whole forward of a batch of 1..kSmallT tokens as one cooperative launch (see
+// decode_fused.cuh).  The split counts are the ones the separate launches would use, with the
+// shared experts in the same GEMMs; both GEMMs always store f32 partial slices.
+static beam_status_t forward_fused(beam_moe* h, const __nv_bfloat16* x, int T_, float* y,
+                                   uint32_t flags, cudaStream_t st)
+{
+    const int D = h->D, F = h->F, Fsh = h->Fsh, K = h->K, E = h->E, S = h->S;
+    const int Tr = ceil_div(T_, S);
+    BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, 2 * sizeof(int), st));  // err, grid_bar
+    const long long mts = ceil_div(T_, tc::BM);
+    const long long groups = std::min<long long>(E, std::max(1LL, ((long long)T_ * K + 1) / 2));
+    const long long t1 = mts * groups * (2LL * F / tc::BN) + (Fsh ? mts * (2LL * Fsh / tc::BN) : 0);
+    const long long t2 = mts * groups * (D / tc::BN) + (Fsh ? mts * ((long long)D / tc::BN) : 0);
+    const int s1 = normalise_splits(choose_splits(h->num_sms, t1), D / tc::BK);
+    const int s2c = choose_splits(h->num_sms, t2);
+    const int s2r = normalise_splits(s2c, F / tc::BK);
+    const int s2s = Fsh ? normalise_splits(s2c, Fsh / tc::BK) : 1;
+
+    FusedDecodeParams P;
+    memset(&P, 0, sizeof P);
+    P.g1 = h->p1s;
+    if (Fsh)
+        BEAM_TRY(encode_map(h, &P.g1.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)T_,
+                            (uint64_t)D, tc::BM));
+    P.g1.n_groups = h->n_groups;
+    P.g1.shared_rows = Fsh ? T_ : 0;
+    P.g1.k_splits_routed = P.g1.k_splits_shared = s1;
+    P.g1.tail_cnt = nullptr;
+    P.g1.tail_ws = nullptr;
+    P.g2 = h->p2;
+    P.g2.n_groups = h->n_groups;
+    P.g2.shared_rows = Fsh ? T_ : 0;
+    P.g2.k_splits_routed = s2r;
+    P.g2.k_splits_shared = s2s;
+    P.g2.tail_cnt = nullptr;
+    P.g2.tail_ws = nullptr;
+    P.g2.out_routed = h->ypart;
+    P.g2.split_stride_routed = (long long)h->split_rows * K * D;
+    P.g2.out_shared = h->ysh_part;
+    P.g2.split_stride_shared = (long long)h->split_rows * D;
+    P.x = x;
+    P.wrm = static_cast<const __nv_bfloat16*>(h->wrm);
+    P.L = h->L;
+    P.lchunk = 256 * ceil_div(D, 256 * kMaxSplits);   // at most kMaxSplits slices of D
+    P.lchunks = ceil_div(D, P.lchunk);
+    P.T = T_; P.Tr = Tr; P.seg = S; P.D = D; P.E = E; P.K = K; P.n2E = h->n2E;
+    P.mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
+    P.topk_id = h->topk_id; P.gate = h->gate; P.mlogit = h->mlogit; P.keep = h->keep;
+    P.ghat = h->ghat; P.nkeep_tok = h->nkeep_tok; P.lreg_tok = h->lreg_tok;
+    P.counts = h->counts; P.offsets = h->offsets; P.groups = h->groups; P.n_groups = h->n_groups;
+    P.stats = h->dstats; P.perm = h->perm; P.inv = h->inv; P.tile_group = h->tile_group;
+    P.xperm = static_cast<__nv_bfloat16*>(h->xperm);
+    P.F = F; P.Fsh = Fsh;
+    P.h = static_cast<__half*>(h->hbuf); P.hsh = static_cast<__half*>(h->hsh);
+    P.y = y;
+    P.grid_bar = &h->dstats->grid_bar;
+    P.err = &h->dstats->err;
+    const dim3 grid(h->num_sms), block(tc::kThreads);
+    const size_t smem = tc::SMEM_BYTES;
+    cudaError_t e;
+    switch ((E + 31) / 32) {
+        case 1: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<1>, grid, block, smem, st, P); break;
+        case 2: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<2>, grid, block, smem, st, P); break;
+        case 3: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<3>, grid, block, smem, st, P); break;
+        case 4: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<4>, grid, block, smem, st, P); break;
+        case 5: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<5>, grid, block, smem, st, P); break;
+        case 6: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<6>, grid, block, smem, st, P); break;
+        case 7: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<7>, grid, block, smem, st, P); break;
+        default: e = launch_ex(h, ST_FUSED_DECODE, true, fused_decode_kernel<8>, grid, block, smem, st, P); break;
+    }
+    BEAM_CUDA(e);
     return BEAM_OK;
 }
 
@@ -1032,7 +1145,7 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
     if (T > 0 && (!x || !y)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
         return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
-    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH))
+    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_FUSED_DECODE))
         return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
     if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
         return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core expert path needs a bf16 layer with "
@@ -1046,7 +1159,10 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
     if (h->prof) ++h->prof_forwards;
-    if (T > 0) {
+    if (T > 0 && fused_eligible(h, T, flags, use_tc)) {
+        // one launch: nothing to gain from a graph
+        BEAM_TRY(forward_fused(h, static_cast<const __nv_bfloat16*>(x), T, y, flags, st));
+    } else if (T > 0) {
         // Replay: the whole forward (8-10 kernels, their tensor maps and split choices) was
         // captured as a CUDA graph for these exact arguments; one launch replays it.  Not
         // used while profiling, on the legacy default stream, or with BEAM_NO_GRAPH.

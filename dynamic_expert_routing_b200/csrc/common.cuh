@@ -34,7 +34,7 @@ struct DevStats {
     int n_kept;           // kept (token, slot) pairs
     int tokens;
     int err;              // nonzero when a bounded wait ran out
-    int pad;
+    unsigned grid_bar;    // arrivals at the fused decode kernel's grid barriers (zeroed with err)
 };
 
 // ---------------------------------------------------------------- storage-type helpers

@@ -255,69 +255,76 @@ compact_scatter_gather_kernel(const int* __restrict__ topk_id, const uint8_t* __
 // The results are bit-identical to the multi-kernel path.
 constexpr int kSmallT = 32;
 
-template <int EPL, typename TW>
-__global__ void __launch_bounds__(1024)
-route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, long long split_stride,
-                           int Tr, int T, int E, int K, int seg, int mask_off,
-                           int* __restrict__ topk_id, float* __restrict__ gate,
-                           float* __restrict__ mlogit, uint8_t* __restrict__ keep,
-                           float* __restrict__ ghat, int* __restrict__ nkeep_tok,
-                           float* __restrict__ lreg_tok, int* __restrict__ counts,
-                           int* __restrict__ offsets, Group* __restrict__ groups,
-                           int* __restrict__ n_groups, DevStats* __restrict__ stats,
-                           int* __restrict__ perm, int* __restrict__ inv,
-                           const TW* __restrict__ x, TW* __restrict__ xperm, int D, int gather,
-                           int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group)
+// Working set of the small-batch routing (one block): at most kSmallT routed tokens.
+struct SmallScratch {
+    int id[kSmallT][32];
+    uint8_t keep[kSmallT][32];
+    uint32_t mask[kSmallT][kMaxE / 32 + 1];  // kept experts of each token (padded row)
+    int nk[kSmallT];
+    float lr[kSmallT];
+    uint32_t word[kMaxE];
+    int cnt[kMaxE];
+    int off[kMaxE + 1];
+    int perm[kSmallT * 32];
+};
+
+// The small-batch routing of one block, steps 1-4 above, on any number of warps.  Only a block
+// with `outputs` set writes the results to global memory (the fused decode kernel runs this in
+// every block and lets one of them publish); every block keeps offsets and perm in `sc`.
+template <int EPL>
+__device__ __forceinline__ void route_compact_small_body(
+    SmallScratch& sc, bool outputs, const float* __restrict__ L, int ldL, int splits,
+    long long split_stride, int Tr, int T, int E, int K, int seg, int mask_off,
+    int* __restrict__ topk_id, float* __restrict__ gate, float* __restrict__ mlogit,
+    uint8_t* __restrict__ keep, float* __restrict__ ghat, int* __restrict__ nkeep_tok,
+    float* __restrict__ lreg_tok, int* __restrict__ counts, int* __restrict__ offsets,
+    Group* __restrict__ groups, int* __restrict__ n_groups, DevStats* __restrict__ stats,
+    int* __restrict__ perm, int* __restrict__ inv, Group* __restrict__ tile_group)
 {
-    __shared__ int s_id[kSmallT][32];
-    __shared__ uint8_t s_keep[kSmallT][32];
-    __shared__ uint32_t s_mask[kSmallT][kMaxE / 32 + 1];  // kept experts of each token (padded row)
-    __shared__ int s_nk[kSmallT];
-    __shared__ float s_lr[kSmallT];
-    __shared__ uint32_t s_word[kMaxE];
-    __shared__ int s_cnt[kMaxE];
-    __shared__ int s_off[kMaxE + 1];
-    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
     for (int i = threadIdx.x; i < kSmallT * (kMaxE / 32 + 1); i += blockDim.x)
-        (&s_mask[0][0])[i] = 0u;
-    // the arrival counters of the grouped GEMMs' tail split start every forward at zero
-    for (int i = threadIdx.x; i < n_tail_cnt; i += blockDim.x) tail_cnt[i] = 0;
+        (&sc.mask[0][0])[i] = 0u;
     __syncthreads();
 
     // 1. selection
-    if (warp < Tr) {
-        const RowDecision d = select_row<EPL>(L + (size_t)warp * ldL, splits, split_stride, E, K,
+    for (int r = warp; r < Tr; r += nwarps) {
+        const RowDecision d = select_row<EPL>(L + (size_t)r * ldL, splits, split_stride, E, K,
                                               mask_off, lane);
         const int S = seg > 1 ? seg : 1;
-        const int t0 = warp * S, t1 = min(T, t0 + S);
+        const int t0 = r * S, t1 = min(T, t0 + S);
         for (int t = t0; t < t1; ++t) {
             if (lane < K) {
-                const size_t o = (size_t)t * K + lane;
-                topk_id[o] = d.id;
-                gate[o] = d.g;
-                mlogit[o] = d.l;
-                keep[o] = d.keep ? 1 : 0;
-                ghat[o] = d.ghat;
-                s_id[t][lane] = d.id;
-                s_keep[t][lane] = d.keep ? 1 : 0;
-                if (d.keep) atomicOr(&s_mask[t][d.id >> 5], 1u << (d.id & 31));  // order-free OR
+                if (outputs) {
+                    const size_t o = (size_t)t * K + lane;
+                    topk_id[o] = d.id;
+                    gate[o] = d.g;
+                    mlogit[o] = d.l;
+                    keep[o] = d.keep ? 1 : 0;
+                    ghat[o] = d.ghat;
+                }
+                sc.id[t][lane] = d.id;
+                sc.keep[t][lane] = d.keep ? 1 : 0;
+                if (d.keep) atomicOr(&sc.mask[t][d.id >> 5], 1u << (d.id & 31));  // order-free OR
             }
             if (lane == 0) {
-                nkeep_tok[t] = d.nkeep;
-                lreg_tok[t] = d.lreg;
-                s_nk[t] = d.nkeep;
-                s_lr[t] = d.lreg;
+                if (outputs) { nkeep_tok[t] = d.nkeep; lreg_tok[t] = d.lreg; }
+                sc.nk[t] = d.nkeep;
+                sc.lr[t] = d.lreg;
             }
         }
     }
     __syncthreads();
 
     // 2. one ballot word per expert (lane = token)
-    for (int e = warp; e < E; e += 32) {
-        const bool has = lane < T && ((s_mask[lane][e >> 5] >> (e & 31)) & 1u);
+    for (int e = warp; e < E; e += nwarps) {
+        const bool has = lane < T && ((sc.mask[lane][e >> 5] >> (e & 31)) & 1u);
         const uint32_t word = __ballot_sync(0xffffffffu, has);
-        if (lane == 0) { s_word[e] = word; s_cnt[e] = __popc(word); counts[e] = __popc(word); }
+        if (lane == 0) {
+            sc.word[e] = word;
+            sc.cnt[e] = __popc(word);
+            if (outputs) counts[e] = __popc(word);
+        }
     }
     __syncthreads();
 
@@ -328,7 +335,7 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
-            loc[j] = (e < E) ? s_cnt[e] : 0;
+            loc[j] = (e < E) ? sc.cnt[e] : 0;
             act[j] = loc[j] > 0;
             sum += loc[j];
             nact += act[j];
@@ -355,16 +362,18 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
             if (e < E) {
-                offsets[e] = run;
-                s_off[e] = run;
+                sc.off[e] = run;
+                if (outputs) offsets[e] = run;
                 if (act[j]) {
-                    Group g;
-                    g.row0 = run; g.m = loc[j]; g.expert = e; g.mt0 = runm;
-                    groups[runa] = g;
-                    ++runa;
-                    // at most 32 tokens: a group has at most 8 tiles, written here directly
                     const int mts = (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
-                    for (int q = 0; q < mts; ++q) tile_group[runm + q] = g;
+                    if (outputs) {
+                        Group g;
+                        g.row0 = run; g.m = loc[j]; g.expert = e; g.mt0 = runm;
+                        groups[runa] = g;
+                        // at most 32 tokens: a group has at most 8 tiles, written here directly
+                        for (int q = 0; q < mts; ++q) tile_group[runm + q] = g;
+                    }
+                    ++runa;
                     runm += mts;
                 }
             }
@@ -373,9 +382,9 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
         const int total = __shfl_sync(0xffffffffu, incl, 31);
         const int tact = __shfl_sync(0xffffffffu, inca, 31);
         const int mt = __shfl_sync(0xffffffffu, inclm, 31);
-        long long ks = lane < T ? s_nk[lane] : 0;
-        double ls = lane < T ? (double)s_lr[lane] : 0.0;
-        int nz = (lane < T && s_nk[lane] == 0) ? 1 : 0;
+        long long ks = lane < T ? sc.nk[lane] : 0;
+        double ls = lane < T ? (double)sc.lr[lane] : 0.0;
+        int nz = (lane < T && sc.nk[lane] == 0) ? 1 : 0;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             ks += __shfl_xor_sync(0xffffffffu, ks, o);
@@ -383,16 +392,18 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
             nz += __shfl_xor_sync(0xffffffffu, nz, o);
         }
         if (lane == 0) {
-            offsets[E] = total;
-            s_off[E] = total;
-            n_groups[0] = tact;
-            n_groups[1] = mt;
-            stats->n_kept = total;
-            stats->n_active = tact;
-            stats->keep_sum = ks;
-            stats->lreg_sum = ls;
-            stats->n_all_masked = nz;
-            stats->tokens = T;
+            sc.off[E] = total;
+            if (outputs) {
+                offsets[E] = total;
+                n_groups[0] = tact;
+                n_groups[1] = mt;
+                stats->n_kept = total;
+                stats->n_active = tact;
+                stats->keep_sum = ks;
+                stats->lreg_sum = ls;
+                stats->n_all_masked = nz;
+                stats->tokens = T;
+            }
         }
     }
     __syncthreads();
@@ -401,24 +412,56 @@ route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, lon
     for (int i = threadIdx.x; i < T * K; i += blockDim.x) {
         const int t = i / K, k = i - t * K;
         int pos = -1;
-        if (s_keep[t][k]) {
-            const int e = s_id[t][k];
-            pos = s_off[e] + __popc(s_word[e] & ((1u << t) - 1u));
-            perm[pos] = i;
+        if (sc.keep[t][k]) {
+            const int e = sc.id[t][k];
+            pos = sc.off[e] + __popc(sc.word[e] & ((1u << t) - 1u));
+            sc.perm[pos] = i;
+            if (outputs) perm[pos] = i;
         }
-        inv[i] = pos;
+        if (outputs) inv[i] = pos;
     }
-    if (gather) {
-        __syncthreads();
-        const int nk = s_off[E];
-        const int nv = D * (int)sizeof(TW) / 16;
-        for (int pos = warp; pos < nk; pos += 32) {
-            const int t = perm[pos] / K;
-            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
-            uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
-            for (int v = lane; v < nv; v += 32) dst[v] = src[v];
-        }
+    __syncthreads();
+}
+
+// X_perm[pos] = x[perm[pos] / K] for the kept pairs pos = w, w + nw, ... (warp w of nw).
+template <typename TW>
+__device__ __forceinline__ void gather_small_rows(const SmallScratch& sc, int E, int K, int D,
+                                                  const TW* __restrict__ x, TW* __restrict__ xperm,
+                                                  int w, int nw)
+{
+    const int lane = threadIdx.x & 31;
+    const int nk = sc.off[E];
+    const int nv = D * (int)sizeof(TW) / 16;
+    for (int pos = w; pos < nk; pos += nw) {
+        const int t = sc.perm[pos] / K;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
+        uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
+        for (int v = lane; v < nv; v += 32) dst[v] = src[v];
     }
+}
+
+template <int EPL, typename TW>
+__global__ void __launch_bounds__(1024)
+route_compact_small_kernel(const float* __restrict__ L, int ldL, int splits, long long split_stride,
+                           int Tr, int T, int E, int K, int seg, int mask_off,
+                           int* __restrict__ topk_id, float* __restrict__ gate,
+                           float* __restrict__ mlogit, uint8_t* __restrict__ keep,
+                           float* __restrict__ ghat, int* __restrict__ nkeep_tok,
+                           float* __restrict__ lreg_tok, int* __restrict__ counts,
+                           int* __restrict__ offsets, Group* __restrict__ groups,
+                           int* __restrict__ n_groups, DevStats* __restrict__ stats,
+                           int* __restrict__ perm, int* __restrict__ inv,
+                           const TW* __restrict__ x, TW* __restrict__ xperm, int D, int gather,
+                           int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group)
+{
+    __shared__ SmallScratch sc;
+    pdl_wait();
+    // the arrival counters of the grouped GEMMs' tail split start every forward at zero
+    for (int i = threadIdx.x; i < n_tail_cnt; i += blockDim.x) tail_cnt[i] = 0;
+    route_compact_small_body<EPL>(sc, true, L, ldL, splits, split_stride, Tr, T, E, K, seg,
+                                  mask_off, topk_id, gate, mlogit, keep, ghat, nkeep_tok, lreg_tok,
+                                  counts, offsets, groups, n_groups, stats, perm, inv, tile_group);
+    if (gather) gather_small_rows(sc, E, K, D, x, xperm, threadIdx.x >> 5, blockDim.x >> 5);
     pdl_launch_dependents();
 }
 

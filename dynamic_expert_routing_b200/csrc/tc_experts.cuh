@@ -385,53 +385,103 @@ struct TileWalker {
 // MODE_PLAIN has neither path compiled in.
 enum Mode { MODE_PLAIN = 0, MODE_TAIL = 1, MODE_SWAP = 2 };
 
-template <int EPI, int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
-tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
-{
-    constexpr bool TAIL = MODE == MODE_TAIL;
-    constexpr bool SWAP = MODE == MODE_SWAP && EPI != EPI_STORE_F32;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* gbase = smem_raw + (base - raw);
-    // layout: [stage s: A (16 KB) | B (32 KB)] x STAGES, epilogue buffers, then the barriers
-    float* epi_buf = reinterpret_cast<float*>(gbase + STAGES * STAGE_BYTES);
-    const uint32_t bar0 = base + STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
-    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
-    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES +
-                                                      8 * (2 * STAGES + 5));
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+// Shared-memory layout of one CTA: [stage s: A (16 KB) | B (32 KB)] x STAGES, the epilogue
+// staging buffers, then the mbarriers, the TMEM address slot and the abort flag.
+struct GemmSmem {
+    uint32_t base;              // shared-window address of the (1024-aligned) stage ring
+    uint8_t* gbase;             // the same, generic
+    float* epi_buf;
+    uint32_t bar0;
+    uint32_t* tmem_slot;
+    volatile int* abort_flag;
+    __device__ uint32_t full_bar(int s) const { return bar0 + 8u * s; }
+    __device__ uint32_t empty_bar(int s) const { return bar0 + 8u * (STAGES + s); }
+    __device__ uint32_t tfull_bar(int a) const { return bar0 + 8u * (2 * STAGES + a); }
+    __device__ uint32_t tempty_bar(int a) const { return bar0 + 8u * (2 * STAGES + 2 + a); }
+    __device__ uint32_t drain_bar() const { return bar0 + 8u * (2 * STAGES + 4); }
+};
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ GemmSmem gemm_smem(uint8_t* smem_raw)
+{
+    GemmSmem m;
+    const uint32_t raw = smem_u32(smem_raw);
+    m.base = (raw + 1023u) & ~1023u;
+    m.gbase = smem_raw + (m.base - raw);
+    m.epi_buf = reinterpret_cast<float*>(m.gbase + STAGES * STAGE_BYTES);
+    m.bar0 = m.base + STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES;
+    m.tmem_slot = reinterpret_cast<uint32_t*>(m.gbase + STAGES * STAGE_BYTES + kEpiWarps * EPI_WARP_BYTES +
+                                              8 * (2 * STAGES + 5));
+    m.abort_flag = reinterpret_cast<volatile int*>(m.tmem_slot + 1);
+    return m;
+}
+
+// Barrier init and TMEM allocation (warp 1), then a block barrier; returns the TMEM base.
+__device__ __forceinline__ uint32_t gemm_setup(const GemmSmem& sm)
+{
+    const int warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), kEpiWarps); }
-        mbar_init(drain_bar, 1);
-        *abort_flag = 0;
+        for (int s = 0; s < STAGES; ++s) { mbar_init(sm.full_bar(s), 1); mbar_init(sm.empty_bar(s), 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(sm.tfull_bar(a), 1); mbar_init(sm.tempty_bar(a), kEpiWarps); }
+        mbar_init(sm.drain_bar(), 1);
+        *sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&p.a_routed); tma_prefetch_desc(&p.b_routed);
-        tma_prefetch_desc(&p.a_shared); tma_prefetch_desc(&p.b_shared);
-        if (SWAP) tma_prefetch_desc(&p.a_routed_tail);
-    }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+                     ::"r"(smem_u32(sm.tmem_slot)), "r"(TMEM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    return *sm.tmem_slot;
+}
 
-    pdl_wait();  // groups, counts and activations come from the previous kernels
+// After the last GEMM phase: a block barrier, the error word on an abort, TMEM freed.
+__device__ __forceinline__ void gemm_teardown(const GemmSmem& sm, uint32_t tmem_base, int* err)
+{
+    const int warp = threadIdx.x >> 5;
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *sm.abort_flag) atomicOr(err, ERR_TC_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// Pipeline position of the thread playing a role (producer: stage s / phase ph; MMA issuer:
+// stage, phase, accumulator acc / aph; epilogue: acc / aph).  It carries over from one GEMM
+// phase of a launch to the next, as the mbarriers do.
+struct RoleState {
+    int s = 0, acc = 0;
+    uint32_t ph = 0, aph = 0;
+    bool ok = true, issued = false;
+    int pend_ph[STAGES] = {0, 0, 0, 0};
+    bool pend[STAGES] = {false, false, false, false};
+};
+
+// One GEMM phase over the tile list of `p`: warp 0 lane 0 issues TMA, warp 1 lane 0 issues
+// MMAs, warps 2.. run the epilogue.  Returns with every tile of this CTA stored (or with
+// rs.ok = false and the abort flag raised after a wait ran out, its copies and MMAs drained).
+template <int EPI, int FMT, int MODE>
+__device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm,
+                                           uint32_t tmem_base, RoleState& rs)
+{
+    constexpr bool TAIL = MODE == MODE_TAIL;
+    constexpr bool SWAP = MODE == MODE_SWAP && EPI != EPI_STORE_F32;
+    const uint32_t base = sm.base;
+    float* epi_buf = sm.epi_buf;
+    volatile int* abort_flag = sm.abort_flag;
+    auto full_bar = [&](int s) { return sm.full_bar(s); };
+    auto empty_bar = [&](int s) { return sm.empty_bar(s); };
+    auto tfull_bar = [&](int a) { return sm.tfull_bar(a); };
+    auto tempty_bar = [&](int a) { return sm.tempty_bar(a); };
+    const uint32_t drain_bar = sm.drain_bar();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_mt = p.n_groups[1];
     // tiles of the launch (used by the tail split): n_groups[1] holds the groups' m tiles
     long long n_tiles = 0;
@@ -445,12 +495,11 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
         TileWalker<TAIL, SWAP> w;
         w.init(&p, total_mt, n_tiles);
         Tile t;
-        int s = 0;
-        uint32_t ph = 0;
-        int pend_ph[STAGES];
-        bool pend[STAGES];
-        for (int i = 0; i < STAGES; ++i) { pend[i] = false; pend_ph[i] = 0; }
-        bool ok = true;
+        int s = rs.s;
+        uint32_t ph = rs.ph;
+        bool ok = rs.ok;
+        int* pend_ph = rs.pend_ph;
+        bool* pend = rs.pend;
         while (ok && w.get(t)) {
             const CUtensorMap* am = t.shared ? &p.a_shared : &p.a_routed;
             const CUtensorMap* bm = t.shared ? &p.b_shared : &p.b_routed;
@@ -474,7 +523,7 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                 if (++s == STAGES) { s = 0; ph ^= 1u; }
             }
         }
-        if (!ok) {
+        if (!ok && rs.ok) {
             // drain: let every copy this thread issued land before the CTA can exit
             for (int i = 0; i < STAGES; ++i) {
                 if (!pend[i]) continue;
@@ -483,14 +532,15 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                        globaltimer() - t0 < kWaitLimitNs) {}
             }
         }
+        rs.s = s; rs.ph = ph; rs.ok = ok;
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
         TileWalker<TAIL, SWAP> w;
         w.init(&p, total_mt, n_tiles);
         Tile t;
-        int s = 0, acc = 0;
-        uint32_t ph = 0, aph = 0;
-        bool ok = true, issued = false;
+        int s = rs.s, acc = rs.acc;
+        uint32_t ph = rs.ph, aph = rs.aph;
+        bool ok = rs.ok, issued = rs.issued;
         constexpr uint32_t idesc = make_idesc(FMT);
         while (ok && w.get(t)) {
             if (!mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) { ok = false; break; }
@@ -527,18 +577,20 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             tc_commit(tfull_bar(acc));
             if (++acc == 2) { acc = 0; aph ^= 1u; }
         }
-        if (!ok && issued) {
+        if (!ok && rs.ok && issued) {
             tc_commit(drain_bar);  // completes when every MMA issued so far has finished
             const unsigned long long t0 = globaltimer();
             while (!mbar_try_wait(drain_bar, 0) && globaltimer() - t0 < kWaitLimitNs) {}
         }
+        rs.s = s; rs.ph = ph; rs.acc = acc; rs.aph = aph; rs.ok = ok; rs.issued = issued;
     } else if (warp >= 2) {
         // ------------------------------------------------ epilogue (TMEM -> registers -> global)
         TileWalker<TAIL, SWAP> w;
         w.init(&p, total_mt, n_tiles);
         Tile t;
-        int acc = 0;
-        uint32_t aph = 0;
+        int acc = rs.acc;
+        uint32_t aph = rs.aph;
+        bool ok = rs.ok;
         const int lb = 32 * (warp & 3);  // TMEM lanes this warp may access
         const int warp_e = warp - 2;     // index of this epilogue warp (its staging buffer)
         const int half = warp_e / 4;     // which half of the tile's columns this warp drains
@@ -549,8 +601,8 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
             return EPI == EPI_SWIGLU ? (c & 1) * (BN / 2) + 32 * (half * 2 + (c >> 1))
                                      : 32 * (half * 4 + c);
         };
-        while (w.get(t)) {
-            if (!mbar_wait(tfull_bar(acc), aph, abort_flag)) break;
+        while (ok && w.get(t)) {
+            if (!mbar_wait(tfull_bar(acc), aph, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)lb << 16) + (uint32_t)(acc * BN);
             // rows lb .. lb+31 of the tile belong to this warp; row_ok(i) = row i of them is
@@ -706,17 +758,28 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
                 if (++acc == 2) { acc = 0; aph ^= 1u; }
             }
         }
+        rs.acc = acc; rs.aph = aph; rs.ok = ok;
     }
 
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) atomicOr(p.err, ERR_TC_TIMEOUT);
-    if (warp == 1) {
-        __syncwarp();
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                     ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+}
+
+template <int EPI, int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
+{
+    constexpr bool SWAP = MODE == MODE_SWAP && EPI != EPI_STORE_F32;
+    extern __shared__ uint8_t smem_raw[];
+    const GemmSmem sm = gemm_smem(smem_raw);
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&p.a_routed); tma_prefetch_desc(&p.b_routed);
+        tma_prefetch_desc(&p.a_shared); tma_prefetch_desc(&p.b_shared);
+        if (SWAP) tma_prefetch_desc(&p.a_routed_tail);
     }
+    const uint32_t tmem_base = gemm_setup(sm);
+    pdl_wait();  // groups, counts and activations come from the previous kernels
+    RoleState rs;
+    gemm_roles<EPI, FMT, MODE>(p, sm, tmem_base, rs);
+    gemm_teardown(sm, tmem_base, p.err);
     pdl_launch_dependents();
 }
 

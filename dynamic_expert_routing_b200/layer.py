@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import (BEAM_DTYPE_BF16, BEAM_DTYPE_F32, BEAM_MASK_OFF, BEAM_NO_GRAPH,
+from ._lib import (BEAM_DTYPE_BF16, BEAM_DTYPE_F32, BEAM_MASK_OFF, BEAM_FUSED_DECODE, BEAM_NO_GRAPH,
                    BEAM_PATH_STREAM, BEAM_PATH_TENSOR, BeamConfig, BeamStats, BeamWeights, check)
 
 _DTYPES = {torch.float32: BEAM_DTYPE_F32, torch.bfloat16: BEAM_DTYPE_BF16}
@@ -64,20 +64,24 @@ class BeamMoE:
 
     # -------------------------------------------------------------- forward
     @staticmethod
-    def flags(mask_off: bool = False, path: str | None = None, graph: bool = True) -> int:
-        return (BEAM_MASK_OFF if mask_off else 0) | _PATHS[path] | (0 if graph else BEAM_NO_GRAPH)
+    def flags(mask_off: bool = False, path: str | None = None, graph: bool = True,
+              fused: bool = False) -> int:
+        return ((BEAM_MASK_OFF if mask_off else 0) | _PATHS[path] | (0 if graph else BEAM_NO_GRAPH)
+                | (BEAM_FUSED_DECODE if fused else 0))
 
     def forward(self, x: torch.Tensor, mask_off: bool = False, path: str | None = None,
-                out: torch.Tensor | None = None, stream=None, graph: bool = True) -> torch.Tensor:
+                out: torch.Tensor | None = None, stream=None, graph: bool = True,
+                fused: bool = False) -> torch.Tensor:
         """y [T][D] float32 of x [T][D] (storage dtype, CUDA), enqueued on the current stream.
-        graph=False launches the kernels directly instead of replaying a captured graph."""
+        graph=False launches the kernels directly instead of replaying a captured graph;
+        fused=True runs a bf16 batch of <= 32 tokens as one cooperative launch (opt-in)."""
         if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype):
             raise ValueError("x must be a contiguous CUDA tensor of the layer's storage dtype")
         T = x.shape[0]
         if out is None:
             out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
         check(_lib.load().beam_moe_forward(self._h, _ptr(x), T, _ptr(out),
-                                           self.flags(mask_off, path, graph),
+                                           self.flags(mask_off, path, graph, fused),
                                            ctypes.c_void_p(_stream_handle(stream))))
         return out
 

@@ -51,6 +51,8 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_PATH_STREAM  0x2u  /* force the weight-streaming (GEMV) expert path */
 #define BEAM_PATH_TENSOR  0x4u  /* force the tcgen05 tensor-core expert path (bf16 only) */
 #define BEAM_NO_GRAPH     0x8u  /* launch the kernels directly instead of replaying a graph */
+#define BEAM_FUSED_DECODE 0x10u /* batches of <= 32 tokens (bf16): one fused cooperative
+                                   launch instead of separate kernels (opt-in; slower on B200) */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
@@ -117,6 +119,11 @@ beam_status_t beam_moe_create(const beam_moe_config_t *cfg, const beam_moe_weigh
  * it).  The contents of x_dev may change between calls; the pointers may not, for a replay.
  * BEAM_NO_GRAPH, the legacy default stream, an already-capturing stream and profiling all use
  * direct kernel launches.
+ * BEAM_FUSED_DECODE: a bf16 forward of 1..32 tokens on the tensor-core path runs as one
+ * cooperative launch of one block per SM (router, routing, compaction, both GEMMs, SwiGLU and
+ * combine, separated by grid barriers) when the device supports cooperative launches; it is
+ * launched directly, not replayed.  Without the flag the same forward runs as separate kernels
+ * chained with programmatic dependent launch, which measured faster.
  */
 beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, float *y_dev,
                                uint32_t flags, void *stream);
@@ -157,9 +164,10 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * off.  beam_moe_stage_name(i) names stage i ("" when out of range).  On the tensor-core path
  * the shared experts' GEMMs run on a second stream, overlapping the routing; they are timed
  * under stages of their own (tc_shared_gateup, tc_shared_down, shared_swiglu_finish), so that
- * each stage's time covers the work of one problem.
+ * each stage's time covers the work of one problem.  A fused decode forward is one launch,
+ * timed as the stage fused_decode.
  */
-#define BEAM_N_STAGES 15
+#define BEAM_N_STAGES 16
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);

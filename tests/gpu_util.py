@@ -27,7 +27,7 @@ def same_decision_tokens(gr: dict, orr) -> np.ndarray:
 
 def run_case(spec: synth.LayerSpec, T: int, seed: int = 0, keep_rate=0.5, mask_off=False,
              path=None, zero_mask=False, mask_bias=None, max_tokens=None, y_tokens=None,
-             layer=None, weights=None, x=None):
+             layer=None, weights=None, x=None, fused=False):
     """Run the CUDA layer and the oracle on the same inputs; assert parity; return details."""
     from dynamic_expert_routing_b200 import BeamMoE
     big = spec.n_experts * spec.d_ff * spec.d_model * 3 > 50_000_000
@@ -47,9 +47,9 @@ def run_case(spec: synth.LayerSpec, T: int, seed: int = 0, keep_rate=0.5, mask_o
                             segment_len=spec.segment_len)
         xd = x.cuda()
         y = torch.empty((T, spec.d_model), dtype=torch.float32, device="cuda")
-        layer.forward(xd, mask_off=mask_off, path=path, out=y)
+        layer.forward(xd, mask_off=mask_off, path=path, out=y, fused=fused)
         y.fill_(float("nan"))
-        layer.forward(xd, mask_off=mask_off, path=path, out=y)
+        layer.forward(xd, mask_off=mask_off, path=path, out=y, fused=fused)
     torch.cuda.synchronize()
     gr = layer.routing(T)
     st = layer.stats()

@@ -271,19 +271,20 @@ def test_profiling_stages_count_every_launch(T):
     """Per-stage timing: every stage launches once per forward and the launches per stage add
     up to the handle's launch counter (so a roofline that divides a stage's time by its
     launches is consistent).  T = 300 runs the shared experts on the second stream, timed
-    under stages of their own; T = 4 splits K and runs them inside the routed launches."""
+    under stages of their own; T = 4 splits K and runs them inside the routed launches (as
+    separate kernels: fused=False, not the one-launch decode path)."""
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=256)
     w = synth.make_layer(spec, keep_rate=0.5)
     layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=T)
     x = synth.make_tokens(spec, T, seed=5).cuda()
     y = torch.empty((T, spec.d_model), device="cuda")
-    layer.forward(x, path="tensor", out=y)
+    layer.forward(x, path="tensor", out=y, fused=False)
     n = 3
     n0 = layer.launch_count()
     layer.profile_begin(n)
     for _ in range(n):
-        layer.forward(x, path="tensor", out=y)
+        layer.forward(x, path="tensor", out=y, fused=False)
     prof = layer.profile_end()
     assert prof["forwards"] == n
     stages = {k: v for k, v in prof.items() if k != "forwards"}
@@ -417,4 +418,54 @@ def test_swapped_many_small_groups():
     y2 = layer.forward(info["x"].cuda(), mask_off=True, graph=False)
     torch.cuda.synchronize()
     assert torch.equal(y2, info["y"])
+    layer.close()
+
+
+# ------------------------------------------------------------------ fused decode launch
+@pytest.mark.parametrize("spec,T,mask_off", [
+    (_small(), 1, False),
+    (_small(n_shared=1, d_ff_shared=256), 7, False),
+    (_small(segment_len=16, n_shared=1, d_ff_shared=128), 32, False),
+    (_small(), 32, True),
+    (synth.LayerSpec("e256", 512, 256, 32, 128), 3, False),
+    (synth.SPECS["dsv2lite"], 1, False),
+    (synth.SPECS["mixtral"], 8, False),
+], ids=["t1", "shared_t7", "segments_t32", "mask_off_t32", "e256_k32", "dsv2lite_t1", "mixtral_t8"])
+def test_fused_decode_matches_oracle_and_separate_kernels(spec, T, mask_off):
+    """BEAM_FUSED_DECODE runs a batch of <= 32 tokens as one cooperative launch (router,
+    routing, compaction, both GEMMs, SwiGLU, combine, separated by grid barriers).  It must meet
+    the oracle like every path, repeat its own bits, and agree with the separate-kernel path,
+    which sums the router logits in another order: routing equal away from near-ties, y within
+    the tolerance."""
+    info = run_case(spec, T, seed=61, mask_off=mask_off, fused=True)
+    layer = info["layer"]
+    x = info["x"].cuda()
+    n0 = layer.launch_count()
+    y1 = layer.forward(x, mask_off=mask_off, fused=True).clone()
+    assert layer.launch_count() == n0 + 1          # one kernel
+    assert torch.equal(y1, info["y"])
+    r_fused = layer.routing(T)
+    y2 = layer.forward(x, mask_off=mask_off, fused=False)
+    r_sep = layer.routing(T)
+    torch.cuda.synchronize()
+    assert layer.launch_count() > n0 + 2
+    same = (r_fused["topk_id"] == r_sep["topk_id"]).all(axis=1)
+    assert same.mean() >= 0.9
+    assert parity.rel_l2(y1.cpu().double().numpy()[same], y2.cpu().double().numpy()[same]) < 2e-3
+    layer.close()
+
+
+def test_fused_decode_is_one_profiled_stage():
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=256)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=8)
+    x = synth.make_tokens(spec, 8, seed=3).cuda()
+    layer.forward(x, fused=True)
+    layer.profile_begin(2)
+    layer.forward(x, fused=True)
+    layer.forward(x, fused=True)
+    prof = layer.profile_end()
+    stages = {k: v for k, v in prof.items() if k != "forwards"}
+    assert list(stages) == ["fused_decode"] and stages["fused_decode"][1] == 2
     layer.close()
