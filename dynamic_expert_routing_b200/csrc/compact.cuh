@@ -32,11 +32,42 @@ compact_bits_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__
         for (int w = 0; w < nw; ++w) smask[warp][w][lane] = 0u;
         const int t = c * 32 + lane;
         if (t < T) {
-            for (int k = 0; k < K; ++k) {
-                size_t o = (size_t)t * K + k;
-                if (keep[o]) {
-                    int e = topk_id[o];
-                    smask[warp][e >> 5][lane] |= 1u << (e & 31);
+            // a token's K slots are contiguous: with K = 4, 8 or 16, read them as 16-byte vectors
+            // (all loads in flight at once); otherwise slot by slot
+            if (K == 4 || K == 8 || K == 16) {
+                const size_t o = (size_t)t * K;
+                uint32_t kp[4];
+                if (K == 16) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(keep + o);
+                    kp[0] = v.x; kp[1] = v.y; kp[2] = v.z; kp[3] = v.w;
+                } else if (K == 8) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(keep + o);
+                    kp[0] = v.x; kp[1] = v.y; kp[2] = kp[3] = 0u;
+                } else {
+                    kp[0] = *reinterpret_cast<const uint32_t*>(keep + o); kp[1] = kp[2] = kp[3] = 0u;
+                }
+                int id[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (q * 4 < K) {
+                        const int4 v = *reinterpret_cast<const int4*>(topk_id + o + q * 4);
+                        id[4 * q] = v.x; id[4 * q + 1] = v.y; id[4 * q + 2] = v.z; id[4 * q + 3] = v.w;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    if (k < K && ((kp[k >> 2] >> (8 * (k & 3))) & 0xffu)) {
+                        const int e = id[k];
+                        smask[warp][e >> 5][lane] |= 1u << (e & 31);
+                    }
+                }
+            } else {
+                for (int k = 0; k < K; ++k) {
+                    const size_t o = (size_t)t * K + k;
+                    if (keep[o]) {
+                        const int e = topk_id[o];
+                        smask[warp][e >> 5][lane] |= 1u << (e & 31);
+                    }
                 }
             }
         }
@@ -56,23 +87,6 @@ compact_bits_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__
     pdl_launch_dependents();
 }
 
-// tile_group[q] = the group that owns tile q (tiles of kGroupTileRows rows, numbered across
-// the groups in order), so that the grouped GEMMs find a tile's group with one 16-byte load.
-// Called by every warp of the block after the group table is written and the block has
-// synchronised.  The table was written by this block, so it is read through L2
-// (ld.global.cg), never through the non-coherent path.
-__device__ __forceinline__ void fill_tile_groups(const Group* groups, const int* n_groups,
-                                                 Group* __restrict__ tile_group, int warp, int lane,
-                                                 int nwarps)
-{
-    const int ng = __ldcg(n_groups);
-    for (int g = warp; g < ng; g += nwarps) {
-        const int4 G = __ldcg(reinterpret_cast<const int4*>(groups + g));  // row0, m, expert, mt0
-        const int mts = (G.y + kGroupTileRows - 1) / kGroupTileRows;
-        for (int q = lane; q < mts; q += 32) reinterpret_cast<int4*>(tile_group)[G.w + q] = G;
-    }
-}
-
 __global__ void __launch_bounds__(1024)
 compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                     const int* __restrict__ nkeep_tok, const float* __restrict__ lreg_tok,
@@ -82,6 +96,8 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                     int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group)
 {
     __shared__ int s_counts[kMaxE];
+    __shared__ Group s_groups[kMaxE];
+    __shared__ int s_ngroups;
     __shared__ long long s_keep[32];
     __shared__ double s_lreg[32];
     __shared__ int s_zero[32];
@@ -91,22 +107,54 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
     // the arrival counters of the grouped GEMMs' tail split start every forward at zero
     for (int i = threadIdx.x; i < n_tail_cnt; i += blockDim.x) tail_cnt[i] = 0;
 
-    // 1. per-expert chunk prefix sums
-    for (int e = warp; e < E; e += nwarps) {
-        int running = 0;
-        for (int c0 = 0; c0 < nch; c0 += 32) {
-            const int c = c0 + lane;
-            const int p = (c < nch) ? __popc(bits[(size_t)e * nch + c]) : 0;
-            int incl = p;
+    // 0. per-thread sums of the token statistics, issued first so their loads overlap the rest
+    long long ks = 0;
+    double ls = 0.0;
+    int nz = 0;
+#pragma unroll 4
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+        const int nk = nkeep_tok[t];
+        ks += nk;
+        ls += (double)lreg_tok[t];
+        nz += (nk == 0);
+    }
+
+    // 1. per-expert chunk prefix sums: a warp takes two experts at a time and loads 8 words of
+    // 32 chunks of each together, then scans them one after the other
+    for (int e0 = warp; e0 < E; e0 += 2 * nwarps) {
+        const int e1 = e0 + nwarps;
+        int run0 = 0, run1 = 0;
+        for (int c0 = 0; c0 < nch; c0 += 32 * 8) {
+            uint32_t w0[8], w1[8];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + 32 * u + lane;
+                w0[u] = (c < nch) ? bits[(size_t)e0 * nch + c] : 0u;
+                w1[u] = (c < nch && e1 < E) ? bits[(size_t)e1 * nch + c] : 0u;
             }
-            if (c < nch) chunk_base[(size_t)e * nch + c] = running + incl - p;
-            running += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + 32 * u + lane;
+                const int p0 = __popc(w0[u]), p1 = __popc(w1[u]);
+                int i0 = p0, i1 = p1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int n0 = __shfl_up_sync(0xffffffffu, i0, o);
+                    const int n1 = __shfl_up_sync(0xffffffffu, i1, o);
+                    if (lane >= o) { i0 += n0; i1 += n1; }
+                }
+                if (c < nch) {
+                    chunk_base[(size_t)e0 * nch + c] = run0 + i0 - p0;
+                    if (e1 < E) chunk_base[(size_t)e1 * nch + c] = run1 + i1 - p1;
+                }
+                run0 += __shfl_sync(0xffffffffu, i0, 31);
+                run1 += __shfl_sync(0xffffffffu, i1, 31);
+            }
         }
-        if (lane == 0) { s_counts[e] = running; counts[e] = running; }
+        if (lane == 0) {
+            s_counts[e0] = run0; counts[e0] = run0;
+            if (e1 < E) { s_counts[e1] = run1; counts[e1] = run1; }
+        }
     }
     __syncthreads();
 
@@ -149,6 +197,7 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                     Group g;
                     g.row0 = run; g.m = loc[j]; g.expert = e; g.mt0 = runm;
                     groups[runa] = g;
+                    s_groups[runa] = g;
                     ++runa;
                     runm += (loc[j] + kGroupTileRows - 1) / kGroupTileRows;
                 }
@@ -162,21 +211,13 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
             offsets[E] = total;
             n_groups[0] = tact;
             n_groups[1] = mt;
+            s_ngroups = tact;
             stats->n_kept = total;
             stats->n_active = tact;
         }
     }
 
-    // 3. statistics: strided per-thread sums, then a fixed-shape tree
-    long long ks = 0;
-    double ls = 0.0;
-    int nz = 0;
-    for (int t = threadIdx.x; t < T; t += blockDim.x) {
-        int nk = nkeep_tok[t];
-        ks += nk;
-        ls += (double)lreg_tok[t];
-        nz += (nk == 0);
-    }
+    // 3. statistics: the per-thread sums of step 0, then a fixed-shape tree
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         ks += __shfl_xor_sync(0xffffffffu, ks, o);
@@ -185,7 +226,12 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
     }
     if (lane == 0) { s_keep[warp] = ks; s_lreg[warp] = ls; s_zero[warp] = nz; }
     __syncthreads();
-    fill_tile_groups(groups, n_groups, tile_group, warp, lane, nwarps);
+    // tile -> group table, from the block's copy of the group table
+    for (int g = warp; g < s_ngroups; g += nwarps) {
+        const Group G = s_groups[g];
+        const int mts = (G.m + kGroupTileRows - 1) / kGroupTileRows;
+        for (int q = lane; q < mts; q += 32) tile_group[G.mt0 + q] = G;
+    }
     if (warp == 0) {
         ks = lane < nwarps ? s_keep[lane] : 0;
         ls = lane < nwarps ? s_lreg[lane] : 0.0;

@@ -93,6 +93,15 @@ struct RowDecision {
     float lreg;    // all lanes: (1/K) sum_k sigmoid(l_k)
 };
 
+// Order key of (logit v, expert e): larger key = larger v, and for equal v the lower e (the
+// float's bits mapped to an unsigned order, above the complemented index).
+__device__ __forceinline__ unsigned long long topk_key(float v, int e)
+{
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)ord << 32) | (uint32_t)(~e);
+}
+
 template <int EPL>
 __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, int splits,
                                                   long long split_stride, int E, int K,
@@ -104,33 +113,41 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
         for (int s = 1; s < splits; ++s) a += Li[s * split_stride + col];
         return a;
     };
-    float v[EPL];
+    // Each lane sorts the keys of its experts lane, lane+32, ... once (descending); then every
+    // round takes the warp maximum of the lanes' first keys, and the lane that owned it drops
+    // its first key.  The keys are distinct (the index is part of them), so the rounds yield
+    // the Top-K in rank order with ties to the lower index.
+    unsigned long long key[EPL];
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
-        int e = lane + 32 * j;
-        v[j] = (e < E) ? logit(e) : -INFINITY;
+        const int e = lane + 32 * j;
+        key[j] = (e < E) ? topk_key(logit(e), e) : 0ull;
     }
-    unsigned chosen = 0;
-    int my_id = 0;
-    float my_v = 0.f;
-    for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) {
-            int e = lane + 32 * j;
-            bool ok = (e < E) && !((chosen >> j) & 1u);
-            if (ok && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
+    for (int pass = 0; pass < EPL; ++pass) {
+#pragma unroll
+        for (int j = pass & 1; j + 1 < EPL; j += 2) {
+            if (key[j + 1] > key[j]) { const unsigned long long t = key[j]; key[j] = key[j + 1]; key[j + 1] = t; }
         }
+    }
+    unsigned long long my_key = 0ull;
+    for (int k = 0; k < K; ++k) {
+        unsigned long long b = key[0];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            const unsigned long long ob = __shfl_xor_sync(0xffffffffu, b, o);
+            b = ob > b ? ob : b;
         }
-        if ((bi & 31) == lane) chosen |= 1u << (bi >> 5);
-        if (lane == k) { my_id = bi; my_v = bv; }
+        if (key[0] == b) {
+#pragma unroll
+            for (int j = 0; j + 1 < EPL; ++j) key[j] = key[j + 1];
+            key[EPL - 1] = 0ull;
+        }
+        if (lane == k) my_key = b;
     }
+    const int my_id = (int)(~(uint32_t)my_key);
+    const uint32_t ord = (uint32_t)(my_key >> 32);
+    const float my_v = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
     RowDecision d;
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
     const bool active = lane < K;
