@@ -128,6 +128,7 @@ struct beam_moe {
     float* lreg_tok = nullptr;
     uint32_t* bits = nullptr;
     int *chunk_base = nullptr, *counts = nullptr, *offsets = nullptr, *perm = nullptr, *inv = nullptr;
+    ScanPart* scan_part = nullptr;  // compact_scan's per-CTA statistics
     Group* groups = nullptr;
     int* n_groups = nullptr;     // [0]: kept groups, [1]: their 128-row tiles
     Group* tile_group = nullptr; // 128-row tile (numbered across the groups) -> its group
@@ -545,6 +546,7 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->lreg_tok, Tm * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->bits, E * h->max_nch * sizeof(uint32_t)));
     BEAM_TRY(dalloc(h, &h->chunk_base, E * h->max_nch * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->scan_part, kScanMaxCtas * sizeof(ScanPart)));
     BEAM_TRY(dalloc(h, &h->counts, E * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->offsets, (E + 1) * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->perm, rows * sizeof(int)));
@@ -884,10 +886,12 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         BEAM_CUDA(e);
         BEAM_CUDA(launch(h, ST_COMPACT_BITS, compact_bits_kernel, dim3(ceil_div(nch, 8)), dim3(256), 0, st,
                          (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, E, nch, h->bits));
-        BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(1), dim3(1024), 0, st,
+        BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(scan_ctas(E, T_)),
+                         dim3(32 * kScanWarps), 0, st,
                          (const uint32_t*)h->bits, nch, E, T_, (const int*)h->nkeep_tok,
                          (const float*)h->lreg_tok, h->counts, h->offsets, h->chunk_base, h->groups,
-                         h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms), h->tile_group));
+                         h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms), h->tile_group,
+                         h->scan_part, &h->dstats->grid_bar));
         BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>,
                          dim3(ceil_div((long long)T_ * K, 8)), dim3(256), 0, st,
                          (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D, nch,

@@ -34,7 +34,8 @@ struct DevStats {
     int n_kept;           // kept (token, slot) pairs
     int tokens;
     int err;              // nonzero when a bounded wait ran out
-    unsigned grid_bar;    // arrivals at the fused decode kernel's grid barriers (zeroed with err)
+    unsigned grid_bar;    // arrival counter, zeroed with err every forward: the fused decode
+                          // kernel's grid barriers, or compact_scan's last-CTA election
 };
 
 // ---------------------------------------------------------------- storage-type helpers

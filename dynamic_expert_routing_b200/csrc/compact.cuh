@@ -2,12 +2,13 @@
 // mask 1 are run (ai-feeds.com summary "BEAM: 用于 MoE 动态路由的二进制专家激活掩码", Method,
 // output and inference acceleration: masked experts' FFNs are skipped).
 //
-// Deterministic and free of atomics: the order of perm is fixed by (expert asc, token asc).
+// Deterministic: the order of perm is fixed by (expert asc, token asc), and no atomic decides
+// any order (the scan's one atomic only elects the CTA that finishes).
 //   1. compact_bits: per 32-token chunk c and expert e, a warp ballot gives the word
 //      bits[e][c] whose bit b says "token 32c+b keeps a slot routed to e".
-//   2. compact_scan (one CTA): per expert, popcount prefix sums over chunks -> chunk_base;
-//      counts; exclusive scan over experts -> offsets; the list of active groups; and the
-//      forward's statistics, reduced in a fixed tree order.
+//   2. compact_scan: per expert (one warp each), popcount prefix sums over chunks ->
+//      chunk_base and counts; then the last CTA: exclusive scan over experts -> offsets, the
+//      list of active groups, and the forward's statistics, reduced in a fixed order.
 //   3. compact_scatter_gather: the position of pair (t, k) routed to e is
 //      offsets[e] + chunk_base[e][t/32] + popc(bits[e][t/32] & lanes_below(t%32)); it writes
 //      perm / inv and copies x[t] into row pos of X_perm.
@@ -87,78 +88,124 @@ compact_bits_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__
     pdl_launch_dependents();
 }
 
-__global__ void __launch_bounds__(1024)
+// compact_scan runs on several CTAs of kScanWarps warps: warp g of the grid scans the chunk
+// words of experts g, g + (grid warps), ...; every thread adds the statistics of a strided set
+// of tokens, and each CTA writes its sums to part[blockIdx.x].  The last CTA to arrive (an
+// atomic counter decides which CTA that is, never the order of any sum) builds the offsets,
+// the active-group list, the tile table and the statistics from the per-expert counts and
+// the per-CTA sums, taken in index order.
+constexpr int kScanWarps = 8;
+constexpr int kScanMaxCtas = 64;
+
+struct ScanPart {
+    long long keep;   // kept slots of this CTA's tokens
+    double lreg;      // their L_reg terms
+    int zero;         // their tokens with no kept slot
+    int pad;
+};
+
+// CTAs of one compact_scan launch: one warp per expert, and one thread per 2048 tokens at most
+// for the statistics.
+__host__ __device__ __forceinline__ int scan_ctas(int E, int T)
+{
+    int n = (E + kScanWarps - 1) / kScanWarps;
+    const int nt = (T + 2047) / 2048;
+    if (nt > n) n = nt;
+    return n < 1 ? 1 : (n > kScanMaxCtas ? kScanMaxCtas : n);
+}
+
+__global__ void __launch_bounds__(32 * kScanWarps)
 compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
                     const int* __restrict__ nkeep_tok, const float* __restrict__ lreg_tok,
                     int* __restrict__ counts, int* __restrict__ offsets,
                     int* __restrict__ chunk_base, Group* __restrict__ groups,
                     int* __restrict__ n_groups, DevStats* __restrict__ stats,
-                    int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group)
+                    int* __restrict__ tail_cnt, int n_tail_cnt, Group* __restrict__ tile_group,
+                    ScanPart* __restrict__ part, unsigned* __restrict__ arrive)
 {
     __shared__ int s_counts[kMaxE];
     __shared__ Group s_groups[kMaxE];
     __shared__ int s_ngroups;
-    __shared__ long long s_keep[32];
-    __shared__ double s_lreg[32];
-    __shared__ int s_zero[32];
+    __shared__ long long s_keep[kScanWarps];
+    __shared__ double s_lreg[kScanWarps];
+    __shared__ int s_zero[kScanWarps];
+    __shared__ int s_last;
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
+    const int nthreads = gridDim.x * blockDim.x;
+    const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
     // the arrival counters of the grouped GEMMs' tail split start every forward at zero
-    for (int i = threadIdx.x; i < n_tail_cnt; i += blockDim.x) tail_cnt[i] = 0;
+    for (int i = gtid; i < n_tail_cnt; i += nthreads) tail_cnt[i] = 0;
 
     // 0. per-thread sums of the token statistics, issued first so their loads overlap the rest
     long long ks = 0;
     double ls = 0.0;
     int nz = 0;
 #pragma unroll 4
-    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    for (int t = gtid; t < T; t += nthreads) {
         const int nk = nkeep_tok[t];
         ks += nk;
         ls += (double)lreg_tok[t];
         nz += (nk == 0);
     }
 
-    // 1. per-expert chunk prefix sums: a warp takes two experts at a time and loads 8 words of
-    // 32 chunks of each together, then scans them one after the other
-    for (int e0 = warp; e0 < E; e0 += 2 * nwarps) {
-        const int e1 = e0 + nwarps;
-        int run0 = 0, run1 = 0;
+    // 1. per-expert chunk prefix sums: 8 words of 32 chunks loaded together, then scanned
+    for (int e = blockIdx.x * kScanWarps + warp; e < E; e += gridDim.x * kScanWarps) {
+        int run = 0;
         for (int c0 = 0; c0 < nch; c0 += 32 * 8) {
-            uint32_t w0[8], w1[8];
+            uint32_t w[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int c = c0 + 32 * u + lane;
-                w0[u] = (c < nch) ? bits[(size_t)e0 * nch + c] : 0u;
-                w1[u] = (c < nch && e1 < E) ? bits[(size_t)e1 * nch + c] : 0u;
+                w[u] = (c < nch) ? bits[(size_t)e * nch + c] : 0u;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int c = c0 + 32 * u + lane;
-                const int p0 = __popc(w0[u]), p1 = __popc(w1[u]);
-                int i0 = p0, i1 = p1;
+                const int pc = __popc(w[u]);
+                int incl = pc;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const int n0 = __shfl_up_sync(0xffffffffu, i0, o);
-                    const int n1 = __shfl_up_sync(0xffffffffu, i1, o);
-                    if (lane >= o) { i0 += n0; i1 += n1; }
+                    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += n;
                 }
-                if (c < nch) {
-                    chunk_base[(size_t)e0 * nch + c] = run0 + i0 - p0;
-                    if (e1 < E) chunk_base[(size_t)e1 * nch + c] = run1 + i1 - p1;
-                }
-                run0 += __shfl_sync(0xffffffffu, i0, 31);
-                run1 += __shfl_sync(0xffffffffu, i1, 31);
+                if (c < nch) chunk_base[(size_t)e * nch + c] = run + incl - pc;
+                run += __shfl_sync(0xffffffffu, incl, 31);
             }
         }
-        if (lane == 0) {
-            s_counts[e0] = run0; counts[e0] = run0;
-            if (e1 < E) { s_counts[e1] = run1; counts[e1] = run1; }
-        }
+        if (lane == 0) counts[e] = run;
     }
+
+    // 2. this CTA's statistics: warp trees, then the warps in index order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ks += __shfl_xor_sync(0xffffffffu, ks, o);
+        ls += __shfl_xor_sync(0xffffffffu, ls, o);
+        nz += __shfl_xor_sync(0xffffffffu, nz, o);
+    }
+    if (lane == 0) { s_keep[warp] = ks; s_lreg[warp] = ls; s_zero[warp] = nz; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        ScanPart q;
+        q.keep = 0; q.lreg = 0.0; q.zero = 0; q.pad = 0;
+        for (int w = 0; w < kScanWarps; ++w) { q.keep += s_keep[w]; q.lreg += s_lreg[w]; q.zero += s_zero[w]; }
+        part[blockIdx.x] = q;
+    }
+
+    // 3. the last CTA to arrive finishes; counts and partial sums are visible to it
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(arrive, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) {
+        pdl_launch_dependents();
+        return;
+    }
+    __threadfence();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_counts[e] = __ldcg(counts + e);
     __syncthreads();
 
-    // 2. offsets and the active-group list (warp 0; each lane owns 8 consecutive experts)
+    // 4. offsets and the active-group list (warp 0; each lane owns 8 consecutive experts)
     if (warp == 0) {
         int loc[8], act[8];
         int sum = 0, nact = 0;
@@ -215,39 +262,27 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
             stats->n_kept = total;
             stats->n_active = tact;
         }
+    } else if (warp == 1 && lane == 0) {
+        // 5. statistics: the CTAs' sums in CTA order
+        long long k = 0;
+        double l = 0.0;
+        int z = 0;
+        for (int b = 0; b < (int)gridDim.x; ++b) {
+            k += __ldcg(&part[b].keep);
+            l += __ldcg(&part[b].lreg);
+            z += __ldcg(&part[b].zero);
+        }
+        stats->keep_sum = k;
+        stats->lreg_sum = l;
+        stats->n_all_masked = z;
+        stats->tokens = T;
     }
-
-    // 3. statistics: the per-thread sums of step 0, then a fixed-shape tree
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        ks += __shfl_xor_sync(0xffffffffu, ks, o);
-        ls += __shfl_xor_sync(0xffffffffu, ls, o);
-        nz += __shfl_xor_sync(0xffffffffu, nz, o);
-    }
-    if (lane == 0) { s_keep[warp] = ks; s_lreg[warp] = ls; s_zero[warp] = nz; }
     __syncthreads();
     // tile -> group table, from the block's copy of the group table
-    for (int g = warp; g < s_ngroups; g += nwarps) {
+    for (int g = warp; g < s_ngroups; g += kScanWarps) {
         const Group G = s_groups[g];
         const int mts = (G.m + kGroupTileRows - 1) / kGroupTileRows;
         for (int q = lane; q < mts; q += 32) tile_group[G.mt0 + q] = G;
-    }
-    if (warp == 0) {
-        ks = lane < nwarps ? s_keep[lane] : 0;
-        ls = lane < nwarps ? s_lreg[lane] : 0.0;
-        nz = lane < nwarps ? s_zero[lane] : 0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            ks += __shfl_xor_sync(0xffffffffu, ks, o);
-            ls += __shfl_xor_sync(0xffffffffu, ls, o);
-            nz += __shfl_xor_sync(0xffffffffu, nz, o);
-        }
-        if (lane == 0) {
-            stats->keep_sum = ks;
-            stats->lreg_sum = ls;
-            stats->n_all_masked = nz;
-            stats->tokens = T;
-        }
     }
     pdl_launch_dependents();
 }

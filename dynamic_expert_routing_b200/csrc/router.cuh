@@ -93,13 +93,17 @@ struct RowDecision {
     float lreg;    // all lanes: (1/K) sum_k sigmoid(l_k)
 };
 
-// Order key of (logit v, expert e): larger key = larger v, and for equal v the lower e (the
-// float's bits mapped to an unsigned order, above the complemented index).
-__device__ __forceinline__ unsigned long long topk_key(float v, int e)
+// Order bits of a logit: a larger value has larger bits (the float's sign-magnitude bits
+// mapped to an unsigned order), and the map is one to one.
+__device__ __forceinline__ uint32_t topk_ord(float v)
 {
     const uint32_t u = __float_as_uint(v);
-    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    return ((unsigned long long)ord << 32) | (uint32_t)(~e);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float topk_value(uint32_t ord)
+{
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
 }
 
 template <int EPL>
@@ -113,41 +117,43 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
         for (int s = 1; s < splits; ++s) a += Li[s * split_stride + col];
         return a;
     };
-    // Each lane sorts the keys of its experts lane, lane+32, ... once (descending); then every
-    // round takes the warp maximum of the lanes' first keys, and the lane that owned it drops
-    // its first key.  The keys are distinct (the index is part of them), so the rounds yield
-    // the Top-K in rank order with ties to the lower index.
-    unsigned long long key[EPL];
+    // Each lane sorts its experts lane, lane+32, ... once by value, descending; the sort is
+    // stable, so equal values keep the lower expert first (lane padding: order 0 and an index
+    // above every expert, after every real expert).  Every round then takes the warp maximum
+    // of the lanes' first values, the lowest expert among the lanes holding that maximum
+    // (two warp reductions), and the lane that owned it drops its first entry.  The rounds
+    // yield the Top-K in rank order with ties to the lower index.
+    uint32_t ord[EPL], idx[EPL];
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
         const int e = lane + 32 * j;
-        key[j] = (e < E) ? topk_key(logit(e), e) : 0ull;
+        ord[j] = (e < E) ? topk_ord(logit(e)) : 0u;
+        idx[j] = (e < E) ? (uint32_t)e : 0xffffffffu;
     }
 #pragma unroll
     for (int pass = 0; pass < EPL; ++pass) {
 #pragma unroll
         for (int j = pass & 1; j + 1 < EPL; j += 2) {
-            if (key[j + 1] > key[j]) { const unsigned long long t = key[j]; key[j] = key[j + 1]; key[j + 1] = t; }
+            if (ord[j + 1] > ord[j]) {
+                const uint32_t to = ord[j]; ord[j] = ord[j + 1]; ord[j + 1] = to;
+                const uint32_t ti = idx[j]; idx[j] = idx[j + 1]; idx[j + 1] = ti;
+            }
         }
     }
-    unsigned long long my_key = 0ull;
+    uint32_t my_ord = 0u, my_idx = 0u;
     for (int k = 0; k < K; ++k) {
-        unsigned long long b = key[0];
+        const uint32_t best = __reduce_max_sync(0xffffffffu, ord[0]);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, ord[0] == best ? idx[0] : 0xffffffffu);
+        if (idx[0] == win) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long ob = __shfl_xor_sync(0xffffffffu, b, o);
-            b = ob > b ? ob : b;
+            for (int j = 0; j + 1 < EPL; ++j) { ord[j] = ord[j + 1]; idx[j] = idx[j + 1]; }
+            ord[EPL - 1] = 0u;
+            idx[EPL - 1] = 0xffffffffu;
         }
-        if (key[0] == b) {
-#pragma unroll
-            for (int j = 0; j + 1 < EPL; ++j) key[j] = key[j + 1];
-            key[EPL - 1] = 0ull;
-        }
-        if (lane == k) my_key = b;
+        if (lane == k) { my_ord = best; my_idx = win; }
     }
-    const int my_id = (int)(~(uint32_t)my_key);
-    const uint32_t ord = (uint32_t)(my_key >> 32);
-    const float my_v = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+    const int my_id = (int)my_idx;
+    const float my_v = topk_value(my_ord);
     RowDecision d;
     const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
     const bool active = lane < K;

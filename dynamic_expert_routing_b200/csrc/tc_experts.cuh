@@ -385,6 +385,45 @@ struct TileWalker {
 // MODE_PLAIN has neither path compiled in.
 enum Mode { MODE_PLAIN = 0, MODE_TAIL = 1, MODE_SWAP = 2 };
 
+// Stores of one 32x32 f32 sub-tile from an epilogue warp's staging buffer (row i at
+// buf + i * EPI_PITCH) to rows 0 .. nrows-1 of `out` (row pitch ld elements), 16 bytes per
+// lane: fp16 takes 4 lanes per row, so one instruction writes 8 rows; f32 takes 8 lanes per
+// row, 4 rows per instruction.  Lane l reads row-chunk (l / lanes_per_row, l % lanes_per_row):
+// with the 33-word pitch the 32 lanes hit 32 different banks.  The column offset of `out`
+// must be a multiple of 8 (fp16) or 4 (f32) elements and ld a multiple of the same.
+__device__ __forceinline__ void store_rows_f16(const float* buf, __half* out, int ld, int nrows,
+                                               int lane)
+{
+    const int cg = (lane & 3) * 8;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        if (8 * q >= nrows) break;   // warp-uniform: no rows left
+        const int r = (lane >> 2) + 8 * q;
+        if (r < nrows) {
+            const float* s = buf + r * EPI_PITCH + cg;
+            __half2 h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(s[2 * j], s[2 * j + 1]);
+            *reinterpret_cast<uint4*>(out + (size_t)r * ld + cg) = *reinterpret_cast<const uint4*>(h);
+        }
+    }
+}
+
+__device__ __forceinline__ void store_rows_f32(const float* buf, float* out, int ld, int nrows,
+                                               int lane)
+{
+    const int cg = (lane & 7) * 4;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        if (4 * q >= nrows) break;   // warp-uniform: no rows left
+        const int r = (lane >> 3) + 4 * q;
+        if (r < nrows) {
+            const float* s = buf + r * EPI_PITCH + cg;
+            *reinterpret_cast<float4*>(out + (size_t)r * ld + cg) = make_float4(s[0], s[1], s[2], s[3]);
+        }
+    }
+}
+
 // Shared-memory layout of one CTA: [stage s: A (16 KB) | B (32 KB)] x STAGES, the epilogue
 // staging buffers, then the mbarriers, the TMEM address slot and the abort flag.
 struct GemmSmem {
@@ -720,9 +759,7 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                         for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] *= v[i];
                     }
                     __syncwarp();
-                    __half* col = out + row_base * ld + (size_t)t.n * (BN / 2) + 32 * j + lane;
-                    for (int i = 0; i < nrows; ++i)
-                        col[(size_t)i * ld] = __float2half_rn(buf[i * EPI_PITCH + lane]);
+                    store_rows_f16(buf, out + row_base * ld + (size_t)t.n * (BN / 2) + 32 * j, ld, nrows, lane);
                     __syncwarp();
                 }
             } else {
@@ -739,15 +776,13 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
 #pragma unroll
                     for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] = v[i];
                     __syncwarp();
-                    const size_t off = (size_t)t.ks * sstride + row_base * ld + (size_t)t.n * BN + 32 * j + lane;
-                    if (EPI == EPI_STORE_F16) {
-                        __half* col = static_cast<__half*>(t.shared ? p.out_shared : p.out_routed) + off;
-                        for (int i = 0; i < nrows; ++i)
-                            col[(size_t)i * ld] = __float2half_rn(buf[i * EPI_PITCH + lane]);
-                    } else {
-                        float* col = static_cast<float*>(t.shared ? p.out_shared : p.out_routed) + off;
-                        for (int i = 0; i < nrows; ++i) col[(size_t)i * ld] = buf[i * EPI_PITCH + lane];
-                    }
+                    const size_t off = (size_t)t.ks * sstride + row_base * ld + (size_t)t.n * BN + 32 * j;
+                    if (EPI == EPI_STORE_F16)
+                        store_rows_f16(buf, static_cast<__half*>(t.shared ? p.out_shared : p.out_routed) + off,
+                                       ld, nrows, lane);
+                    else
+                        store_rows_f32(buf, static_cast<float*>(t.shared ? p.out_shared : p.out_routed) + off,
+                                       ld, nrows, lane);
                     __syncwarp();
                 }
             }
