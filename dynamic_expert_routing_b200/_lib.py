@@ -50,6 +50,18 @@ class BeamStats(ctypes.Structure):
                 ("tokens", ctypes.c_int32), ("n_kept", ctypes.c_int32)]
 
 
+class BeamGenConfig(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("segment_len", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32)]
+
+
+class BeamRouting(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("topk_id", "gate", "mask_logit", "keep", "ghat",
+                                               "n_keep", "lreg", "active")]
+
+
 class BeamError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
@@ -85,13 +97,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.beam_moe_stage_name.restype = ctypes.c_char_p
     lib.beam_moe_launch_count.argtypes = [P]
     lib.beam_moe_launch_count.restype = ctypes.c_int64
+    lib.beam_gen_create.argtypes = [ctypes.POINTER(BeamGenConfig), P, P, P, ctypes.POINTER(P)]
+    lib.beam_gen_route.argtypes = [P, P, I, ctypes.POINTER(BeamRouting), U, P]
+    lib.beam_gen_sync.argtypes = [P]
+    lib.beam_gen_destroy.argtypes = [P]
+    lib.beam_gen_destroy.restype = None
+    lib.beam_moe_forward_routed.argtypes = [P, P, I, ctypes.POINTER(BeamRouting), P, U, P]
     lib.beam_moe_destroy.argtypes = [P]
     lib.beam_moe_destroy.restype = None
     lib.beam_moe_last_error.restype = ctypes.c_char_p
     lib.beam_moe_version.restype = ctypes.c_char_p
     for f in (lib.beam_moe_create, lib.beam_moe_forward, lib.beam_moe_forward_host,
               lib.beam_moe_stats, lib.beam_moe_get_routing, lib.beam_moe_profile_begin,
-              lib.beam_moe_profile_end):
+              lib.beam_moe_profile_end, lib.beam_gen_create, lib.beam_gen_route,
+              lib.beam_gen_sync, lib.beam_moe_forward_routed):
         f.restype = ctypes.c_int
     _lib = lib
     return lib

@@ -50,18 +50,23 @@ static beam_status_t fail(beam_status_t st, const char* fmt, ...)
     } while (0)
 
 // ---------------------------------------------------------------- repack kernels
-// Wrm [n2E_pad][D]: row j < E is column j of W_r, row E + j is column j of W_m, rest zero.
+// Wrm [n_pad][D] for nL layers (W_r, W_m [nL][D][E]): row 2lE + j (j < E) is column j of layer
+// l's W_r, row 2lE + E + j column j of its W_m; rows from 2E*nL on are zero.  One layer: the
+// layer's router; nL layers: the cross-layer mask generator.
 template <typename T>
 __global__ void repack_router_kernel(const T* __restrict__ wr, const T* __restrict__ wm, int D,
-                                     int E, int n2E_pad, T* __restrict__ out)
+                                     int E, int nL, int n_pad, T* __restrict__ out)
 {
-    const size_t n = (size_t)n2E_pad * D;
+    const size_t n = (size_t)n_pad * D;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x) {
         const int j = (int)(i / D), d = (int)(i % D);
+        const int l = j / (2 * E), c = j % (2 * E);
         T v = from_float<T>(0.f);
-        if (j < E) v = wr[(size_t)d * E + j];
-        else if (j < 2 * E) v = wm[(size_t)d * E + (j - E)];
+        if (l < nL) {
+            const size_t base = ((size_t)l * D + d) * E;
+            v = c < E ? wr[base + c] : wm[base + (c - E)];
+        }
         out[i] = v;
     }
 }
@@ -109,6 +114,25 @@ __global__ void repack_down_kernel(const TI* __restrict__ w, long long n, int S,
 }
 
 // ---------------------------------------------------------------- the handle
+// Routing given by the caller (beam_moe_forward_routed): the forward then starts at the
+// compaction.  gate and mlogit are optional (only beam_moe_get_routing reads them).
+struct RouteIn {
+    const int* topk_id = nullptr;
+    const uint8_t* keep = nullptr;
+    const float* ghat = nullptr;
+    const int* nkeep = nullptr;
+    const float* lreg = nullptr;
+    const float* gate = nullptr;
+    const float* mlogit = nullptr;
+    bool operator==(const RouteIn& o) const {
+        return topk_id == o.topk_id && keep == o.keep && ghat == o.ghat && nkeep == o.nkeep &&
+               lreg == o.lreg && gate == o.gate && mlogit == o.mlogit;
+    }
+};
+
+struct beam_moe;
+static RouteIn own_routing(const beam_moe* h);
+
 struct beam_moe {
     beam_moe_config_t cfg;
     int E, K, D, F, Fsh, Tmax, S;
@@ -170,7 +194,10 @@ struct beam_moe {
     int g_T = -1;
     uint32_t g_flags = 0;
     bool g_tc = false;
+    RouteIn cur;         // the routing arrays the last forward read (beam_moe_get_routing)
     int g_kernels = 0;   // kernels in the captured graph
+    bool g_routed = false;
+    RouteIn g_rin;       // routing pointers of a captured routed forward
     // launch accounting and optional per-stage timing
     long long launches = 0;
     bool prof = false;
@@ -295,6 +322,15 @@ constexpr int kTcRouterMinRows = 64;
 // Counter regions of the tail split: routed gate/up, routed down.  (The shared problem runs
 // concurrently with the routing on a second stream, so its last wave has no idle SMs to fill.)
 constexpr int kTailCntRegions = 2;
+// The handle's own routing arrays (written by its router and Top-K/mask kernels).
+static RouteIn own_routing(const beam_moe* h)
+{
+    RouteIn r;
+    r.topk_id = h->topk_id; r.keep = h->keep; r.ghat = h->ghat; r.nkeep = h->nkeep_tok;
+    r.lreg = h->lreg_tok; r.gate = h->gate; r.mlogit = h->mlogit;
+    return r;
+}
+
 static int tail_cnt_ints(int num_sms) { return kTailCntRegions * num_sms * tc::kEpiWarps; }
 
 // Small batches gather their kept rows inside the fused routing kernel up to this many bytes.
@@ -339,8 +375,8 @@ static beam_status_t repack(beam_moe* h, const beam_moe_weights_t* w, cudaStream
     using TH = typename HType<T>::type;
     const int D = h->D, E = h->E, F = h->F;
     repack_router_kernel<T><<<1024, 256, 0, st>>>(static_cast<const T*>(w->w_router),
-                                                  static_cast<const T*>(w->w_mask), D, E, h->ldL,
-                                                  static_cast<T*>(h->wrm));
+                                                  static_cast<const T*>(w->w_mask), D, E, 1,
+                                                  h->ldL, static_cast<T*>(h->wrm));
     BEAM_CUDA(cudaGetLastError());
     repack_gateup_kernel<T><<<(unsigned)((long long)E * 2 * F), 128, 0, st>>>(
         static_cast<const T*>(w->w_gate), static_cast<const T*>(w->w_up), E, F, D,
@@ -653,7 +689,7 @@ static cudaError_t launch_select(beam_moe* h, int Tr, int T, int mask_off, int s
     return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256), 0, st,
                   (const float*)h->L, h->ldL, splits, split_stride, Tr, T, h->E, h->K, h->S,
                   mask_off, h->topk_id, h->gate, h->mlogit, h->keep, h->ghat, h->nkeep_tok,
-                  h->lreg_tok);
+                  h->lreg_tok, 0LL, 0LL, (uint32_t*)nullptr);
 }
 
 template <int EPL, typename T>
@@ -793,19 +829,19 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
 }
 
 template <typename TR, typename TS>
-static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, int T_, float* y,
-                                  cudaStream_t st)
+static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, const float* ghat,
+                                  int T_, float* y, cudaStream_t st)
 {
     // few tokens: split each token's columns over several CTAs so the combine spans the SMs
     const dim3 cgrid(T_, T_ < h->num_sms ? ceil_div(h->D / 4, 256) : 1);
     return launch(h, ST_COMBINE, combine_kernel<TR, TS>, cgrid, dim3(256), 0, st,
                   (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
-                  (const int*)h->inv, (const float*)h->ghat, T_, h->K, h->D, y);
+                  (const int*)h->inv, ghat, T_, h->K, h->D, y);
 }
 
 template <typename T>
 static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uint32_t flags,
-                                  bool use_tc, cudaStream_t st)
+                                  bool use_tc, cudaStream_t st, const RouteIn* rin = nullptr)
 {
     const int E = h->E, K = h->K, D = h->D;
     const int S = h->S;
@@ -829,10 +865,16 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         BEAM_CUDA(cudaEventRecord(h->ev_join, h->side));
     }
 
+    // the routing this forward reads: computed below, or given by the caller
+    const RouteIn rt = rin ? *rin : own_routing(h);
+    h->cur = rt;
+
     // 1. router logits L = x [W_r | W_m]  (routed rows only: segment leaders when S > 1)
     int lsplits = 1;
     long long lstride = 0;
-    if (h->tc_ok && Tr >= kTcRouterMinRows) {
+    if (rin) {
+        // the routing is given: no router
+    } else if (h->tc_ok && Tr >= kTcRouterMinRows) {
         tc::TcParams& p0 = h->p0;
         BEAM_TRY(encode_map(h, &p0.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)Tr,
                             (uint64_t)D, tc::BM, (uint64_t)S * D));
@@ -855,7 +897,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     // 2-3. routing decision and compaction.  Small batches (one 32-token chunk) run them as one
     // single-CTA kernel; larger ones as select -> bit planes -> scan -> scatter + gather.
     cudaError_t e;
-    if (T_ <= kSmallT) {
+    if (!rin && T_ <= kSmallT) {
         const int gather_inline = (long long)T_ * K * D * (long long)sizeof(T) <= kInlineGatherBytes;
         switch ((E + 31) / 32) {
             case 1: e = launch_small<1>(h, x, Tr, T_, mask_off, lsplits, lstride, gather_inline, st); break;
@@ -873,28 +915,30 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                              dim3(256), 0, st, (const int*)h->perm, (const int*)(h->offsets + E),
                              K, D, x, (T*)h->xperm));
     } else {
-        switch ((E + 31) / 32) {
-            case 1: e = launch_select<1>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            case 2: e = launch_select<2>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            case 3: e = launch_select<3>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            case 4: e = launch_select<4>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            case 5: e = launch_select<5>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            case 6: e = launch_select<6>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            case 7: e = launch_select<7>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
-            default: e = launch_select<8>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+        if (!rin) {
+            switch ((E + 31) / 32) {
+                case 1: e = launch_select<1>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                case 2: e = launch_select<2>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                case 3: e = launch_select<3>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                case 4: e = launch_select<4>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                case 5: e = launch_select<5>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                case 6: e = launch_select<6>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                case 7: e = launch_select<7>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+                default: e = launch_select<8>(h, Tr, T_, mask_off, lsplits, lstride, st); break;
+            }
+            BEAM_CUDA(e);
         }
-        BEAM_CUDA(e);
         BEAM_CUDA(launch(h, ST_COMPACT_BITS, compact_bits_kernel, dim3(ceil_div(nch, 8)), dim3(256), 0, st,
-                         (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, E, nch, h->bits));
+                         rt.topk_id, rt.keep, T_, K, E, nch, h->bits));
         BEAM_CUDA(launch(h, ST_COMPACT_SCAN, compact_scan_kernel, dim3(scan_ctas(E, T_)),
                          dim3(32 * kScanWarps), 0, st,
-                         (const uint32_t*)h->bits, nch, E, T_, (const int*)h->nkeep_tok,
-                         (const float*)h->lreg_tok, h->counts, h->offsets, h->chunk_base, h->groups,
+                         (const uint32_t*)h->bits, nch, E, T_, rt.nkeep,
+                         rt.lreg, h->counts, h->offsets, h->chunk_base, h->groups,
                          h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms), h->tile_group,
                          h->scan_part, &h->dstats->grid_bar));
         BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>,
                          dim3(ceil_div((long long)T_ * K, 8)), dim3(256), 0, st,
-                         (const int*)h->topk_id, (const uint8_t*)h->keep, T_, K, D, nch,
+                         rt.topk_id, rt.keep, T_, K, D, nch,
                          (const uint32_t*)h->bits, (const int*)h->offsets,
                          (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     }
@@ -921,10 +965,10 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     if (fork) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_join, 0));
     if (!h->Fsh) ysh_out.f16 = yr.f16;  // no shared term: only its (unused) type must match
     cudaError_t ce;
-    if (yr.f16 && ysh_out.f16) ce = launch_combine<__half, __half>(h, yr, ysh_out, T_, y, st);
-    else if (yr.f16) ce = launch_combine<__half, float>(h, yr, ysh_out, T_, y, st);
-    else if (ysh_out.f16) ce = launch_combine<float, __half>(h, yr, ysh_out, T_, y, st);
-    else ce = launch_combine<float, float>(h, yr, ysh_out, T_, y, st);
+    if (yr.f16 && ysh_out.f16) ce = launch_combine<__half, __half>(h, yr, ysh_out, rt.ghat, T_, y, st);
+    else if (yr.f16) ce = launch_combine<__half, float>(h, yr, ysh_out, rt.ghat, T_, y, st);
+    else if (ysh_out.f16) ce = launch_combine<float, __half>(h, yr, ysh_out, rt.ghat, T_, y, st);
+    else ce = launch_combine<float, float>(h, yr, ysh_out, rt.ghat, T_, y, st);
     BEAM_CUDA(ce);
     return BEAM_OK;
 }
@@ -945,6 +989,7 @@ static beam_status_t forward_fused(beam_moe* h, const __nv_bfloat16* x, int T_, 
 {
     const int D = h->D, F = h->F, Fsh = h->Fsh, K = h->K, E = h->E, S = h->S;
     const int Tr = ceil_div(T_, S);
+    h->cur = own_routing(h);
     BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, 2 * sizeof(int), st));  // err, grid_bar
     const long long mts = ceil_div(T_, tc::BM);
     const long long groups = std::min<long long>(E, std::max(1LL, ((long long)T_ * K + 1) / 2));
@@ -1051,7 +1096,7 @@ static cudaError_t launch_select_into(beam_moe* h, const float* L, int Tr, int T
 {
     return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256),
                   0, st, L, h->n2E, 1, 0LL, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate,
-                  mlogit, keep, ghat, nkeep_tok, lreg_tok);
+                  mlogit, keep, ghat, nkeep_tok, lreg_tok, 0LL, 0LL, (uint32_t*)nullptr);
 }
 
 template <typename T>
@@ -1078,6 +1123,182 @@ static beam_status_t route_noalloc_impl(beam_moe* h, const T* x, int T_, int32_t
         case 6: e = launch_select_into<6>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
         case 7: e = launch_select_into<7>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
         default: e = launch_select_into<8>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
+    }
+    BEAM_CUDA(e);
+    return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- cross-layer routing
+// The mask generator ("Stepped MoE: Segment-Level Routing with Configurable Inference
+// Complexity", core method): the logits of every layer from one GEMM over the segment
+// leaders' rows of z, G = z_lead [W_r^(1) | W_m^(1) | ... | W_r^(L) | W_m^(L)], then one warp per
+// (segment, layer) takes BEAM's Top-K / softmax / mask decision (route_select_kernel with a
+// layer grid dimension) and marks the layer's kept experts.
+struct beam_gen {
+    beam_moe core;          // device plumbing shared with the layer handle (allocations, tensor
+                            // maps, launches, error word); its expert fields stay unused
+    int L = 0;
+    int nlog = 0;           // L * 2E logit columns
+    int ldG = 0;            // row pitch of G: nlog, padded to the tile width on the tensor path
+    void* wgen = nullptr;   // [ldG][D] repacked generator weights
+    float* G = nullptr;     // logits [splits][Tr][ldG] (K-split slices when the GEMM splits)
+};
+
+static beam_status_t gen_validate(const beam_gen_config_t* c)
+{
+    if (!c) return fail(BEAM_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->dtype != BEAM_DTYPE_F32 && c->dtype != BEAM_DTYPE_BF16)
+        return fail(BEAM_ERR_INVALID_ARG, "dtype must be BEAM_DTYPE_F32 or BEAM_DTYPE_BF16");
+    const int dmul = c->dtype == BEAM_DTYPE_BF16 ? 64 : 4;
+    const int dmax = c->dtype == BEAM_DTYPE_BF16 ? 8192 : 4096;
+    if (c->d_model <= 0 || c->d_model % dmul || c->d_model > dmax)
+        return fail(BEAM_ERR_INVALID_ARG, "d_model=%d must be a positive multiple of %d, <= %d",
+                    c->d_model, dmul, dmax);
+    if (c->n_layers < 1 || c->n_layers > 512)
+        return fail(BEAM_ERR_INVALID_ARG, "n_layers=%d must be in [1, 512]", c->n_layers);
+    if (c->n_experts < 1 || c->n_experts > kMaxE)
+        return fail(BEAM_ERR_INVALID_ARG, "n_experts=%d must be in [1, %d]", c->n_experts, kMaxE);
+    if (c->top_k < 1 || c->top_k > std::min(c->n_experts, 32))
+        return fail(BEAM_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E, 32)]", c->top_k);
+    if (c->segment_len < 0 || c->segment_len > 65536)
+        return fail(BEAM_ERR_INVALID_ARG, "segment_len=%d out of range", c->segment_len);
+    if (c->max_tokens < 1 || c->max_tokens > 65536)
+        return fail(BEAM_ERR_INVALID_ARG, "max_tokens=%d must be in [1, 65536]", c->max_tokens);
+    return BEAM_OK;
+}
+
+static beam_status_t gen_create_impl(const beam_gen_config_t* c, const void* wr, const void* wm,
+                                     cudaStream_t st, beam_gen* g)
+{
+    beam_moe* h = &g->core;
+    memset(&h->cfg, 0, sizeof h->cfg);
+    h->cfg.d_model = c->d_model; h->cfg.n_experts = c->n_experts; h->cfg.top_k = c->top_k;
+    h->cfg.dtype = c->dtype; h->cfg.segment_len = c->segment_len; h->cfg.max_tokens = c->max_tokens;
+    h->D = c->d_model; h->E = c->n_experts; h->K = c->top_k; h->F = h->Fsh = 0;
+    h->Tmax = c->max_tokens;
+    h->S = c->segment_len > 1 ? c->segment_len : 1;
+    h->n2E = 2 * h->E;
+    h->esz = h->hsz = c->dtype == BEAM_DTYPE_BF16 ? 2 : 4;
+    int dev = 0;
+    BEAM_CUDA(cudaGetDevice(&dev));
+    BEAM_CUDA(cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev));
+    g->L = c->n_layers;
+    g->nlog = g->L * h->n2E;
+    // the tensor-core GEMM under the same condition as a layer's router
+    const bool tc = c->dtype == BEAM_DTYPE_BF16 && h->D % tc::BN == 0;
+    g->ldG = tc ? ceil_div(g->nlog, tc::BN) * tc::BN : g->nlog;
+    const int Trmax = ceil_div(h->Tmax, h->S);
+    // room for the largest K-split the GEMM takes: the split count depends on the 128-row
+    // tile count, so the largest row count of each tile count bounds it
+    size_t gfloats = (size_t)Trmax * g->ldG;
+    if (tc) {
+        for (int mt = 1; mt <= ceil_div(Trmax, tc::BM); ++mt) {
+            const int rows = std::min(mt * tc::BM, Trmax);
+            if (rows < kTcRouterMinRows) continue;
+            const int s = normalise_splits(choose_splits(h->num_sms, (long long)mt * (g->ldG / tc::BN)),
+                                           h->D / tc::BK);
+            gfloats = std::max(gfloats, (size_t)s * rows * g->ldG);
+        }
+    }
+    BEAM_TRY(dalloc(h, &g->wgen, (size_t)g->ldG * h->D * h->esz));
+    BEAM_TRY(dalloc(h, &g->G, gfloats * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->zero_int, 2 * sizeof(int)));
+    BEAM_TRY(dalloc(h, &h->groups, sizeof(Group)));
+    BEAM_TRY(dalloc(h, &h->dstats, sizeof(DevStats)));
+    BEAM_CUDA(cudaMemsetAsync(h->dstats, 0, sizeof(DevStats), st));
+    BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, 2 * sizeof(int), st));
+    BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
+    if (c->dtype == BEAM_DTYPE_BF16)
+        repack_router_kernel<__nv_bfloat16><<<2048, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(wr), static_cast<const __nv_bfloat16*>(wm), h->D,
+            h->E, g->L, g->ldG, static_cast<__nv_bfloat16*>(g->wgen));
+    else
+        repack_router_kernel<float><<<2048, 256, 0, st>>>(
+            static_cast<const float*>(wr), static_cast<const float*>(wm), h->D, h->E, g->L,
+            g->ldG, static_cast<float*>(g->wgen));
+    BEAM_CUDA(cudaGetLastError());
+    if (tc) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        BEAM_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+        if (!fn || q != cudaDriverEntryPointSuccess)
+            return fail(BEAM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        h->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        BEAM_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+        // one dense problem: G [Tr][ldG] = z_lead [Tr][D] . Wgen [ldG][D]^T
+        tc::TcParams& r = h->p0;
+        memset(&r, 0, sizeof r);
+        BEAM_TRY(encode_map(h, &r.b_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g->wgen,
+                            (uint64_t)g->ldG, (uint64_t)h->D, tc::BN));
+        r.b_routed = r.b_shared;
+        r.groups = h->groups;
+        r.n_groups = h->zero_int;          // no routed groups
+        r.out_routed = r.out_shared = g->G;
+        r.ld_routed = r.ld_shared = g->ldG;
+        r.n_tiles_routed = r.n_tiles_shared = g->ldG / tc::BN;
+        r.k_steps_routed = r.k_steps_shared = h->D / tc::BK;
+        r.k_splits_routed = r.k_splits_shared = 1;
+        r.store_cols = g->nlog;            // columns past L*2E are padding nobody reads
+        r.err = &h->dstats->err;
+        h->tc_ok = true;
+    }
+    BEAM_CUDA(cudaStreamSynchronize(st));
+    return BEAM_OK;
+}
+
+template <int EPL>
+static cudaError_t launch_select_layers(beam_gen* g, const float* G, int splits, long long sstride,
+                                        int Tr, int T, int mask_off, const beam_routing_t* o,
+                                        cudaStream_t st)
+{
+    beam_moe* h = &g->core;
+    return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8), g->L),
+                  dim3(256), 0, st, G, g->ldG, splits, sstride, Tr, T, h->E, h->K, h->S, mask_off,
+                  o->topk_id, o->gate, o->mask_logit, o->keep, o->ghat, o->n_keep, o->lreg,
+                  (long long)T * h->K, (long long)T, o->active);
+}
+
+template <typename T>
+static beam_status_t gen_route_impl(beam_gen* g, const T* z, int T_, const beam_routing_t* o,
+                                    int mask_off, cudaStream_t st)
+{
+    beam_moe* h = &g->core;
+    const int S = h->S, Tr = ceil_div(T_, S), E = h->E, D = h->D;
+    BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, 2 * sizeof(int), st));
+    if (o->active)
+        BEAM_CUDA(cudaMemsetAsync(o->active, 0, (size_t)g->L * ((E + 31) / 32) * sizeof(uint32_t), st));
+    int splits = 1;
+    long long sstride = 0;
+    if (h->tc_ok && Tr >= kTcRouterMinRows) {
+        tc::TcParams& p = h->p0;
+        BEAM_TRY(encode_map(h, &p.a_shared, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, z, (uint64_t)Tr,
+                            (uint64_t)D, tc::BM, (uint64_t)S * D));
+        p.a_routed = p.a_shared;
+        p.shared_rows = Tr;
+        const long long tiles = (long long)ceil_div(Tr, tc::BM) * p.n_tiles_shared;
+        splits = normalise_splits(choose_splits(h->num_sms, tiles), D / tc::BK);
+        sstride = (long long)Tr * g->ldG;
+        p.k_splits_routed = p.k_splits_shared = splits;
+        p.split_stride_routed = p.split_stride_shared = sstride;
+        BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
+                         dim3((unsigned)std::min<long long>(h->num_sms, tiles * splits)),
+                         dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
+    } else {
+        BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
+                         dim3(g->nlog, ceil_div(Tr, kGemvRows)), dim3(256), 0, st, z, S, Tr, D,
+                         (const T*)g->wgen, g->nlog, g->ldG, g->G));
+    }
+    cudaError_t e;
+    switch ((E + 31) / 32) {
+        case 1: e = launch_select_layers<1>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        case 2: e = launch_select_layers<2>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        case 3: e = launch_select_layers<3>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        case 4: e = launch_select_layers<4>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        case 5: e = launch_select_layers<5>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        case 6: e = launch_select_layers<6>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        case 7: e = launch_select_layers<7>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
+        default: e = launch_select_layers<8>(g, g->G, splits, sstride, Tr, T_, mask_off, o, st); break;
     }
     BEAM_CUDA(e);
     return BEAM_OK;
@@ -1117,6 +1338,68 @@ beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, in
                                      mask_logit, keep, ghat, mask_off, sc, st);
 }
 
+beam_status_t beam_gen_create(const beam_gen_config_t* cfg, const void* w_router,
+                              const void* w_mask, void* stream, beam_gen_t** out)
+{
+    g_err[0] = 0;
+    BEAM_TRY(gen_validate(cfg));
+    if (!w_router || !w_mask || !out) return fail(BEAM_ERR_INVALID_ARG, "weights or out is NULL");
+    beam_gen* g = new (std::nothrow) beam_gen();
+    if (!g) return fail(BEAM_ERR_OOM, "host allocation failed");
+    beam_status_t s = gen_create_impl(cfg, w_router, w_mask, static_cast<cudaStream_t>(stream), g);
+    if (s != BEAM_OK) {
+        cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+        free_all(&g->core);
+        delete g;
+        return s;
+    }
+    *out = g;
+    return BEAM_OK;
+}
+
+beam_status_t beam_gen_route(beam_gen_t* g, const void* z, int32_t T, const beam_routing_t* out,
+                             uint32_t flags, void* stream)
+{
+    g_err[0] = 0;
+    if (!g || !out) return fail(BEAM_ERR_INVALID_ARG, "generator or out is NULL");
+    beam_moe* h = &g->core;
+    if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
+    if (flags & ~BEAM_MASK_OFF)
+        return fail(BEAM_ERR_INVALID_ARG, "only BEAM_MASK_OFF is accepted, got flags 0x%x", flags);
+    if (T == 0) return BEAM_OK;
+    if (!z || !out->topk_id || !out->gate || !out->mask_logit || !out->keep || !out->ghat ||
+        !out->n_keep || !out->lreg)
+        return fail(BEAM_ERR_INVALID_ARG, "z and every routing array except active must be non-NULL");
+    if (reinterpret_cast<uintptr_t>(z) & 15) return fail(BEAM_ERR_INVALID_ARG, "z must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
+    if (h->cfg.dtype == BEAM_DTYPE_BF16)
+        BEAM_TRY(gen_route_impl<__nv_bfloat16>(g, static_cast<const __nv_bfloat16*>(z), T, out, mask_off, st));
+    else
+        BEAM_TRY(gen_route_impl<float>(g, static_cast<const float*>(z), T, out, mask_off, st));
+    BEAM_CUDA(cudaEventRecord(h->done, st));
+    return BEAM_OK;
+}
+
+beam_status_t beam_gen_sync(beam_gen_t* g)
+{
+    g_err[0] = 0;
+    if (!g) return fail(BEAM_ERR_INVALID_ARG, "generator is NULL");
+    BEAM_CUDA(cudaEventSynchronize(g->core.done));
+    DevStats ds;
+    BEAM_CUDA(cudaMemcpy(&ds, g->core.dstats, sizeof ds, cudaMemcpyDeviceToHost));
+    if (ds.err) return fail(BEAM_ERR_TIMEOUT, "a bounded device wait ran out (code %d)", ds.err);
+    return BEAM_OK;
+}
+
+void beam_gen_destroy(beam_gen_t* g)
+{
+    if (!g) return;
+    if (g->core.done) cudaEventSynchronize(g->core.done);
+    free_all(&g->core);
+    delete g;
+}
+
 beam_status_t beam_moe_create(const beam_moe_config_t* cfg, const beam_moe_weights_t* w,
                               void* stream, beam_moe_t** out)
 {
@@ -1140,11 +1423,11 @@ beam_status_t beam_moe_create(const beam_moe_config_t* cfg, const beam_moe_weigh
     return BEAM_OK;
 }
 
-beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y, uint32_t flags,
-                               void* stream)
+// The forward behind beam_moe_forward (rin == nullptr) and beam_moe_forward_routed: argument
+// checks shared by both, then the fused decode launch, a graph replay, or direct launches.
+static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float* y, uint32_t flags,
+                                   const RouteIn* rin, void* stream)
 {
-    g_err[0] = 0;
-    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
     if (T > 0 && (!x || !y)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
@@ -1163,7 +1446,12 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
     if (h->prof) ++h->prof_forwards;
-    if (T > 0 && fused_eligible(h, T, flags, use_tc)) {
+    auto run = [&]() -> beam_status_t {
+        return (h->cfg.dtype == BEAM_DTYPE_BF16)
+            ? forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y, flags, use_tc, st, rin)
+            : forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st, rin);
+    };
+    if (T > 0 && !rin && fused_eligible(h, T, flags, use_tc)) {
         // one launch: nothing to gain from a graph
         BEAM_TRY(forward_fused(h, static_cast<const __nv_bfloat16*>(x), T, y, flags, st));
     } else if (T > 0) {
@@ -1172,10 +1460,12 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
         // used while profiling, on the legacy default stream, or with BEAM_NO_GRAPH.
         const bool graphable = !(flags & BEAM_NO_GRAPH) && !h->prof && st != nullptr;
         const uint32_t key_flags = flags & ~BEAM_NO_GRAPH;
+        const bool same_routing = rin ? (h->g_routed && h->g_rin == *rin) : !h->g_routed;
         if (graphable && h->graph_exec && h->g_x == x && h->g_y == y && h->g_T == T &&
-            h->g_flags == key_flags && h->g_tc == use_tc) {
+            h->g_flags == key_flags && h->g_tc == use_tc && same_routing) {
             BEAM_CUDA(cudaGraphLaunch(h->graph_exec, st));
             h->launches += h->g_kernels;
+            h->cur = rin ? *rin : own_routing(h);
         } else {
             bool captured = false;
             if (graphable) {
@@ -1183,9 +1473,7 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
                 if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone &&
                     cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
                     const long long n0 = h->launches;
-                    beam_status_t s1 = (h->cfg.dtype == BEAM_DTYPE_BF16)
-                        ? forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y, flags, use_tc, st)
-                        : forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st);
+                    beam_status_t s1 = run();
                     cudaGraph_t g = nullptr;
                     cudaError_t e1 = cudaStreamEndCapture(st, &g);
                     h->launches = n0;  // counted again when the graph runs
@@ -1200,6 +1488,8 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
                         drop_graph(h);
                         h->graph_exec = ex;
                         h->g_x = x; h->g_y = y; h->g_T = T; h->g_flags = key_flags; h->g_tc = use_tc;
+                        h->g_routed = rin != nullptr;
+                        h->g_rin = rin ? *rin : RouteIn();
                         h->g_kernels = (int)nn;
                         captured = true;
                     }
@@ -1213,18 +1503,47 @@ beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y
                     cudaGetLastError();
                 }
             }
-            if (!captured) {
-                if (h->cfg.dtype == BEAM_DTYPE_BF16)
-                    BEAM_TRY(forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, y,
-                                                         flags, use_tc, st));
-                else
-                    BEAM_TRY(forward_impl<float>(h, static_cast<const float*>(x), T, y, flags, use_tc, st));
-            }
+            if (!captured) BEAM_TRY(run());
         }
     }
     h->last_T = T;
     BEAM_CUDA(cudaEventRecord(h->done, st));
     return BEAM_OK;
+}
+
+beam_status_t beam_moe_forward(beam_moe_t* h, const void* x, int32_t T, float* y, uint32_t flags,
+                               void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    return forward_entry(h, x, T, y, flags, nullptr, stream);
+}
+
+beam_status_t beam_moe_forward_routed(beam_moe_t* h, const void* x, int32_t T,
+                                      const beam_routing_t* r, float* y, uint32_t flags,
+                                      void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (!r) return fail(BEAM_ERR_INVALID_ARG, "routing is NULL");
+    if (flags & (BEAM_MASK_OFF | BEAM_FUSED_DECODE))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_MASK_OFF and BEAM_FUSED_DECODE do not apply to a "
+                    "forward with given routing (the mask is part of the routing)");
+    if (T > 0 && (!r->topk_id || !r->keep || !r->ghat || !r->n_keep || !r->lreg))
+        return fail(BEAM_ERR_INVALID_ARG, "routing needs topk_id, keep, ghat, n_keep and lreg");
+    // the compaction reads a token's K slots as one vector when K is 4, 8 or 16
+    const bool vec = h->K == 4 || h->K == 8 || h->K == 16;
+    if (T > 0 && ((reinterpret_cast<uintptr_t>(r->topk_id) & (vec ? 15 : 3)) ||
+                  (reinterpret_cast<uintptr_t>(r->keep) & (vec ? h->K - 1 : 0))))
+        return fail(BEAM_ERR_INVALID_ARG, "topk_id must be 4-byte aligned and keep 1-byte aligned "
+                    "(top_k 4, 8 or 16: topk_id 16-byte, keep top_k-byte aligned)");
+    if (T > 0 && ((reinterpret_cast<uintptr_t>(r->ghat) | reinterpret_cast<uintptr_t>(r->n_keep) |
+                   reinterpret_cast<uintptr_t>(r->lreg)) & 3))
+        return fail(BEAM_ERR_INVALID_ARG, "ghat, n_keep and lreg must be 4-byte aligned");
+    RouteIn rin;
+    rin.topk_id = r->topk_id; rin.keep = r->keep; rin.ghat = r->ghat; rin.nkeep = r->n_keep;
+    rin.lreg = r->lreg; rin.gate = r->gate; rin.mlogit = r->mask_logit;
+    return forward_entry(h, x, T, y, flags, &rin, stream);
 }
 
 beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T, float* y_host,
@@ -1280,10 +1599,14 @@ beam_status_t beam_moe_get_routing(beam_moe_t* h, int32_t* topk_id, float* gate,
         if (offsets) memset(offsets, 0, sizeof(int32_t) * (h->E + 1));
         return BEAM_OK;
     }
-    if (topk_id) BEAM_CUDA(cudaMemcpy(topk_id, h->topk_id, n * 4, cudaMemcpyDeviceToHost));
-    if (gate) BEAM_CUDA(cudaMemcpy(gate, h->gate, n * 4, cudaMemcpyDeviceToHost));
-    if (mask_logit) BEAM_CUDA(cudaMemcpy(mask_logit, h->mlogit, n * 4, cudaMemcpyDeviceToHost));
-    if (keep) BEAM_CUDA(cudaMemcpy(keep, h->keep, n, cudaMemcpyDeviceToHost));
+    // the arrays the last forward read: its own, or those given to beam_moe_forward_routed
+    const RouteIn& c = h->cur;
+    if ((gate && !c.gate) || (mask_logit && !c.mlogit))
+        return fail(BEAM_ERR_INVALID_ARG, "the last forward was given no gate / mask_logit array");
+    if (topk_id) BEAM_CUDA(cudaMemcpy(topk_id, c.topk_id, n * 4, cudaMemcpyDeviceToHost));
+    if (gate) BEAM_CUDA(cudaMemcpy(gate, c.gate, n * 4, cudaMemcpyDeviceToHost));
+    if (mask_logit) BEAM_CUDA(cudaMemcpy(mask_logit, c.mlogit, n * 4, cudaMemcpyDeviceToHost));
+    if (keep) BEAM_CUDA(cudaMemcpy(keep, c.keep, n, cudaMemcpyDeviceToHost));
     if (inv) BEAM_CUDA(cudaMemcpy(inv, h->inv, n * 4, cudaMemcpyDeviceToHost));
     int nk = 0;
     BEAM_CUDA(cudaMemcpy(&nk, h->offsets + h->E, sizeof nk, cudaMemcpyDeviceToHost));

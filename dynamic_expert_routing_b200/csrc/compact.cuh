@@ -18,7 +18,7 @@
 
 namespace beam {
 
-constexpr int kMaxE = 256;
+constexpr int kMaxE = kRouteMaxE;
 
 __global__ void __launch_bounds__(256)
 compact_bits_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__ keep, int T,

@@ -21,6 +21,7 @@ namespace beam {
 // weight row with 16-byte loads, each thread keeps one partial per row, and the partials are
 // reduced in a fixed order (warp butterfly, then the 8 warps in index order).
 constexpr int kGemvRows = 16;
+constexpr int kRouteMaxE = 256;  // most routed experts per layer
 
 template <typename TW>
 __global__ void __launch_bounds__(256)
@@ -170,13 +171,18 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
     return d;
 }
 
-// One warp per routed row i (row i of L, leading dimension ldL: router logits in columns
-// [0, E), mask logits in [E, 2E); `splits` K-split slices split_stride floats apart, added in
-// slice order).  Lane l holds logits of experts l, l+32, ... (EPL per lane).
+// One warp per (routed row i, layer l = blockIdx.y).  Row i of L has leading dimension ldL;
+// layer l's router logits are its columns [2lE, 2lE + E), its mask logits [2lE + E, 2lE + 2E)
+// (one layer: l = 0); `splits` K-split slices split_stride floats apart are added in slice
+// order.  Lane l holds logits of experts l, l+32, ... (EPL per lane).
 // K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
 // rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
 // L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
-// to every token of the routed row's segment (S = 1: the row's own token).
+// to every token of the routed row's segment (S = 1: the row's own token), layer l's outputs
+// out_ls ([T][K] arrays) or tok_ls ([T] arrays) elements after layer 0's.  With `active` set,
+// bit e of layer l's word e/32 of active[l][nw] (nw = (E+31)/32, zeroed by the caller) is
+// set for every expert e kept by one of the block's tokens (an OR: the result does not depend
+// on the order of the updates).
 template <int EPL>
 __global__ void __launch_bounds__(256)
 route_select_kernel(const float* __restrict__ L, int ldL, int splits, long long split_stride,
@@ -184,27 +190,42 @@ route_select_kernel(const float* __restrict__ L, int ldL, int splits, long long 
                     int mask_off, int* __restrict__ topk_id, float* __restrict__ gate,
                     float* __restrict__ mlogit, uint8_t* __restrict__ keep,
                     float* __restrict__ ghat, int* __restrict__ nkeep_tok,
-                    float* __restrict__ lreg_tok)
+                    float* __restrict__ lreg_tok, long long out_ls, long long tok_ls,
+                    uint32_t* __restrict__ active)
 {
+    __shared__ uint32_t s_act[kRouteMaxE / 32];
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x * 8 + warp;
+    const int layer = blockIdx.y;
+    const int nw = (E + 31) >> 5;
+    if (active) {
+        if (threadIdx.x < nw) s_act[threadIdx.x] = 0u;
+        __syncthreads();
+    }
     if (i < Tr) {
-        const RowDecision d = select_row<EPL>(L + (size_t)i * ldL, splits, split_stride, E, K,
-                                              mask_off, lane);
+        const RowDecision d = select_row<EPL>(L + (size_t)i * ldL + (size_t)layer * 2 * E, splits,
+                                              split_stride, E, K, mask_off, lane);
         const int S = seg > 1 ? seg : 1;
         const int t0 = i * S, t1 = min(T, t0 + S);
+        const size_t lo = (size_t)layer * out_ls, lt = (size_t)layer * tok_ls;
         for (int t = t0; t < t1; ++t) {
             if (lane < K) {
-                size_t o = (size_t)t * K + lane;
+                size_t o = lo + (size_t)t * K + lane;
                 topk_id[o] = d.id;
                 gate[o] = d.g;
                 mlogit[o] = d.l;
                 keep[o] = d.keep ? 1 : 0;
                 ghat[o] = d.ghat;
             }
-            if (lane == 0) { nkeep_tok[t] = d.nkeep; lreg_tok[t] = d.lreg; }
+            if (lane == 0) { nkeep_tok[lt + t] = d.nkeep; lreg_tok[lt + t] = d.lreg; }
         }
+        if (active && d.keep) atomicOr(&s_act[d.id >> 5], 1u << (d.id & 31));
+    }
+    if (active) {
+        __syncthreads();
+        if (threadIdx.x < nw && s_act[threadIdx.x])
+            atomicOr(active + (size_t)layer * nw + threadIdx.x, s_act[threadIdx.x]);
     }
     pdl_launch_dependents();
 }

@@ -12,7 +12,8 @@ import torch
 
 from . import _lib
 from ._lib import (BEAM_DTYPE_BF16, BEAM_DTYPE_F32, BEAM_MASK_OFF, BEAM_FUSED_DECODE, BEAM_NO_GRAPH,
-                   BEAM_PATH_STREAM, BEAM_PATH_TENSOR, BeamConfig, BeamStats, BeamWeights, check)
+                   BEAM_PATH_STREAM, BEAM_PATH_TENSOR, BeamConfig, BeamGenConfig, BeamRouting,
+                   BeamStats, BeamWeights, check)
 
 _DTYPES = {torch.float32: BEAM_DTYPE_F32, torch.bfloat16: BEAM_DTYPE_BF16}
 _PATHS = {None: 0, "auto": 0, "stream": BEAM_PATH_STREAM, "tensor": BEAM_PATH_TENSOR}
@@ -87,6 +88,27 @@ class BeamMoE:
 
     __call__ = forward
 
+    def forward_routed(self, x: torch.Tensor, routing: dict, path: str | None = None,
+                       out: torch.Tensor | None = None, stream=None, graph: bool = True) -> torch.Tensor:
+        """y [T][D] float32 of x [T][D] with the routing given (one layer's slice of
+        BeamGenerator.route, see BeamGenerator.layer): the router and the Top-K/mask step are
+        skipped, the compaction, experts and combine run as in forward."""
+        if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype):
+            raise ValueError("x must be a contiguous CUDA tensor of the layer's storage dtype")
+        T = x.shape[0]
+        for k, dt in (("topk_id", torch.int32), ("keep", torch.uint8), ("ghat", torch.float32),
+                      ("n_keep", torch.int32), ("lreg", torch.float32)):
+            t = routing[k]
+            if not (t.is_cuda and t.is_contiguous() and t.dtype == dt and t.shape[0] == T):
+                raise ValueError(f"routing[{k!r}] must be a contiguous CUDA {dt} tensor of {T} rows")
+        if out is None:
+            out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
+        r = _routing_struct(routing)
+        check(_lib.load().beam_moe_forward_routed(self._h, _ptr(x), T, ctypes.byref(r), _ptr(out),
+                                                  self.flags(False, path, graph),
+                                                  ctypes.c_void_p(_stream_handle(stream))))
+        return out
+
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, mask_off: bool = False,
                      path: str | None = None, stream=None) -> torch.Tensor:
         """Host-buffer variant: copies x in, runs the layer, copies y out, synchronises."""
@@ -143,6 +165,88 @@ class BeamMoE:
     def close(self) -> None:
         if getattr(self, "_h", None):
             _lib.load().beam_moe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+_ROUTING_FIELDS = ("topk_id", "gate", "mask_logit", "keep", "ghat", "n_keep", "lreg", "active")
+
+
+def _routing_struct(routing: dict) -> BeamRouting:
+    return BeamRouting(*[_ptr(routing.get(k)) for k in _ROUTING_FIELDS])
+
+
+class BeamGenerator:
+    """Cross-layer mask generator held by the CUDA library.
+
+    w_router, w_mask: [L][D][E] CUDA tensors of one storage type (float32 or bfloat16), layer
+    l's router and mask-router matrices.  route(z) gives every layer's routing of the token
+    batch z [T][D] at once (one decision per segment of `segment_len` tokens, taken at the
+    segment's first token, when segment_len > 1).
+    """
+
+    def __init__(self, w_router: torch.Tensor, w_mask: torch.Tensor, top_k: int, max_tokens: int,
+                 segment_len: int = 0, stream=None):
+        lib = _lib.load()
+        dt = _DTYPES.get(w_router.dtype)
+        if dt is None:
+            raise TypeError(f"unsupported storage dtype {w_router.dtype}")
+        for name, t in (("w_router", w_router), ("w_mask", w_mask)):
+            if not (t.is_cuda and t.is_contiguous() and t.dtype == w_router.dtype and t.dim() == 3
+                    and t.shape == w_router.shape):
+                raise ValueError(f"{name} must be a contiguous [L][D][E] CUDA tensor of dtype {w_router.dtype}")
+        L, D, E = w_router.shape
+        self.cfg = BeamGenConfig(D, L, E, top_k, dt, segment_len, max_tokens)
+        h = ctypes.c_void_p()
+        check(lib.beam_gen_create(ctypes.byref(self.cfg), _ptr(w_router), _ptr(w_mask),
+                                  ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(h)))
+        self._h = h
+        self.dtype = w_router.dtype
+        self.n_layers, self.d_model, self.n_experts, self.top_k = L, D, E, top_k
+        self.max_tokens = max_tokens
+
+    def route(self, z: torch.Tensor, mask_off: bool = False, out: dict | None = None,
+              stream=None) -> dict:
+        """Every layer's routing of z [T][D]: topk_id [L][T][K] int32, gate, mask_logit, ghat
+        [L][T][K] float32, keep [L][T][K] uint8, n_keep [L][T] int32, lreg [L][T] float32 and
+        active [L][(E+31)/32] int32 (bit e%32 of word e/32: expert e kept in that layer)."""
+        if not (z.is_cuda and z.is_contiguous() and z.dtype == self.dtype):
+            raise ValueError("z must be a contiguous CUDA tensor of the generator's storage dtype")
+        T = z.shape[0]
+        L, K, nw = self.n_layers, self.top_k, (self.n_experts + 31) // 32
+        if out is None:
+            dev = z.device
+            out = dict(topk_id=torch.empty((L, T, K), dtype=torch.int32, device=dev),
+                       gate=torch.empty((L, T, K), dtype=torch.float32, device=dev),
+                       mask_logit=torch.empty((L, T, K), dtype=torch.float32, device=dev),
+                       keep=torch.empty((L, T, K), dtype=torch.uint8, device=dev),
+                       ghat=torch.empty((L, T, K), dtype=torch.float32, device=dev),
+                       n_keep=torch.empty((L, T), dtype=torch.int32, device=dev),
+                       lreg=torch.empty((L, T), dtype=torch.float32, device=dev),
+                       active=torch.empty((L, nw), dtype=torch.int32, device=dev))
+        r = _routing_struct(out)
+        check(_lib.load().beam_gen_route(self._h, _ptr(z), T, ctypes.byref(r),
+                                         BEAM_MASK_OFF if mask_off else 0,
+                                         ctypes.c_void_p(_stream_handle(stream))))
+        return out
+
+    @staticmethod
+    def layer(routing: dict, l: int) -> dict:
+        """Layer l's slice of a route() result (views), as BeamMoE.forward_routed takes it."""
+        return {k: v[l] for k, v in routing.items()}
+
+    def sync(self) -> None:
+        """Wait for the last route(); raises if one of its bounded device waits ran out."""
+        check(_lib.load().beam_gen_sync(self._h))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _lib.load().beam_gen_destroy(self._h)
             self._h = None
 
     def __del__(self):

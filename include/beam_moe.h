@@ -209,6 +209,93 @@ beam_status_t beam_moe_route_noalloc(beam_moe_t *h, const void *x_dev, int32_t T
  */
 beam_status_t beam_moe_wait_selftest(int32_t timeout_us, void *stream);
 
+/*
+ * ---------------------------------------------------------------- cross-layer routing
+ * The mask generator of "Stepped MoE: Segment-Level Routing with Configurable Inference
+ * Complexity" (core method and its inference paragraph): one pass over the output z of the
+ * model's dense prefix gives the routing logits of every MoE layer at once, one decision per
+ * segment of S tokens taken at the segment's first token, so that every layer's experts are
+ * known before the first MoE layer runs (and their weights can be fetched ahead).
+ * Combined with BEAM, layer l's decision is BEAM's Steps 1-3 with that layer's generator
+ * weights: r = z W_r^(l), mask logits z W_m^(l); Top-K of r (ties to the lower index), a
+ * softmax over the K, keep = mask logit >= 0 on the Top-K set, g_hat = g * keep.  The logits of
+ * all layers come from one GEMM, z_leaders [W_r^(1) | W_m^(1) | ... | W_r^(L) | W_m^(L)].
+ */
+typedef struct beam_gen beam_gen_t;
+
+typedef struct {
+    int32_t d_model;      /* D of z; same rules as beam_moe_config_t.d_model */
+    int32_t n_layers;     /* L, 1..512 */
+    int32_t n_experts;    /* E per layer, 1..256 */
+    int32_t top_k;        /* K, 1..min(E, 32) */
+    int32_t dtype;        /* BEAM_DTYPE_F32 or BEAM_DTYPE_BF16: storage of z and the weights */
+    int32_t segment_len;  /* 0 or 1: one decision per token; S > 1: per segment of S tokens */
+    int32_t max_tokens;   /* largest T any call will pass, 1..65536 */
+} beam_gen_config_t;
+
+/*
+ * Routing of L layers (or of one layer: every pointer offset to that layer), device arrays,
+ * layer-major:
+ *   topk_id [L][T][K] int32 (rank order)   gate [L][T][K] f32 (softmax over the K)
+ *   mask_logit [L][T][K] f32               keep [L][T][K] uint8
+ *   ghat [L][T][K] f32 (gate * keep)       n_keep [L][T] int32 (kept slots per token)
+ *   lreg [L][T] f32 ((1/K) sum_{TK} sigmoid(mask logit))
+ *   active [L][(E+31)/32] uint32: bit e%32 of word e/32 of layer l is set when some token of
+ *          the call keeps expert e in layer l (the experts whose weights that layer will read)
+ * A token of segment s carries the decision of the segment's first token, S*s.
+ */
+typedef struct {
+    int32_t *topk_id;
+    float *gate;
+    float *mask_logit;
+    uint8_t *keep;
+    float *ghat;
+    int32_t *n_keep;
+    float *lreg;
+    uint32_t *active;
+} beam_routing_t;
+
+/*
+ * Build a mask generator from w_router_dev[L][D][E] and w_mask_dev[L][D][E] (device, storage
+ * type, row-major per layer; borrowed during the call only: they are repacked into one
+ * [L*2E][D] matrix owned by the handle), on `stream` (then synchronised).  Errors as for
+ * beam_moe_create.
+ */
+beam_status_t beam_gen_create(const beam_gen_config_t *cfg, const void *w_router_dev,
+                              const void *w_mask_dev, void *stream, beam_gen_t **out);
+
+/*
+ * Routing of every layer for z_dev[T][D]: every array of *out except `active` (which may be
+ * NULL) must hold L*T*K (or L*T) elements; enqueued on `stream` without synchronising.  bf16
+ * generators with d_model a multiple of 64 compute the logits on the tensor cores (tcgen05),
+ * others with a CUDA-core GEMV; then one warp per (segment, layer) takes the decision.
+ * flags: 0 or BEAM_MASK_OFF (every Top-K slot kept).  T = 0 is a no-op.  Returns
+ * BEAM_ERR_TIMEOUT (from beam_gen_sync) if a bounded device wait ran out.
+ */
+beam_status_t beam_gen_route(beam_gen_t *g, const void *z_dev, int32_t T,
+                             const beam_routing_t *out, uint32_t flags, void *stream);
+
+/* Wait for the generator's last call; BEAM_ERR_TIMEOUT if one of its bounded waits ran out. */
+beam_status_t beam_gen_sync(beam_gen_t *g);
+
+/* Free the generator's device buffers (waits for its pending work).  NULL is ignored. */
+void beam_gen_destroy(beam_gen_t *g);
+
+/*
+ * beam_moe_forward with the routing given instead of computed: r points at one layer's
+ * topk_id, keep, ghat, n_keep and lreg (required; gate and mask_logit optional, only kept for
+ * beam_moe_get_routing; active unused), e.g. layer l's slice of a beam_gen_route output.  The
+ * forward skips the router and the Top-K/mask step and runs the compaction, the experts, the
+ * shared experts and the combine exactly as beam_moe_forward does; beam_moe_stats then
+ * describes the given routing.  flags: BEAM_PATH_STREAM / BEAM_PATH_TENSOR / BEAM_NO_GRAPH
+ * (BEAM_MASK_OFF and BEAM_FUSED_DECODE are rejected: the mask is part of the routing).  The
+ * graph replay key includes the routing pointers.  The routing arrays must stay valid until
+ * the stream reaches the end of the call's work.
+ */
+beam_status_t beam_moe_forward_routed(beam_moe_t *h, const void *x_dev, int32_t T,
+                                      const beam_routing_t *r, float *y_dev, uint32_t flags,
+                                      void *stream);
+
 /* Free every device buffer of the handle (waits for its pending work).  NULL is ignored. */
 void beam_moe_destroy(beam_moe_t *h);
 

@@ -119,6 +119,26 @@ def route(x, w_router, w_mask, top_k: int, segment_len: int = 0, mask_off: bool 
     return out
 
 
+def route_layers(z, w_router, w_mask, top_k: int, segment_len: int = 0,
+                 mask_off: bool = False) -> list:
+    """Cross-layer routing: the mask generator of "Stepped MoE: Segment-Level Routing with
+    Configurable Inference Complexity" (core method) decides every MoE layer's experts at once
+    from the dense prefix's output z, one decision per segment taken at its first token.
+    Combined with BEAM, layer l's routing is Steps 1-3 of z with layer l's router and
+    mask-router matrices.  w_router, w_mask: [L][D][E].  Returns one Routing per layer."""
+    if w_router.shape != w_mask.shape or len(w_router.shape) != 3:
+        raise ValueError("w_router and w_mask must both be [L][D][E]")
+    return [route(z, w_router[l], w_mask[l], top_k, segment_len=segment_len, mask_off=mask_off)
+            for l in range(w_router.shape[0])]
+
+
+def active_experts(routing: Routing, n_experts: int) -> np.ndarray:
+    """bool [E]: the experts some token keeps (the experts whose weights the layer reads)."""
+    act = np.zeros(int(n_experts), bool)
+    act[routing.topk_id[routing.keep.astype(bool)]] = True
+    return act
+
+
 def stats(routing: Routing):
     """(Avg-K, L_reg, tokens with every Top-K slot masked)."""
     lib = _load()

@@ -4,7 +4,7 @@ Shared by both sides of every parity check: the CPU oracle and the CUDA library 
 same tensors from here.  Nothing in this package computes any part of the MoE layer.
 """
 from .layers import (LayerSpec, SPECS, make_layer, make_tokens, make_router, make_experts,
-                     mask_bias_for_keep_rate)
+                     make_generator, mask_bias_for_keep_rate)
 
 __all__ = ["LayerSpec", "SPECS", "make_layer", "make_tokens", "make_router", "make_experts",
-           "mask_bias_for_keep_rate"]
+           "make_generator", "mask_bias_for_keep_rate"]

@@ -188,3 +188,20 @@ def make_layer(spec: LayerSpec, seed: int = 0, keep_rate: float | None = 0.5,
     wg, wu, wd, wsg, wsu, wsd = make_experts(spec, seed, device)
     return dict(w_router=wr, w_mask=wm, w_gate=wg, w_up=wu, w_down=wd,
                 ws_gate=wsg, ws_up=wsu, ws_down=wsd, mask_bias=c)
+
+
+def make_generator(spec: LayerSpec, n_layers: int, seed: int = 0,
+                   keep_rate: float | None = 0.5, mask_bias: float | None = None):
+    """Weights of a cross-layer mask generator: (W_r, W_m), each [L][D][E] in the storage type.
+
+    Layer l's pair is `make_router` of the same spec with seed 1000 * (seed + 1) + l, so every
+    layer draws its own streams; the mask bias follows `make_layer`'s rule.
+    """
+    if mask_bias is not None:
+        c = float(mask_bias)
+    elif keep_rate is None or keep_rate >= 1.0:
+        c = 0.0
+    else:
+        c = mask_bias_for_keep_rate(spec, keep_rate)
+    wr, wm = zip(*[make_router(spec, 1000 * (seed + 1) + l, c) for l in range(n_layers)])
+    return torch.stack(wr).contiguous(), torch.stack(wm).contiguous()

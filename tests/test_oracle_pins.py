@@ -334,3 +334,54 @@ def test_bf16_inputs_widen_exactly():
     b = oracle.route(x.float(), w32["w_router"], w32["w_mask"], spec.top_k)
     np.testing.assert_array_equal(a.g, b.g)
     np.testing.assert_array_equal(oracle.layer(x, w, a), oracle.layer(x.float(), w32, b))
+
+
+def test_cross_layer_routing_closed_form():
+    """Cross-layer routing ('Stepped MoE: Segment-Level Routing with Configurable Inference
+    Complexity', core method: one generator pass gives every layer's experts, once per
+    segment, from the segment's first position).  Layer l's router reads channel
+    1 + (e + l) mod 7 of z for expert e, so its Top-K in rank order are the channels holding
+    the K largest values, mapped back through the shift by l.  Its mask router reads the
+    constant channel z[:, 0] = 1 with sign + (even l) or - (odd l): every Top-K slot is kept
+    in even layers and none in odd ones, with L_reg = sigmoid(+1) or sigmoid(-1)."""
+    D, E, K, L, S, T = 8, 7, 3, 4, 2, 9     # the last segment is partial
+    rs = np.random.default_rng(5)
+    z = np.zeros((T, D), np.float32)
+    z[:, 0] = 1.0
+    for t in range(T):
+        z[t, 1:] = rs.permutation(7).astype(np.float32) * 0.5 - 1.0   # distinct, exact
+    wr = np.zeros((L, D, E), np.float32)
+    wm = np.zeros((L, D, E), np.float32)
+    for l in range(L):
+        for e in range(E):
+            wr[l, 1 + (e + l) % 7, e] = 1.0
+        wm[l, 0, :] = 1.0 if l % 2 == 0 else -1.0
+    rl = oracle.route_layers(torch.from_numpy(z), torch.from_numpy(wr), torch.from_numpy(wm), K,
+                             segment_len=S)
+    assert len(rl) == L
+    sig = {1: 1.0 / (1.0 + math.exp(-1.0)), 0: 1.0 / (1.0 + math.exp(1.0))}
+    for l, r in enumerate(rl):
+        kept = 1 if l % 2 == 0 else 0
+        want_act = np.zeros(E, bool)
+        for t in range(T):
+            lead = (t // S) * S
+            channels = sorted(range(7), key=lambda j: -z[lead, 1 + j])[:K]
+            want = [(j - l) % 7 for j in channels]
+            assert list(r.topk_id[t]) == want
+            assert (r.keep[t] == kept).all()
+            assert r.nkeep[t] == K * kept
+            assert r.lreg[t] == pytest.approx(sig[kept], abs=1e-15)
+            if kept:
+                want_act[want] = True
+        np.testing.assert_array_equal(oracle.active_experts(r, E), want_act)
+
+
+def test_cross_layer_routing_single_layer_is_layer_routing():
+    """With one layer the generator's decision is the layer's own routing of the same input."""
+    spec = _small_spec()
+    x = synth.make_tokens(spec, 30, seed=21)
+    w = synth.make_layer(spec, seed=21, keep_rate=0.5)
+    (g,) = oracle.route_layers(x, w["w_router"][None], w["w_mask"][None], spec.top_k, segment_len=4)
+    r = oracle.route(x, w["w_router"], w["w_mask"], spec.top_k, segment_len=4)
+    for f in ("topk_id", "g", "keep", "ghat", "nkeep", "lreg"):
+        np.testing.assert_array_equal(getattr(g, f), getattr(r, f))
