@@ -64,6 +64,11 @@ DEFAULT_WORKLOAD = "mixtral-prefill"
 # supplementary points measured after the headline in the default run
 EXTRA_POINTS = ["mixtral-decode1", "mixtral-decode8", "mixtral-decode64", "dsv2lite-decode1",
                 "fine-decode32"]
+# cross-layer routing (the mask generator) points: name -> (layer spec, MoE layers, tokens,
+# segment length, keep rate).  The Stepped-MoE shape: 44 MoE layers of 212 experts (K = 16,
+# D = 1536), one decision per 16-token segment, over an 8192-token context or one decode token.
+GEN_POINTS = {"gen-fine44-prefill": ("fine", 44, 8192, 16, 0.5),
+              "gen-fine44-decode": ("fine", 44, 1, 16, 0.5)}
 # every workload, one JSON line each (--sweep)
 SWEEP = ["mixtral-prefill", "mixtral-prefill-high", "mixtral-prefill-plain", "mixtral-decode1",
          "mixtral-decode1-high", "mixtral-decode8", "mixtral-decode64", "dsv2lite-prefill",
@@ -218,6 +223,71 @@ def layer_work(spec, T, st, tc_path=True, joint=False):
 
 
 TENSOR_STAGES = {"tc_gateup", "tc_down", "tc_router", "tc_shared_gateup", "tc_shared_down"}
+
+
+def gen_work(spec, L: int, T: int, S: int) -> dict:
+    """Algorithmic work of one cross-layer routing call: the generator matrix [L*2E][D] read
+    once, the segment leaders' rows of z read once, every layer's routing arrays written once
+    (topk_id, gate, mask_logit, ghat: 4 B, keep: 1 B per slot; n_keep, lreg: 4 B per token;
+    the active bitsets), and the logit GEMM's FLOPs."""
+    es = 2 if spec.storage == "bf16" else 4
+    D, E, K = spec.d_model, spec.n_experts, spec.top_k
+    Tr = -(-T // max(1, S))
+    cols = L * 2 * E
+    bytes_ = (cols * D * es + Tr * D * es + L * T * K * (4 * 4 + 1) + L * T * 8
+              + L * ((E + 31) // 32) * 4)
+    return {"bytes": bytes_, "flops": 2 * Tr * D * cols}
+
+
+def gen_point(torch, name, steps, warmup, device, peaks):
+    """Time beam_gen_route on one GPU: each timed call has its own event pair, and between
+    calls, outside the timed region, a 256 MB buffer is written and then read, so the L2 holds
+    none of the call's data and no dirty lines whose write-back would land in the next call."""
+    import synth
+    from dynamic_expert_routing_b200 import BeamGenerator
+    spec_name, L, T, S, keep = GEN_POINTS[name]
+    spec = synth.SPECS[spec_name].with_(segment_len=S)
+    wr, wm = synth.make_generator(spec, L, seed=0, keep_rate=keep)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)
+    with torch.cuda.stream(torch.cuda.Stream(device)):
+        gen = BeamGenerator(wr.to(device), wm.to(device), spec.top_k, max_tokens=T, segment_len=S)
+        del wr, wm
+        z = synth.make_tokens(spec, T, seed=1, device=device)
+        out = gen.route(z)
+        for _ in range(warmup):
+            gen.route(z, out=out)
+        st = torch.cuda.current_stream()
+        pairs = []
+        sink = torch.empty((), dtype=torch.float32, device=device)
+        for _ in range(steps):
+            flush.zero_()
+            torch.sum(flush, dim=0, out=sink)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            gen.route(z, out=out)
+            b.record(st)
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        gen.sync()
+        ms = sum(a.elapsed_time(b) for a, b in pairs) / steps
+        keep_sum = int(out["keep"].sum().item())
+        act = out["active"].cpu().numpy().astype("int64") & 0xffffffff
+        n_act = [sum(bin(int(w)).count("1") for w in row) for row in act]
+        gen.close()
+    del flush
+    work = gen_work(spec, L, T, S)
+    t_hbm = work["bytes"] / (peaks["hbm"] * 1e9)
+    t_tc = work["flops"] / (peaks["tc"] * 1e12)
+    return dict(workload=name, metric="cross-layer routing tokens/s", unit="tokens/s",
+                layers=L, tokens=T, segment_len=S, keep_rate=keep,
+                value=round(T / (ms * 1e-3), 2), ms_per_step=round(ms, 5),
+                layer_roofline_frac=round(max(t_hbm, t_tc) / (ms * 1e-3), 4),
+                bound="hbm" if t_hbm >= t_tc else "tensor",
+                algorithmic_bytes=work["bytes"], algorithmic_flops=work["flops"],
+                avg_k=round(keep_sum / (L * T), 4),
+                mean_active_experts=round(sum(n_act) / L, 2),
+                l2="flushed (256 MB written, then read) between timed calls")
 
 
 def roofline_for(stage, work, ms_per_launch, peaks, workload):
@@ -447,11 +517,15 @@ def _run_ours(args):
     torch.cuda.empty_cache()
 
     points = []
+    gen_points = []
     if not args.no_points:
         for p in EXTRA_POINTS:
             if p == name:
                 continue
             points.append(point(torch, dist, p, max(10, args.steps), args.warmup, world, device, peaks))
+        if world == 1:
+            for p in GEN_POINTS:
+                gen_points.append(gen_point(torch, p, max(10, args.steps), args.warmup, device, peaks))
 
     if rank == 0:
         line = {
@@ -490,6 +564,7 @@ def _run_ours(args):
             "clocks": clocks,
             "cpu_baseline": cpu,
             "points": points,
+            "gen_points": gen_points,
             "peaks": peaks,
         }
         print(json.dumps(line), flush=True)
@@ -514,6 +589,8 @@ def run_sweep(args):
         r["metric"] = "masked MoE-layer tokens/s"
         r["unit"] = "tokens/s"
         print(json.dumps(r), flush=True)
+    for name in GEN_POINTS:
+        print(json.dumps(gen_point(torch, name, args.steps, args.warmup, device, peaks)), flush=True)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)

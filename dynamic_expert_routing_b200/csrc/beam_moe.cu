@@ -682,6 +682,32 @@ static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3
     return launch_ex(h, stage, false, kernel, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
+// Router logits on the CUDA cores, L[r][j] (leading dimension ld) for ncols columns of the
+// repacked matrix w [ncols][D]: one CTA per column, or one warp per column from
+// kGemvWarpCols columns on (the choice depends on the column count alone, so a one-layer
+// generator and the layer with the same matrices compute the same bits).
+constexpr int kGemvWarpCols = 2048;
+
+template <typename T>
+static cudaError_t launch_router_gemv(beam_moe* h, const T* x, int S, int Tr, int D, const T* w,
+                                      int ncols, int ld, float* L, cudaStream_t st)
+{
+    if (ncols >= kGemvWarpCols) {
+        const dim3 grid1(ceil_div(ncols, 8), Tr);
+        if (Tr == 1)
+            return launch(h, ST_ROUTER_LOGITS, router_gemv_warp_kernel<T, 1>, grid1, dim3(256), 0,
+                          st, x, S, Tr, D, w, ncols, ld, L);
+        if (Tr <= 4)
+            return launch(h, ST_ROUTER_LOGITS, router_gemv_warp_kernel<T, 4>,
+                          dim3(ceil_div(ncols, 8), 1), dim3(256), 0, st, x, S, Tr, D, w, ncols, ld, L);
+        return launch(h, ST_ROUTER_LOGITS, router_gemv_warp_kernel<T, kGemvRows>,
+                      dim3(ceil_div(ncols, 8), ceil_div(Tr, kGemvRows)), dim3(256), 0, st, x, S,
+                      Tr, D, w, ncols, ld, L);
+    }
+    return launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>, dim3(ncols, ceil_div(Tr, kGemvRows)),
+                  dim3(256), 0, st, x, S, Tr, D, w, ncols, ld, L);
+}
+
 template <int EPL>
 static cudaError_t launch_select(beam_moe* h, int Tr, int T, int mask_off, int splits,
                                  long long split_stride, cudaStream_t st)
@@ -890,9 +916,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
     } else {
-        BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
-                         dim3(h->n2E, ceil_div(Tr, kGemvRows)),
-                         dim3(256), 0, st, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->ldL, h->L));
+        BEAM_CUDA(launch_router_gemv<T>(h, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->ldL, h->L, st));
     }
     // 2-3. routing decision and compaction.  Small batches (one 32-token chunk) run them as one
     // single-CTA kernel; larger ones as select -> bit planes -> scan -> scatter + gather.
@@ -1110,9 +1134,7 @@ static beam_status_t route_noalloc_impl(beam_moe* h, const T* x, int T_, int32_t
     float* L = reinterpret_cast<float*>(scratch);
     int* nkeep = reinterpret_cast<int*>(scratch + l_bytes);
     float* lreg = reinterpret_cast<float*>(scratch + l_bytes + (size_t)T_ * sizeof(int));
-    BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
-                     dim3(h->n2E, ceil_div(Tr, kGemvRows)),
-                     dim3(256), 0, st, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, h->n2E, L));
+    BEAM_CUDA(launch_router_gemv<T>(h, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, h->n2E, L, st));
     cudaError_t e;
     switch ((h->E + 31) / 32) {
         case 1: e = launch_select_into<1>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
@@ -1285,9 +1307,7 @@ static beam_status_t gen_route_impl(beam_gen* g, const T* z, int T_, const beam_
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * splits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
     } else {
-        BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_gemv_kernel<T>,
-                         dim3(g->nlog, ceil_div(Tr, kGemvRows)), dim3(256), 0, st, z, S, Tr, D,
-                         (const T*)g->wgen, g->nlog, g->ldG, g->G));
+        BEAM_CUDA(launch_router_gemv<T>(h, z, S, Tr, D, (const T*)g->wgen, g->nlog, g->ldG, g->G, st));
     }
     cudaError_t e;
     switch ((E + 31) / 32) {

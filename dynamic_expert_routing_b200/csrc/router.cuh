@@ -74,6 +74,70 @@ router_gemv_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
     pdl_launch_dependents();
 }
 
+// The same logits for many columns (a cross-layer generator has L*2E of them, where one CTA
+// per column would launch thousands of CTAs of a few hundred bytes each): one warp per column
+// j and block of ROWS routed rows (1 for a single routed row, so that the warp keeps one
+// partial and few registers); the lanes split the D-long weight row with 16-byte loads, each
+// lane keeps one partial per row, and a warp butterfly reduces them.
+template <typename TW, int ROWS>
+__global__ void __launch_bounds__(256)
+router_gemv_warp_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
+                        const TW* __restrict__ wrm, int n2E, int ldL, float* __restrict__ L)
+{
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = blockIdx.x * 8 + warp;
+    const int row0 = blockIdx.y * ROWS;
+    const int nrows = min(ROWS, Tr - row0);
+    if (j < n2E) {
+        const size_t xstride = (size_t)(seg > 1 ? seg : 1) * D;
+        constexpr int VN = Vec<TW>::N;
+        float acc[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) acc[r] = 0.f;
+        const TW* wrow = wrm + (size_t)j * D;
+        const TW* x0 = x + (size_t)row0 * xstride;
+        // kU weight vectors per lane are loaded before any is used, so a warp has kU 512-byte
+        // requests in flight instead of one load round trip per vector
+        constexpr int kU = 4;
+        for (int d0 = lane * VN; d0 < D; d0 += kU * 32 * VN) {
+            uint4 wv[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int d = d0 + u * 32 * VN;
+                wv[u] = d < D ? ldg_stream(wrow + d) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int d = d0 + u * 32 * VN;
+                if (d < D) {
+                    float w[VN];
+                    Vec<TW>::widen(wv[u], w);
+#pragma unroll
+                    for (int r = 0; r < ROWS; ++r) {
+                        if (r < nrows) {
+                            float xv[VN];
+                            Vec<TW>::widen(__ldg(reinterpret_cast<const uint4*>(x0 + r * xstride + d)), xv);
+                            float s = 0.f;
+#pragma unroll
+                            for (int v = 0; v < VN; ++v) s = fmaf(w[v], xv[v], s);
+                            acc[r] += s;
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) {
+            if (r < nrows) {
+                const float s = warp_sum(acc[r]);
+                if (lane == 0) L[(size_t)(row0 + r) * ldL + j] = s;
+            }
+        }
+    }
+    pdl_launch_dependents();
+}
+
 // ---------------------------------------------------------------- Top-K, softmax, mask
 // One warp per routed row i (row i of L, leading dimension ldL: router logits in columns
 // [0, E), mask logits in [E, 2E); `splits` K-split slices split_stride floats apart, added in
@@ -209,16 +273,46 @@ route_select_kernel(const float* __restrict__ L, int ldL, int splits, long long 
         const int S = seg > 1 ? seg : 1;
         const int t0 = i * S, t1 = min(T, t0 + S);
         const size_t lo = (size_t)layer * out_ls, lt = (size_t)layer * tok_ls;
-        for (int t = t0; t < t1; ++t) {
+        if (S == 1) {
             if (lane < K) {
-                size_t o = lo + (size_t)t * K + lane;
+                const size_t o = lo + (size_t)t0 * K + lane;
                 topk_id[o] = d.id;
                 gate[o] = d.g;
                 mlogit[o] = d.l;
                 keep[o] = d.keep ? 1 : 0;
                 ghat[o] = d.ghat;
             }
-            if (lane == 0) { nkeep_tok[lt + t] = d.nkeep; lreg_tok[lt + t] = d.lreg; }
+            if (lane == 0) { nkeep_tok[lt + t0] = d.nkeep; lreg_tok[lt + t0] = d.lreg; }
+        } else {
+            // the segment's rows [t0, t1) x K are one contiguous range of each output, holding
+            // the same K slots per token: lane q writes elements q, q + 32, ..., taking slot
+            // (element mod K) from the lane that owns it, so every store is a whole-warp run
+            const int n = (t1 - t0) * K;
+            const size_t base = lo + (size_t)t0 * K;
+            // slot of element q = q mod K, carried from one pass to the next (no division)
+            const int step = 32 % K;
+            int src = lane % K;
+            for (int q0 = 0; q0 < n; q0 += 32) {   // the same trip count on every lane
+                const int q = q0 + lane;
+                const int id = __shfl_sync(0xffffffffu, d.id, src);
+                const float g = __shfl_sync(0xffffffffu, d.g, src);
+                const float l = __shfl_sync(0xffffffffu, d.l, src);
+                const int kp = __shfl_sync(0xffffffffu, d.keep ? 1 : 0, src);
+                const float gh = __shfl_sync(0xffffffffu, d.ghat, src);
+                if (q < n) {
+                    topk_id[base + q] = id;
+                    gate[base + q] = g;
+                    mlogit[base + q] = l;
+                    keep[base + q] = (uint8_t)kp;
+                    ghat[base + q] = gh;
+                }
+                src += step;
+                if (src >= K) src -= K;
+            }
+            for (int t = t0 + lane; t < t1; t += 32) {
+                nkeep_tok[lt + t] = d.nkeep;
+                lreg_tok[lt + t] = d.lreg;
+            }
         }
         if (active && d.keep) atomicOr(&s_act[d.id >> 5], 1u << (d.id & 31));
     }

@@ -105,3 +105,16 @@ def test_spread_sample_covers_the_batch():
     assert (s[1:] > s[:-1]).all()
     assert list(bench.spread_sample(5, 100)) == [0, 1, 2, 3, 4]
     assert list(bench.spread_sample(64, 1)) == [0]
+
+
+def test_gen_work_counts_generator_matrix_leaders_and_outputs():
+    """One cross-layer routing call: the [L*2E][D] matrix and the leaders' rows read once, the
+    per-layer routing arrays written once, 2*Tr*D*L*2E FLOPs."""
+    spec = synth.SPECS["fine"]                  # D 1536, E 212, K 16, bf16
+    w = bench.gen_work(spec, 44, 8192, 16)
+    cols = 44 * 2 * 212
+    assert w["flops"] == 2 * 512 * 1536 * cols
+    assert w["bytes"] == (cols * 1536 * 2 + 512 * 1536 * 2 + 44 * 8192 * 16 * 17 + 44 * 8192 * 8
+                          + 44 * 7 * 4)
+    one = bench.gen_work(spec, 44, 1, 16)        # one decode token: one leader row
+    assert one["flops"] == 2 * 1536 * cols

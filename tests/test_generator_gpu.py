@@ -75,7 +75,10 @@ GEN_CASES = [
     ("mixtral-l4", synth.SPECS["mixtral"], 4, 200),
     ("dsv2lite-l2", synth.SPECS["dsv2lite"], 2, 130),
     ("tiny-fp32-l2", synth.SPECS["tiny"], 2, 64),
+    # 5 layers x 424 logit columns: one warp per column, with 1, 4 and 16 rows per warp
     ("fine-decode1", synth.SPECS["fine"], 5, 1),
+    ("fine-l5-t3", synth.SPECS["fine"], 5, 3),
+    ("fine-l5-t40", synth.SPECS["fine"], 5, 40),
 ]
 
 
