@@ -858,9 +858,15 @@ template <typename TR, typename TS>
 static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, const float* ghat,
                                   int T_, float* y, cudaStream_t st)
 {
-    // few tokens: split each token's columns over several CTAs so the combine spans the SMs
-    const dim3 cgrid(T_, T_ < h->num_sms ? ceil_div(h->D / 4, 256) : 1);
-    return launch(h, ST_COMBINE, combine_kernel<TR, TS>, cgrid, dim3(256), 0, st,
+    // few tokens: split each token's columns over several CTAs so the combine spans the SMs;
+    // otherwise one CTA per token whose threads take the row's float4 columns in equal passes
+    // (D/4 = 384: 192 threads x 2 rather than 256 + 128)
+    const int d4 = h->D / 4;
+    const bool split_cols = T_ < h->num_sms;
+    const int passes = ceil_div(d4, 256);
+    const int nthr = split_cols ? 256 : std::min(256, ceil_div(ceil_div(d4, passes), 32) * 32);
+    const dim3 cgrid(T_, split_cols ? ceil_div(d4, 256) : 1);
+    return launch(h, ST_COMBINE, combine_kernel<TR, TS>, cgrid, dim3(nthr), 0, st,
                   (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
                   (const int*)h->inv, ghat, T_, h->K, h->D, y);
 }
