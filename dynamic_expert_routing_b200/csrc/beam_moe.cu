@@ -1345,6 +1345,11 @@ beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, in
     if (T == 0) return BEAM_OK;
     if (!x || !topk_id || !gate || !mask_logit || !keep || !ghat)
         return fail(BEAM_ERR_INVALID_ARG, "x and every output pointer must be non-NULL");
+    if ((reinterpret_cast<uintptr_t>(topk_id) | reinterpret_cast<uintptr_t>(gate) |
+         reinterpret_cast<uintptr_t>(mask_logit) | reinterpret_cast<uintptr_t>(ghat)) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "topk_id, gate, mask_logit and ghat must be 4-byte aligned");
+    if (reinterpret_cast<uintptr_t>(x) & 15)
+        return fail(BEAM_ERR_INVALID_ARG, "x must be 16-byte aligned");
     const long long Tr = (T + h->S - 1) / h->S;
     const long long need = ((Tr * h->n2E * 4 + 255) & ~255LL) + 8LL * T;
     if (need > (long long)BEAM_ROUTE_NOALLOC_SCRATCH_BYTES)
@@ -1397,6 +1402,11 @@ beam_status_t beam_gen_route(beam_gen_t* g, const void* z, int32_t T, const beam
         !out->n_keep || !out->lreg)
         return fail(BEAM_ERR_INVALID_ARG, "z and every routing array except active must be non-NULL");
     if (reinterpret_cast<uintptr_t>(z) & 15) return fail(BEAM_ERR_INVALID_ARG, "z must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(out->topk_id) | reinterpret_cast<uintptr_t>(out->gate) |
+         reinterpret_cast<uintptr_t>(out->mask_logit) | reinterpret_cast<uintptr_t>(out->ghat) |
+         reinterpret_cast<uintptr_t>(out->n_keep) | reinterpret_cast<uintptr_t>(out->lreg) |
+         reinterpret_cast<uintptr_t>(out->active)) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "the 32-bit routing arrays must be 4-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
     if (h->cfg.dtype == BEAM_DTYPE_BF16)

@@ -180,7 +180,7 @@ int64_t beam_moe_launch_count(const beam_moe_t *h);
  * Routing only, without allocating: Steps 1-3 (Top-K, K-way softmax, mask) for x_dev[T][D]
  * into caller-provided device arrays topk_id[T][K] int32, gate[T][K] f32, mask_logit[T][K]
  * f32, keep[T][K] uint8 and ghat[T][K] f32 (same values and layout as beam_moe_forward
- * produces), enqueued on `stream`.  The BEAM pages have no counterpart to this call; it exists
+ * produces; the 32-bit arrays 4-byte aligned, x 16-byte aligned), enqueued on `stream`.  The BEAM pages have no counterpart to this call; it exists
  * for callers that cannot allocate device memory when they route, e.g. a serving engine that
  * reserves all free device memory for its own pools up front, so any later cudaMalloc fails.
  * The call allocates nothing: its only scratch (the router logits and per-token statistics)
@@ -269,8 +269,9 @@ beam_status_t beam_gen_create(const beam_gen_config_t *cfg, const void *w_router
  * NULL) must hold L*T*K (or L*T) elements; enqueued on `stream` without synchronising.  bf16
  * generators with d_model a multiple of 64 compute the logits on the tensor cores (tcgen05),
  * others with a CUDA-core GEMV; then one warp per (segment, layer) takes the decision.
- * flags: 0 or BEAM_MASK_OFF (every Top-K slot kept).  T = 0 is a no-op.  Returns
- * BEAM_ERR_TIMEOUT (from beam_gen_sync) if a bounded device wait ran out.
+ * flags: 0 or BEAM_MASK_OFF (every Top-K slot kept).  T = 0 is a no-op.  z must be 16-byte
+ * aligned and the 32-bit arrays 4-byte aligned (else BEAM_ERR_INVALID_ARG).  A bounded device
+ * wait that ran out is reported by beam_gen_sync (BEAM_ERR_TIMEOUT).
  */
 beam_status_t beam_gen_route(beam_gen_t *g, const void *z_dev, int32_t T,
                              const beam_routing_t *out, uint32_t flags, void *stream);
@@ -290,7 +291,9 @@ void beam_gen_destroy(beam_gen_t *g);
  * describes the given routing.  flags: BEAM_PATH_STREAM / BEAM_PATH_TENSOR / BEAM_NO_GRAPH
  * (BEAM_MASK_OFF and BEAM_FUSED_DECODE are rejected: the mask is part of the routing).  The
  * graph replay key includes the routing pointers.  The routing arrays must stay valid until
- * the stream reaches the end of the call's work.
+ * the stream reaches the end of the call's work, and, for beam_moe_get_routing, until that
+ * call.  Alignment: topk_id 4 bytes (16 when top_k is 4, 8 or 16), keep top_k bytes when
+ * top_k is 4, 8 or 16, ghat / n_keep / lreg 4 bytes.
  */
 beam_status_t beam_moe_forward_routed(beam_moe_t *h, const void *x_dev, int32_t T,
                                       const beam_routing_t *r, float *y_dev, uint32_t flags,

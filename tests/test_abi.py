@@ -13,7 +13,7 @@ HEADER = os.path.join(ROOT, "include", "beam_moe.h")
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(beam_moe_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(beam_(?:moe|gen)_\w+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -25,7 +25,8 @@ def lib():
 
 def test_header_declares_the_named_calls():
     names = _declared_functions()
-    for n in ("beam_moe_create", "beam_moe_forward", "beam_moe_stats"):
+    for n in ("beam_moe_create", "beam_moe_forward", "beam_moe_stats", "beam_gen_create",
+              "beam_gen_route", "beam_moe_forward_routed"):
         assert n in names
 
 
@@ -65,6 +66,38 @@ def test_null_handle_calls(lib):
     lib.beam_moe_destroy(None)
     assert lib.beam_moe_wait_selftest(0, None) == BEAM_ERR_INVALID_ARG
     assert b"sm_100a" in lib.beam_moe_version()
+
+
+def test_invalid_generator_config_is_rejected_without_cuda(lib):
+    from dynamic_expert_routing_b200._lib import BeamGenConfig, BEAM_ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    w = ctypes.c_void_p(16)
+    bad = [
+        BeamGenConfig(100, 4, 8, 2, 1, 0, 64),     # d_model not a multiple of 64 (bf16)
+        BeamGenConfig(256, 0, 8, 2, 1, 0, 64),     # no layers
+        BeamGenConfig(256, 513, 8, 2, 1, 0, 64),   # too many layers
+        BeamGenConfig(256, 4, 0, 2, 1, 0, 64),     # no experts
+        BeamGenConfig(256, 4, 8, 9, 1, 0, 64),     # K > E
+        BeamGenConfig(256, 4, 8, 2, 7, 0, 64),     # unknown dtype
+        BeamGenConfig(256, 4, 8, 2, 1, -1, 64),    # negative segment length
+        BeamGenConfig(256, 4, 8, 2, 1, 0, 0),      # max_tokens 0
+    ]
+    for cfg in bad:
+        assert lib.beam_gen_create(ctypes.byref(cfg), w, w, None, ctypes.byref(h)) == BEAM_ERR_INVALID_ARG
+        assert lib.beam_moe_last_error()
+        assert not h.value
+    good = BeamGenConfig(256, 4, 8, 2, 1, 0, 64)
+    assert lib.beam_gen_create(ctypes.byref(good), None, w, None, ctypes.byref(h)) == BEAM_ERR_INVALID_ARG
+    assert lib.beam_gen_create(ctypes.byref(good), w, w, None, None) == BEAM_ERR_INVALID_ARG
+
+
+def test_generator_and_routed_forward_null_handles(lib):
+    from dynamic_expert_routing_b200._lib import BeamRouting, BEAM_ERR_INVALID_ARG
+    r = BeamRouting()
+    assert lib.beam_gen_route(None, None, 1, ctypes.byref(r), 0, None) == BEAM_ERR_INVALID_ARG
+    assert lib.beam_gen_sync(None) == BEAM_ERR_INVALID_ARG
+    lib.beam_gen_destroy(None)
+    assert lib.beam_moe_forward_routed(None, None, 1, ctypes.byref(r), None, 0, None) == BEAM_ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(tmp_path):
