@@ -45,8 +45,10 @@ def _load():
         lib.oracle_compact.argtypes = [I, I, I, P, P, P, P, P, P]
         lib.oracle_layer.argtypes = [I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, I, P, P]
         lib.oracle_expert.argtypes = [I, I, I, P, P, P, P, I, P]
+        lib.oracle_route_backward.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P,
+                                              ctypes.c_double, I, P, P, P, P, P, P, P]
         for f in (lib.oracle_route, lib.oracle_stats, lib.oracle_compact, lib.oracle_layer,
-                  lib.oracle_expert, lib.oracle_num_threads):
+                  lib.oracle_expert, lib.oracle_route_backward, lib.oracle_num_threads):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -207,4 +209,51 @@ def expert(x_vec, wg, wu, wd, e: int = 0) -> np.ndarray:
     rc = lib.oracle_expert(D, F, dt, _p(xv), _p(wga), _p(wua), _p(wda), int(e), _p(out))
     if rc != 0:
         raise RuntimeError(f"oracle_expert failed with code {rc}")
+    return out
+
+
+@dataclass
+class RouteGrad:
+    s: np.ndarray      # float64 [T][K]: <dy_t, E_i(x_t)> of every Top-K slot (= dL/dg_hat)
+    d_r: np.ndarray    # float64 [T][K]: dL/d(router logit) of slot k at routed rows, else 0
+    d_l: np.ndarray    # float64 [T][K]: dL/d(mask logit) of slot k at routed rows, else 0
+    dw_r: np.ndarray   # float64 [D][E] (None when only some rows were asked for)
+    dw_m: np.ndarray   # float64 [D][E] (None when only some rows were asked for)
+    dx: np.ndarray     # float64 [T][D]: the routing's share of dL/dx (0 off the routed rows)
+
+
+def route_backward(x, weights: dict, routing: Routing, dy, reg_scale: float = 0.0,
+                   segment_len: int = 0, rows=None) -> RouteGrad:
+    """Training-side gradient of the router and the mask router under the straight-through
+    estimator, plus the L_reg term (BEAM article on aitrends.kr, training paragraph; ai-feeds
+    summary, Method, binarisation and straight-through estimator).  dy: float64 [T][D] upstream
+    gradient of the output; reg_scale: dL/dL_reg with L_reg the mean over tokens.  The experts
+    of every Top-K slot are evaluated (training runs them all; the mask only scales gates).
+    `rows` (token indices of routed rows) restricts the work to those rows and skips dW."""
+    lib = _load()
+    xa, dt = _host(x)
+    T, D = xa.shape
+    wr, _ = _host(weights["w_router"])
+    wm, _ = _host(weights["w_mask"])
+    wg, _ = _host(weights["w_gate"])
+    wu, _ = _host(weights["w_up"])
+    wd, _ = _host(weights["w_down"])
+    E, F, _ = wg.shape
+    K = routing.topk_id.shape[1]
+    dya = np.ascontiguousarray(dy, np.float64)
+    if dya.shape != (T, D):
+        raise ValueError("dy must be [T][D]")
+    sel = None if rows is None else np.ascontiguousarray(rows, np.int32)
+    out = RouteGrad(np.zeros((T, K)), np.zeros((T, K)), np.zeros((T, K)),
+                    np.zeros((D, E)), np.zeros((D, E)), np.zeros((T, D)))
+    rc = lib.oracle_route_backward(
+        T, D, E, K, F, dt, int(segment_len), _p(xa), _p(wr), _p(wm), _p(wg), _p(wu), _p(wd),
+        _p(np.ascontiguousarray(routing.topk_id)), _p(np.ascontiguousarray(routing.g)),
+        _p(np.ascontiguousarray(routing.mask_logit)), _p(dya), float(reg_scale),
+        -1 if sel is None else int(sel.shape[0]), _p(sel), _p(out.s), _p(out.d_r), _p(out.d_l),
+        _p(out.dw_r), _p(out.dw_m), _p(out.dx))
+    if rc != 0:
+        raise RuntimeError(f"oracle_route_backward failed with code {rc}")
+    if sel is not None:
+        out.dw_r = out.dw_m = None
     return out

@@ -286,3 +286,111 @@ int oracle_layer(int T, int D, int E, int K, int F, int S_sh, int Fs, int dtype,
     }
     return bad ? 1 : 0;
 }
+
+/*
+ * Training-side gradient of the routing ([BEAM-KR] training paragraph: the loss
+ * L = L_lm + alpha L_bal + beta L_reg with L_reg = (1/K) sum_{i in TK} |m_hat_i|, and the
+ * straight-through estimator that lets the binary mask's gradient flow to m_hat; [BEAM-CN]
+ * Method, "二值化与直通估计器": a step function forward, the continuous version's gradient
+ * backward).  Readings: L_bal is not defined on the pages and is left out; L_reg is the mean
+ * over tokens of the per-token term (as in the forward's statistics), so with reg_scale =
+ * dL/dL_reg every (token, slot) adds reg_scale / (T K) to dL/dm_hat; the straight-through
+ * estimator sets dm/dm_hat = 1; during training every Top-K expert is evaluated (the mask's
+ * gradient needs E_i(x) of masked slots too) while the output uses g_hat = g * m.
+ *
+ * Given dy = dL_lm/dy [T][D], per token t and Top-K slot k (expert i):
+ *   s_tk   = <dy_t, E_i(x_t)>                        (= dL/dg_hat_tk)
+ *   dg_k   = sum over the routed row's tokens of s_tk * m_k
+ *   dmh_k  = sum over the routed row's tokens of (s_tk * g_k + reg_scale / (T K))
+ *   d_l_k  = dmh_k * sigmoid(l_k) (1 - sigmoid(l_k))       (mask logit)
+ *   d_r_k  = g_k (dg_k - sum_j g_j dg_j)                  (softmax over the K)
+ * with m_k = (l_k >= 0); logits outside TK get no gradient (the Top-K selection is piecewise
+ * constant).  The routed row of token t is t itself, or its segment's first token ([SMoE]):
+ * the segment's tokens share one decision, so their terms are summed at the leader.  Then
+ *   dW_r[d][i] = sum over routed rows of x[row][d] d_r_k;  dW_m likewise with d_l_k
+ *   dx[row][d] = sum_k d_r_k W_r[d][i_k] + d_l_k W_m[d][i_k]   (the routing's share of dx;
+ *                rows that are not routed rows get 0)
+ * s, d_r and d_l are [T][K] (d_r, d_l at routed rows, 0 elsewhere); dw_r, dw_m [D][E];
+ * dx [T][D].  sel == NULL: every routed row and dW; otherwise only the n_sel routed rows
+ * listed in sel (token indices of routed rows) and dw_r / dw_m are left untouched.
+ * topk_id, g and mlogit are oracle_route's outputs (already carrying the leader's decision).
+ */
+int oracle_route_backward(int T, int D, int E, int K, int F, int dtype, int seg,
+                          const void *x, const void *w_router, const void *w_mask,
+                          const void *wg, const void *wu, const void *wd,
+                          const int32_t *topk_id, const double *g, const double *mlogit,
+                          const double *dy, double reg_scale, int n_sel, const int32_t *sel,
+                          double *s_out, double *d_r, double *d_l,
+                          double *dw_r, double *dw_m, double *dx)
+{
+    if (T < 0 || D <= 0 || E <= 0 || K <= 0 || K > E || K > 256 || F <= 0) return 1;
+    const int S = seg > 1 ? seg : 1;
+    const int n_rows = (T + S - 1) / S;
+    const int n = sel ? n_sel : n_rows;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int q = 0; q < n; ++q) {
+        const int src = sel ? sel[q] : q * S;
+        double *xv = (double *)malloc(sizeof(double) * (size_t)D);
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        double *o = (double *)malloc(sizeof(double) * (size_t)D);
+        double dg[256], dmh[256];
+        if (!xv || !h || !o || src < 0 || src >= T || src % S) {
+            bad = 1;
+            free(xv); free(h); free(o);
+            continue;
+        }
+        for (int k = 0; k < K; ++k) dg[k] = dmh[k] = 0.0;
+        const int t_end = src + S < T ? src + S : T;
+        for (int t = src; t < t_end; ++t) {
+            for (int d = 0; d < D; ++d) xv[d] = load_elem(x, dtype, (size_t)t * D + d);
+            for (int k = 0; k < K; ++k) {
+                const size_t sl = (size_t)t * K + k;
+                const int e = topk_id[sl];
+                expert_ffn(D, F, dtype, xv, wg, wu, wd, (size_t)e * F * D, (size_t)e * D * F, h, o);
+                double s = 0.0;
+                for (int d = 0; d < D; ++d) s += dy[(size_t)t * D + d] * o[d];
+                s_out[sl] = s;
+                const double m = mlogit[sl] >= 0.0 ? 1.0 : 0.0;
+                dg[k] += s * m;
+                dmh[k] += s * g[sl] + reg_scale / ((double)T * (double)K);
+                if (t != src) { d_r[sl] = 0.0; d_l[sl] = 0.0; }
+            }
+        }
+        double c = 0.0;
+        for (int k = 0; k < K; ++k) c += g[(size_t)src * K + k] * dg[k];
+        for (int k = 0; k < K; ++k) {
+            const size_t sl = (size_t)src * K + k;
+            const double sg = sigmoid(mlogit[sl]);
+            d_l[sl] = dmh[k] * sg * (1.0 - sg);
+            d_r[sl] = g[sl] * (dg[k] - c);
+        }
+        for (int d = 0; d < D; ++d) {
+            double a = 0.0;
+            for (int k = 0; k < K; ++k) {
+                const size_t sl = (size_t)src * K + k;
+                const int e = topk_id[sl];
+                a += d_r[sl] * load_elem(w_router, dtype, (size_t)d * E + e) +
+                     d_l[sl] * load_elem(w_mask, dtype, (size_t)d * E + e);
+            }
+            dx[(size_t)src * D + d] = a;
+        }
+        for (int t = src + 1; t < t_end; ++t)
+            for (int d = 0; d < D; ++d) dx[(size_t)t * D + d] = 0.0;
+        free(xv); free(h); free(o);
+    }
+    if (bad) return 2;
+    if (sel) return 0;
+    for (size_t i = 0; i < (size_t)D * E; ++i) dw_r[i] = dw_m[i] = 0.0;
+    for (int src = 0; src < T; src += S)
+        for (int k = 0; k < K; ++k) {
+            const size_t sl = (size_t)src * K + k;
+            const int e = topk_id[sl];
+            for (int d = 0; d < D; ++d) {
+                const double xd = load_elem(x, dtype, (size_t)src * D + d);
+                dw_r[(size_t)d * E + e] += xd * d_r[sl];
+                dw_m[(size_t)d * E + e] += xd * d_l[sl];
+            }
+        }
+    return 0;
+}
