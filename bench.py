@@ -33,6 +33,9 @@ WORKLOADS = {
     # device) for ncu captures of the same kernels
     "profile-prefill": ("mixtral", 1024, 0.5, {"n_experts": 4}),
     "profile-decode": ("mixtral", 2, None, {"n_experts": 4}),
+    # reduced Mixtral-like training step (4 experts, 2048 tokens) for ncu captures of the
+    # routing-gradient kernels
+    "profile-train": ("mixtral", 2048, 0.5, {"n_experts": 4}),
     # reduced fine-grained prefill (2048 tokens) for ncu captures of the small-K down GEMM
     "profile-fine": ("fine", 2048, 0.5),
     "mixtral-prefill": ("mixtral", 4096, 0.5),
@@ -69,6 +72,11 @@ EXTRA_POINTS = ["mixtral-decode1", "mixtral-decode8", "mixtral-decode64", "dsv2l
 # D = 1536), one decision per 16-token segment, over an 8192-token context or one decode token.
 GEN_POINTS = {"gen-fine44-prefill": ("fine", 44, 8192, 16, 0.5),
               "gen-fine44-decode": ("fine", 44, 1, 16, 0.5)}
+# training-side points (BEAM_TRAIN forward, then the routing gradient): name -> workload
+TRAIN_POINTS = {"train-mixtral-prefill": "mixtral-prefill",
+                "train-dsv2lite-prefill": "dsv2lite-prefill",
+                "train-fine-seg16-prefill": "fine-seg16-prefill",
+                "train-profile": "profile-train"}
 # every workload, one JSON line each (--sweep)
 SWEEP = ["mixtral-prefill", "mixtral-prefill-high", "mixtral-prefill-plain", "mixtral-decode1",
          "mixtral-decode1-high", "mixtral-decode8", "mixtral-decode64", "dsv2lite-prefill",
@@ -288,6 +296,86 @@ def gen_point(torch, name, steps, warmup, device, peaks):
                 avg_k=round(keep_sum / (L * T), 4),
                 mean_active_experts=round(sum(n_act) / L, 2),
                 l2="flushed (256 MB written, then read) between timed calls")
+
+
+def grad_work(spec, T, tc_path=True) -> dict:
+    """Algorithmic bytes of the routing gradient's kernels (all HBM-bound; their FLOPs are a
+    few per byte).  route_grad: dy and dx rows (fp32), every Top-K slot's expert output row
+    (fp16 on the tensor-core path, fp32 otherwise), the router rows read once, the routing
+    arrays (ids, gate, mask logit, inv: 16 B per slot) and the per-slot outputs (pair
+    gradients 8 B, d_gate_logit / d_mask_logit / s 12 B).  route_dw: the routed rows of x
+    once, perm and the pair gradients, the partial columns written.  route_dw_reduce: the
+    partial columns read, dW_r and dW_m written."""
+    D, E, K = spec.d_model, spec.n_experts, spec.top_k
+    es = 2 if spec.storage == "bf16" else 4
+    ys = 2 if tc_path else 4
+    S = max(1, spec.segment_len)
+    Tr = -(-T // S)
+    w = {}
+    w["route_grad"] = dict(bytes=2 * T * D * 4 + T * K * D * ys + 2 * E * D * es + T * K * 36,
+                           flops=2 * T * K * D + 4 * Tr * K * D)
+    units = 2 * 148 + E
+    w["route_dw"] = dict(bytes=Tr * D * es + T * K * 12 + units * 2 * D * 4, flops=4 * Tr * K * D)
+    w["route_dw_reduce"] = dict(bytes=units * 2 * D * 4 + 2 * D * E * 4, flops=0)
+    return w
+
+
+def train_point(torch, name, steps, warmup, device, peaks):
+    """One training step of the routing: the BEAM_TRAIN forward (every Top-K expert evaluated,
+    the mask scaling the gates) and the routing gradient.  The forward and the gradient are
+    timed with their own event pairs, call by call; the forward between two gradient calls
+    streams the expert weights (more than the 126 MB L2), so no gradient call finds the
+    previous one's data in L2."""
+    wl = TRAIN_POINTS[name]
+    spec, T, keep, layer, x = build_layer(torch, wl, device)
+    y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+    dy = torch.randn((T, spec.d_model), generator=g, device=device, dtype=torch.float32)
+    st_ = torch.cuda.current_stream()
+    for _ in range(warmup):
+        layer.forward(x, out=y, train=True)
+        layer.backward_router(x, dy, reg_scale=0.5)
+    torch.cuda.synchronize()
+    fw, bw = [], []
+    n0 = layer.launch_count()
+    for _ in range(steps):
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(st_)
+        layer.forward(x, out=y, train=True)
+        b.record(st_)
+        layer.backward_router(x, dy, reg_scale=0.5)
+        c.record(st_)
+        fw.append((a, b))
+        bw.append((b, c))
+    torch.cuda.synchronize()
+    launches = (layer.launch_count() - n0) / steps
+    ms_f = sum(p.elapsed_time(q) for p, q in fw) / steps
+    ms_b = sum(p.elapsed_time(q) for p, q in bw) / steps
+    st = layer.stats()
+    # masked inference forward at the same shape, for the training forward's extra cost
+    ms_inf, _ = time_steps(torch, None, layer, x, y, steps, warmup, False, 1)
+    layer.profile_begin(steps)
+    for _ in range(steps):
+        layer.forward(x, out=y, train=True)
+        layer.backward_router(x, dy, reg_scale=0.5)
+    prof = layer.profile_end()
+    work = grad_work(spec, T, tc_path="tc_gateup" in prof)
+    kernels = {}
+    for k in ("route_grad", "route_dw", "route_dw_reduce"):
+        if k in prof:
+            kernels[k] = roofline_for(k, work[k], prof[k][0] / prof[k][1], peaks, name)
+    layer.close()
+    grad_bytes = sum(v["bytes"] for v in work.values())
+    return dict(workload=name, metric="routing-gradient tokens/s", unit="tokens/s", tokens=T,
+                keep_rate=keep, value=round(T / (ms_b * 1e-3), 2), ms_per_step=round(ms_b, 5),
+                roofline_frac=round(grad_bytes / (peaks["hbm"] * 1e9) / (ms_b * 1e-3), 4),
+                train_forward_ms=round(ms_f, 5), inference_forward_ms=round(ms_inf, 5),
+                avg_k=round(st["avg_k"], 4), evaluated_slots_per_token=round(st["n_kept"] / T, 4),
+                launches_per_step=launches,
+                gradient_launches=sum(prof[k][1] for k in kernels) // max(1, prof["forwards"]),
+                kernels=kernels,
+                l2="a training forward (expert weights > 126 MB) runs between gradient calls")
 
 
 def roofline_for(stage, work, ms_per_launch, peaks, workload):
@@ -518,6 +606,7 @@ def _run_ours(args):
 
     points = []
     gen_points = []
+    train_points = []
     if not args.no_points:
         for p in EXTRA_POINTS:
             if p == name:
@@ -526,6 +615,8 @@ def _run_ours(args):
         if world == 1:
             for p in GEN_POINTS:
                 gen_points.append(gen_point(torch, p, max(10, args.steps), args.warmup, device, peaks))
+            train_points.append(train_point(torch, "train-mixtral-prefill", max(10, args.steps),
+                                            args.warmup, device, peaks))
 
     if rank == 0:
         line = {
@@ -565,6 +656,7 @@ def _run_ours(args):
             "cpu_baseline": cpu,
             "points": points,
             "gen_points": gen_points,
+            "train_points": train_points,
             "peaks": peaks,
         }
         print(json.dumps(line), flush=True)
@@ -591,6 +683,10 @@ def run_sweep(args):
         print(json.dumps(r), flush=True)
     for name in GEN_POINTS:
         print(json.dumps(gen_point(torch, name, args.steps, args.warmup, device, peaks)), flush=True)
+    for name in TRAIN_POINTS:
+        if name != "train-profile":
+            print(json.dumps(train_point(torch, name, args.steps, args.warmup, device, peaks)),
+                  flush=True)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
@@ -709,6 +805,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
     ap.add_argument("--sweep", action="store_true",
                     help="measure every workload (one JSON line each) instead of the headline")
+    ap.add_argument("--train", choices=sorted(TRAIN_POINTS), action="append",
+                    help="measure only these training points (one JSON line each)")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="store a kernel's DRAM bytes per launch from an ncu CSV log (no GPU work)")
     ap.add_argument("--traffic-kernel", default=r"tc_grouped_gemm_kernel<(\(int\))?0,",
@@ -723,6 +821,14 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.train:
+        import torch
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(device)
+        with torch.cuda.stream(torch.cuda.Stream(device)):
+            for name in args.train:
+                print(json.dumps(train_point(torch, name, args.steps, args.warmup, device,
+                                             load_peaks())), flush=True)
     elif args.sweep:
         run_sweep(args)
     else:

@@ -23,8 +23,9 @@ BEAM_PATH_STREAM = 0x2
 BEAM_PATH_TENSOR = 0x4
 BEAM_NO_GRAPH = 0x8
 BEAM_FUSED_DECODE = 0x10
+BEAM_TRAIN = 0x20
 
-BEAM_N_STAGES = 16
+BEAM_N_STAGES = 19
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 STATUS_NAMES = {0: "BEAM_OK", 1: "BEAM_ERR_INVALID_ARG", 2: "BEAM_ERR_OOM", 3: "BEAM_ERR_CUDA",
@@ -103,6 +104,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.beam_gen_destroy.argtypes = [P]
     lib.beam_gen_destroy.restype = None
     lib.beam_moe_forward_routed.argtypes = [P, P, I, ctypes.POINTER(BeamRouting), P, U, P]
+    lib.beam_moe_backward_router.argtypes = [P, P, P, I, ctypes.c_float, P, P, P, P, P, P, P]
     lib.beam_moe_destroy.argtypes = [P]
     lib.beam_moe_destroy.restype = None
     lib.beam_moe_last_error.restype = ctypes.c_char_p
@@ -110,7 +112,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for f in (lib.beam_moe_create, lib.beam_moe_forward, lib.beam_moe_forward_host,
               lib.beam_moe_stats, lib.beam_moe_get_routing, lib.beam_moe_profile_begin,
               lib.beam_moe_profile_end, lib.beam_gen_create, lib.beam_gen_route,
-              lib.beam_gen_sync, lib.beam_moe_forward_routed):
+              lib.beam_gen_sync, lib.beam_moe_forward_routed, lib.beam_moe_backward_router):
         f.restype = ctypes.c_int
     _lib = lib
     return lib

@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdlib>
 #include <cstdio>
@@ -26,6 +27,7 @@
 #include "stream_experts.cuh"
 #include "tc_experts.cuh"
 #include "decode_fused.cuh"
+#include "route_grad.cuh"
 
 using namespace beam;
 
@@ -133,6 +135,15 @@ struct RouteIn {
 struct beam_moe;
 static RouteIn own_routing(const beam_moe* h);
 
+// Where a forward left the routed experts' outputs Y_perm: `splits` slices `stride` elements
+// apart (added in slice order), fp16 or fp32.
+struct YOut {
+    const void* base = nullptr;
+    int splits = 1;
+    long long stride = 0;
+    bool f16 = false;
+};
+
 struct beam_moe {
     beam_moe_config_t cfg;
     int E, K, D, F, Fsh, Tmax, S;
@@ -186,6 +197,12 @@ struct beam_moe {
     cudaStream_t side = nullptr;
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     int last_T = -1;
+    // training: the last forward's mode and where it left Y_perm (read by the routing
+    // gradient), the per-pair logit gradients and the dW partial columns
+    bool last_train = false;
+    YOut last_yr;
+    float2* pair_grad = nullptr;  // [Tmax*K] (d_gate_logit, d_mask_logit) of routed rows
+    float* dw_part = nullptr;     // [2*num_sms + E][2][D]
     std::vector<void*> allocs;
     // replay cache: the last forward captured as a CUDA graph, keyed by its arguments
     cudaGraphExec_t graph_exec = nullptr;
@@ -198,6 +215,7 @@ struct beam_moe {
     int g_kernels = 0;   // kernels in the captured graph
     bool g_routed = false;
     RouteIn g_rin;       // routing pointers of a captured routed forward
+    YOut g_yr;           // Y_perm of the captured forward
     // launch accounting and optional per-stage timing
     long long launches = 0;
     bool prof = false;
@@ -210,14 +228,15 @@ struct beam_moe {
 enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
-    ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE, ST_COUNT
+    ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE,
+    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_ROUTE_DW_REDUCE, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
     "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish",
-    "fused_decode"};
+    "fused_decode", "route_grad", "route_dw", "route_dw_reduce"};
 
 static void prof_release(beam_moe* h)
 {
@@ -597,6 +616,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->yperm, rows * D * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->x_stage, Tm * D * es));
     BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->pair_grad, rows * sizeof(float2)));
+    BEAM_TRY(dalloc(h, &h->dw_part, (2 * (size_t)h->num_sms + E) * 2 * D * sizeof(float)));
     BEAM_CUDA(cudaMemsetAsync(h->dstats, 0, sizeof(DevStats), st));
     BEAM_CUDA(cudaMemsetAsync(h->tail_cnt, 0, tail_cnt_ints(h->num_sms) * sizeof(int), st));
     BEAM_CUDA(cudaMemsetAsync(h->range_flag, 0, sizeof(int), st));
@@ -732,13 +753,6 @@ static cudaError_t launch_small(beam_moe* h, const T* x, int Tr, int T_, int mas
 
 // Output of one expert problem for the combine: `splits` slices `stride` elements apart,
 // fp16 (unsplit tensor-core output) or fp32 (split-K partials, GEMV path).
-struct YOut {
-    const void* base = nullptr;
-    int splits = 1;
-    long long stride = 0;
-    bool f16 = false;
-};
-
 // GEMM1 (+ SwiGLU finish when split) and GEMM2 on the tensor cores, on stream `st`, for the
 // routed groups (PROB_ROUTED), the always-on shared group (PROB_SHARED), or both in the same
 // launches (PROB_BOTH: the shared tiles first, then the routed ones; used for small batches,
@@ -879,7 +893,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     const int S = h->S;
     const int Tr = ceil_div(T_, S);
     const int nch = ceil_div(T_, 32);
-    const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
+    const int mask_off = (flags & BEAM_TRAIN) ? 2 : (flags & BEAM_MASK_OFF) ? 1 : 0;
 
     // 0. shared experts: they need only x, so for larger batches on the tensor path they run on
     // a side stream, concurrently with the router and the compaction, and join before the
@@ -991,6 +1005,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         yr.base = h->yperm; yr.f16 = false;
         if (h->Fsh) { ysh_out.base = h->ysh; ysh_out.f16 = false; }
     }
+    h->last_yr = yr;
     // 5. fixed-order combine (after the side stream joins)
     if (fork) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_join, 0));
     if (!h->Fsh) ysh_out.f16 = yr.f16;  // no shared term: only its (unused) type must match
@@ -1331,6 +1346,66 @@ static beam_status_t gen_route_impl(beam_gen* g, const T* z, int T_, const beam_
 }
 
 // ---------------------------------------------------------------- C ABI
+// ---------------------------------------------------------------- training: routing gradient
+// Pairs per unit of the dW pass: about two CTAs per SM over all column slices, at least 16.
+// Then ceil(pairs / R) <= 2 * num_sms / slices, so the units (at most that plus one partial
+// unit per expert) fit the handle's 2 * num_sms + E partial columns.
+static int dw_rows_per_unit(const beam_moe* h, int T_, int slices)
+{
+    const long long pairs = (long long)T_ * h->K;
+    long long r = (pairs * slices + 2LL * h->num_sms - 1) / (2LL * h->num_sms);
+    r = ((r + 15) / 16) * 16;
+    return (int)std::max<long long>(16, r);
+}
+
+template <typename TY, typename TX>
+static cudaError_t launch_route_grad(beam_moe* h, const TX* x, const float* dy, int T_, float reg,
+                                     float* dx, float* dgl, float* dml, float* dgh, cudaStream_t st)
+{
+    (void)x;
+    const YOut& yr = h->last_yr;
+    const int Tr = ceil_div(T_, h->S);
+    const int K = h->K;
+#define BEAM_RG(KM)                                                                              \
+    launch(h, ST_ROUTE_GRAD, route_grad_kernel<TY, TX, KM>, dim3(Tr), dim3(kGradThreads), 0, st, \
+           (const TY*)yr.base, yr.splits, yr.stride, (const int*)h->inv, (const int*)h->topk_id, \
+           (const float*)h->gate, (const float*)h->mlogit, dy, (const TX*)h->wrm, T_, K, h->E,  \
+           h->D, h->S, reg, dgh, dgl, dml, h->pair_grad, dx)
+    if (K <= 4) return BEAM_RG(4);
+    if (K <= 8) return BEAM_RG(8);
+    if (K <= 16) return BEAM_RG(16);
+    return BEAM_RG(32);
+#undef BEAM_RG
+}
+
+template <typename TX>
+static beam_status_t backward_impl(beam_moe* h, const TX* x, const float* dy, int T_,
+                                   float reg_scale, float* dwr, float* dwm, float* dx, float* dgl,
+                                   float* dml, float* dgh, cudaStream_t st)
+{
+    const int K = h->K, E = h->E, D = h->D;
+    // dL/dm_hat of every (token, slot) from L_reg = mean over tokens of (1/K) sum_TK m_hat
+    const float reg = (float)((double)reg_scale / ((double)T_ * (double)K));
+    // 1. per routed row: the K dots with dy, the logit gradients, dx
+    const cudaError_t e1 = h->last_yr.f16
+        ? launch_route_grad<__half, TX>(h, x, dy, T_, reg, dx, dgl, dml, dgh, st)
+        : launch_route_grad<float, TX>(h, x, dy, T_, reg, dx, dgl, dml, dgh, st);
+    BEAM_CUDA(e1);
+    // 2. per (unit of one expert's pairs, column slice): partial dW columns
+    constexpr int N = Vec<TX>::N;
+    const int slices = ceil_div(D, 256 * N);
+    const int R = dw_rows_per_unit(h, T_, slices);
+    const int units = ceil_div((long long)T_ * K, R) + E;
+    BEAM_CUDA(launch(h, ST_ROUTE_DW, route_dw_partial_kernel<TX>, dim3(units, slices), dim3(256), 0,
+                     st, (const int*)h->offsets, (const int*)h->perm,
+                     (const float2*)h->pair_grad, x, K, E, D, h->S, R, h->dw_part));
+    // 3. each expert's partials in unit order
+    BEAM_CUDA(launch(h, ST_ROUTE_DW_REDUCE, route_dw_reduce_kernel,
+                     dim3(ceil_div((long long)E * D, 256)), dim3(256), 0, st,
+                     (const int*)h->offsets, (const float*)h->dw_part, E, D, R, dwr, dwm));
+    return BEAM_OK;
+}
+
 extern "C" {
 
 beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, int32_t* topk_id,
@@ -1468,8 +1543,11 @@ static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float*
     if (T > 0 && (!x || !y)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
         return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
-    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_FUSED_DECODE))
+    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH |
+                  BEAM_FUSED_DECODE | BEAM_TRAIN))
         return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & BEAM_TRAIN) && (flags & (BEAM_MASK_OFF | BEAM_FUSED_DECODE)))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_TRAIN excludes BEAM_MASK_OFF and BEAM_FUSED_DECODE");
     if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
         return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core expert path needs a bf16 layer with "
                     "d_model a multiple of 256");
@@ -1502,6 +1580,7 @@ static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float*
             BEAM_CUDA(cudaGraphLaunch(h->graph_exec, st));
             h->launches += h->g_kernels;
             h->cur = rin ? *rin : own_routing(h);
+            h->last_yr = h->g_yr;
         } else {
             bool captured = false;
             if (graphable) {
@@ -1527,6 +1606,7 @@ static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float*
                         h->g_routed = rin != nullptr;
                         h->g_rin = rin ? *rin : RouteIn();
                         h->g_kernels = (int)nn;
+                        h->g_yr = h->last_yr;
                         captured = true;
                     }
                     if (g) cudaGraphDestroy(g);
@@ -1543,6 +1623,7 @@ static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float*
         }
     }
     h->last_T = T;
+    h->last_train = (flags & BEAM_TRAIN) != 0;
     BEAM_CUDA(cudaEventRecord(h->done, st));
     return BEAM_OK;
 }
@@ -1562,9 +1643,9 @@ beam_status_t beam_moe_forward_routed(beam_moe_t* h, const void* x, int32_t T,
     g_err[0] = 0;
     if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
     if (!r) return fail(BEAM_ERR_INVALID_ARG, "routing is NULL");
-    if (flags & (BEAM_MASK_OFF | BEAM_FUSED_DECODE))
-        return fail(BEAM_ERR_INVALID_ARG, "BEAM_MASK_OFF and BEAM_FUSED_DECODE do not apply to a "
-                    "forward with given routing (the mask is part of the routing)");
+    if (flags & (BEAM_MASK_OFF | BEAM_FUSED_DECODE | BEAM_TRAIN))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_MASK_OFF, BEAM_FUSED_DECODE and BEAM_TRAIN do not "
+                    "apply to a forward with given routing (the mask is part of the routing)");
     if (T > 0 && (!r->topk_id || !r->keep || !r->ghat || !r->n_keep || !r->lreg))
         return fail(BEAM_ERR_INVALID_ARG, "routing needs topk_id, keep, ghat, n_keep and lreg");
     // the compaction reads a token's K slots as one vector when K is 4, 8 or 16
@@ -1708,6 +1789,41 @@ const char* beam_moe_stage_name(int32_t stage)
 int64_t beam_moe_launch_count(const beam_moe_t* h) { return h ? h->launches : 0; }
 
 static __device__ int g_wait_selftest_result;
+
+beam_status_t beam_moe_backward_router(beam_moe_t* h, const void* x, const float* dy, int32_t T,
+                                       float reg_scale, float* dw_router, float* dw_mask,
+                                       float* dx, float* d_gate_logit, float* d_mask_logit,
+                                       float* dghat, void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
+    if (T == 0) return BEAM_OK;
+    if (!h->last_train || h->last_T != T)
+        return fail(BEAM_ERR_NO_FORWARD, "the routing gradient needs the handle's last forward to "
+                    "be a BEAM_TRAIN forward of the same T (last forward: T=%d, %s)", h->last_T,
+                    h->last_train ? "training" : "not training");
+    if (!x || !dy || !dw_router || !dw_mask || !dx)
+        return fail(BEAM_ERR_INVALID_ARG, "x, dy, dw_router, dw_mask and dx are required");
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dy) |
+         reinterpret_cast<uintptr_t>(dx)) & 15)
+        return fail(BEAM_ERR_INVALID_ARG, "x, dy and dx must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(dw_router) | reinterpret_cast<uintptr_t>(dw_mask) |
+         reinterpret_cast<uintptr_t>(d_gate_logit) | reinterpret_cast<uintptr_t>(d_mask_logit) |
+         reinterpret_cast<uintptr_t>(dghat)) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "the float32 outputs must be 4-byte aligned");
+    if (!std::isfinite(reg_scale))
+        return fail(BEAM_ERR_INVALID_ARG, "reg_scale must be finite");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (h->cfg.dtype == BEAM_DTYPE_BF16)
+        BEAM_TRY(backward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), dy, T,
+                                              reg_scale, dw_router, dw_mask, dx, d_gate_logit,
+                                              d_mask_logit, dghat, st));
+    else
+        BEAM_TRY(backward_impl<float>(h, static_cast<const float*>(x), dy, T, reg_scale, dw_router,
+                                      dw_mask, dx, d_gate_logit, d_mask_logit, dghat, st));
+    return BEAM_OK;
+}
 
 beam_status_t beam_moe_wait_selftest(int32_t timeout_us, void* stream)
 {

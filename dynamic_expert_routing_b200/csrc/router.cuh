@@ -144,17 +144,18 @@ router_gemv_warp_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
 // slice order).  Lane l holds logits of experts l, l+32, ... (EPL per lane).
 // K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
 // rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
-// L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
-// to every token of the routed row's segment (S = 1: the row's own token).
+// L[i][E + id_k], m = (logit >= 0) (1 for plain Top-K), g_hat = g * m, keep = m (1 for plain
+// Top-K and in training mode).  The decision is written to every token of the routed row's
+// segment (S = 1: the row's own token).
 // Decision for one routed row, computed by one warp (all lanes return the same values except
 // the per-slot ones, which lane k < K holds for slot k).
 struct RowDecision {
     int id;        // lane k: expert of slot k
     float g;       // lane k: softmax gate of slot k
     float l;       // lane k: mask logit of slot k
-    bool keep;     // lane k: slot kept
-    float ghat;    // lane k: g * keep
-    int nkeep;     // all lanes: kept slots of the row
+    bool keep;     // lane k: slot's expert evaluated (kept; every slot in training mode)
+    float ghat;    // lane k: g * m (the mask)
+    int nkeep;     // all lanes: slots of the row whose mask is 1
     float lreg;    // all lanes: (1/K) sum_k sigmoid(l_k)
 };
 
@@ -227,10 +228,13 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
     d.id = my_id;
     d.g = ex / den;
     d.l = active ? logit(E + my_id) : 0.f;
-    d.keep = active && (mask_off || d.l >= 0.f);
-    d.ghat = d.keep ? d.g : 0.f;
+    // mask_off: 0 = BEAM mask, 1 = plain Top-K, 2 = training (every Top-K slot is evaluated,
+    // so keep = 1 for the compaction, while the gate still carries the mask: g_hat = g * m)
+    const bool m = active && (mask_off == 1 || d.l >= 0.f);
+    d.keep = active && (mask_off != 0 || d.l >= 0.f);
+    d.ghat = m ? d.g : 0.f;
     const float sg = active ? sigmoid_f(d.l) : 0.f;
-    d.nkeep = __popc(__ballot_sync(0xffffffffu, d.keep));
+    d.nkeep = __popc(__ballot_sync(0xffffffffu, m));
     d.lreg = warp_sum(sg) / (float)K;
     return d;
 }
@@ -241,7 +245,7 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
 // order.  Lane l holds logits of experts l, l+32, ... (EPL per lane).
 // K rounds of a warp arg-max under the total order (value desc, index asc) give the Top-K in
 // rank order.  Lane k < K then owns slot k: g_k = exp(r_k - r_0) / sum, mask logit
-// L[i][E + id_k], keep = mask_off | (logit >= 0), g_hat = g * keep.  The decision is written
+// L[i][E + id_k], keep and g_hat as select_row gives them.  The decision is written
 // to every token of the routed row's segment (S = 1: the row's own token), layer l's outputs
 // out_ls ([T][K] arrays) or tok_ls ([T] arrays) elements after layer 0's.  With `active` set,
 // bit e of layer l's word e/32 of active[l][nw] (nw = (E+31)/32, zeroed by the caller) is

@@ -12,8 +12,8 @@ import torch
 
 from . import _lib
 from ._lib import (BEAM_DTYPE_BF16, BEAM_DTYPE_F32, BEAM_MASK_OFF, BEAM_FUSED_DECODE, BEAM_NO_GRAPH,
-                   BEAM_PATH_STREAM, BEAM_PATH_TENSOR, BeamConfig, BeamGenConfig, BeamRouting,
-                   BeamStats, BeamWeights, check)
+                   BEAM_PATH_STREAM, BEAM_PATH_TENSOR, BEAM_TRAIN, BeamConfig, BeamGenConfig,
+                   BeamRouting, BeamStats, BeamWeights, check)
 
 _DTYPES = {torch.float32: BEAM_DTYPE_F32, torch.bfloat16: BEAM_DTYPE_BF16}
 _PATHS = {None: 0, "auto": 0, "stream": BEAM_PATH_STREAM, "tensor": BEAM_PATH_TENSOR}
@@ -66,27 +66,55 @@ class BeamMoE:
     # -------------------------------------------------------------- forward
     @staticmethod
     def flags(mask_off: bool = False, path: str | None = None, graph: bool = True,
-              fused: bool = False) -> int:
+              fused: bool = False, train: bool = False) -> int:
         return ((BEAM_MASK_OFF if mask_off else 0) | _PATHS[path] | (0 if graph else BEAM_NO_GRAPH)
-                | (BEAM_FUSED_DECODE if fused else 0))
+                | (BEAM_FUSED_DECODE if fused else 0) | (BEAM_TRAIN if train else 0))
 
     def forward(self, x: torch.Tensor, mask_off: bool = False, path: str | None = None,
                 out: torch.Tensor | None = None, stream=None, graph: bool = True,
-                fused: bool = False) -> torch.Tensor:
+                fused: bool = False, train: bool = False) -> torch.Tensor:
         """y [T][D] float32 of x [T][D] (storage dtype, CUDA), enqueued on the current stream.
         graph=False launches the kernels directly instead of replaying a captured graph;
-        fused=True runs a bf16 batch of <= 32 tokens as one cooperative launch (opt-in)."""
+        fused=True runs a bf16 batch of <= 32 tokens as one cooperative launch (opt-in);
+        train=True evaluates every Top-K slot's expert (the mask only scales the gates) so
+        that backward_router can follow."""
         if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype):
             raise ValueError("x must be a contiguous CUDA tensor of the layer's storage dtype")
         T = x.shape[0]
         if out is None:
             out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
         check(_lib.load().beam_moe_forward(self._h, _ptr(x), T, _ptr(out),
-                                           self.flags(mask_off, path, graph, fused),
+                                           self.flags(mask_off, path, graph, fused, train),
                                            ctypes.c_void_p(_stream_handle(stream))))
         return out
 
     __call__ = forward
+
+    def backward_router(self, x: torch.Tensor, dy: torch.Tensor, reg_scale: float = 0.0,
+                        slots: bool = False, stream=None) -> dict:
+        """Gradient of the routing after a forward(train=True) of the same x: dW_router,
+        dW_mask [D][E] and the routing's share of dx [T][D] (float32), for the upstream
+        gradient dy [T][D] (float32) and reg_scale = dL/dL_reg.  slots=True also returns the
+        per-slot d_gate_logit, d_mask_logit and dghat [T][K]."""
+        if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype):
+            raise ValueError("x must be a contiguous CUDA tensor of the layer's storage dtype")
+        T = x.shape[0]
+        if not (dy.is_cuda and dy.is_contiguous() and dy.dtype == torch.float32
+                and tuple(dy.shape) == (T, self.d_model)):
+            raise ValueError("dy must be a contiguous CUDA float32 tensor of shape [T][D]")
+        D, E, K = self.d_model, self.n_experts, self.top_k
+        f32 = dict(dtype=torch.float32, device=x.device)
+        out = dict(dw_router=torch.empty((D, E), **f32), dw_mask=torch.empty((D, E), **f32),
+                   dx=torch.empty((T, D), **f32))
+        if slots:
+            for k in ("d_gate_logit", "d_mask_logit", "dghat"):
+                out[k] = torch.empty((T, K), **f32)
+        check(_lib.load().beam_moe_backward_router(
+            self._h, _ptr(x), _ptr(dy), T, ctypes.c_float(reg_scale), _ptr(out["dw_router"]),
+            _ptr(out["dw_mask"]), _ptr(out["dx"]), _ptr(out.get("d_gate_logit")),
+            _ptr(out.get("d_mask_logit")), _ptr(out.get("dghat")),
+            ctypes.c_void_p(_stream_handle(stream))))
+        return out
 
     def forward_routed(self, x: torch.Tensor, routing: dict, path: str | None = None,
                        out: torch.Tensor | None = None, stream=None, graph: bool = True) -> torch.Tensor:

@@ -53,6 +53,9 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_NO_GRAPH     0x8u  /* launch the kernels directly instead of replaying a graph */
 #define BEAM_FUSED_DECODE 0x10u /* batches of <= 32 tokens (bf16): one fused cooperative
                                    launch instead of separate kernels (opt-in; slower on B200) */
+#define BEAM_TRAIN        0x20u /* training forward: every Top-K slot's expert is evaluated
+                                   and the mask only scales the gates (g_hat = g * m), so that
+                                   beam_moe_backward_router can follow (see there) */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
@@ -110,8 +113,11 @@ beam_status_t beam_moe_create(const beam_moe_config_t *cfg, const beam_moe_weigh
  * expert-grouping compaction, the grouped SwiGLU experts (kept experts only), the shared
  * experts and the fixed-order combine.  Deterministic: the same inputs give the same bits.
  * T = 0 is a no-op.  T > max_tokens or NULL pointers -> BEAM_ERR_INVALID_ARG.
- * flags: BEAM_MASK_OFF, and at most one of BEAM_PATH_STREAM / BEAM_PATH_TENSOR (by default the
- * path is chosen from T), BEAM_NO_GRAPH.  x_dev and y_dev must stay valid until the stream
+ * flags: BEAM_MASK_OFF or BEAM_TRAIN (not both), and at most one of BEAM_PATH_STREAM /
+ * BEAM_PATH_TENSOR (by default the path is chosen from T), BEAM_NO_GRAPH.  BEAM_TRAIN gives the
+ * same y (up to rounding: masked slots add 0 * E_i(x)) at the cost of every Top-K expert; its
+ * statistics count the mask (avg_k, l_reg, all-masked tokens) but n_active_experts, n_kept,
+ * the counts and beam_moe_get_routing's keep / perm describe the evaluated slots (all of them).  x_dev and y_dev must stay valid until the stream
  * reaches the end of the call's work.
  * Replay: on a non-default stream that is not being captured, the first forward with a given
  * (x_dev, y_dev, T, flags) is captured into a CUDA graph owned by the handle, and later calls
@@ -167,7 +173,7 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * each stage's time covers the work of one problem.  A fused decode forward is one launch,
  * timed as the stage fused_decode.
  */
-#define BEAM_N_STAGES 16
+#define BEAM_N_STAGES 19
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);
@@ -298,6 +304,44 @@ void beam_gen_destroy(beam_gen_t *g);
 beam_status_t beam_moe_forward_routed(beam_moe_t *h, const void *x_dev, int32_t T,
                                       const beam_routing_t *r, float *y_dev, uint32_t flags,
                                       void *stream);
+
+/*
+ * ---------------------------------------------------------------- training: routing gradient
+ * The gradient of the routing under BEAM's training recipe (BEAM article on aitrends.kr,
+ * training paragraph: L = L_lm + alpha L_bal + beta L_reg, L_reg = (1/K) sum_{i in TK}
+ * |m_hat_i|, the straight-through estimator carrying the binary mask's gradient to m_hat;
+ * ai-feeds.com summary, Method, binarisation and straight-through estimator).  With
+ * dy = dL/dy, for token t and Top-K slot k (expert i, gate g_k, mask logit l_k, m_k = l_k >= 0):
+ *   s_tk = <dy_t, E_i(x_t)>  (= dL/dg_hat),   dL/dg_k = s_tk m_k,
+ *   dL/dm_hat_k = s_tk g_k + reg_scale / (T K)       (straight through: dm/dm_hat = 1; L_reg
+ *                                                     the mean over tokens of the per-token term)
+ *   d_mask_logit_k = dL/dm_hat_k sigmoid(l_k) (1 - sigmoid(l_k))
+ *   d_gate_logit_k = g_k (dL/dg_k - sum_j g_j dL/dg_j)   (softmax over the K; logits outside
+ *                                                     the Top-K get nothing)
+ *   dW_r[d][i] = sum_t x_t[d] d_gate_logit_tk,  dW_m[d][i] = sum_t x_t[d] d_mask_logit_tk,
+ *   dx_t = sum_k d_gate_logit_tk W_r[:, i] + d_mask_logit_tk W_m[:, i]   (the routing's share
+ *          of dL/dx; the experts' own backward is not part of this call).
+ * With segment routing the segment's tokens share their first token's decision: their terms
+ * are summed at that token, which alone gets logit gradients and a nonzero dx row.  L_bal is
+ * not defined on the pages and has no term here.
+ *
+ * Precondition: the handle's last forward was a beam_moe_forward with BEAM_TRAIN (flags may
+ * add BEAM_PATH_* / BEAM_NO_GRAPH; not BEAM_MASK_OFF or BEAM_FUSED_DECODE) on the same x_dev
+ * contents and the same T, and no forward ran since (else BEAM_ERR_NO_FORWARD).  That forward
+ * evaluated every Top-K slot's expert and kept the outputs in the handle.
+ * Arguments (device pointers, enqueued on `stream`, no host synchronisation):
+ *   x_dev [T][D] storage type (16-byte aligned), dy_dev [T][D] float32 (16-byte aligned),
+ *   reg_scale = dL/dL_reg (beta), dw_router_dev / dw_mask_dev [D][E] float32 (overwritten),
+ *   dx_dev [T][D] float32 (overwritten, 16-byte aligned); d_gate_logit_dev,
+ *   d_mask_logit_dev and dghat_dev [T][K] float32 are optional outputs (NULL to skip) holding
+ *   the per-slot gradients above (0 at the tokens of a segment after its first) and s.
+ * Every sum runs in a fixed order: the same inputs give the same bits.  T = 0 is a no-op.
+ */
+beam_status_t beam_moe_backward_router(beam_moe_t *h, const void *x_dev, const float *dy_dev,
+                                       int32_t T, float reg_scale, float *dw_router_dev,
+                                       float *dw_mask_dev, float *dx_dev,
+                                       float *d_gate_logit_dev, float *d_mask_logit_dev,
+                                       float *dghat_dev, void *stream);
 
 /* Free every device buffer of the handle (waits for its pending work).  NULL is ignored. */
 void beam_moe_destroy(beam_moe_t *h);

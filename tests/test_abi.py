@@ -100,6 +100,21 @@ def test_generator_and_routed_forward_null_handles(lib):
     assert lib.beam_moe_forward_routed(None, None, 1, ctypes.byref(r), None, 0, None) == BEAM_ERR_INVALID_ARG
 
 
+def test_routing_gradient_null_handle(lib):
+    from dynamic_expert_routing_b200._lib import BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_backward_router(None, None, None, 1, ctypes.c_float(0.0), None, None,
+                                        None, None, None, None, None) == BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_last_error()
+
+
+def test_stage_table_matches_the_header(lib):
+    from dynamic_expert_routing_b200 import _lib
+    names = [lib.beam_moe_stage_name(i).decode() for i in range(_lib.BEAM_N_STAGES)]
+    assert all(names) and len(set(names)) == len(names)
+    assert lib.beam_moe_stage_name(_lib.BEAM_N_STAGES) == b""
+    assert names[-3:] == ["route_grad", "route_dw", "route_dw_reduce"]
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from dynamic_expert_routing_b200 import _lib
     with pytest.raises(RuntimeError):
