@@ -100,10 +100,19 @@ def load_peaks():
                     tc_sustained=FALLBACK_BF16_TFLOPS, source="fallback")
 
 
-def kernel_source_hash() -> str:
+# Sources that do not take part in a stage's kernels or launches: the forward's kernels never
+# run the routing-gradient code, so its file is left out of their hash.
+GRAD_SOURCES = {"route_grad.cuh"}
+GRAD_STAGES = {"route_grad", "route_dw"}
+
+
+def kernel_source_hash(stage: str = "") -> str:
+    """Hash of the CUDA sources a stage's kernels are built and launched from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dynamic_expert_routing_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
+        if f in GRAD_SOURCES and stage not in GRAD_STAGES:
+            continue
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -119,7 +128,7 @@ def recorded_traffic(kernel: str, workload: str):
     except Exception:
         return None
     rec = d.get(workload, {}).get(kernel)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -304,8 +313,8 @@ def grad_work(spec, T, tc_path=True) -> dict:
     (fp16 on the tensor-core path, fp32 otherwise), the router rows read once, the routing
     arrays (ids, gate, mask logit, inv: 16 B per slot) and the per-slot outputs (pair
     gradients 8 B, d_gate_logit / d_mask_logit / s 12 B).  route_dw: the routed rows of x
-    once, perm and the pair gradients, the partial columns written.  route_dw_reduce: the
-    partial columns read, dW_r and dW_m written."""
+    once, perm and the pair gradients, dW_r and dW_m written (the partial columns it adds up
+    are scratch, not algorithmic traffic)."""
     D, E, K = spec.d_model, spec.n_experts, spec.top_k
     es = 2 if spec.storage == "bf16" else 4
     ys = 2 if tc_path else 4
@@ -314,9 +323,7 @@ def grad_work(spec, T, tc_path=True) -> dict:
     w = {}
     w["route_grad"] = dict(bytes=2 * T * D * 4 + T * K * D * ys + 2 * E * D * es + T * K * 36,
                            flops=2 * T * K * D + 4 * Tr * K * D)
-    units = 2 * 148 + E
-    w["route_dw"] = dict(bytes=Tr * D * es + T * K * 12 + units * 2 * D * 4, flops=4 * Tr * K * D)
-    w["route_dw_reduce"] = dict(bytes=units * 2 * D * 4 + 2 * D * E * 4, flops=0)
+    w["route_dw"] = dict(bytes=Tr * D * es + T * K * 12 + 2 * D * E * 4, flops=4 * Tr * K * D)
     return w
 
 
@@ -362,7 +369,7 @@ def train_point(torch, name, steps, warmup, device, peaks):
     prof = layer.profile_end()
     work = grad_work(spec, T, tc_path="tc_gateup" in prof)
     kernels = {}
-    for k in ("route_grad", "route_dw", "route_dw_reduce"):
+    for k in ("route_grad", "route_dw"):
         if k in prof:
             kernels[k] = roofline_for(k, work[k], prof[k][0] / prof[k][1], peaks, name)
     layer.close()
@@ -780,17 +787,18 @@ def record_traffic(args):
             d = json.load(f)
     except FileNotFoundError:
         d = {}
-    d.setdefault(args.workload, {})[args.traffic_stage] = {
+    key = getattr(args, "traffic_workload", None) or args.workload
+    d.setdefault(key, {})[args.traffic_stage] = {
         "dram_bytes_per_launch": int(round(sum(totals) / len(totals))),
         "launches": len(totals),
         "kernel": args.traffic_kernel,
-        "source_hash": kernel_source_hash(),
+        "source_hash": kernel_source_hash(args.traffic_stage),
         "command": args.traffic_command,
     }
     with open(path, "w") as f:
         json.dump(d, f, indent=1, sort_keys=True)
         f.write("\n")
-    print(json.dumps(d[args.workload][args.traffic_stage]))
+    print(json.dumps(d[key][args.traffic_stage]))
 
 
 def main():
@@ -813,6 +821,8 @@ def main():
                     help="regex of the kernel name in the CSV (gate/up: EPI 0, down: EPI 2)")
     ap.add_argument("--traffic-stage", default="tc_gateup", help="bench stage of that kernel")
     ap.add_argument("--traffic-command", default="", help="the ncu command that wrote the CSV")
+    ap.add_argument("--traffic-workload", default=None,
+                    help="workload or point key to store it under (default: --workload)")
     args = ap.parse_args()
     if args.record_traffic:
         record_traffic(args)

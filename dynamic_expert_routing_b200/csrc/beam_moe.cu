@@ -201,8 +201,11 @@ struct beam_moe {
     // gradient), the per-pair logit gradients and the dW partial columns
     bool last_train = false;
     YOut last_yr;
-    float2* pair_grad = nullptr;  // [Tmax*K] (d_gate_logit, d_mask_logit) of routed rows
-    float* dw_part = nullptr;     // [2*num_sms + E][2][D]
+    float2* pair_grad = nullptr;  // [Tmax*K] (d_gate_logit, d_mask_logit) of routed rows, at
+                                  // each pair's position in perm
+    int dw_chunks = 0;            // column chunks of the dW pass (32 vectors of x each)
+    float* dw_part = nullptr;     // [16*num_sms/dw_chunks + E + 1][2][D] partial columns
+    int* dw_cnt = nullptr;        // [E][dw_chunks] arrival counters, zero between calls
     std::vector<void*> allocs;
     // replay cache: the last forward captured as a CUDA graph, keyed by its arguments
     cudaGraphExec_t graph_exec = nullptr;
@@ -229,14 +232,14 @@ enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
     ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE,
-    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_ROUTE_DW_REDUCE, ST_COUNT
+    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
     "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish",
-    "fused_decode", "route_grad", "route_dw", "route_dw_reduce"};
+    "fused_decode", "route_grad", "route_dw"};
 
 static void prof_release(beam_moe* h)
 {
@@ -617,10 +620,14 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->x_stage, Tm * D * es));
     BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->pair_grad, rows * sizeof(float2)));
-    BEAM_TRY(dalloc(h, &h->dw_part, (2 * (size_t)h->num_sms + E) * 2 * D * sizeof(float)));
+    h->dw_chunks = ceil_div((long long)D, cfg->dtype == BEAM_DTYPE_BF16 ? dw_chunk_cols<__nv_bfloat16>()
+                                                                       : dw_chunk_cols<float>());
+    BEAM_TRY(dalloc(h, &h->dw_part, (16 * (size_t)h->num_sms / h->dw_chunks + E + 1) * 2 * D * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->dw_cnt, E * (size_t)h->dw_chunks * sizeof(int)));
     BEAM_CUDA(cudaMemsetAsync(h->dstats, 0, sizeof(DevStats), st));
     BEAM_CUDA(cudaMemsetAsync(h->tail_cnt, 0, tail_cnt_ints(h->num_sms) * sizeof(int), st));
     BEAM_CUDA(cudaMemsetAsync(h->range_flag, 0, sizeof(int), st));
+    BEAM_CUDA(cudaMemsetAsync(h->dw_cnt, 0, E * (size_t)h->dw_chunks * sizeof(int), st));
     BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, 2 * sizeof(int), st));
     BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
     if (h->Fsh > 0) {
@@ -1347,30 +1354,32 @@ static beam_status_t gen_route_impl(beam_gen* g, const T* z, int T_, const beam_
 
 // ---------------------------------------------------------------- C ABI
 // ---------------------------------------------------------------- training: routing gradient
-// Pairs per unit of the dW pass: about two CTAs per SM over all column slices, at least 16.
-// Then ceil(pairs / R) <= 2 * num_sms / slices, so the units (at most that plus one partial
-// unit per expert) fit the handle's 2 * num_sms + E partial columns.
-static int dw_rows_per_unit(const beam_moe* h, int T_, int slices)
+// Pairs per unit of the dW pass: about 16 warps per SM over all column chunks, at least 32.
+// Then ceil(pairs / R) <= 16 * num_sms / chunks, so the units (at most that plus one partial
+// unit per expert) fit the handle's 16 * num_sms / chunks + E + 1 partial column pairs.
+static int dw_rows_per_unit(const beam_moe* h, int T_)
 {
     const long long pairs = (long long)T_ * h->K;
-    long long r = (pairs * slices + 2LL * h->num_sms - 1) / (2LL * h->num_sms);
-    r = ((r + 15) / 16) * 16;
-    return (int)std::max<long long>(16, r);
+    const long long warps = 16LL * h->num_sms;
+    long long r = (pairs * h->dw_chunks + warps - 1) / warps;
+    r = ((r + 31) / 32) * 32;
+    return (int)std::max<long long>(32, r);
 }
 
 template <typename TY, typename TX>
-static cudaError_t launch_route_grad(beam_moe* h, const TX* x, const float* dy, int T_, float reg,
-                                     float* dx, float* dgl, float* dml, float* dgh, cudaStream_t st)
+static cudaError_t launch_route_grad(beam_moe* h, const float* dy, int T_, float reg, float* dx,
+                                     float* dgl, float* dml, float* dgh, cudaStream_t st)
 {
-    (void)x;
     const YOut& yr = h->last_yr;
-    const int Tr = ceil_div(T_, h->S);
-    const int K = h->K;
+    const int S = h->S, K = h->K;
+    // one CTA per routed row (a token, or a segment)
+    const unsigned grid = (unsigned)ceil_div(T_, S);
 #define BEAM_RG(KM)                                                                              \
-    launch(h, ST_ROUTE_GRAD, route_grad_kernel<TY, TX, KM>, dim3(Tr), dim3(kGradThreads), 0, st, \
+    launch(h, ST_ROUTE_GRAD, route_grad_kernel<TY, TX, KM>, dim3(grid), dim3(kGradThreads), 0, st, \
            (const TY*)yr.base, yr.splits, yr.stride, (const int*)h->inv, (const int*)h->topk_id, \
            (const float*)h->gate, (const float*)h->mlogit, dy, (const TX*)h->wrm, T_, K, h->E,  \
-           h->D, h->S, reg, dgh, dgl, dml, h->pair_grad, dx)
+           h->D, S, reg, dgh, dgl, dml, h->pair_grad, dx)
+    if (K <= 2) return BEAM_RG(2);
     if (K <= 4) return BEAM_RG(4);
     if (K <= 8) return BEAM_RG(8);
     if (K <= 16) return BEAM_RG(16);
@@ -1388,21 +1397,17 @@ static beam_status_t backward_impl(beam_moe* h, const TX* x, const float* dy, in
     const float reg = (float)((double)reg_scale / ((double)T_ * (double)K));
     // 1. per routed row: the K dots with dy, the logit gradients, dx
     const cudaError_t e1 = h->last_yr.f16
-        ? launch_route_grad<__half, TX>(h, x, dy, T_, reg, dx, dgl, dml, dgh, st)
-        : launch_route_grad<float, TX>(h, x, dy, T_, reg, dx, dgl, dml, dgh, st);
+        ? launch_route_grad<__half, TX>(h, dy, T_, reg, dx, dgl, dml, dgh, st)
+        : launch_route_grad<float, TX>(h, dy, T_, reg, dx, dgl, dml, dgh, st);
     BEAM_CUDA(e1);
-    // 2. per (unit of one expert's pairs, column slice): partial dW columns
-    constexpr int N = Vec<TX>::N;
-    const int slices = ceil_div(D, 256 * N);
-    const int R = dw_rows_per_unit(h, T_, slices);
-    const int units = ceil_div((long long)T_ * K, R) + E;
-    BEAM_CUDA(launch(h, ST_ROUTE_DW, route_dw_partial_kernel<TX>, dim3(units, slices), dim3(256), 0,
-                     st, (const int*)h->offsets, (const int*)h->perm,
-                     (const float2*)h->pair_grad, x, K, E, D, h->S, R, h->dw_part));
-    // 3. each expert's partials in unit order
-    BEAM_CUDA(launch(h, ST_ROUTE_DW_REDUCE, route_dw_reduce_kernel,
-                     dim3(ceil_div((long long)E * D, 256)), dim3(256), 0, st,
-                     (const int*)h->offsets, (const float*)h->dw_part, E, D, R, dwr, dwm));
+    // 2. dW: one warp per (unit of one expert's pairs, column chunk), then the expert's
+    // partials in unit order
+    const int R = dw_rows_per_unit(h, T_);
+    const long long items = ((long long)ceil_div((long long)T_ * K, R) + E) * h->dw_chunks;
+    BEAM_CUDA(launch(h, ST_ROUTE_DW, route_dw_kernel<TX>, dim3((unsigned)ceil_div(items, 8)),
+                     dim3(256), 0, st, (const int*)h->offsets, (const int*)h->perm,
+                     (const float2*)h->pair_grad, x, K, E, D, h->S, R, h->dw_chunks, h->dw_part,
+                     h->dw_cnt, dwr, dwm));
     return BEAM_OK;
 }
 

@@ -173,7 +173,7 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * each stage's time covers the work of one problem.  A fused decode forward is one launch,
  * timed as the stage fused_decode.
  */
-#define BEAM_N_STAGES 19
+#define BEAM_N_STAGES 18
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);

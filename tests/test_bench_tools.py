@@ -88,14 +88,14 @@ def test_record_traffic_reads_ncu_csv(tmp_path, monkeypatch):
     ])
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda stage="": "abc")
     args = types.SimpleNamespace(record_traffic=str(csv), traffic_kernel=r"tc_grouped_gemm_kernel<(\(int\))?0,",
                                  traffic_stage="tc_gateup", traffic_command="ncu ...",
                                  workload="mixtral-prefill")
     bench.record_traffic(args)
     assert bench.recorded_traffic("tc_gateup", "mixtral-prefill") == 1_650_000_000
     assert bench.recorded_traffic("tc_down", "mixtral-prefill") is None
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "changed")
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda stage="": "changed")
     assert bench.recorded_traffic("tc_gateup", "mixtral-prefill") is None
 
 
