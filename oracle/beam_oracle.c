@@ -1,5 +1,6 @@
 /*
- * beam_oracle.c -- plain, slow, fp64 CPU oracle of the BEAM masked MoE-layer forward.
+ * beam_oracle.c -- plain, slow, fp64 CPU oracle of the BEAM masked MoE-layer forward, and of
+ * the training-side gradient of its routing (oracle_route_backward, at the end of the file).
  *
  * TEST INFRASTRUCTURE ONLY.  This file is the correctness reference for the CUDA library.
  * Only the test suite, the package smoke check and the bench's CPU-baseline leg may load it.

@@ -50,6 +50,34 @@ def test_layer_work_joint_launches_carry_both_problems():
     assert jnt["swiglu_finish"]["bytes"] == sep["swiglu_finish"]["bytes"] + sep["shared_swiglu_finish"]["bytes"]
 
 
+def test_grad_work_counts_each_array_once():
+    """The routing gradient's algorithmic bytes: route_grad reads dy and every Top-K slot's
+    expert row and writes dx once; segment routing only changes the routed rows of x that the
+    dW pass reads, and the fp32 streaming path keeps expert rows in fp32."""
+    spec = synth.SPECS["mixtral"]
+    T, D, E, K = 4096, 4096, 8, 2
+    w = bench.grad_work(spec, T)
+    assert w["route_grad"]["bytes"] == 2 * T * D * 4 + T * K * D * 2 + 2 * E * D * 2 + 36 * T * K
+    assert w["route_dw"]["bytes"] == T * D * 2 + 12 * T * K + 8 * D * E
+    w32 = bench.grad_work(spec, T, tc_path=False)
+    assert w32["route_grad"]["bytes"] - w["route_grad"]["bytes"] == T * K * D * 2
+    seg = spec.with_(segment_len=16)
+    ws = bench.grad_work(seg, T)
+    assert ws["route_grad"]["bytes"] == w["route_grad"]["bytes"]
+    assert w["route_dw"]["bytes"] - ws["route_dw"]["bytes"] == (T - T // 16) * D * 2
+    assert set(w) == bench.GRAD_STAGES
+
+
+def test_forward_traffic_hash_ignores_the_gradient_source():
+    """Recorded DRAM traffic of a forward kernel stays valid when only the routing gradient's
+    source changes; the gradient's own stages hash it."""
+    fwd = bench.kernel_source_hash("tc_gateup")
+    grad = bench.kernel_source_hash("route_grad")
+    assert fwd != grad
+    assert bench.kernel_source_hash("tc_down") == fwd
+    assert bench.kernel_source_hash("route_dw") == grad
+
+
 def test_layer_work_without_shared_experts_has_empty_shared_problem():
     spec = synth.LayerSpec("w", 1024, 8, 2, 512)
     w, _ = bench.layer_work(spec, 64, STATS)
