@@ -19,6 +19,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -143,7 +144,9 @@ class ClockSampler:
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # raw samples: BEAM_BENCH_OUT if set, else the system temporary directory
+        out = os.environ.get("BEAM_BENCH_OUT") or tempfile.gettempdir()
+        self.path = os.path.join(out, f"clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         try:

@@ -336,6 +336,7 @@ beam_status_t beam_moe_forward_routed(beam_moe_t *h, const void *x_dev, int32_t 
  *   d_mask_logit_dev and dghat_dev [T][K] float32 are optional outputs (NULL to skip) holding
  *   the per-slot gradients above (0 at the tokens of a segment after its first) and s.
  * Every sum runs in a fixed order: the same inputs give the same bits.  T = 0 is a no-op.
+ * The call allocates nothing: its workspace was allocated with the handle.
  */
 beam_status_t beam_moe_backward_router(beam_moe_t *h, const void *x_dev, const float *dy_dev,
                                        int32_t T, float reg_scale, float *dw_router_dev,
