@@ -12,12 +12,18 @@ the mask m by m0 + sigmoid(l) - sigmoid(l0), which equals m at the base point an
 d/dl = sigmoid'(l); the Top-K set and the expert outputs are held at their base values (the
 selection is piecewise constant; the experts' own gradient is not part of the routing's).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synth
+from tests.test_oracle_pins import closed_form
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 def _f64(t):
@@ -188,3 +194,22 @@ def test_selected_rows_agree_with_the_full_pass():
     for t in (2, 6, 8):
         assert np.array_equal(part.dx[t], full.dx[t])
         assert np.array_equal(part.d_l[t], full.d_l[t])
+
+
+def test_hand_worked_gradient():
+    """A one-token layer whose gradient is derived by hand in tests/golden (closed forms)."""
+    with open(os.path.join(GOLDEN, "hand_worked_backward.json")) as f:
+        case = json.load(f)["cases"][0]
+    f32 = lambda a: torch.tensor(np.array(a, dtype=np.float64), dtype=torch.float32)
+    cf = lambda rows: np.array([[closed_form(v) for v in row] for row in rows])
+    w = dict(w_router=f32(cf(case["w_router"])), w_mask=f32(cf(case["w_mask"])),
+             w_gate=f32(case["w_gate"]), w_up=f32(case["w_up"]), w_down=f32(case["w_down"]))
+    x = f32(case["x"])
+    r = oracle.route(x, w["w_router"], w["w_mask"], case["K"])
+    ex = case["expect"]
+    np.testing.assert_array_equal(r.topk_id, np.array(ex["topk_id"]))
+    got = oracle.route_backward(x, w, r, np.array(case["dy"]), reg_scale=case["reg_scale"])
+    # ln 3 and 1/2 pass through float32 inputs, hence rtol 1e-6
+    for name, val in (("s", got.s), ("d_gate_logit", got.d_r), ("d_mask_logit", got.d_l),
+                      ("dw_router", got.dw_r), ("dw_mask", got.dw_m), ("dx", got.dx)):
+        np.testing.assert_allclose(val, cf(ex[name]), rtol=1e-6, atol=1e-12, err_msg=name)
