@@ -390,13 +390,20 @@ def train_point(torch, name, steps, warmup, device, peaks):
 
 def roofline_for(stage, work, ms_per_launch, peaks, workload):
     """Roofline of one kernel against its binding resource: tensor peak for a tensor-core
-    kernel whose FLOPs take longer than its bytes at HBM speed, HBM bandwidth otherwise."""
+    kernel whose FLOPs take longer than its bytes at HBM speed, HBM bandwidth otherwise.
+    The tensor peak is the measured burst bf16 figure: every kernel here is timed inside a
+    loop of steps far shorter than the seconds-long loop that settles the sustained figure (the
+    clocks sampled during the timed region stay at the maximum); the sustained peak is given
+    beside it (`peak_sustained`, `frac_of_sustained`).  frac = algorithmic FLOPs (or bytes) per
+    launch / ms_per_launch / peak."""
     t_bytes = work["bytes"] / (peaks["hbm"] * 1e9)
-    t_flops = work["flops"] / (peaks["tc_sustained"] * 1e12)
+    t_flops = work["flops"] / (peaks["tc"] * 1e12)
     if stage in TENSOR_STAGES and t_flops >= t_bytes:
         achieved = work["flops"] / (ms_per_launch * 1e-3) / 1e12
-        peak = peaks["tc_sustained"]
-        out = dict(bound="tensor", achieved=round(achieved, 2), peak=peak, unit="TFLOP/s")
+        peak = peaks["tc"]
+        out = dict(bound="tensor", achieved=round(achieved, 2), peak=peak, unit="TFLOP/s",
+                   peak_sustained=peaks["tc_sustained"],
+                   frac_of_sustained=round(achieved / peaks["tc_sustained"], 4))
     else:
         achieved = work["bytes"] / (ms_per_launch * 1e-3) / 1e9
         peak = peaks["hbm"]
@@ -407,11 +414,29 @@ def roofline_for(stage, work, ms_per_launch, peaks, workload):
     out["ms_per_launch"] = round(ms_per_launch, 5)
     out["algorithmic_bytes"] = int(work["bytes"])
     out["algorithmic_flops"] = int(work["flops"])
-    out["peak_source"] = peaks["source"] + (" (sustained bf16)" if out["bound"] == "tensor" else "")
+    out["peak_source"] = peaks["source"] + (" (burst bf16)" if out["bound"] == "tensor" else " (HBM copy)")
     return out
 
 
 # ------------------------------------------------------------------ our arm
+def workload_config(spec, T, keep, world, sbytes) -> dict:
+    """The `config` of a workload's JSON line, the same on both arms: the layer shape, the batch,
+    the keep rate and mask setting, how the L2 is kept from serving one step from the last, and
+    the parallelism (N independent replicas)."""
+    return {
+        "workload": f"{spec.name}-like layer, {'prefill' if T > 64 else 'decode'} T={T}, "
+                    f"keep rate {keep if keep else 1.0}",
+        "d_model": spec.d_model, "n_experts": spec.n_experts, "top_k": spec.top_k,
+        "d_ff": spec.d_ff, "n_shared": spec.n_shared, "d_ff_shared": spec.d_ff_shared,
+        "segment_len": spec.segment_len, "tokens_per_gpu": T, "keep_rate": keep,
+        "mask": "off" if keep is None else "on",
+        "l2": L2_LABEL_FLUSHED if sbytes < L2_FLUSH_BELOW_BYTES else
+              "inputs larger than L2 (the expert weights one step reads exceed the 126 MB L2); "
+              "no flush between steps",
+        "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
+    }
+
+
 def workload_spec(name):
     import synth
     entry = WORKLOADS[name]
@@ -449,26 +474,88 @@ def job_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
     return tokens_per_rank * world / (ms_max * 1e-3)
 
 
-def time_steps(torch, dist, layer, x, y, steps, warmup, mask_off, world):
+# A point whose algorithmic bytes per step are below this is timed with the L2 flushed between
+# steps (its working set could otherwise stay in the 126 MB L2 from one step to the next).
+L2_FLUSH_BELOW_BYTES = 1 << 30
+L2_LABEL_FLUSHED = "flushed between timed steps (256 MB written, then read; each step has its own event pair)"
+
+
+def l2_label(step_bytes: int) -> str:
+    return (L2_LABEL_FLUSHED if step_bytes < L2_FLUSH_BELOW_BYTES else
+            f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB of algorithmic bytes per step against "
+            "the 126 MB L2); no flush between steps")
+
+
+def reference_step_bytes(spec, T, keep, w, x) -> int:
+    """Algorithmic bytes per step from the oracle's routing of the whole batch (the reference
+    arm runs no GPU forward to read them from)."""
+    import oracle
+    r = oracle.route(x, w["w_router"], w["w_mask"], spec.top_k, segment_len=spec.segment_len,
+                     mask_off=keep is None)
+    counts, _, _, _ = oracle.compact(r, spec.n_experts)
+    st = dict(n_active_experts=int((counts > 0).sum()), n_kept=int(counts.sum()))
+    _, total = layer_work(spec, T, st)
+    return total["bytes"]
+
+
+class L2Flush:
+    """Evicts the L2 between timed steps: a 256 MB buffer written, then read (no dirty line of
+    it is left to be written back inside the next step's time)."""
+
+    def __init__(self, torch, device):
+        self.buf = torch.empty(64 << 20, dtype=torch.float32, device=device)
+        self.sink = torch.empty((), dtype=torch.float32, device=device)
+        self.torch = torch
+
+    def __call__(self):
+        self.buf.zero_()
+        self.torch.sum(self.buf, dim=0, out=self.sink)
+
+
+def time_steps(torch, dist, layer, x, y, steps, warmup, mask_off, world, flush=None):
+    """ms per step over `steps` forwards after `warmup` ones, max over ranks.  Without `flush`
+    the steps run back to back between one event pair; with it, each step has its own event
+    pair and the L2 is flushed before it, outside the timed region."""
     for _ in range(warmup):
         layer.forward(x, mask_off=mask_off, out=y)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     st = torch.cuda.current_stream()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
     n0 = layer.launch_count()
-    a.record(st)
-    for _ in range(steps):
-        layer.forward(x, mask_off=mask_off, out=y)
-    b.record(st)
-    torch.cuda.synchronize()
+    if flush is None:
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(steps):
+            layer.forward(x, mask_off=mask_off, out=y)
+        b.record(st)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+    else:
+        pairs = []
+        for _ in range(steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            layer.forward(x, mask_off=mask_off, out=y)
+            b.record(st)
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in pairs) / steps
     launches = layer.launch_count() - n0
-    ms = a.elapsed_time(b) / steps
     if world > 1:
         dist.barrier()
     return max_over_ranks(torch, dist, ms, world, x.device), launches
+
+
+def step_bytes(torch, layer, x, y, spec, T, mask_off):
+    """Algorithmic bytes of one forward of this layer on x (from one untimed forward's stats)."""
+    layer.forward(x, mask_off=mask_off, out=y)
+    st = layer.stats()
+    _, total = layer_work(spec, T, st)
+    return total["bytes"]
 
 
 def point(torch, dist, name, steps, warmup, world, device, peaks, mask_off=False):
@@ -481,10 +568,14 @@ def _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off):
     spec, T, keep, layer, x = build_layer(torch, name, device)
     y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
     mo = mask_off or keep is None
-    ms, _ = time_steps(torch, dist, layer, x, y, steps, warmup, mo, world)
+    sb = step_bytes(torch, layer, x, y, spec, T, mo)
+    flush = L2Flush(torch, device) if sb < L2_FLUSH_BELOW_BYTES else None
+    ms, _ = time_steps(torch, dist, layer, x, y, steps, warmup, mo, world, flush=flush)
     st = layer.stats()
     layer.profile_begin(steps)
     for _ in range(steps):
+        if flush is not None:
+            flush()
         layer.forward(x, mask_off=mo, out=y)
     prof = layer.profile_end()
     work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof,
@@ -496,6 +587,7 @@ def _point(torch, dist, name, steps, warmup, world, device, peaks, mask_off):
     t_roof = max(total["bytes"] / (peaks["hbm"] * 1e9), total["flops"] / (peaks["tc"] * 1e12))
     layer.close()
     return dict(workload=name, tokens=T, keep_rate=keep, mask="off" if mo else "on",
+                l2=l2_label(sb),
                 value=round(job_throughput(T, world, ms), 2), ms_per_step=round(ms, 5),
                 avg_k=round(st["avg_k"], 4), n_active_experts=st["n_active_experts"],
                 layer_roofline_frac=round(t_roof / (ms * 1e-3), 4), roofline=rl,
@@ -510,8 +602,11 @@ def spread_sample(T: int, n: int):
     return np.unique(np.linspace(0, T - 1, n).round().astype(np.int64))
 
 
-def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_steps=None):
-    """Time the fp64 oracle on a bounded sample of the workload (tokens/s on host cores)."""
+def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_steps=None,
+                 keep_outputs=None):
+    """Time the fp64 oracle on a bounded sample of the workload (tokens/s on host cores).
+    keep_outputs (a dict), if given, receives the sample, the oracle's y on it, the weights and
+    x on the host, for the parity leg."""
     import numpy as np
     import torch
     import oracle
@@ -526,12 +621,66 @@ def cpu_baseline(spec, T, keep, weights_dev, x_dev, budget_s=15.0, reference_ste
     threads = oracle.num_threads()
     sel = spread_sample(T, int(budget_s * threads / per_tok))
     t0 = time.perf_counter()
-    xs = x[torch.from_numpy(sel).long()]
-    r = oracle.route(xs, w["w_router"], w["w_mask"], spec.top_k, mask_off=keep is None)
-    oracle.layer(xs, w, r)
+    # the routing of every token (cheap next to the experts; segment routing needs the
+    # leaders), then Step 4 for the sampled tokens
+    r = oracle.route(x, w["w_router"], w["w_mask"], spec.top_k, segment_len=spec.segment_len,
+                     mask_off=keep is None)
+    y_ref = oracle.layer(x, w, r, tokens=sel)
     dt = time.perf_counter() - t0
+    if keep_outputs is not None:
+        keep_outputs.update(sel=sel, y_ref=y_ref, w=w, x=x)
     return dict(value=round(len(sel) / dt, 4), unit="tokens/s", cores=threads, kind="oracle",
-                sample=f"{len(sel)} of {T} tokens spread evenly over the batch, routing + experts, fp64")
+                sample=f"routing of all {T} tokens, then the experts of {len(sel)} tokens spread "
+                       "evenly over the batch (tokens/s counts the sampled tokens), fp64")
+
+
+def parity_leg(spec, T, keep, y_gpu, gr, ref) -> dict:
+    """The timed forward's output against the fp64 oracle, outside any timed region: routing
+    on every token (bit-exact ids / keep / perm on clean tokens, unclean ones counted), y on the
+    CPU baseline's token sample.  A sampled token whose decision differs from the oracle's (only
+    possible inside the 1e-3 margin) is compared under the GPU's decision, which must itself be
+    valid within the margin; the error against the oracle's own decisions is given beside."""
+    import numpy as np
+    import oracle
+    from tests import parity
+    w, x, sel, y_own = ref["w"], ref["x"], ref["sel"], ref["y_ref"]
+    mask_off = keep is None
+    out = dict(routing_tokens=T, y_tokens=int(len(sel)), tolerance=(
+        dict(max_abs=parity.TOL_BF16_ABS, rel_l2=parity.TOL_BF16_REL) if spec.storage == "bf16"
+        else dict(rel_l2=parity.TOL_F32_REL)))
+    orr = oracle.route(x, w["w_router"], w["w_mask"], spec.top_k, segment_len=spec.segment_len,
+                       mask_off=mask_off)
+    ok = True
+    try:
+        info = parity.compare_routing(gr, orr, spec.n_experts)
+        parity.check_structure(gr, T, spec.top_k, spec.n_experts)
+    except AssertionError as e:
+        ok = False
+        clean = orr.clean()
+        info = dict(clean=int(clean.sum()), unclean=int((~clean).sum()))
+        out["routing_error"] = str(e)[:200]
+    out.update(clean=info["clean"], unclean=info["unclean"])
+    ids_same = np.array([set(gr["topk_id"][t].tolist()) == set(orr.topk_id[t].tolist()) and
+                         {int(e): int(k) for e, k in zip(gr["topk_id"][t], gr["keep"][t])} ==
+                         {int(e): int(k) for e, k in zip(orr.topk_id[t], orr.keep[t])}
+                         for t in sel])
+    yg = np.asarray(y_gpu, np.float64)[sel]
+    y_ref = np.array(y_own, np.float64, copy=True)
+    differ = np.nonzero(~ids_same)[0]
+    out["differing_tokens"] = int(differ.size)
+    if differ.size:
+        try:
+            gdec, _ = parity.gpu_decision_routing(gr, x, w["w_router"], w["w_mask"], spec.top_k,
+                                                  spec.segment_len, mask_off)
+            y_ref[differ] = oracle.layer(x, w, gdec, tokens=sel[differ])
+        except AssertionError as e:
+            ok = False
+            out["decision_error"] = str(e)[:200]
+    rep = parity.y_report(yg, y_ref, spec.storage)
+    own = parity.y_report(yg, y_own, spec.storage)
+    out.update(max_abs=rep["max_abs"], rel_l2=rep["rel_l2"], max_abs_own_decision=own["max_abs"],
+               rel_l2_own_decision=own["rel_l2"], ok=bool(ok and rep["ok"]))
+    return out
 
 
 def run_ours(args):
@@ -561,16 +710,25 @@ def _run_ours(args):
     spec, T, keep, layer, x = build_layer(torch, name, device)
     y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
     mask_off = keep is None
+    sb = step_bytes(torch, layer, x, y, spec, T, mask_off)
+    flush = L2Flush(torch, device) if sb < L2_FLUSH_BELOW_BYTES else None
     sampler = ClockSampler(gpu_uuid(torch, device))
     with sampler:
-        ms, launches = time_steps(torch, dist, layer, x, y, args.steps, args.warmup, mask_off, world)
+        ms, launches = time_steps(torch, dist, layer, x, y, args.steps, args.warmup, mask_off,
+                                  world, flush=flush)
     clocks = sampler.summary()
     st = layer.stats()
     # per-kernel timing pass (same K steps, events around every kernel)
     layer.profile_begin(args.steps)
     for _ in range(args.steps):
+        if flush is not None:
+            flush()
         layer.forward(x, mask_off=mask_off, out=y)
     prof = layer.profile_end()
+    # the timed forward's output and routing, for the parity leg (deterministic: every step
+    # gives the same bits)
+    y_head = y.cpu().numpy() if rank == 0 and world == 1 and not args.no_cpu_baseline else None
+    gr_head = layer.routing(T) if y_head is not None else None
     work, total = layer_work(spec, T, st, tc_path="tc_gateup" in prof,
                              joint=spec.n_shared > 0 and "tc_gateup" in prof
                              and "tc_shared_gateup" not in prof)
@@ -605,11 +763,15 @@ def _run_ours(args):
     ms_off, _ = time_steps(torch, dist, layer, x, y, args.steps, args.warmup, True, world)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    par = None
+    if y_head is not None:
         import synth
         wcpu = synth.make_layer(spec, seed=0, keep_rate=keep if keep else 0.5, device=device)
-        cpu = cpu_baseline(spec, T, keep, wcpu, x, budget_s=args.cpu_budget)
+        ref = {}
+        cpu = cpu_baseline(spec, T, keep, wcpu, x, budget_s=args.cpu_budget, keep_outputs=ref)
         del wcpu
+        par = parity_leg(spec, T, keep, y_head, gr_head, ref)
+        del ref
     layer.close()
     del layer, x, y
     torch.cuda.empty_cache()
@@ -642,16 +804,11 @@ def _run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16" if spec.storage == "bf16" else "f32",
             "data": "synthetic (seeded; random-init weights of the layer shape)",
-            "config": {
-                "workload": f"{spec.name}-like layer, {'prefill' if T > 64 else 'decode'} T={T}, "
-                            f"keep rate {keep if keep else 1.0}",
-                "d_model": spec.d_model, "n_experts": spec.n_experts, "top_k": spec.top_k,
-                "d_ff": spec.d_ff, "n_shared": spec.n_shared, "d_ff_shared": spec.d_ff_shared,
-                "tokens_per_gpu": T, "keep_rate": keep, "mask": "off" if mask_off else "on",
-                "avg_k": round(st["avg_k"], 4), "n_active_experts": st["n_active_experts"],
-                "l2": "expert weights exceed the 126 MB L2; no flush between steps",
-                "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
-            },
+            "config": workload_config(spec, T, keep, world, sb),
+            "routing_stats": {"avg_k": round(st["avg_k"], 4), "l_reg": round(st["l_reg"], 6),
+                              "n_active_experts": st["n_active_experts"], "n_kept": st["n_kept"],
+                              "n_tokens_all_masked": st["n_tokens_all_masked"]},
+            "parity": par,
             "roofline": rl,
             "layer_roofline_frac": round(t_roof / (ms * 1e-3), 4),
             "mask_off": {"value": round(job_throughput(T, world, ms_off), 2),
@@ -721,13 +878,13 @@ def run_reference(args):
     oracle.layer(x[:1], w, r1)
     per_tok = max(time.perf_counter() - t0, 1e-4) / threads
     budget = 150.0 / (args.steps + args.warmup)
-    sel = torch.from_numpy(spread_sample(T, int(budget / per_tok))).long()
-    xs = x[sel]
+    sel = spread_sample(T, int(budget / per_tok))
 
     def step():
-        r = oracle.route(xs, w["w_router"], w["w_mask"], spec.top_k,
-                         segment_len=0, mask_off=keep is None)
-        oracle.layer(xs, w, r)
+        # the routing of every token, then Step 4 of the sampled ones (as the CPU-baseline leg)
+        r = oracle.route(x, w["w_router"], w["w_mask"], spec.top_k,
+                         segment_len=spec.segment_len, mask_off=keep is None)
+        oracle.layer(x, w, r, tokens=sel)
 
     for _ in range(args.warmup):
         step()
@@ -743,12 +900,12 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; random-init weights of the layer shape)",
-        "config": {"workload": f"{spec.name}-like layer, T={T}, keep rate {keep}",
-                   "d_model": spec.d_model, "n_experts": spec.n_experts, "top_k": spec.top_k,
-                   "d_ff": spec.d_ff, "tokens_per_gpu": T, "keep_rate": keep},
+        "config": workload_config(spec, T, keep, int(os.environ.get("WORLD_SIZE", "1")),
+                                  reference_step_bytes(spec, T, keep, w, x)),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{len(sel)} of {T} tokens per step, spread evenly over the "
-                                   "batch, routing + experts, fp64"},
+                         "sample": f"per step: routing of all {T} tokens, then the experts of "
+                                   f"{len(sel)} tokens spread evenly over the batch (tokens/s counts "
+                                   "the sampled tokens), fp64"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -14,6 +14,7 @@ BEAM_ERR_CUDA = 3
 BEAM_ERR_UNSUPPORTED = 4
 BEAM_ERR_TIMEOUT = 5
 BEAM_ERR_NO_FORWARD = 6
+BEAM_ERR_RANGE = 7
 
 BEAM_DTYPE_F32 = 0
 BEAM_DTYPE_BF16 = 1
@@ -29,7 +30,8 @@ BEAM_N_STAGES = 18
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 STATUS_NAMES = {0: "BEAM_OK", 1: "BEAM_ERR_INVALID_ARG", 2: "BEAM_ERR_OOM", 3: "BEAM_ERR_CUDA",
-                4: "BEAM_ERR_UNSUPPORTED", 5: "BEAM_ERR_TIMEOUT", 6: "BEAM_ERR_NO_FORWARD"}
+                4: "BEAM_ERR_UNSUPPORTED", 5: "BEAM_ERR_TIMEOUT", 6: "BEAM_ERR_NO_FORWARD",
+                7: "BEAM_ERR_RANGE"}
 
 
 class BeamConfig(ctypes.Structure):

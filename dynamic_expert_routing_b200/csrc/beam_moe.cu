@@ -666,19 +666,21 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
 
 // ---------------------------------------------------------------- launch helper (PDL)
 // Every forward kernel goes through here: it is counted, launched with programmatic stream
-// serialisation, and (while profiling) bracketed by an event pair of its stage.
+// serialisation, and (while profiling) bracketed by an event pair of its stage.  h == nullptr
+// launches the kernel the same way without touching any handle state (no count, no events):
+// the allocation-free routing call uses that, so it never writes to the handle.
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_ex(beam_moe* h, int stage, bool coop, void (*kernel)(KArgs...), dim3 grid,
                              dim3 block, size_t smem, cudaStream_t st, Args&&... args)
 {
     cudaEvent_t ea = nullptr, eb = nullptr;
-    if (h->prof && h->prof_pool.size() >= 2) {
+    if (h && h->prof && h->prof_pool.size() >= 2) {
         ea = h->prof_pool.back(); h->prof_pool.pop_back();
         eb = h->prof_pool.back(); h->prof_pool.pop_back();
         cudaError_t e = cudaEventRecord(ea, st);
         if (e != cudaSuccess) return e;
     }
-    ++h->launches;
+    if (h) ++h->launches;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = grid;
     lc.blockDim = block;
@@ -827,7 +829,7 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
                          dim3(256), 0, st, (const float*)h->g1part, s1n, p.split_stride_routed,
                          (const int*)(routed ? h->offsets + E : h->zero_int), F, (__half*)h->hbuf,
                          (const float*)h->g1part_sh, s1n, p.split_stride_shared, rows_sh, Fsh,
-                         (__half*)h->hsh));
+                         (__half*)h->hsh, &h->dstats->err));
     } else if (swap1) {
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_SWAP>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
@@ -1120,15 +1122,20 @@ static __device__ __align__(256) unsigned char g_route_scratch[BEAM_ROUTE_NOALLO
 static std::mutex g_route_scratch_mu;
 static void* g_route_scratch_dev[256] = {};  // device address of the array, per device
 
-// Device address of the scratch array on the current device, looked up once per device (the
-// host-side name of a __device__ array is not a device address).
-static beam_status_t route_scratch_address(void** out)
+// Device address of the scratch array on the current device (the host-side name of a
+// __device__ array is not a device address).  It is looked up with cudaGetSymbolAddress on the
+// first call on each device, and again on every later call made while `st` is not capturing,
+// so a context that was reset and reloaded the module gets the new address; during a stream
+// capture (where the lookup could have to load the module) the cached address is used.
+static beam_status_t route_scratch_address(void** out, cudaStream_t st)
 {
     int dev = -1;
     BEAM_CUDA(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 256) return fail(BEAM_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    BEAM_CUDA(cudaStreamIsCapturing(st, &cs));
     std::lock_guard<std::mutex> lock(g_route_scratch_mu);
-    if (!g_route_scratch_dev[dev]) {
+    if (!g_route_scratch_dev[dev] || cs == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
         if (e != cudaSuccess || !p)
@@ -1146,7 +1153,8 @@ static cudaError_t launch_select_into(beam_moe* h, const float* L, int Tr, int T
                                       float* ghat, int* nkeep_tok, float* lreg_tok,
                                       cudaStream_t st)
 {
-    return launch(h, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256),
+    // launched without the handle (nullptr): the call leaves its launch count and profile alone
+    return launch(nullptr, ST_ROUTE_SELECT, route_select_kernel<EPL>, dim3(ceil_div(Tr, 8)), dim3(256),
                   0, st, L, h->n2E, 1, 0LL, Tr, T, h->E, h->K, h->S, mask_off, topk_id, gate,
                   mlogit, keep, ghat, nkeep_tok, lreg_tok, 0LL, 0LL, (uint32_t*)nullptr);
 }
@@ -1162,7 +1170,7 @@ static beam_status_t route_noalloc_impl(beam_moe* h, const T* x, int T_, int32_t
     float* L = reinterpret_cast<float*>(scratch);
     int* nkeep = reinterpret_cast<int*>(scratch + l_bytes);
     float* lreg = reinterpret_cast<float*>(scratch + l_bytes + (size_t)T_ * sizeof(int));
-    BEAM_CUDA(launch_router_gemv<T>(h, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, h->n2E, L, st));
+    BEAM_CUDA(launch_router_gemv<T>(nullptr, x, S, Tr, h->D, (const T*)h->wrm, h->n2E, h->n2E, L, st));
     cudaError_t e;
     switch ((h->E + 31) / 32) {
         case 1: e = launch_select_into<1>(h, L, Tr, T_, mask_off, topk_id, gate, mlogit, keep, ghat, nkeep, lreg, st); break;
@@ -1437,8 +1445,8 @@ beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, in
                     "T=%d needs %lld bytes of routing scratch; the static buffer holds %u bytes",
                     T, need, (unsigned)BEAM_ROUTE_NOALLOC_SCRATCH_BYTES);
     void* scratch = nullptr;
-    BEAM_TRY(route_scratch_address(&scratch));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    BEAM_TRY(route_scratch_address(&scratch, st));
     const int mask_off = (flags & BEAM_MASK_OFF) ? 1 : 0;
     unsigned char* sc = static_cast<unsigned char*>(scratch);
     if (h->cfg.dtype == BEAM_DTYPE_BF16)
@@ -1504,7 +1512,11 @@ beam_status_t beam_gen_sync(beam_gen_t* g)
     BEAM_CUDA(cudaEventSynchronize(g->core.done));
     DevStats ds;
     BEAM_CUDA(cudaMemcpy(&ds, g->core.dstats, sizeof ds, cudaMemcpyDeviceToHost));
-    if (ds.err) return fail(BEAM_ERR_TIMEOUT, "a bounded device wait ran out (code %d)", ds.err);
+    if (ds.err & ~ERR_FP16_RANGE)
+        return fail(BEAM_ERR_TIMEOUT, "a bounded device wait ran out (code %d)", ds.err);
+    if (ds.err & ERR_FP16_RANGE)
+        return fail(BEAM_ERR_RANGE, "an fp16 intermediate of the last forward (H = silu(gate) * up, "
+                    "or an expert output) was outside the fp16 range; y holds infinities");
     return BEAM_OK;
 }
 
@@ -1697,7 +1709,11 @@ beam_status_t beam_moe_stats(beam_moe_t* h, beam_moe_stats_t* out, int32_t* coun
     }
     DevStats ds;
     BEAM_CUDA(cudaMemcpy(&ds, h->dstats, sizeof ds, cudaMemcpyDeviceToHost));
-    if (ds.err) return fail(BEAM_ERR_TIMEOUT, "a bounded device wait ran out (code %d)", ds.err);
+    if (ds.err & ~ERR_FP16_RANGE)
+        return fail(BEAM_ERR_TIMEOUT, "a bounded device wait ran out (code %d)", ds.err);
+    if (ds.err & ERR_FP16_RANGE)
+        return fail(BEAM_ERR_RANGE, "an fp16 intermediate of the last forward (H = silu(gate) * up, "
+                    "or an expert output) was outside the fp16 range; y holds infinities");
     out->tokens = ds.tokens;
     out->avg_k = ds.tokens ? (double)ds.keep_sum / ds.tokens : 0.0;
     out->l_reg = ds.tokens ? ds.lreg_sum / ds.tokens : 0.0;

@@ -90,6 +90,14 @@ template <> __device__ __forceinline__ __half from_float<__half>(float v) {
 template <typename TX> struct HType { using type = float; };
 template <> struct HType<__nv_bfloat16> { using type = __half; };
 
+// fp16 range of the stored intermediates (H = silu(gate) * up and the unsplit expert outputs
+// of bf16 layers): a value that rounds to a finite fp16 has magnitude below 65520 (the midpoint
+// between the largest fp16, 65504, and the next power of two).  A kernel that stores a value
+// outside that range (or a NaN) sets this bit in the forward's error word; beam_moe_stats then
+// reports BEAM_ERR_RANGE instead of returning numbers that hold an infinity.
+constexpr int ERR_FP16_RANGE = 0x400;
+__device__ __forceinline__ bool fp16_out_of_range(float v) { return !(fabsf(v) < 65520.0f); }
+
 // Streaming 16-byte load through the read-only path, not kept in L1.
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     uint4 r;

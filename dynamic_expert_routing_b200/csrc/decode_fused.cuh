@@ -185,7 +185,9 @@ fused_decode_kernel(const __grid_constant__ FusedDecodeParams P)
                 g += __ldcg(src + q * st + b);
                 u += __ldcg(src + q * st + b + 128);
             }
-            (shared ? P.hsh : P.h)[r * FF + f] = __float2half_rn(silu_f(g) * u);
+            const float hv = silu_f(g) * u;
+            if (fp16_out_of_range(hv)) atomicOr(P.err, ERR_FP16_RANGE);
+            (shared ? P.hsh : P.h)[r * FF + f] = __float2half_rn(hv);
         }
         fence_for_tma_readers();
     }

@@ -71,7 +71,7 @@ __device__ __forceinline__ ItemView stream_item(const StreamArgs& a, long item, 
 
 // ---------------------------------------------------------------- warp-private TMA ring
 // Each warp streams its weight rows through its own ring of kRingNS shared-memory stages,
-// filled by 1-D bulk copies (cp.async.bulk, no multicast) that lane 0 issues kRingNS segments
+// filled by 1-D bulk copies (cp.async.bulk, one per segment) that lane 0 issues kRingNS segments
 // ahead of the computation; an mbarrier per stage signals arrival (transaction bytes).  A
 // stage is refilled once every lane of the warp has read it (__syncwarp + proxy fence).
 // This keeps kRingNS x (segment bytes) x (rows) in flight per warp independently of
@@ -312,8 +312,11 @@ stream_gateup_kernel(StreamArgs a)
                     if (i < mp) {
                         const float g = warp_sum(acc[2 * q][i]);
                         const float u = warp_sum(acc[2 * q + 1][i]);
-                        if (lane == 0)
-                            hout[(size_t)(p0 + i) * v.FF + f0 + q] = from_float<TH>(silu_f(g) * u);
+                        if (lane == 0) {
+                            const float hv = silu_f(g) * u;
+                            if (sizeof(TH) == 2 && fp16_out_of_range(hv)) atomicOr(a.err, ERR_FP16_RANGE);
+                            hout[(size_t)(p0 + i) * v.FF + f0 + q] = from_float<TH>(hv);
+                        }
                     }
                 }
             }

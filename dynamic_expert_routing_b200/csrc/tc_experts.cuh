@@ -21,8 +21,8 @@
 //     into K pieces run on otherwise idle SMs.  Each piece stores an f32 partial; the epilogue
 //     warp that arrives last at a sub-block (an atomic counter decides who, never the order)
 //     adds the pieces' partials in piece order and runs the normal epilogue on the sum;
-//   * tile 128 (tokens) x 256 x 64, TMA (cp.async.bulk.tensor, 128-byte swizzle, no cluster
-//     multicast) fills a 4-stage shared-memory ring guarded by mbarriers;
+//   * tile 128 (tokens) x 256 x 64; each CTA issues its own TMA loads (cp.async.bulk.tensor,
+//     128-byte swizzle) into a 4-stage shared-memory ring guarded by mbarriers;
 //   * warp 0 lane 0 issues TMA, warp 1 lane 0 issues tcgen05.mma (kind::f16, fp32
 //     accumulation in TMEM, double-buffered accumulators of 256 columns), warps 2..9 drain
 //     TMEM with tcgen05.ld (two warps per lane quadrant, each half the columns) and run the
@@ -392,7 +392,7 @@ enum Mode { MODE_PLAIN = 0, MODE_TAIL = 1, MODE_SWAP = 2 };
 // with the 33-word pitch the 32 lanes hit 32 different banks.  The column offset of `out`
 // must be a multiple of 8 (fp16) or 4 (f32) elements and ld a multiple of the same.
 __device__ __forceinline__ void store_rows_f16(const float* buf, __half* out, int ld, int nrows,
-                                               int lane)
+                                               int lane, bool& bad)
 {
     const int cg = (lane & 3) * 8;
 #pragma unroll
@@ -403,7 +403,10 @@ __device__ __forceinline__ void store_rows_f16(const float* buf, __half* out, in
             const float* s = buf + r * EPI_PITCH + cg;
             __half2 h[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(s[2 * j], s[2 * j + 1]);
+            for (int j = 0; j < 4; ++j) {
+                bad |= fp16_out_of_range(s[2 * j]) | fp16_out_of_range(s[2 * j + 1]);
+                h[j] = __floats2half2_rn(s[2 * j], s[2 * j + 1]);
+            }
             *reinterpret_cast<uint4*>(out + (size_t)r * ld + cg) = *reinterpret_cast<const uint4*>(h);
         }
     }
@@ -630,6 +633,7 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
         int acc = rs.acc;
         uint32_t aph = rs.aph;
         bool ok = rs.ok;
+        bool bad = false;                // an fp16 store of this thread was out of range
         const int lb = 32 * (warp & 3);  // TMEM lanes this warp may access
         const int warp_e = warp - 2;     // index of this epilogue warp (its staging buffer)
         const int half = warp_e / 4;     // which half of the tile's columns this warp drains
@@ -672,7 +676,11 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                         __half* col = out + (size_t)(t.row0 + r0h) * ld + (size_t)t.n * (BN / 2) + lb + lane;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            if (i < nr) *col = __float2half_rn(silu_f(g[i]) * u[i]);
+                            if (i < nr) {
+                                const float hv = silu_f(g[i]) * u[i];
+                                bad |= fp16_out_of_range(hv);
+                                *col = __float2half_rn(hv);
+                            }
                             col += ld;
                         }
                     }
@@ -686,7 +694,10 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                                       half * BM + lb + lane;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            if (i < nr) *col = __float2half_rn(v[i]);
+                            if (i < nr) {
+                                bad |= fp16_out_of_range(v[i]);
+                                *col = __float2half_rn(v[i]);
+                            }
                             col += ld;
                         }
                     }
@@ -759,7 +770,7 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                         for (int i = 0; i < 32; ++i) buf[lane * EPI_PITCH + i] *= v[i];
                     }
                     __syncwarp();
-                    store_rows_f16(buf, out + row_base * ld + (size_t)t.n * (BN / 2) + 32 * j, ld, nrows, lane);
+                    store_rows_f16(buf, out + row_base * ld + (size_t)t.n * (BN / 2) + 32 * j, ld, nrows, lane, bad);
                     __syncwarp();
                 }
             } else {
@@ -779,7 +790,7 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                     const size_t off = (size_t)t.ks * sstride + row_base * ld + (size_t)t.n * BN + 32 * j;
                     if (EPI == EPI_STORE_F16)
                         store_rows_f16(buf, static_cast<__half*>(t.shared ? p.out_shared : p.out_routed) + off,
-                                       ld, nrows, lane);
+                                       ld, nrows, lane, bad);
                     else
                         store_rows_f32(buf, static_cast<float*>(t.shared ? p.out_shared : p.out_routed) + off,
                                        ld, nrows, lane);
@@ -793,6 +804,7 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                 if (++acc == 2) { acc = 0; aph ^= 1u; }
             }
         }
+        if (bad) atomicOr(p.err, ERR_FP16_RANGE);
         rs.acc = acc; rs.aph = aph; rs.ok = ok;
     }
 
@@ -826,9 +838,10 @@ __global__ void __launch_bounds__(256)
 swiglu_finish_kernel(const float* __restrict__ g, int splits, long long stride,
                      const int* __restrict__ n_rows_ptr, int F, __half* __restrict__ h,
                      const float* __restrict__ gsh, int splits_sh, long long stride_sh,
-                     int rows_sh, int Fsh, __half* __restrict__ hsh)
+                     int rows_sh, int Fsh, __half* __restrict__ hsh, int* __restrict__ err)
 {
     pdl_wait();
+    bool bad = false;
     const long long nr = (long long)(*n_rows_ptr) * F;
     const long long ns = (long long)rows_sh * Fsh;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nr + ns;
@@ -847,8 +860,11 @@ swiglu_finish_kernel(const float* __restrict__ g, int splits, long long stride,
             gate += src[s * st + base];
             up += src[s * st + base + 128];
         }
-        (shared ? hsh : h)[r * FF + f] = __float2half_rn(silu_f(gate) * up);
+        const float hv = silu_f(gate) * up;
+        bad |= fp16_out_of_range(hv);
+        (shared ? hsh : h)[r * FF + f] = __float2half_rn(hv);
     }
+    if (bad) atomicOr(err, ERR_FP16_RANGE);
     pdl_launch_dependents();
 }
 

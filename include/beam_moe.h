@@ -41,7 +41,9 @@ typedef enum {
     BEAM_ERR_CUDA = 3,         /* a CUDA runtime error; the message has the CUDA error string */
     BEAM_ERR_UNSUPPORTED = 4,  /* valid request this build cannot serve (e.g. tensor path in fp32) */
     BEAM_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out; outputs are not valid */
-    BEAM_ERR_NO_FORWARD = 6    /* beam_moe_stats / get_routing before any forward */
+    BEAM_ERR_NO_FORWARD = 6,   /* beam_moe_stats / get_routing before any forward */
+    BEAM_ERR_RANGE = 7         /* bf16 layers: an fp16 intermediate of the last forward (H, or an
+                                  expert output) overflowed; its y is not valid */
 } beam_status_t;
 
 enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
@@ -145,7 +147,10 @@ beam_status_t beam_moe_forward_host(beam_moe_t *h, const void *x_host, int32_t T
 /*
  * Statistics of the last forward; waits for it to finish.  counts_host, if not NULL,
  * receives the per-expert kept-slot counts (E int32).  Returns BEAM_ERR_TIMEOUT if a
- * bounded device wait of that forward ran out.
+ * bounded device wait of that forward ran out, and BEAM_ERR_RANGE if, in a bf16 layer, a value
+ * the forward stored in fp16 (H = silu(W_g x) * (W_u x), or an expert's unsplit output) had a
+ * magnitude of 65520 or more (it rounds to infinity) or was NaN: the kernels check every such
+ * store and set a bit of the forward's error word, so an overflow is reported, not silent.
  */
 beam_status_t beam_moe_stats(beam_moe_t *h, beam_moe_stats_t *out, int32_t *counts_host);
 
@@ -195,9 +200,14 @@ int64_t beam_moe_launch_count(const beam_moe_t *h);
  * ceil(ceil(T/S)*2E*4 / 256)*256 + 8*T bytes (S = segment length, 1 when off); a larger T is
  * rejected with BEAM_ERR_INVALID_ARG and a message giving both sizes.  The first call on
  * each device looks up the array's device address (cudaGetSymbolAddress) and caches it; make
- * that first call before any stream capture.  All calls share the array, so calls whose GPU
- * work overlaps (different streams or threads) race on it and must be serialised by the
- * caller.  flags: 0 or BEAM_MASK_OFF.  The handle's own buffers and statistics are untouched.
+ * that first call before any stream capture.  Later calls on a stream that is not capturing
+ * look it up again (so a reset context that reloaded the library's module is served); calls
+ * during a capture use the cached address.  All calls share the array and it keeps the last
+ * call's contents, so calls whose GPU work overlaps (different streams or threads) race on it
+ * and must be serialised by the caller.  flags: 0 or BEAM_MASK_OFF.  The handle's own buffers,
+ * statistics, launch count and profile are untouched (its weights are only read), so the call
+ * may be enqueued between forwards; like every call on a handle it must not run concurrently
+ * with another call on the same handle from a second host thread.
  */
 #define BEAM_ROUTE_NOALLOC_SCRATCH_BYTES (2u << 20)
 beam_status_t beam_moe_route_noalloc(beam_moe_t *h, const void *x_dev, int32_t T,

@@ -17,3 +17,22 @@ def pytest_configure(config):
 def _build_oracle():
     import oracle
     oracle.build()
+
+
+# One line per GPU parity case (filled by tests.gpu_util.run_case), printed at the end of the
+# run: the clean / unclean token counts of the routing comparison, the tokens whose decision
+# differs from the oracle's (inside the 1e-3 margin), and the y errors.
+PARITY_REPORT: list = []
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    if not PARITY_REPORT:
+        return
+    tr = terminalreporter
+    tr.section("parity report (GPU vs fp64 oracle)")
+    tr.write_line("case | tokens | clean | unclean | differing | y tokens | max|err| | rel-L2 | "
+                  "max|err| vs oracle decision | rel-L2 vs oracle decision")
+    for r in PARITY_REPORT:
+        tr.write_line(f"{r['case']} | {r['T']} | {r['clean']} | {r['unclean']} | {r['differing']} | "
+                      f"{r['y_tokens']} | {r['max_abs']:.3e} | {r['rel_l2']:.3e} | "
+                      f"{r['max_abs_own']:.3e} | {r['rel_l2_own']:.3e}")

@@ -27,7 +27,7 @@ def same_decision_tokens(gr: dict, orr) -> np.ndarray:
 
 def run_case(spec: synth.LayerSpec, T: int, seed: int = 0, keep_rate=0.5, mask_off=False,
              path=None, zero_mask=False, mask_bias=None, max_tokens=None, y_tokens=None,
-             layer=None, weights=None, x=None, fused=False):
+             layer=None, weights=None, x=None, fused=False, case=None):
     """Run the CUDA layer and the oracle on the same inputs; assert parity; return details."""
     from dynamic_expert_routing_b200 import BeamMoE
     big = spec.n_experts * spec.d_ff * spec.d_model * 3 > 50_000_000
@@ -65,9 +65,31 @@ def run_case(spec: synth.LayerSpec, T: int, seed: int = 0, keep_rate=0.5, mask_o
     assert abs(st["l_reg"] - l_reg) <= 1e-5 + info["unclean"] / T
     assert st["n_kept"] == int(gr["keep"].sum())
     np.testing.assert_array_equal(st["counts"], np.diff(gr["offsets"]))
+    # y on every compared token: the GPU's decision (checked to be valid within the margin;
+    # equal to the oracle's on every clean token) through the oracle's Step 4
     same = same_decision_tokens(gr, orr)
-    sel = np.nonzero(same)[0] if y_tokens is None else np.intersect1d(np.asarray(y_tokens), np.nonzero(same)[0])
-    y_ref = oracle.layer(x, weights, orr, tokens=sel)
-    info.update(parity.compare_y(y.cpu().numpy()[sel], y_ref, spec.storage))
+    sel = np.arange(T) if y_tokens is None else np.unique(np.asarray(y_tokens, np.int64))
+    gdec, near = parity.gpu_decision_routing(gr, x, weights["w_router"], weights["w_mask"],
+                                             spec.top_k, spec.segment_len, mask_off)
+    y_gpu = y.cpu().numpy()[sel]
+    y_ref = oracle.layer(x, weights, gdec, tokens=sel)
+    info.update(parity.compare_y(y_gpu, y_ref, spec.storage))
+    # reported: the error against the oracle's own decision on every compared token, and the
+    # tokens whose decision differs (all inside the margin)
+    differ = sel[~same[sel]]
+    if differ.size:
+        y_own = oracle.layer(x, weights, orr, tokens=sel)
+        own = parity.y_report(y_gpu, y_own, spec.storage)
+    else:
+        own = parity.y_report(y_gpu, y_ref, spec.storage)
+    info.update(y_tokens=int(sel.size), differing_tokens=differ.tolist(),
+                near_margin_tokens=int(near.sum()), max_abs_own_decision=own["max_abs"],
+                rel_l2_own_decision=own["rel_l2"])
+    from tests.conftest import PARITY_REPORT
+    PARITY_REPORT.append(dict(case=case or f"{spec.name} T={T}", T=T, clean=info["clean"],
+                              unclean=info["unclean"], differing=int(differ.size),
+                              y_tokens=int(sel.size), max_abs=info["max_abs"],
+                              rel_l2=info["rel_l2"], max_abs_own=own["max_abs"],
+                              rel_l2_own=own["rel_l2"]))
     info.update(layer=layer, y=y, routing=gr, oracle=orr, stats=st, weights=weights, x=x)
     return info

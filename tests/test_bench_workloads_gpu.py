@@ -1,0 +1,30 @@
+"""Parity on every workload the bench times: the same layer, token count, keep rate, mask
+setting and launch configuration (a non-default stream, the forward captured as a CUDA graph
+and replayed) as `bench.py --sweep`, against the fp64 oracle.
+
+Routing is compared on every token (bit-exact on clean tokens, unclean ones counted); y on 256
+tokens spread evenly over the batch (every token when the batch is at most 256), each under
+the GPU's decision after that decision is checked to be valid within the margin, with the
+error against the oracle's own decision reported alongside (tests/conftest.py prints one line
+per case at the end of the run).
+"""
+import numpy as np
+import pytest
+
+import bench
+from tests.gpu_util import run_case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", bench.SWEEP)
+def test_bench_workload_matches_oracle(name):
+    spec, T, keep = bench.workload_spec(name)
+    sample = bench.spread_sample(T, 256)
+    info = run_case(spec, T, keep_rate=keep if keep else 0.5, mask_off=keep is None,
+                    y_tokens=sample, case=name)
+    # an unclean leader makes its whole segment unclean
+    assert info["unclean"] <= 0.05 * T * max(1, spec.segment_len)
+    assert info["clean"] + info["unclean"] == T
+    layer = info["layer"]
+    layer.close()

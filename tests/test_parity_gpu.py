@@ -237,10 +237,10 @@ def test_model_shapes_decode(name, T, keep):
     ("fine_seg16", 8192, 0.5, False),
 ])
 def test_model_shapes_prefill(name, T, keep, mask_off):
-    """Full-size prefill on the path the bench times: routing on every token, y on a sample of
-    tokens spread over the batch (every 97th, plus the last)."""
+    """Full-size prefill on the path the bench times: routing on every token, y on 256 tokens
+    spread evenly over the batch (first and last included)."""
     spec = synth.SPECS[name]
-    sample = np.unique(np.concatenate([np.arange(0, T, 97), [T - 1]]))
+    sample = np.unique(np.linspace(0, T - 1, 256).round().astype(np.int64))
     info = run_case(spec, T, keep_rate=keep, mask_off=mask_off, y_tokens=sample)
     # with segment routing an unclean leader makes its whole segment unclean
     assert info["unclean"] <= 0.05 * T * max(1, spec.segment_len)
@@ -506,4 +506,32 @@ def test_exact_ties_go_to_the_lower_expert(T, path):
     orr = oracle.route(x.cpu(), wr, w["w_mask"], spec.top_k)
     agree = (np.sort(ids, axis=1) == np.sort(orr.topk_id, axis=1)).all(axis=1)
     assert agree.mean() >= 0.95
+    layer.close()
+
+
+# ------------------------------------------------------------------ fp16 range of intermediates
+@pytest.mark.parametrize("T,path,fused", [(300, "tensor", False), (5, "tensor", False),
+                                          (5, "tensor", True), (40, "stream", False)],
+                         ids=["tensor_whole_k", "tensor_split_k", "fused_decode", "stream"])
+def test_fp16_overflow_of_h_is_reported(T, path, fused):
+    """bf16 layers store H = silu(W_g x) * (W_u x) (and the unsplit expert outputs) in fp16.
+    One token scaled by 1000 drives its shared expert's H far past 65504 (gate and up grow with
+    the scale, H with its square); the forward must then report BEAM_ERR_RANGE from
+    beam_moe_stats, on every expert path, while ordinary inputs before and after give BEAM_OK
+    (the error word is cleared by every forward)."""
+    from dynamic_expert_routing_b200 import BeamMoE, BeamError, _lib
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=T)
+    x = synth.make_tokens(spec, T, seed=3)
+    xs = x.clone()
+    xs[T // 2] *= 1000.0
+    layer.forward(x.cuda(), path=path, fused=fused)
+    assert layer.stats()["tokens"] == T
+    layer.forward(xs.cuda(), path=path, fused=fused)
+    with pytest.raises(BeamError) as ei:
+        layer.stats()
+    assert ei.value.status == _lib.BEAM_ERR_RANGE
+    layer.forward(x.cuda(), path=path, fused=fused)
+    assert layer.stats()["tokens"] == T
     layer.close()

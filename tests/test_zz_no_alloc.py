@@ -8,7 +8,9 @@ produces for the same tokens, twice in a row on different tokens, so the second 
 scratch the first one filled.  The two may compute the logits with a different fp32
 summation order (large bf16 batches use the tensor cores in the forward), so the comparison
 uses the routing tolerance of the parity tests: Top-K ids and keep bits equal wherever the
-decision margin exceeds 1e-3, gates and mask logits within 1e-4.
+decision margin exceeds 1e-3, gates and mask logits within 1e-4.  Each call is also compared
+with the fp64 oracle's routing: ids (in rank order where the ranks are 1e-3 apart) and keep
+bits exact on every clean token, gates and mask logits within 1e-4.
 
 This file is collected last so that a run stopping at the first failure has run every other
 test before it.
@@ -39,6 +41,19 @@ def _route_noalloc(lib, layer, x, flags=0):
     return st, {k: v.cpu().numpy() for k, v in out.items()}
 
 
+def _compare_oracle(got, orr, msg, margin=1e-3):
+    clean = orr.clean(margin)
+    assert clean.mean() >= 0.9, msg
+    for t in np.nonzero(clean)[0]:
+        assert set(got["topk_id"][t].tolist()) == set(orr.topk_id[t].tolist()), f"{msg}: token {t}"
+        if orr.rank_gap[t] > margin:
+            np.testing.assert_array_equal(got["topk_id"][t], orr.topk_id[t], err_msg=f"{msg}: token {t}")
+            np.testing.assert_array_equal(got["keep"][t], orr.keep[t], err_msg=f"{msg}: token {t}")
+            np.testing.assert_allclose(got["gate"][t], orr.g[t], atol=1e-4, err_msg=f"{msg}: token {t}")
+            np.testing.assert_allclose(got["mask_logit"][t], orr.mask_logit[t], atol=1e-4,
+                                       err_msg=f"{msg}: token {t}")
+
+
 def _compare(got, ref, msg, margin=1e-3):
     same_ids = (got["topk_id"] == ref["topk_id"]).all(axis=1)
     # a differing Top-K row is only acceptable at a near-tie of two gates
@@ -65,13 +80,20 @@ def test_route_noalloc_matches_forward_twice(spec, T):
     w = synth.make_layer(spec, keep_rate=0.5)
     layer = BeamMoE({k: v.cuda() for k, v in w.items() if isinstance(v, torch.Tensor)},
                     spec.top_k, max_tokens=T, segment_len=spec.segment_len)
+    import oracle
     for call, seed in enumerate((11, 12)):
-        x = synth.make_tokens(spec, T, seed=seed).cuda()
+        xc = synth.make_tokens(spec, T, seed=seed)
+        x = xc.cuda()
         layer.forward(x)
         ref = layer.routing(T)
+        n0 = layer.launch_count()
         st, got = _route_noalloc(lib, layer, x)
         assert st == _lib.BEAM_OK, lib.beam_moe_last_error()
+        assert layer.launch_count() == n0          # the handle's state is left alone
         _compare(got, ref, f"call {call}")
+        orr = oracle.route(xc, w["w_router"], w["w_mask"], spec.top_k,
+                           segment_len=spec.segment_len)
+        _compare_oracle(got, orr, f"call {call} vs oracle")
     # the mask-off flag keeps every Top-K slot
     st, got = _route_noalloc(lib, layer, x, flags=_lib.BEAM_MASK_OFF)
     assert st == _lib.BEAM_OK and got["keep"].all()
