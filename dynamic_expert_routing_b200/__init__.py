@@ -5,7 +5,7 @@ is its Python binding.  There is no CPU fallback: importing `BeamMoE` and creati
 requires the built library and a CUDA device.
 """
 from ._lib import (BEAM_MASK_OFF, BEAM_PATH_STREAM, BEAM_PATH_TENSOR, BeamError, LIB_PATH, load)
-from .layer import BeamGenerator, BeamMoE
+from .layer import BeamGenerator, BeamMoE, softtopk, softtopk_backward
 
-__all__ = ["BeamMoE", "BeamGenerator", "BeamError", "load", "LIB_PATH", "BEAM_MASK_OFF", "BEAM_PATH_STREAM",
+__all__ = ["BeamMoE", "BeamGenerator", "softtopk", "softtopk_backward", "BeamError", "load", "LIB_PATH", "BEAM_MASK_OFF", "BEAM_PATH_STREAM",
            "BEAM_PATH_TENSOR"]

@@ -107,6 +107,19 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.beam_gen_destroy.restype = None
     lib.beam_moe_forward_routed.argtypes = [P, P, I, ctypes.POINTER(BeamRouting), P, U, P]
     lib.beam_moe_backward_router.argtypes = [P, P, P, I, ctypes.c_float, P, P, P, P, P, P, P]
+    lib.beam_softtopk_forward.argtypes = [P, I, I, I, ctypes.c_float, P, P, P, P]
+    lib.beam_softtopk_backward.argtypes = [P, P, I, I, ctypes.c_float, P, P]
+    lib.beam_softtopk_forward.restype = ctypes.c_int
+    lib.beam_softtopk_backward.restype = ctypes.c_int
+    lib.beam_moe_create_ep.argtypes = [ctypes.POINTER(BeamConfig), ctypes.POINTER(BeamWeights), P,
+                                       ctypes.POINTER(P)]
+    lib.beam_moe_ep_dispatch.argtypes = [P, P, I, U, P, P, P]
+    lib.beam_moe_ep_combine.argtypes = [P, P, P, P]
+    lib.beam_ep_expert_range.argtypes = [I, I, I, ctypes.POINTER(I), ctypes.POINTER(I)]
+    lib.beam_ep_recv_routing.argtypes = [P, I, I, I, P, P, P, P, P, P]
+    for f in (lib.beam_moe_create_ep, lib.beam_moe_ep_dispatch, lib.beam_moe_ep_combine,
+              lib.beam_ep_expert_range, lib.beam_ep_recv_routing):
+        f.restype = ctypes.c_int
     lib.beam_moe_destroy.argtypes = [P]
     lib.beam_moe_destroy.restype = None
     lib.beam_moe_last_error.restype = ctypes.c_char_p

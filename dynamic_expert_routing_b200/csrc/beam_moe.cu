@@ -28,6 +28,7 @@
 #include "tc_experts.cuh"
 #include "decode_fused.cuh"
 #include "route_grad.cuh"
+#include "softtopk.cuh"
 
 using namespace beam;
 
@@ -147,6 +148,8 @@ struct YOut {
 struct beam_moe {
     beam_moe_config_t cfg;
     int E, K, D, F, Fsh, Tmax, S;
+    int Ew = 0;          // routed experts whose weights the handle holds: E, or 0 for the
+                         // routing-only handle of expert parallelism (beam_moe_create_ep)
     int n2E;             // 2E: router + mask logit columns
     int ldL;             // leading dimension of the logits and rows of the repacked router
     size_t esz;
@@ -218,6 +221,11 @@ struct beam_moe {
     int g_kernels = 0;   // kernels in the captured graph
     bool g_routed = false;
     RouteIn g_rin;       // routing pointers of a captured routed forward
+    // expert parallelism: the last beam_moe_ep_dispatch (token count, where the shared experts'
+    // output is, whether they ran on the side stream), read by beam_moe_ep_combine
+    int ep_T = -1;
+    YOut ep_ysh;
+    bool ep_fork = false;
     YOut g_yr;           // Y_perm of the captured forward
     // launch accounting and optional per-stage timing
     long long launches = 0;
@@ -395,19 +403,21 @@ template <typename T>
 static beam_status_t repack(beam_moe* h, const beam_moe_weights_t* w, cudaStream_t st)
 {
     using TH = typename HType<T>::type;
-    const int D = h->D, E = h->E, F = h->F;
+    const int D = h->D, E = h->E, F = h->F, Ew = h->Ew;
     repack_router_kernel<T><<<1024, 256, 0, st>>>(static_cast<const T*>(w->w_router),
                                                   static_cast<const T*>(w->w_mask), D, E, 1,
                                                   h->ldL, static_cast<T*>(h->wrm));
     BEAM_CUDA(cudaGetLastError());
-    repack_gateup_kernel<T><<<(unsigned)((long long)E * 2 * F), 128, 0, st>>>(
-        static_cast<const T*>(w->w_gate), static_cast<const T*>(w->w_up), E, F, D,
-        static_cast<T*>(h->wgu));
-    BEAM_CUDA(cudaGetLastError());
-    repack_down_kernel<T, TH><<<2048, 256, 0, st>>>(static_cast<const T*>(w->w_down),
-                                                    (long long)E * D * F, 1, D, F, 0,
-                                                    static_cast<TH*>(h->wd), h->range_flag);
-    BEAM_CUDA(cudaGetLastError());
+    if (Ew > 0) {
+        repack_gateup_kernel<T><<<(unsigned)((long long)Ew * 2 * F), 128, 0, st>>>(
+            static_cast<const T*>(w->w_gate), static_cast<const T*>(w->w_up), Ew, F, D,
+            static_cast<T*>(h->wgu));
+        BEAM_CUDA(cudaGetLastError());
+        repack_down_kernel<T, TH><<<2048, 256, 0, st>>>(static_cast<const T*>(w->w_down),
+                                                        (long long)Ew * D * F, 1, D, F, 0,
+                                                        static_cast<TH*>(h->wd), h->range_flag);
+        BEAM_CUDA(cudaGetLastError());
+    }
     if (h->Fsh > 0) {
         repack_gateup_kernel<T><<<(unsigned)(2LL * h->Fsh), 128, 0, st>>>(
             static_cast<const T*>(w->ws_gate), static_cast<const T*>(w->ws_up), 1, h->Fsh, D,
@@ -456,13 +466,20 @@ static beam_status_t setup_tc(beam_moe* h)
     memset(&b, 0, sizeof b);
     // GEMM1: X_perm [rows][D] x W_gu [E*2F][D] -> H (fp16) [rows][F]
     BEAM_TRY(encode_map(h, &a.a_routed, BF, h->xperm, rows, D, tc::BM));
-    BEAM_TRY(encode_map(h, &a.b_routed, BF, h->wgu, E * 2 * F, D, tc::BN));
+    if (h->Ew > 0) BEAM_TRY(encode_map(h, &a.b_routed, BF, h->wgu, E * 2 * F, D, tc::BN));
     // GEMM2: H [rows][F] x W_d [E*D][F] -> Y_perm (f32) [rows][D]
     BEAM_TRY(encode_map(h, &b.a_routed, HF, h->hbuf, rows, F, tc::BM));
-    BEAM_TRY(encode_map(h, &b.b_routed, HF, h->wd, E * D, F, tc::BN));
+    if (h->Ew > 0) BEAM_TRY(encode_map(h, &b.b_routed, HF, h->wd, E * D, F, tc::BN));
     // the same activations in boxes of kSwapBox rows, for the swapped small groups
     BEAM_TRY(encode_map(h, &a.a_routed_tail, BF, h->xperm, rows, D, tc::kSwapBox));
     BEAM_TRY(encode_map(h, &b.a_routed_tail, HF, h->hbuf, rows, F, tc::kSwapBox));
+    if (h->Ew == 0) {
+        // a routing-only handle holds no routed expert weights: its launches carry no routed
+        // group, so these maps are never read; they point at the router matrix so that every
+        // map a kernel is given (and prefetches) is a valid one
+        BEAM_TRY(encode_map(h, &a.b_routed, BF, h->wrm, (uint64_t)h->ldL, D, tc::BN));
+        BEAM_TRY(encode_map(h, &b.b_routed, BF, h->wrm, (uint64_t)h->ldL, D, tc::BN));
+    }
     if (Fsh) {
         BEAM_TRY(encode_map(h, &a.b_shared, BF, h->wsgu, 2 * Fsh, D, tc::BN));
         BEAM_TRY(encode_map(h, &b.a_shared, HF, h->hsh, Tm, Fsh, tc::BM));
@@ -562,10 +579,11 @@ static beam_status_t setup_tc(beam_moe* h)
 }
 
 static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_weights_t* w,
-                                 cudaStream_t st, beam_moe* h)
+                                 cudaStream_t st, beam_moe* h, bool routing_only = false)
 {
     h->cfg = *cfg;
     h->E = cfg->n_experts; h->K = cfg->top_k; h->D = cfg->d_model; h->F = cfg->d_ff;
+    h->Ew = routing_only ? 0 : h->E;
     h->Fsh = cfg->n_shared * cfg->d_ff_shared;
     h->Tmax = cfg->max_tokens;
     h->S = cfg->segment_len > 1 ? cfg->segment_len : 1;
@@ -584,8 +602,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     const size_t rows = Tm * K;  // upper bound on kept pairs
     BEAM_TRY(dalloc(h, &h->wrm, (size_t)h->ldL * D * es));
     BEAM_TRY(dalloc(h, &h->zero_int, 2 * sizeof(int)));
-    BEAM_TRY(dalloc(h, &h->wgu, E * 2 * F * D * es));
-    BEAM_TRY(dalloc(h, &h->wd, E * D * F * hs));
+    BEAM_TRY(dalloc(h, &h->wgu, (size_t)h->Ew * 2 * F * D * es));
+    BEAM_TRY(dalloc(h, &h->wd, (size_t)h->Ew * D * F * hs));
     BEAM_TRY(dalloc(h, &h->range_flag, sizeof(int)));
     if (Fsh) {
         BEAM_TRY(dalloc(h, &h->wsgu, 2 * Fsh * D * es));
@@ -894,9 +912,13 @@ static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, co
                   (const int*)h->inv, ghat, T_, h->K, h->D, y);
 }
 
+// ep_dispatch: stop after the compaction (expert parallelism, beam_moe_ep_dispatch): the kept
+// rows stay in X_perm for the caller's exchange, and the shared experts run on their own (on
+// the side stream on the tensor path), their output kept for beam_moe_ep_combine.
 template <typename T>
 static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uint32_t flags,
-                                  bool use_tc, cudaStream_t st, const RouteIn* rin = nullptr)
+                                  bool use_tc, cudaStream_t st, const RouteIn* rin = nullptr,
+                                  bool ep_dispatch = false)
 {
     const int E = h->E, K = h->K, D = h->D;
     const int S = h->S;
@@ -910,7 +932,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     // are short, and two streams of them would only add launches that wait for each other.
     BEAM_CUDA(cudaMemsetAsync(&h->dstats->err, 0, 2 * sizeof(int), st));  // err, grid_bar
     YOut ysh_out;
-    const bool fork = use_tc && h->Fsh > 0 && T_ > kSplitMaxTokens;
+    const bool fork = use_tc && h->Fsh > 0 && (T_ > kSplitMaxTokens || ep_dispatch);
     const bool joint = use_tc && h->Fsh > 0 && !fork;
     if (fork) {
         YOut unused;
@@ -995,8 +1017,27 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          (const uint32_t*)h->bits, (const int*)h->offsets,
                          (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));
     }
-    // 4. experts: kept groups only (plus the shared group when it is not on the side stream)
     using TH = typename HType<T>::type;
+    if (ep_dispatch) {
+        // the routed experts run on the ranks that hold them; only the shared ones run here
+        if (!use_tc && h->Fsh > 0) {
+            StreamArgs a;
+            a.xperm = h->xperm; a.x = x; a.wgu = h->wgu; a.wsgu = h->wsgu; a.wd = h->wd; a.wsd = h->wsd;
+            a.h = h->hbuf; a.hsh = h->hsh; a.yperm = h->yperm; a.ysh = h->ysh;
+            a.groups = h->groups; a.n_groups = h->zero_int; a.err = &h->dstats->err;
+            a.D = D; a.F = h->F; a.Fsh = h->Fsh; a.T = T_;
+            BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(h->num_sms), dim3(256),
+                             (size_t)stream_gateup_smem(), st, a));
+            BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(h->num_sms), dim3(256),
+                             (size_t)stream_down_smem(), st, a));
+            ysh_out.base = h->ysh; ysh_out.f16 = false;
+        }
+        h->ep_T = T_;
+        h->ep_ysh = ysh_out;
+        h->ep_fork = fork;
+        return BEAM_OK;
+    }
+    // 4. experts: kept groups only (plus the shared group when it is not on the side stream)
     YOut yr;
     if (use_tc) {
         BEAM_TRY(tc_problem(h, x, T_, joint ? PROB_BOTH : PROB_ROUTED, st, yr, ysh_out));
@@ -1419,6 +1460,103 @@ static beam_status_t backward_impl(beam_moe* h, const TX* x, const float* dy, in
     return BEAM_OK;
 }
 
+// ---------------------------------------------------------------- expert parallelism
+// Routing of the rows an expert rank received: source s sent recv_counts[s][e] rows of its local
+// expert e, source-major and expert-minor (the order of the sender's X_perm), so row j belongs
+// to the (s, e) block whose range holds j.  Each row becomes a one-slot "token" routed to that
+// expert with gate 1 (topk_id = e, keep = 1, g_hat = 1, n_keep = 1, lreg = 0), which a routed
+// forward of the expert handle (K = 1) turns into the expert's output row: the compaction groups
+// the rows by expert, the grouped GEMMs run, and the combine writes 1 * Y row back in place.
+// Every block scans the nblk <= kEpMaxBlocks counts into shared memory (256 threads, each a run
+// of consecutive counts, then a scan of the 256 run totals), then finds each row's block by a
+// binary search.
+constexpr int kEpMaxBlocks = 4096;
+
+__global__ void __launch_bounds__(256)
+ep_recv_routing_kernel(const int* __restrict__ recv_counts, int nblk, int El, int n_rows,
+                       int* __restrict__ topk_id, uint8_t* __restrict__ keep,
+                       float* __restrict__ ghat, int* __restrict__ nkeep, float* __restrict__ lreg)
+{
+    __shared__ int s_off[kEpMaxBlocks + 1];
+    __shared__ int s_run[256];
+    pdl_wait();
+    const int tid = threadIdx.x;
+    const int per = (nblk + 255) / 256;
+    const int b0 = tid * per, b1 = min(nblk, b0 + per);
+    int run = 0;
+    for (int b = b0; b < b1; ++b) run += recv_counts[b];
+    s_run[tid] = run;
+    __syncthreads();
+    if (tid < 32) {
+        // exclusive scan of the 256 run totals by one warp, 8 per lane
+        int v[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { v[i] = s_run[tid * 8 + i]; sum += v[i]; }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (tid >= o) incl += n;
+        }
+        int ex = incl - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { s_run[tid * 8 + i] = ex; ex += v[i]; }
+    }
+    __syncthreads();
+    int off = s_run[tid];
+    for (int b = b0; b < b1; ++b) { s_off[b] = off; off += recv_counts[b]; }
+    if (b1 == nblk && b0 < b1) s_off[nblk] = off;
+    if (nblk == 0 && tid == 0) s_off[0] = 0;
+    __syncthreads();
+    for (int j = blockIdx.x * blockDim.x + tid; j < n_rows; j += gridDim.x * blockDim.x) {
+        int lo = 0, hi = nblk;   // s_off[lo] <= j < s_off[hi] for every j below the total
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_off[mid] <= j) lo = mid; else hi = mid;
+        }
+        topk_id[j] = lo % El;
+        keep[j] = 1;
+        ghat[j] = 1.f;
+        nkeep[j] = 1;
+        lreg[j] = 0.f;
+    }
+    pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------- SoftTopK
+template <int EPL>
+static cudaError_t launch_softtopk_fwd(const float* r, int T, int E, int K, float tau, float* y,
+                                       uint8_t* mask, float* nu, cudaStream_t st)
+{
+    return launch(nullptr, 0, softtopk_fwd_kernel<EPL>, dim3(ceil_div(T, 8)), dim3(256), 0, st,
+                  r, T, E, K, tau, y, mask, nu);
+}
+
+template <int EPL>
+static cudaError_t launch_softtopk_bwd(const float* y, const float* dy, int T, int E, float tau,
+                                       float* dr, cudaStream_t st)
+{
+    return launch(nullptr, 0, softtopk_bwd_kernel<EPL>, dim3(ceil_div(T, 8)), dim3(256), 0, st,
+                  y, dy, T, E, tau, dr);
+}
+
+static beam_status_t softtopk_check(int32_t T, int32_t E, float tau, const void* a, const void* b,
+                                    const void* c)
+{
+    if (T < 0) return fail(BEAM_ERR_INVALID_ARG, "T=%d is negative", T);
+    if (E < 1 || E > kSoftTopkMaxE)
+        return fail(BEAM_ERR_INVALID_ARG, "E=%d must be in [1, %d]", E, kSoftTopkMaxE);
+    if (!(tau > 0.f) || !std::isfinite(tau))
+        return fail(BEAM_ERR_INVALID_ARG, "tau must be a positive finite number");
+    if ((long long)T * E > (1LL << 31) - 1)
+        return fail(BEAM_ERR_INVALID_ARG, "T*E=%lld is too large", (long long)T * E);
+    if (T > 0 && (!a || !b || !c)) return fail(BEAM_ERR_INVALID_ARG, "a required pointer is NULL");
+    if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) |
+         reinterpret_cast<uintptr_t>(c)) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "the float arrays must be 4-byte aligned");
+    return BEAM_OK;
+}
+
 extern "C" {
 
 beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, int32_t* topk_id,
@@ -1551,11 +1689,142 @@ beam_status_t beam_moe_create(const beam_moe_config_t* cfg, const beam_moe_weigh
     return BEAM_OK;
 }
 
+beam_status_t beam_moe_create_ep(const beam_moe_config_t* cfg, const beam_moe_weights_t* w,
+                                 void* stream, beam_moe_t** out)
+{
+    g_err[0] = 0;
+    BEAM_TRY(validate(cfg));
+    if (!w || !out) return fail(BEAM_ERR_INVALID_ARG, "weights or out is NULL");
+    if (!w->w_router || !w->w_mask)
+        return fail(BEAM_ERR_INVALID_ARG, "w_router and w_mask are required");
+    if (cfg->n_shared > 0 && (!w->ws_gate || !w->ws_up || !w->ws_down))
+        return fail(BEAM_ERR_INVALID_ARG, "a shared-expert weight pointer is NULL");
+    beam_moe* h = new (std::nothrow) beam_moe();
+    if (!h) return fail(BEAM_ERR_OOM, "host allocation failed");
+    beam_status_t s = create_impl(cfg, w, static_cast<cudaStream_t>(stream), h, true);
+    if (s != BEAM_OK) {
+        cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+        free_all(h);
+        delete h;
+        return s;
+    }
+    *out = h;
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_ep_dispatch(beam_moe_t* h, const void* x, int32_t T, uint32_t flags,
+                                   void* xperm, int32_t* counts, void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
+    if (!counts) return fail(BEAM_ERR_INVALID_ARG, "counts is required");
+    if (T > 0 && (!xperm || (reinterpret_cast<uintptr_t>(xperm) & 15)))
+        return fail(BEAM_ERR_INVALID_ARG, "xperm must be non-NULL and 16-byte aligned");
+    if (T > 0 && !x) return fail(BEAM_ERR_INVALID_ARG, "x is NULL");
+    if (T > 0 && (reinterpret_cast<uintptr_t>(x) & 15))
+        return fail(BEAM_ERR_INVALID_ARG, "x must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(counts) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "counts must be 4-byte aligned");
+    if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR))
+        return fail(BEAM_ERR_INVALID_ARG, "flags: BEAM_MASK_OFF, BEAM_PATH_STREAM or BEAM_PATH_TENSOR");
+    if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
+    if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
+        return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core path needs a bf16 layer with d_model a "
+                    "multiple of 256");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false : h->tc_ok;
+    if (T > 0) {
+        // the compaction gathers the kept rows straight into the caller's buffer (the handle's
+        // own X_perm is only read by its expert GEMMs, which a dispatch does not run)
+        void* own = h->xperm;
+        h->xperm = xperm;
+        beam_status_t r = (h->cfg.dtype == BEAM_DTYPE_BF16)
+            ? forward_impl<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x), T, nullptr, flags,
+                                          use_tc, st, nullptr, true)
+            : forward_impl<float>(h, static_cast<const float*>(x), T, nullptr, flags, use_tc, st,
+                                  nullptr, true);
+        h->xperm = own;
+        BEAM_TRY(r);
+        BEAM_CUDA(cudaMemcpyAsync(counts, h->counts, sizeof(int32_t) * h->E,
+                                  cudaMemcpyDeviceToDevice, st));
+    } else {
+        BEAM_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * h->E, st));
+        h->ep_T = 0;
+        h->ep_fork = false;
+    }
+    h->cur = own_routing(h);
+    h->last_T = T;
+    h->last_train = false;
+    BEAM_CUDA(cudaEventRecord(h->done, st));
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_ep_combine(beam_moe_t* h, const float* y_perm, float* y, void* stream)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (h->ep_T < 0) return fail(BEAM_ERR_NO_FORWARD, "no beam_moe_ep_dispatch has run on this handle");
+    const int T_ = h->ep_T;
+    if (T_ == 0) return BEAM_OK;
+    if (!y || (reinterpret_cast<uintptr_t>(y) & 15) || (reinterpret_cast<uintptr_t>(y_perm) & 15))
+        return fail(BEAM_ERR_INVALID_ARG, "y and y_perm must be non-NULL and 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (h->ep_fork) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_join, 0));
+    YOut yr;
+    yr.base = y_perm; yr.splits = 1; yr.stride = 0; yr.f16 = false;
+    YOut ysh = h->ep_ysh;
+    if (!h->Fsh) ysh.f16 = false;
+    cudaError_t e = ysh.f16 ? launch_combine<float, __half>(h, yr, ysh, h->ghat, T_, y, st)
+                            : launch_combine<float, float>(h, yr, ysh, h->ghat, T_, y, st);
+    BEAM_CUDA(e);
+    BEAM_CUDA(cudaEventRecord(h->done, st));
+    return BEAM_OK;
+}
+
+beam_status_t beam_ep_expert_range(int32_t E, int32_t P, int32_t q, int32_t* first, int32_t* count)
+{
+    g_err[0] = 0;
+    if (E < 1 || P < 1 || q < 0 || q >= P || !first || !count)
+        return fail(BEAM_ERR_INVALID_ARG, "need E >= 1, P >= 1, 0 <= q < P and output pointers");
+    const long long a = (long long)q * E / P, b = (long long)(q + 1) * E / P;
+    *first = (int32_t)a;
+    *count = (int32_t)(b - a);
+    return BEAM_OK;
+}
+
+beam_status_t beam_ep_recv_routing(const int32_t* recv_counts, int32_t P, int32_t E_local,
+                                   int32_t n_rows, int32_t* topk_id, uint8_t* keep, float* ghat,
+                                   int32_t* n_keep, float* lreg, void* stream)
+{
+    g_err[0] = 0;
+    if (P < 1 || E_local < 0 || (long long)P * E_local > kEpMaxBlocks || n_rows < 0)
+        return fail(BEAM_ERR_INVALID_ARG, "need P >= 1, E_local >= 0, P*E_local <= %d, n_rows >= 0",
+                    kEpMaxBlocks);
+    if (n_rows == 0) return BEAM_OK;
+    if (E_local == 0) return fail(BEAM_ERR_INVALID_ARG, "rows received for a rank with no experts");
+    if (!recv_counts || !topk_id || !keep || !ghat || !n_keep || !lreg)
+        return fail(BEAM_ERR_INVALID_ARG, "a pointer is NULL");
+    if ((reinterpret_cast<uintptr_t>(recv_counts) | reinterpret_cast<uintptr_t>(topk_id) |
+         reinterpret_cast<uintptr_t>(ghat) | reinterpret_cast<uintptr_t>(n_keep) |
+         reinterpret_cast<uintptr_t>(lreg)) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "the 32-bit arrays must be 4-byte aligned");
+    const int grid = std::min(ceil_div(n_rows, 256), 148 * 4);
+    BEAM_CUDA(launch(nullptr, 0, ep_recv_routing_kernel, dim3(grid), dim3(256), 0,
+                     static_cast<cudaStream_t>(stream), (const int*)recv_counts, P * E_local,
+                     (int)E_local, (int)n_rows, (int*)topk_id, keep, ghat, (int*)n_keep, lreg));
+    return BEAM_OK;
+}
+
 // The forward behind beam_moe_forward (rin == nullptr) and beam_moe_forward_routed: argument
 // checks shared by both, then the fused decode launch, a graph replay, or direct launches.
 static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float* y, uint32_t flags,
                                    const RouteIn* rin, void* stream)
 {
+    if (h->Ew == 0)
+        return fail(BEAM_ERR_UNSUPPORTED, "a routing-only handle (beam_moe_create_ep) runs "
+                    "beam_moe_ep_dispatch / beam_moe_ep_combine, not a forward");
     if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
     if (T > 0 && (!x || !y)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
@@ -1816,6 +2085,9 @@ beam_status_t beam_moe_backward_router(beam_moe_t* h, const void* x, const float
                                        float* dx, float* d_gate_logit, float* d_mask_logit,
                                        float* dghat, void* stream)
 {
+    if (h && h->Ew == 0)
+        return fail(BEAM_ERR_UNSUPPORTED, "a routing-only handle (beam_moe_create_ep) has no "
+                    "expert outputs to differentiate");
     g_err[0] = 0;
     if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
@@ -1843,6 +2115,54 @@ beam_status_t beam_moe_backward_router(beam_moe_t* h, const void* x, const float
     else
         BEAM_TRY(backward_impl<float>(h, static_cast<const float*>(x), dy, T, reg_scale, dw_router,
                                       dw_mask, dx, d_gate_logit, d_mask_logit, dghat, st));
+    return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- SoftTopK
+beam_status_t beam_softtopk_forward(const float* logits, int32_t T, int32_t E, int32_t K,
+                                    float tau, float* y, uint8_t* mask, float* nu, void* stream)
+{
+    g_err[0] = 0;
+    BEAM_TRY(softtopk_check(T, E, tau, logits, y, y));
+    if (K < 1 || K > E) return fail(BEAM_ERR_INVALID_ARG, "K=%d must be in [1, E=%d]", K, E);
+    if (reinterpret_cast<uintptr_t>(nu) & 3)
+        return fail(BEAM_ERR_INVALID_ARG, "nu must be 4-byte aligned");
+    if (T == 0) return BEAM_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch ((E + 31) / 32) {
+        case 1: e = launch_softtopk_fwd<1>(logits, T, E, K, tau, y, mask, nu, st); break;
+        case 2: e = launch_softtopk_fwd<2>(logits, T, E, K, tau, y, mask, nu, st); break;
+        case 3: e = launch_softtopk_fwd<3>(logits, T, E, K, tau, y, mask, nu, st); break;
+        case 4: e = launch_softtopk_fwd<4>(logits, T, E, K, tau, y, mask, nu, st); break;
+        case 5: e = launch_softtopk_fwd<5>(logits, T, E, K, tau, y, mask, nu, st); break;
+        case 6: e = launch_softtopk_fwd<6>(logits, T, E, K, tau, y, mask, nu, st); break;
+        case 7: e = launch_softtopk_fwd<7>(logits, T, E, K, tau, y, mask, nu, st); break;
+        default: e = launch_softtopk_fwd<8>(logits, T, E, K, tau, y, mask, nu, st); break;
+    }
+    BEAM_CUDA(e);
+    return BEAM_OK;
+}
+
+beam_status_t beam_softtopk_backward(const float* y, const float* dy, int32_t T, int32_t E,
+                                     float tau, float* dlogits, void* stream)
+{
+    g_err[0] = 0;
+    BEAM_TRY(softtopk_check(T, E, tau, y, dy, dlogits));
+    if (T == 0) return BEAM_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch ((E + 31) / 32) {
+        case 1: e = launch_softtopk_bwd<1>(y, dy, T, E, tau, dlogits, st); break;
+        case 2: e = launch_softtopk_bwd<2>(y, dy, T, E, tau, dlogits, st); break;
+        case 3: e = launch_softtopk_bwd<3>(y, dy, T, E, tau, dlogits, st); break;
+        case 4: e = launch_softtopk_bwd<4>(y, dy, T, E, tau, dlogits, st); break;
+        case 5: e = launch_softtopk_bwd<5>(y, dy, T, E, tau, dlogits, st); break;
+        case 6: e = launch_softtopk_bwd<6>(y, dy, T, E, tau, dlogits, st); break;
+        case 7: e = launch_softtopk_bwd<7>(y, dy, T, E, tau, dlogits, st); break;
+        default: e = launch_softtopk_bwd<8>(y, dy, T, E, tau, dlogits, st); break;
+    }
+    BEAM_CUDA(e);
     return BEAM_OK;
 }
 

@@ -1,0 +1,138 @@
+// softtopk.cuh -- SoftTopK, the differentiable top-k of "Stepped MoE: Segment-Level Routing with
+// Configurable Inference Complexity" (SoftTopK entry and core method: the mask generator's
+// routing logits pass through a continuous relaxation of the top-k indicator, so the expert
+// choice is trained end to end, while the layers receive the {0,1} top-k mask).
+//
+// The page gives no formula; the relaxation used is the limited-multi-label projection (Amos,
+// Xu and Kolter, 2019): y_i = sigmoid((r_i - nu) / tau) with nu set so that sum_i y_i = K (the
+// entropy-regularised projection of r / tau onto {0 <= y <= 1, sum y = K}).  Its backward,
+// through nu, is dr_j = h_j (dy_j - sum_i h_i dy_i / sum_i h_i) with h_i = y_i (1 - y_i) / tau.
+//
+// One warp per token row; lane l holds logits l, l + 32, ... (EPL = ceil(E/32) per lane).
+//   forward:  nu by bisection in fp32 on f(nu) = sum_i sigmoid((r_i - nu)/tau) - K (strictly
+//             decreasing) from [min r - 40 tau, max r + 40 tau] until the midpoint equals an
+//             end of the bracket; every lane evaluates f with the same xor-butterfly sum, so the
+//             bracket is bitwise identical across the warp.  Then y, and the hard Top-K
+//             indicator (K rounds of a warp arg-max under (value desc, index asc)).
+//   backward: two butterfly sums per row (sum h, sum h dy), then dr.
+// Deterministic: fixed reduction order, no atomics.  HBM-bound: 4 B per logit read, 4 + 1 B
+// written (y, mask) forward; 8 B read and 4 B written per logit backward.
+#pragma once
+#include "common.cuh"
+#include "router.cuh"
+
+namespace beam {
+
+constexpr int kSoftTopkMaxE = 256;
+
+template <int EPL>
+__global__ void __launch_bounds__(256)
+softtopk_fwd_kernel(const float* __restrict__ r, int T, int E, int K, float tau,
+                    float* __restrict__ y, uint8_t* __restrict__ mask, float* __restrict__ nu_out)
+{
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long t = (long long)blockIdx.x * 8 + warp;
+    if (t < T) {
+        const float* rt = r + t * E;
+        float v[EPL];
+        float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = e < E ? __ldg(rt + e) : 0.f;
+            if (e < E) { lo = fminf(lo, v[j]); hi = fmaxf(hi, v[j]); }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        const float inv_tau = 1.0f / tau;
+        float nu;
+        if (K >= E) {
+            nu = -INFINITY;   // y = 1 everywhere: the constraint leaves no freedom
+        } else {
+            lo -= 40.f * tau;
+            hi += 40.f * tau;
+            for (int it = 0; it < 200; ++it) {
+                const float mid = 0.5f * (lo + hi);
+                if (mid <= lo || mid >= hi) break;   // the bracket is two adjacent floats
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < EPL; ++j)
+                    if (lane + 32 * j < E) s += sigmoid_f((v[j] - mid) * inv_tau);
+                s = warp_sum(s);
+                if (s > (float)K) lo = mid; else hi = mid;
+            }
+            nu = 0.5f * (lo + hi);
+        }
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) y[t * E + e] = K >= E ? 1.f : sigmoid_f((v[j] - nu) * inv_tau);
+        }
+        if (nu_out && lane == 0) nu_out[t] = nu;
+        if (mask) {
+            // hard Top-K indicator: K rounds, each taking the largest remaining value, the
+            // lowest expert among equal ones
+            uint32_t ord[EPL];
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) ord[j] = (lane + 32 * j < E) ? topk_ord(v[j]) : 0u;
+            uint32_t sel = 0u;   // bit j: this lane's expert lane + 32 j is selected
+            for (int k = 0; k < K; ++k) {
+                uint32_t best = 0u, bidx = 0xffffffffu;
+#pragma unroll
+                for (int j = 0; j < EPL; ++j) {
+                    const uint32_t e = (uint32_t)(lane + 32 * j);
+                    if (!((sel >> j) & 1u) && e < (uint32_t)E && ord[j] > best) { best = ord[j]; bidx = e; }
+                    else if (!((sel >> j) & 1u) && e < (uint32_t)E && ord[j] == best && e < bidx) bidx = e;
+                }
+                const uint32_t wbest = __reduce_max_sync(0xffffffffu, best);
+                const uint32_t widx = __reduce_min_sync(0xffffffffu, best == wbest ? bidx : 0xffffffffu);
+                if ((widx & 31u) == (uint32_t)lane) sel |= 1u << (widx >> 5);
+            }
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E) mask[t * E + e] = (uint8_t)((sel >> j) & 1u);
+            }
+        }
+    }
+    pdl_launch_dependents();
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256)
+softtopk_bwd_kernel(const float* __restrict__ y, const float* __restrict__ dy, int T, int E,
+                    float tau, float* __restrict__ dr)
+{
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long t = (long long)blockIdx.x * 8 + warp;
+    if (t < T) {
+        const float inv_tau = 1.0f / tau;
+        float h[EPL], g[EPL];
+        float hs = 0.f, hd = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            const float yv = e < E ? __ldg(y + t * E + e) : 0.f;
+            g[j] = e < E ? __ldg(dy + t * E + e) : 0.f;
+            h[j] = yv * (1.f - yv) * inv_tau;
+            hs += h[j];
+            hd += h[j] * g[j];
+        }
+        hs = warp_sum(hs);
+        hd = warp_sum(hd);
+        const float mean = hs > 0.f ? hd / hs : 0.f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) dr[t * E + e] = h[j] * (g[j] - mean);
+        }
+    }
+    pdl_launch_dependents();
+}
+
+}  // namespace beam

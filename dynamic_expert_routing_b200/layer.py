@@ -282,3 +282,38 @@ class BeamGenerator:
             self.close()
         except Exception:
             pass
+
+
+def softtopk(logits: torch.Tensor, top_k: int, tau: float, mask: bool = True, nu: bool = False,
+             stream=None) -> dict:
+    """SoftTopK of routing logits [T][E] (float32, CUDA): the relaxed mask y [T][E] float32,
+    y_i = sigmoid((r_i - nu) / tau) with sum_i y_i = top_k, plus (mask=True) the hard Top-K
+    indicator [T][E] uint8 and (nu=True) nu [T] float32.  See beam_softtopk_forward."""
+    if not (logits.is_cuda and logits.is_contiguous() and logits.dtype == torch.float32
+            and logits.dim() == 2):
+        raise ValueError("logits must be a contiguous [T][E] CUDA float32 tensor")
+    T, E = logits.shape
+    out = dict(y=torch.empty((T, E), dtype=torch.float32, device=logits.device))
+    if mask:
+        out["mask"] = torch.empty((T, E), dtype=torch.uint8, device=logits.device)
+    if nu:
+        out["nu"] = torch.empty((T,), dtype=torch.float32, device=logits.device)
+    check(_lib.load().beam_softtopk_forward(_ptr(logits), T, E, int(top_k), ctypes.c_float(tau),
+                                            _ptr(out["y"]), _ptr(out.get("mask")),
+                                            _ptr(out.get("nu")),
+                                            ctypes.c_void_p(_stream_handle(stream))))
+    return out
+
+
+def softtopk_backward(y: torch.Tensor, dy: torch.Tensor, tau: float, stream=None) -> torch.Tensor:
+    """d logits [T][E] float32 for the upstream gradient dy [T][E] of SoftTopK's y (the
+    relaxation's Jacobian through nu).  See beam_softtopk_backward."""
+    for name, t in (("y", y), ("dy", dy)):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.float32 and t.dim() == 2
+                and t.shape == y.shape):
+            raise ValueError(f"{name} must be a contiguous [T][E] CUDA float32 tensor")
+    T, E = y.shape
+    dr = torch.empty_like(y)
+    check(_lib.load().beam_softtopk_backward(_ptr(y), _ptr(dy), T, E, ctypes.c_float(tau),
+                                             _ptr(dr), ctypes.c_void_p(_stream_handle(stream))))
+    return dr

@@ -354,6 +354,102 @@ beam_status_t beam_moe_backward_router(beam_moe_t *h, const void *x_dev, const f
                                        float *d_gate_logit_dev, float *d_mask_logit_dev,
                                        float *dghat_dev, void *stream);
 
+/*
+ * ---------------------------------------------------------------- expert parallelism
+ * The BEAM article on aitrends.kr names multi-GPU interaction as future work (limitation (D)).
+ * Here the routed experts are split over P ranks in contiguous blocks (beam_ep_expert_range:
+ * rank q holds experts [floor(qE/P), floor((q+1)E/P))); every rank routes its own tokens over
+ * all E experts and runs the shared experts itself.  One forward of a rank's batch:
+ *   1. beam_moe_ep_dispatch on the rank's routing handle: Steps 1-3 and the compaction.  X_perm
+ *      (the kept rows, sorted by expert and then token) stays on the device; the rows for rank
+ *      q's experts are the contiguous range given by the per-expert counts.
+ *   2. the caller exchanges the counts of each rank's experts and the rows (all-to-all);
+ *   3. each rank turns the rows it received into one-slot tokens (beam_ep_recv_routing) and runs
+ *      its expert handle (an ordinary handle over its E_local experts with top_k = 1 and no
+ *      shared experts) with beam_moe_forward_routed: the compaction groups the rows by expert,
+ *      the grouped GEMMs run, and y holds each row's expert output in the received order;
+ *   4. the caller sends those rows back (the reverse all-to-all): the rank gets its own rows'
+ *      expert outputs in X_perm order;
+ *   5. beam_moe_ep_combine: y = sum over the token's kept slots in rank order of g_hat Y + the
+ *      shared experts (the same fixed order as beam_moe_forward, so the result is deterministic).
+ * dynamic_expert_routing_b200/ep.py drives the exchange with torch.distributed (NCCL).
+ */
+
+/*
+ * A routing-only handle: as beam_moe_create, but w_gate / w_up / w_down are ignored (may be
+ * NULL) and no routed expert weights are held.  It routes over cfg->n_experts experts and runs
+ * the shared experts; beam_moe_forward / _routed / backward_router on it give
+ * BEAM_ERR_UNSUPPORTED.  beam_moe_stats and beam_moe_get_routing describe its last dispatch.
+ */
+beam_status_t beam_moe_create_ep(const beam_moe_config_t *cfg, const beam_moe_weights_t *w_dev,
+                                 void *stream, beam_moe_t **out);
+
+/*
+ * Steps 1-3, the compaction and the shared experts for x_dev[T][D] on `stream`, without host
+ * synchronisation.  xperm_dev (caller-owned device buffer of T*K rows of D elements in the
+ * storage type, 16-byte aligned) receives X_perm: its first n_kept rows are the kept rows,
+ * sorted by expert and then token; counts_dev [E] int32 (device) the kept rows per expert.
+ * flags: BEAM_MASK_OFF, BEAM_PATH_STREAM or BEAM_PATH_TENSOR (the path of the shared experts).
+ * Works on any handle.  The shared experts' output and the dispatch's gates stay in the handle
+ * for beam_moe_ep_combine.
+ */
+beam_status_t beam_moe_ep_dispatch(beam_moe_t *h, const void *x_dev, int32_t T, uint32_t flags,
+                                   void *xperm_dev, int32_t *counts_dev, void *stream);
+
+/*
+ * y_dev[T][D] float32 of the last dispatch: the fixed-order combine of y_perm_dev [n_kept][D]
+ * float32 (the expert outputs of the dispatched rows, in X_perm order; 16-byte aligned) with
+ * the dispatch's gates, plus the shared experts.  BEAM_ERR_NO_FORWARD before any dispatch.
+ */
+beam_status_t beam_moe_ep_combine(beam_moe_t *h, const float *y_perm_dev, float *y_dev,
+                                  void *stream);
+
+/* Host only: the experts of rank q of P, [*first, *first + *count), for E experts. */
+beam_status_t beam_ep_expert_range(int32_t E, int32_t P, int32_t q, int32_t *first,
+                                   int32_t *count);
+
+/*
+ * The routing of the n_rows rows an expert rank received, as one-slot tokens: source s sent
+ * recv_counts_dev[s][e] rows (device, [P][E_local] int32) of local expert e, source-major and
+ * expert-minor; n_rows must be their sum.  Writes topk_id [n_rows] int32 (the local expert),
+ * keep [n_rows] uint8 (1), ghat [n_rows] float32 (1), n_keep [n_rows] int32 (1) and lreg
+ * [n_rows] float32 (0), device arrays (4-byte aligned), for beam_moe_forward_routed of the
+ * expert handle.  P * E_local <= 4096.
+ */
+beam_status_t beam_ep_recv_routing(const int32_t *recv_counts_dev, int32_t P, int32_t E_local,
+                                   int32_t n_rows, int32_t *topk_id_dev, uint8_t *keep_dev,
+                                   float *ghat_dev, int32_t *n_keep_dev, float *lreg_dev,
+                                   void *stream);
+
+/*
+ * ---------------------------------------------------------------- training: SoftTopK
+ * The differentiable top-k of "Stepped MoE: Segment-Level Routing with Configurable Inference
+ * Complexity" (its SoftTopK entry and core method): the routing logits pass through a continuous
+ * relaxation of the top-k indicator, so the choice of experts trains end to end, while the
+ * layers use the {0,1} top-k mask.  The page names the relaxation but gives no formula; the one
+ * used is the limited-multi-label projection (Amos, Xu and Kolter, "The Limited Multi-Label
+ * Projection Layer", 2019), for logits r of one row, 1 <= K <= E and temperature tau > 0:
+ *   y_i = sigmoid((r_i - nu) / tau),  nu such that sum_i y_i = K
+ * (y = 1 everywhere when K = E).  As tau -> 0, y tends to the top-k indicator.
+ * beam_softtopk_forward: logits_dev [T][E] float32 -> y_dev [T][E] float32, and optionally
+ *   mask_dev [T][E] uint8 (the hard Top-K indicator, ties to the lower index, as the layer's
+ *   router) and nu_dev [T] float32.  nu is found by bisection in float32 to the resolution of
+ *   float32; results agree with a float64 solution to about 1e-6 relative in y.
+ * beam_softtopk_backward: dlogits_dev [T][E] = the Jacobian of y (through nu) applied to
+ *   dy_dev [T][E]: with h_i = y_i (1 - y_i) / tau,
+ *   dlogits_j = h_j (dy_j - sum_i h_i dy_i / sum_i h_i)   (0 when sum_i h_i = 0);
+ *   y_dev is the forward's y.  Used as the straight-through gradient of the hard mask, or as the
+ *   exact gradient of the relaxation.
+ * Device pointers, row-major, 4-byte aligned; E <= 256; enqueued on `stream` without host
+ * synchronisation; T = 0 is a no-op.  Bad sizes, tau <= 0 or NULL pointers give
+ * BEAM_ERR_INVALID_ARG.  Deterministic (fixed reduction order).
+ */
+beam_status_t beam_softtopk_forward(const float *logits_dev, int32_t T, int32_t E, int32_t K,
+                                    float tau, float *y_dev, uint8_t *mask_dev, float *nu_dev,
+                                    void *stream);
+beam_status_t beam_softtopk_backward(const float *y_dev, const float *dy_dev, int32_t T,
+                                     int32_t E, float tau, float *dlogits_dev, void *stream);
+
 /* Free every device buffer of the handle (waits for its pending work).  NULL is ignored. */
 void beam_moe_destroy(beam_moe_t *h);
 

@@ -19,13 +19,11 @@ def _build_oracle():
     oracle.build()
 
 
-# One line per GPU parity case (filled by tests.gpu_util.run_case), printed at the end of the
-# run: the clean / unclean token counts of the routing comparison, the tokens whose decision
-# differs from the oracle's (inside the 1e-3 margin), and the y errors.
-PARITY_REPORT: list = []
-
-
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """One line per GPU parity case (tests.parity.REPORT, filled by tests.gpu_util.run_case):
+    the clean / unclean token counts of the routing comparison, the tokens whose decision
+    differs from the oracle's (inside the 1e-3 margin), and the y errors."""
+    from tests.parity import REPORT as PARITY_REPORT
     if not PARITY_REPORT:
         return
     tr = terminalreporter

@@ -85,8 +85,7 @@ def run_case(spec: synth.LayerSpec, T: int, seed: int = 0, keep_rate=0.5, mask_o
     info.update(y_tokens=int(sel.size), differing_tokens=differ.tolist(),
                 near_margin_tokens=int(near.sum()), max_abs_own_decision=own["max_abs"],
                 rel_l2_own_decision=own["rel_l2"])
-    from tests.conftest import PARITY_REPORT
-    PARITY_REPORT.append(dict(case=case or f"{spec.name} T={T}", T=T, clean=info["clean"],
+    parity.REPORT.append(dict(case=case or f"{spec.name} T={T}", T=T, clean=info["clean"],
                               unclean=info["unclean"], differing=int(differ.size),
                               y_tokens=int(sel.size), max_abs=info["max_abs"],
                               rel_l2=info["rel_l2"], max_abs_own=own["max_abs"],

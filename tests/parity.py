@@ -21,6 +21,8 @@ from __future__ import annotations
 import numpy as np
 
 MARGIN = 1e-3
+# one dict per GPU parity case of the test run (printed by tests/conftest.py at the end)
+REPORT: list = []
 TOL_BF16_ABS = 2e-2
 TOL_BF16_REL = 5e-3
 TOL_F32_REL = 1e-5
