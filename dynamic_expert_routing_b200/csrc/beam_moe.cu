@@ -687,10 +687,32 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
 // serialisation, and (while profiling) bracketed by an event pair of its stage.  h == nullptr
 // launches the kernel the same way without touching any handle state (no count, no events):
 // the allocation-free routing call uses that, so it never writes to the handle.
+// BEAM_TRACE=1 in the environment prints every launch (stage, grid, block, shared memory) to
+// stderr before it is made, and its launch status after: a host-side fault can then be placed.
+static bool trace_on()
+{
+    static const bool on = getenv("BEAM_TRACE") != nullptr;
+    return on;
+}
+
+static void trace(const char* fmt, ...)
+{
+    if (!trace_on()) return;
+    va_list ap;
+    va_start(ap, fmt);
+    fputs("[beam] ", stderr);
+    vfprintf(stderr, fmt, ap);
+    fputc('\n', stderr);
+    fflush(stderr);
+    va_end(ap);
+}
+
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_ex(beam_moe* h, int stage, bool coop, void (*kernel)(KArgs...), dim3 grid,
                              dim3 block, size_t smem, cudaStream_t st, Args&&... args)
 {
+    trace("launch stage %d grid (%u,%u,%u) block %u smem %zu stream %p", stage, grid.x, grid.y,
+          grid.z, block.x, smem, (void*)st);
     cudaEvent_t ea = nullptr, eb = nullptr;
     if (h && h->prof && h->prof_pool.size() >= 2) {
         ea = h->prof_pool.back(); h->prof_pool.pop_back();
@@ -716,6 +738,7 @@ static cudaError_t launch_ex(beam_moe* h, int stage, bool coop, void (*kernel)(K
     lc.attrs = attr;
     lc.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+    trace("  -> %s", cudaGetErrorString(e));
     if (e == cudaSuccess && ea) {
         e = cudaEventRecord(eb, st);
         h->prof_recs.push_back({stage, ea, eb});
@@ -1735,6 +1758,8 @@ beam_status_t beam_moe_ep_dispatch(beam_moe_t* h, const void* x, int32_t T, uint
                     "multiple of 256");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false : h->tc_ok;
+    trace("ep_dispatch T=%d flags=0x%x tc=%d Ew=%d Fsh=%d xperm=%p counts=%p", T, flags, (int)use_tc,
+          h->Ew, h->Fsh, xperm, (void*)counts);
     if (T > 0) {
         // the compaction gathers the kept rows straight into the caller's buffer (the handle's
         // own X_perm is only read by its expert GEMMs, which a dispatch does not run)
@@ -1746,6 +1771,7 @@ beam_status_t beam_moe_ep_dispatch(beam_moe_t* h, const void* x, int32_t T, uint
             : forward_impl<float>(h, static_cast<const float*>(x), T, nullptr, flags, use_tc, st,
                                   nullptr, true);
         h->xperm = own;
+        trace("ep_dispatch forward status %d", (int)r);
         BEAM_TRY(r);
         BEAM_CUDA(cudaMemcpyAsync(counts, h->counts, sizeof(int32_t) * h->E,
                                   cudaMemcpyDeviceToDevice, st));
