@@ -612,7 +612,11 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
         BEAM_TRY(dalloc(h, &h->ysh, Tm * D * sizeof(float)));
     }
     // logits; bf16 layers keep room for K-split slices of the tensor-core router
-    BEAM_TRY(dalloc(h, &h->L, (cfg->dtype == BEAM_DTYPE_BF16 ? kMaxSplits : 1) * Tm * h->ldL * sizeof(float)));
+    // logits; room for K-split slices of the tensor-core router (bf16) and for the D-chunk
+    // slices of the small-batch router (at most 16 chunks of kRouterChunkBytes)
+    static_assert(8192 * 2 / kRouterChunkBytes <= kMaxSplits && 4096 * 4 / kRouterChunkBytes <= kMaxSplits,
+                  "the logit slices of the small-batch router must fit the L buffer");
+    BEAM_TRY(dalloc(h, &h->L, (size_t)kMaxSplits * Tm * h->ldL * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->topk_id, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->gate, rows * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->mlogit, rows * sizeof(float)));
@@ -926,6 +930,15 @@ static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, co
     // otherwise one CTA per token whose threads take the row's float4 columns in equal passes
     // (D/4 = 384: 192 threads x 2 rather than 256 + 128)
     const int d4 = h->D / 4;
+    if (T_ < h->num_sms && (r.splits > 1 || sh.splits > 1) && h->K <= 32 &&
+        r.splits <= kCombineMaxSplits && sh.splits <= kCombineMaxSplits) {
+        // a small batch with split-K slices: slots and slices read in parallel
+        return launch(h, ST_COMBINE, combine_small_kernel<TR, TS>,
+                      dim3(T_, ceil_div(d4, kCombineSmallCols)),
+                      dim3(kCombineSmallCols, h->K + 1), 0, st,
+                      (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
+                      (const int*)h->inv, ghat, T_, h->K, h->D, y);
+    }
     const bool split_cols = T_ < h->num_sms;
     const int passes = ceil_div(d4, 256);
     const int nthr = split_cols ? 256 : std::min(256, ceil_div(ceil_div(d4, passes), 32) * 32);
@@ -989,6 +1002,14 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
+    } else if (Tr <= kRouterSmallRows) {
+        // a few routed rows: per-chunk slices of D, added in chunk order by the selection
+        constexpr int DC = kRouterChunkBytes / (int)sizeof(T);
+        lsplits = ceil_div(D, DC);
+        lstride = (long long)Tr * h->ldL;
+        BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_small_kernel<T>,
+                         dim3(ceil_div(h->n2E, 8), lsplits), dim3(256), 0, st, x, S, Tr, D,
+                         (const T*)h->wrm, h->n2E, h->ldL, lstride, h->L));
     } else {
         BEAM_CUDA(launch_router_gemv<T>(h, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->ldL, h->L, st));
     }

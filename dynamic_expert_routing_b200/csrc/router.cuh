@@ -138,6 +138,87 @@ router_gemv_warp_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
     pdl_launch_dependents();
 }
 
+// The same logits for a small batch (at most kRouterSmallRows routed rows), as per-chunk
+// partial slices: CTA (column block b, chunk c) covers columns [8b, 8b + 8) and the D-range
+// [c DC, (c + 1) DC), DC = kRouterChunk.  Its threads first stage the chunk of every routed row
+// in shared memory (one read of x per CTA), then warp w takes column 8b + w: lane l reads the
+// 16-byte weight vectors v*32 + l of the chunk (coalesced; consecutive lanes hit consecutive
+// shared-memory words) and keeps one partial per row.  The 32 row partials are reduced across
+// the lanes by a transposing butterfly (lane r ends with row r, 31 shuffles), and lane r writes
+// L[c][r][column], slice c at c * slice_stride.  The selection adds the slices in chunk order,
+// so the result is deterministic.  One read of each weight row; x is read once per column
+// block from L2 instead of once per column.
+constexpr int kRouterSmallRows = 32;
+constexpr int kRouterChunkBytes = 1024;   // a chunk of D: 512 bf16 or 256 fp32 elements
+
+template <typename TW>
+__global__ void __launch_bounds__(256)
+router_small_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
+                    const TW* __restrict__ wrm, int n2E, int ldL, long long slice_stride,
+                    float* __restrict__ L)
+{
+    constexpr int DC = kRouterChunkBytes / (int)sizeof(TW);   // elements per chunk
+    constexpr int VN = Vec<TW>::N;                            // elements per 16-byte vector
+    constexpr int NV = DC / (32 * VN);                        // vectors per lane
+    __shared__ __align__(16) TW xs[kRouterSmallRows][DC];
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.y;
+    const int d0 = c * DC;
+    const int dn = min(DC, D - d0);                           // a multiple of VN
+    const size_t xstride = (size_t)(seg > 1 ? seg : 1) * D;
+    // stage the chunk of every routed row (zero beyond D and beyond Tr)
+    for (int i = threadIdx.x; i < kRouterSmallRows * (DC / VN); i += blockDim.x) {
+        const int r = i / (DC / VN), v = i % (DC / VN);
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (r < Tr && v * VN < dn)
+            val = __ldg(reinterpret_cast<const uint4*>(x + r * xstride + d0) + v);
+        reinterpret_cast<uint4*>(&xs[r][0])[v] = val;
+    }
+    __syncthreads();
+    const int j = blockIdx.x * 8 + warp;
+    if (j < n2E) {
+        float w[NV][VN];
+        const TW* wrow = wrm + (size_t)j * D + d0;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            const int e = (v * 32 + lane) * VN;
+            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+            if (e < dn) raw = ldg_stream(wrow + e);
+            Vec<TW>::widen(raw, w[v]);
+        }
+        float acc[kRouterSmallRows];
+#pragma unroll
+        for (int r = 0; r < kRouterSmallRows; ++r) {
+            float a = 0.f;
+            if (r < Tr) {
+#pragma unroll
+                for (int v = 0; v < NV; ++v) {
+                    float xv[VN];
+                    Vec<TW>::widen(reinterpret_cast<const uint4*>(&xs[r][0])[v * 32 + lane], xv);
+#pragma unroll
+                    for (int q = 0; q < VN; ++q) a = fmaf(w[v][q], xv[q], a);
+                }
+            }
+            acc[r] = a;
+        }
+        // transposing butterfly: at step o the lanes with bit o set keep rows [o, 2o) of the
+        // current numbering and send rows [0, o); after the five steps lane r holds row r
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const bool hi = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < o; ++i) {
+                const float send = hi ? acc[i] : acc[i + o];
+                const float keep = hi ? acc[i + o] : acc[i];
+                acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        if (lane < Tr) L[(size_t)c * slice_stride + (size_t)lane * ldL + j] = acc[0];
+    }
+    pdl_launch_dependents();
+}
+
 // ---------------------------------------------------------------- Top-K, softmax, mask
 // One warp per routed row i (row i of L, leading dimension ldL: router logits in columns
 // [0, E), mask logits in [E, 2E); `splits` K-split slices split_stride floats apart, added in

@@ -562,4 +562,79 @@ combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
     pdl_launch_dependents();
 }
 
+// The combine of a small batch (fewer tokens than SMs) whose expert outputs are split-K slices:
+// the per-column chain of slot x slice loads of combine_kernel is a long dependent walk there.
+// CTA (token t, 16-column block) has 16 x (K + 1) threads: thread (c, k < K) adds the slices of
+// slot k's row in slice order (their loads all issued first), thread (c, K) the slices of the
+// shared term; then thread (c, 0) takes y = sum over the slots in rank order of g_hat * v_k
+// (fmaf, as combine_kernel) + the shared sum.  Deterministic.  K <= 32, splits <= 16.
+constexpr int kCombineSmallCols = 16;
+constexpr int kCombineMaxSplits = 16;
+
+template <typename TY>
+__device__ __forceinline__ float4 sum_slices(const TY* base, int splits, long long s4, size_t i)
+{
+    float4 v[kCombineMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kCombineMaxSplits; ++s)
+        if (s < splits) v[s] = load4(base, s * s4 + i);
+    float4 a = v[0];
+#pragma unroll
+    for (int s = 1; s < kCombineMaxSplits; ++s) {
+        if (s < splits) { a.x += v[s].x; a.y += v[s].y; a.z += v[s].z; a.w += v[s].w; }
+    }
+    return a;
+}
+
+template <typename TY, typename TS>
+__global__ void __launch_bounds__(kCombineSmallCols * 33)
+combine_small_kernel(const TY* __restrict__ yperm, int splits, long long stride,
+                     const TS* __restrict__ ysh, int splits_sh, long long stride_sh,
+                     const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K,
+                     int D, float* __restrict__ y)
+{
+    __shared__ float4 red[33][kCombineSmallCols];
+    __shared__ int s_inv[32];
+    __shared__ float s_g[32];
+    pdl_wait();
+    const int t = blockIdx.x;
+    const int cx = threadIdx.x, k = threadIdx.y;
+    const int D4 = D >> 2;
+    const int c = blockIdx.y * kCombineSmallCols + cx;
+    const int tid = k * kCombineSmallCols + cx;
+    if (tid < K) {
+        s_inv[tid] = inv[(size_t)t * K + tid];
+        s_g[tid] = ghat[(size_t)t * K + tid];
+    }
+    __syncthreads();
+    if (c < D4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k < K) {
+            const int p = s_inv[k];
+            if (p >= 0) v = sum_slices(yperm, splits, stride >> 2, (size_t)p * D4 + c);
+        } else if (ysh) {
+            v = sum_slices(ysh, splits_sh, stride_sh >> 2, (size_t)t * D4 + c);
+        }
+        red[k][cx] = v;
+    }
+    __syncthreads();
+    if (k == 0 && c < D4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < K; ++q) {
+            if (s_inv[q] >= 0) {
+                const float g = s_g[q];
+                const float4 v = red[q][cx];
+                acc.x = fmaf(g, v.x, acc.x); acc.y = fmaf(g, v.y, acc.y);
+                acc.z = fmaf(g, v.z, acc.z); acc.w = fmaf(g, v.w, acc.w);
+            }
+        }
+        if (ysh) {
+            const float4 v = red[K][cx];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        __stcs(reinterpret_cast<float4*>(y) + (size_t)t * D4 + c, acc);
+    }
+    pdl_launch_dependents();
+}
+
 }  // namespace beam
