@@ -195,6 +195,8 @@ struct beam_moe {
     int* tail_cnt = nullptr;     // [kTailCntRegions][num_sms][kEpiWarps]
     int* zero_int = nullptr;     // two zeros: an empty group table
     int* range_flag = nullptr;
+    unsigned* rcnt = nullptr;    // arrival counters of the small-batch router, one per block of
+                                 // 8 logit columns; zero between calls
     cudaEvent_t done = nullptr;
     // side stream for the shared experts (they depend on x only, so they overlap routing)
     cudaStream_t side = nullptr;
@@ -617,6 +619,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     static_assert(8192 * 2 / kRouterChunkBytes <= kMaxSplits && 4096 * 4 / kRouterChunkBytes <= kMaxSplits,
                   "the logit slices of the small-batch router must fit the L buffer");
     BEAM_TRY(dalloc(h, &h->L, (size_t)kMaxSplits * Tm * h->ldL * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->rcnt, (size_t)ceil_div(h->ldL, 8) * sizeof(unsigned)));
+    BEAM_CUDA(cudaMemsetAsync(h->rcnt, 0, (size_t)ceil_div(h->ldL, 8) * sizeof(unsigned), st));
     BEAM_TRY(dalloc(h, &h->topk_id, rows * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->gate, rows * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->mlogit, rows * sizeof(float)));
@@ -1003,13 +1007,11 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
     } else if (Tr <= kRouterSmallRows) {
-        // a few routed rows: per-chunk slices of D, added in chunk order by the selection
+        // a few routed rows: per-chunk slices of D, added in chunk order inside the kernel
         constexpr int DC = kRouterChunkBytes / (int)sizeof(T);
-        lsplits = ceil_div(D, DC);
-        lstride = (long long)Tr * h->ldL;
         BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_small_kernel<T>,
-                         dim3(ceil_div(h->n2E, 8), lsplits), dim3(256), 0, st, x, S, Tr, D,
-                         (const T*)h->wrm, h->n2E, h->ldL, lstride, h->L));
+                         dim3(ceil_div(h->n2E, 8), ceil_div(D, DC)), dim3(256), 0, st, x, S, Tr, D,
+                         (const T*)h->wrm, h->n2E, h->ldL, (long long)Tr * h->ldL, h->L, h->rcnt));
     } else {
         BEAM_CUDA(launch_router_gemv<T>(h, x, S, Tr, D, (const T*)h->wrm, h->n2E, h->ldL, h->L, st));
     }
@@ -1343,8 +1345,16 @@ static beam_status_t gen_create_impl(const beam_gen_config_t* c, const void* wr,
             gfloats = std::max(gfloats, (size_t)s * rows * g->ldG);
         }
     }
+    // and for the D-chunk slices of the small-batch router (at most kRouterSmallRows rows)
+    {
+        const int rows = std::min(Trmax, kRouterSmallRows);
+        const int chunks = ceil_div((long long)h->D * h->esz, kRouterChunkBytes);
+        gfloats = std::max(gfloats, (size_t)chunks * rows * g->ldG);
+    }
     BEAM_TRY(dalloc(h, &g->wgen, (size_t)g->ldG * h->D * h->esz));
     BEAM_TRY(dalloc(h, &g->G, gfloats * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->rcnt, (size_t)ceil_div(g->ldG, 8) * sizeof(unsigned)));
+    BEAM_CUDA(cudaMemsetAsync(h->rcnt, 0, (size_t)ceil_div(g->ldG, 8) * sizeof(unsigned), st));
     BEAM_TRY(dalloc(h, &h->zero_int, 2 * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->groups, sizeof(Group)));
     BEAM_TRY(dalloc(h, &h->dstats, sizeof(DevStats)));
@@ -1427,6 +1437,13 @@ static beam_status_t gen_route_impl(beam_gen* g, const T* z, int T_, const beam_
         BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * splits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
+    } else if (Tr <= kRouterSmallRows) {
+        // the layer's small-batch router, so that a one-layer generator and its layer compute
+        // the same bits
+        constexpr int DC = kRouterChunkBytes / (int)sizeof(T);
+        BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_small_kernel<T>,
+                         dim3(ceil_div(g->nlog, 8), ceil_div(D, DC)), dim3(256), 0, st, z, S, Tr, D,
+                         (const T*)g->wgen, g->nlog, g->ldG, (long long)Tr * g->ldG, g->G, h->rcnt));
     } else {
         BEAM_CUDA(launch_router_gemv<T>(h, z, S, Tr, D, (const T*)g->wgen, g->nlog, g->ldG, g->G, st));
     }

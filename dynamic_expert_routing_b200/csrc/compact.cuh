@@ -20,6 +20,26 @@ namespace beam {
 
 constexpr int kMaxE = kRouteMaxE;
 
+// One warp copies a row of nv 16-byte vectors, 8 vectors per lane in flight at a time (all
+// loads of a batch are issued before its stores).
+__device__ __forceinline__ void copy_row_warp(uint4* __restrict__ dst, const uint4* __restrict__ src,
+                                              int nv, int lane)
+{
+    for (int v0 = 0; v0 < nv; v0 += 32 * 8) {
+        uint4 r[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < nv) r[u] = __ldg(src + v);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < nv) dst[v] = r[u];
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256)
 compact_bits_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__ keep, int T,
                     int K, int E, int nch, uint32_t* __restrict__ bits)
@@ -317,7 +337,7 @@ compact_scatter_gather_kernel(const int* __restrict__ topk_id, const uint8_t* __
             const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
             uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
             const int nv = D * (int)sizeof(TW) / 16;
-            for (int v = lane; v < nv; v += 32) dst[v] = src[v];
+            copy_row_warp(dst, src, nv, lane);
         }
     }
     pdl_launch_dependents();
@@ -517,7 +537,7 @@ __device__ __forceinline__ void gather_small_rows(const SmallScratch& sc, int E,
         const int t = sc.perm[pos] / K;
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
         uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
-        for (int v = lane; v < nv; v += 32) dst[v] = src[v];
+        copy_row_warp(dst, src, nv, lane);
     }
 }
 
@@ -561,7 +581,7 @@ gather_rows_kernel(const int* __restrict__ perm, const int* __restrict__ n_kept_
         const int t = perm[pos] / K;
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
         uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
-        for (int v = lane; v < nv; v += 32) dst[v] = src[v];
+        copy_row_warp(dst, src, nv, lane);
     }
     pdl_launch_dependents();
 }

@@ -138,32 +138,36 @@ router_gemv_warp_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
     pdl_launch_dependents();
 }
 
-// The same logits for a small batch (at most kRouterSmallRows routed rows), as per-chunk
-// partial slices: CTA (column block b, chunk c) covers columns [8b, 8b + 8) and the D-range
-// [c DC, (c + 1) DC), DC = kRouterChunk.  Its threads first stage the chunk of every routed row
-// in shared memory (one read of x per CTA), then warp w takes column 8b + w: lane l reads the
-// 16-byte weight vectors v*32 + l of the chunk (coalesced; consecutive lanes hit consecutive
-// shared-memory words) and keeps one partial per row.  The 32 row partials are reduced across
-// the lanes by a transposing butterfly (lane r ends with row r, 31 shuffles), and lane r writes
-// L[c][r][column], slice c at c * slice_stride.  The selection adds the slices in chunk order,
-// so the result is deterministic.  One read of each weight row; x is read once per column
-// block from L2 instead of once per column.
+// The same logits for a small batch (at most kRouterSmallRows routed rows).  CTA (column block
+// b, chunk c) covers columns [8b, 8b + 8) and the D-range [c DC, (c + 1) DC), DC =
+// kRouterChunkBytes: its threads first stage the chunk of every routed row in shared memory (one
+// read of x per CTA), then warp w takes column 8b + w: lane l reads the 16-byte weight vectors
+// v*32 + l of the chunk (coalesced; consecutive lanes hit consecutive shared-memory words) and
+// keeps one partial per row.  The 32 row partials are reduced across the lanes by a transposing
+// butterfly (lane r ends with row r, 31 shuffles).  With one chunk lane r writes L[r][column].
+// With several, lane r writes its chunk's partial into slice c of L (slice c at c * slice_stride;
+// slice 0 is L itself), and the CTA counts itself in on the block's arrival counter; the CTA
+// that arrives last (the atomic only elects it) adds the block's slices in chunk order into
+// slice 0 and resets the counter to zero for the next call.  The selection then reads one
+// value per logit.  Deterministic; one read of each weight row; x read once per column block.
 constexpr int kRouterSmallRows = 32;
 constexpr int kRouterChunkBytes = 1024;   // a chunk of D: 512 bf16 or 256 fp32 elements
+constexpr int kRouterMaxChunks = 16;      // D <= 8192 bf16 / 4096 fp32
 
 template <typename TW>
 __global__ void __launch_bounds__(256)
 router_small_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
                     const TW* __restrict__ wrm, int n2E, int ldL, long long slice_stride,
-                    float* __restrict__ L)
+                    float* __restrict__ L, unsigned* __restrict__ arrive)
 {
     constexpr int DC = kRouterChunkBytes / (int)sizeof(TW);   // elements per chunk
     constexpr int VN = Vec<TW>::N;                            // elements per 16-byte vector
     constexpr int NV = DC / (32 * VN);                        // vectors per lane
     __shared__ __align__(16) TW xs[kRouterSmallRows][DC];
+    __shared__ int s_last;
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.y;
+    const int c = blockIdx.y, nchunks = gridDim.y;
     const int d0 = c * DC;
     const int dn = min(DC, D - d0);                           // a multiple of VN
     const size_t xstride = (size_t)(seg > 1 ? seg : 1) * D;
@@ -215,6 +219,27 @@ router_small_kernel(const TW* __restrict__ x, int seg, int Tr, int D,
             }
         }
         if (lane < Tr) L[(size_t)c * slice_stride + (size_t)lane * ldL + j] = acc[0];
+    }
+    if (nchunks > 1) {
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) s_last = atomicAdd(arrive + blockIdx.x, 1u) == (unsigned)(nchunks - 1);
+        __syncthreads();
+        if (s_last) {
+            __threadfence();   // the other chunks' slices are visible past this point
+            if (j < n2E && lane < Tr) {
+                float p[kRouterMaxChunks];
+#pragma unroll
+                for (int q = 0; q < kRouterMaxChunks; ++q)
+                    if (q < nchunks) p[q] = __ldcg(L + (size_t)q * slice_stride + (size_t)lane * ldL + j);
+                float a = p[0];
+#pragma unroll
+                for (int q = 1; q < kRouterMaxChunks; ++q)
+                    if (q < nchunks) a += p[q];
+                L[(size_t)lane * ldL + j] = a;
+            }
+            if (threadIdx.x == 0) arrive[blockIdx.x] = 0u;
+        }
     }
     pdl_launch_dependents();
 }
@@ -271,11 +296,29 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
     // (two warp reductions), and the lane that owned it drops its first entry.  The rounds
     // yield the Top-K in rank order with ties to the lower index.
     uint32_t ord[EPL], idx[EPL];
+    float mv[EPL];   // one slice: this lane's mask logits, loaded with the router logits
+    if (splits == 1) {
+        float rv[EPL];
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        ord[j] = (e < E) ? topk_ord(logit(e)) : 0u;
-        idx[j] = (e < E) ? (uint32_t)e : 0xffffffffu;
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            rv[j] = (e < E) ? Li[e] : 0.f;
+            mv[j] = (e < E) ? Li[E + e] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            ord[j] = (e < E) ? topk_ord(rv[j]) : 0u;
+            idx[j] = (e < E) ? (uint32_t)e : 0xffffffffu;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const int e = lane + 32 * j;
+            ord[j] = (e < E) ? topk_ord(logit(e)) : 0u;
+            idx[j] = (e < E) ? (uint32_t)e : 0xffffffffu;
+            mv[j] = 0.f;
+        }
     }
 #pragma unroll
     for (int pass = 0; pass < EPL; ++pass) {
@@ -308,7 +351,18 @@ __device__ __forceinline__ RowDecision select_row(const float* __restrict__ Li, 
     const float den = warp_sum(ex);
     d.id = my_id;
     d.g = ex / den;
-    d.l = active ? logit(E + my_id) : 0.f;
+    if (splits == 1) {
+        // the mask logit of expert my_id is held by lane my_id % 32, entry my_id / 32
+        float ml = 0.f;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+            const float v = __shfl_sync(0xffffffffu, mv[j], my_id & 31);
+            if ((my_id >> 5) == j) ml = v;
+        }
+        d.l = active ? ml : 0.f;
+    } else {
+        d.l = active ? logit(E + my_id) : 0.f;
+    }
     // mask_off: 0 = BEAM mask, 1 = plain Top-K, 2 = training (every Top-K slot is evaluated,
     // so keep = 1 for the compaction, while the gate still carries the mask: g_hat = g * m)
     const bool m = active && (mask_off == 1 || d.l >= 0.f);
