@@ -26,6 +26,7 @@
 #include "compact.cuh"
 #include "stream_experts.cuh"
 #include "tc_experts.cuh"
+#include "tc_down_astat.cuh"
 #include "decode_fused.cuh"
 #include "route_grad.cuh"
 #include "softtopk.cuh"
@@ -560,6 +561,8 @@ static beam_status_t setup_tc(beam_moe* h)
             (const void*)tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_SWAP>};
         for (const void* k : kernels)
             BEAM_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+        BEAM_CUDA(cudaFuncSetAttribute((const void*)tc::tc_down_astat_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, tc::AS_SMEM_BYTES));
     }
     // the fused decode kernel: one resident block per SM is required for its grid barriers
     {
@@ -766,6 +769,10 @@ static cudaError_t launch(beam_moe* h, int stage, void (*kernel)(KArgs...), dim3
 // kGemvWarpCols columns on (the choice depends on the column count alone, so a one-layer
 // generator and the layer with the same matrices compute the same bits).
 constexpr int kGemvWarpCols = 2048;
+// Up to this many routed rows the one-CTA-per-column GEMV is faster than the small-batch router
+// (measured on B200: 4.8 against 7.1 us for one token of the Mixtral-like layer): with so few
+// rows the shared-memory staging and the cross-chunk sum do not pay.
+constexpr int kRouterGemvMaxRows = 4;
 
 template <typename T>
 static cudaError_t launch_router_gemv(beam_moe* h, const T* x, int S, int Tr, int D, const T* w,
@@ -916,6 +923,10 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
         if (swap2)
             BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_SWAP>,
                              dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
+        else if (which == PROB_ROUTED && F / tc::BK <= tc::AS_MAX_KSTEPS)
+            // short K: the unit's H rows stay in shared memory for all of its N-tiles
+            BEAM_CUDA(launch(h, st_dn, tc::tc_down_astat_kernel, dim3(h->num_sms), dim3(tc::kThreads),
+                             (size_t)tc::AS_SMEM_BYTES, st, q));
         else if (tail2)
             BEAM_CUDA(launch(h, st_dn, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F16, 0, tc::MODE_TAIL>,
                              dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, q));
@@ -1006,7 +1017,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * lsplits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
-    } else if (Tr <= kRouterSmallRows) {
+    } else if (Tr > kRouterGemvMaxRows && Tr <= kRouterSmallRows) {
         // a few routed rows: per-chunk slices of D, added in chunk order inside the kernel
         constexpr int DC = kRouterChunkBytes / (int)sizeof(T);
         BEAM_CUDA(launch(h, ST_ROUTER_LOGITS, router_small_kernel<T>,
@@ -1437,7 +1448,7 @@ static beam_status_t gen_route_impl(beam_gen* g, const T* z, int T_, const beam_
         BEAM_CUDA(launch(h, ST_TC_ROUTER, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3((unsigned)std::min<long long>(h->num_sms, tiles * splits)),
                          dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, h->p0));
-    } else if (Tr <= kRouterSmallRows) {
+    } else if (Tr > kRouterGemvMaxRows && Tr <= kRouterSmallRows) {
         // the layer's small-batch router, so that a one-layer generator and its layer compute
         // the same bits
         constexpr int DC = kRouterChunkBytes / (int)sizeof(T);

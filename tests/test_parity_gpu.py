@@ -535,3 +535,25 @@ def test_fp16_overflow_of_h_is_reported(T, path, fused):
     layer.forward(x.cuda(), path=path, fused=fused)
     assert layer.stats()["tokens"] == T
     layer.close()
+
+
+# ------------------------------------------------------------------ short-K down projection
+@pytest.mark.parametrize("F,T,E,K", [(256, 1600, 8, 2), (128, 900, 16, 4), (256, 3000, 60, 4),
+                                     (64, 600, 8, 1), (256, 2000, 212, 16)],
+                         ids=["f256_e8", "f128_e16", "f256_e60", "f64_one_kstep", "f256_e212"])
+def test_short_k_down_projection(F, T, E, K):
+    """Routed down projections with F <= 256 (at most 4 k-steps per tile) run the kernel that
+    keeps a unit's H rows in shared memory for all of its N-tiles (groups of more than 64 rows on
+    average: T*K > 64 E).  Groups span one to many 128-row M-tiles; y against the oracle on a
+    spread sample, and a direct launch repeats the graph replay's bits."""
+    spec = synth.LayerSpec("astat", 512, E, K, F, n_shared=1, d_ff_shared=128)
+    assert T * K > 64 * E
+    sample = np.unique(np.linspace(0, T - 1, 200).round().astype(np.int64))
+    info = run_case(spec, T, seed=F + T, path="tensor", y_tokens=sample)
+    if T * K / (2 * E) > 150:
+        assert info["stats"]["counts"].max() > 128      # groups span several M-tiles
+    layer = info["layer"]
+    y2 = layer.forward(info["x"].cuda(), path="tensor", graph=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, info["y"])
+    layer.close()
