@@ -25,6 +25,7 @@ BEAM_PATH_TENSOR = 0x4
 BEAM_NO_GRAPH = 0x8
 BEAM_FUSED_DECODE = 0x10
 BEAM_TRAIN = 0x20
+BEAM_HOST_PIPELINE = 0x40
 
 BEAM_N_STAGES = 18
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20

@@ -178,6 +178,14 @@ struct beam_moe {
     // host-call staging
     void* x_stage = nullptr;
     float* y_stage = nullptr;
+    // pipelined host calls (BEAM_HOST_PIPELINE): copy streams, per-chunk events, statistics
+    // accumulated over the chunks
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t ev_in[4] = {}, ev_out[4] = {};
+    cudaEvent_t ev_copied = nullptr;
+    DevStats* acc_stats = nullptr;
+    int* acc_counts = nullptr;
+    bool last_pipelined = false;
     size_t hsz;          // bytes per element of H and of the stored down projections
     bool tc_ok = false;  // tensor-core expert path available (bf16, D % 256 == 0)
     bool fused_ok = false;  // fused decode launch available (tc_ok and cooperative launches)
@@ -281,6 +289,16 @@ static void free_all(beam_moe* h)
     if (h->side) cudaStreamDestroy(h->side);
     h->ev_fork = h->ev_join = nullptr;
     h->side = nullptr;
+    for (int i = 0; i < 4; ++i) {
+        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+        if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+        h->ev_in[i] = h->ev_out[i] = nullptr;
+    }
+    if (h->ev_copied) cudaEventDestroy(h->ev_copied);
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
+    h->ev_copied = nullptr;
+    h->copy_in = h->copy_out = nullptr;
 }
 
 // Test hook: BEAM_TEST_FAIL_ALLOC=n makes the n-th device allocation of a create fail as if
@@ -648,6 +666,8 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->yperm, rows * D * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->x_stage, Tm * D * es));
     BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->acc_stats, sizeof(DevStats)));
+    BEAM_TRY(dalloc(h, &h->acc_counts, E * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->pair_grad, rows * sizeof(float2)));
     h->dw_chunks = ceil_div((long long)D, cfg->dtype == BEAM_DTYPE_BF16 ? dw_chunk_cols<__nv_bfloat16>()
                                                                        : dw_chunk_cols<float>());
@@ -659,6 +679,13 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_CUDA(cudaMemsetAsync(h->dw_cnt, 0, E * (size_t)h->dw_chunks * sizeof(int), st));
     BEAM_CUDA(cudaMemsetAsync(h->zero_int, 0, 2 * sizeof(int), st));
     BEAM_CUDA(cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming));
+    BEAM_CUDA(cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking));
+    BEAM_CUDA(cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking));
+    for (int i = 0; i < 4; ++i) {
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming));
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming));
+    }
+    BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_copied, cudaEventDisableTiming));
     if (h->Fsh > 0) {
         BEAM_CUDA(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
         BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
@@ -1123,6 +1150,51 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     else ce = launch_combine<float, float>(h, yr, ysh_out, rt.ghat, T_, y, st);
     BEAM_CUDA(ce);
     return BEAM_OK;
+}
+
+// ---------------------------------------------------------------- pipelined host calls
+// Statistics of a host call run as several chunks: after each chunk's forward, mode 0 (the
+// first chunk) copies its statistics and per-expert counts into the accumulator, mode 1 adds
+// them (integer sums, the L_reg sum in chunk order; error bits OR-ed); mode 2 writes the
+// accumulated values back as the statistics of the whole call (the active experts recounted
+// from the summed counts).  One block.
+__global__ void __launch_bounds__(256)
+stats_accumulate_kernel(DevStats* __restrict__ st, const int* __restrict__ counts,
+                        DevStats* __restrict__ acc, int* __restrict__ acc_counts, int E, int mode)
+{
+    pdl_wait();
+    __shared__ int s_act;
+    if (threadIdx.x == 0) s_act = 0;
+    __syncthreads();
+    int act = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        if (mode == 0) acc_counts[e] = counts[e];
+        else if (mode == 1) acc_counts[e] += counts[e];
+        else { const_cast<int*>(counts)[e] = acc_counts[e]; act += acc_counts[e] > 0; }
+    }
+    if (mode == 2) atomicAdd(&s_act, act);   // an integer count: order-free
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (mode == 0) {
+            *acc = *st;
+        } else if (mode == 1) {
+            acc->keep_sum += st->keep_sum;
+            acc->lreg_sum += st->lreg_sum;
+            acc->n_all_masked += st->n_all_masked;
+            acc->n_kept += st->n_kept;
+            acc->tokens += st->tokens;
+            acc->err |= st->err;
+        } else {
+            st->keep_sum = acc->keep_sum;
+            st->lreg_sum = acc->lreg_sum;
+            st->n_all_masked = acc->n_all_masked;
+            st->n_kept = acc->n_kept;
+            st->tokens = acc->tokens;
+            st->err |= acc->err;
+            st->n_active = s_act;
+        }
+    }
+    pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------- fused decode
@@ -1629,6 +1701,71 @@ static beam_status_t softtopk_check(int32_t T, int32_t E, float tau, const void*
     return BEAM_OK;
 }
 
+// A pipelined host call: the batch as C chunks of whole segments.  Chunk c's x copy runs on
+// copy_in, its forward on `st` once the copy has landed, and its y copy on copy_out once the
+// forward is done, so the copies of one chunk overlap the forwards of its neighbours.  The
+// routing arrays of chunk c are written at the chunk's offset (the handle's pointers are
+// shifted for the call), so the routing of every token is kept; the statistics are added up
+// over the chunks on the device.
+constexpr int kHostChunkTokens = 1366;   // about 3 chunks for a 4096-token batch
+constexpr int kHostMaxChunks = 4;
+constexpr int kHostPipelineMinTokens = 1024;   // smaller batches are copied and run whole
+
+template <typename T>
+static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_, float* y_host,
+                                            uint32_t flags, cudaStream_t st)
+{
+    const int D = h->D, K = h->K, E = h->E;
+    const int align = h->S > 1 ? h->S : 32;
+    const int C = std::min(kHostMaxChunks, std::max(2, ceil_div(T_, kHostChunkTokens)));
+    const int tc = ceil_div(ceil_div(T_, C), align) * align;
+    const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false
+                                                                                        : h->tc_ok;
+    const uint32_t fflags = flags & ~(BEAM_HOST_PIPELINE | BEAM_NO_GRAPH);
+    // the copy streams start after the work already on `st` (x_stage / y_stage are free)
+    BEAM_CUDA(cudaEventRecord(h->ev_copied, st));
+    BEAM_CUDA(cudaStreamWaitEvent(h->copy_in, h->ev_copied, 0));
+    BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_copied, 0));
+    const RouteIn base = own_routing(h);
+    int nchunks = 0;
+    for (int c = 0, off = 0; off < T_; ++c, off += tc) {
+        const int n = std::min(tc, T_ - off);
+        const size_t xo = (size_t)off * D;
+        BEAM_CUDA(cudaMemcpyAsync(static_cast<T*>(h->x_stage) + xo, x_host + xo, (size_t)n * D * sizeof(T),
+                                  cudaMemcpyHostToDevice, h->copy_in));
+        BEAM_CUDA(cudaEventRecord(h->ev_in[c], h->copy_in));
+        BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_in[c], 0));
+        // the chunk's routing lands at its offset of the handle's routing arrays
+        h->topk_id = const_cast<int*>(base.topk_id) + (size_t)off * K;
+        h->gate = const_cast<float*>(base.gate) + (size_t)off * K;
+        h->mlogit = const_cast<float*>(base.mlogit) + (size_t)off * K;
+        h->keep = const_cast<uint8_t*>(base.keep) + (size_t)off * K;
+        h->ghat = const_cast<float*>(base.ghat) + (size_t)off * K;
+        h->nkeep_tok = const_cast<int*>(base.nkeep) + off;
+        h->lreg_tok = const_cast<float*>(base.lreg) + off;
+        beam_status_t r = forward_impl<T>(h, static_cast<const T*>(h->x_stage) + xo, n, h->y_stage + xo,
+                                          fflags, use_tc, st);
+        h->topk_id = const_cast<int*>(base.topk_id); h->gate = const_cast<float*>(base.gate);
+        h->mlogit = const_cast<float*>(base.mlogit); h->keep = const_cast<uint8_t*>(base.keep);
+        h->ghat = const_cast<float*>(base.ghat); h->nkeep_tok = const_cast<int*>(base.nkeep);
+        h->lreg_tok = const_cast<float*>(base.lreg);
+        BEAM_TRY(r);
+        BEAM_CUDA(launch(h, ST_COMPACT_SCAN, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
+                         h->dstats, (const int*)h->counts, h->acc_stats, h->acc_counts, E, c == 0 ? 0 : 1));
+        BEAM_CUDA(cudaEventRecord(h->ev_out[c], st));
+        BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_out[c], 0));
+        BEAM_CUDA(cudaMemcpyAsync(y_host + xo, h->y_stage + xo, (size_t)n * D * sizeof(float),
+                                  cudaMemcpyDeviceToHost, h->copy_out));
+        ++nchunks;
+    }
+    BEAM_CUDA(launch(h, ST_COMPACT_SCAN, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
+                     h->dstats, (const int*)h->counts, h->acc_stats, h->acc_counts, E, 2));
+    BEAM_CUDA(cudaEventRecord(h->ev_copied, h->copy_out));
+    BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_copied, 0));
+    (void)nchunks;
+    return BEAM_OK;
+}
+
 extern "C" {
 
 beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, int32_t* topk_id,
@@ -1832,6 +1969,7 @@ beam_status_t beam_moe_ep_dispatch(beam_moe_t* h, const void* x, int32_t T, uint
     h->cur = own_routing(h);
     h->last_T = T;
     h->last_train = false;
+    h->last_pipelined = false;
     BEAM_CUDA(cudaEventRecord(h->done, st));
     return BEAM_OK;
 }
@@ -1985,6 +2123,7 @@ static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float*
     }
     h->last_T = T;
     h->last_train = (flags & BEAM_TRAIN) != 0;
+    h->last_pipelined = false;
     BEAM_CUDA(cudaEventRecord(h->done, st));
     return BEAM_OK;
 }
@@ -2032,9 +2171,34 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
     if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
     if (T > 0 && (!x_host || !y_host)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((flags & BEAM_HOST_PIPELINE) && T >= kHostPipelineMinTokens && h->Ew > 0) {
+        if (flags & (BEAM_TRAIN | BEAM_FUSED_DECODE))
+            return fail(BEAM_ERR_INVALID_ARG, "BEAM_HOST_PIPELINE excludes BEAM_TRAIN and BEAM_FUSED_DECODE");
+        if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_HOST_PIPELINE))
+            return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+        if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
+            return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
+        if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
+            return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core expert path needs a bf16 layer with "
+                        "d_model a multiple of 256");
+        if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
+        if (h->prof) ++h->prof_forwards;
+        beam_status_t r = (h->cfg.dtype == BEAM_DTYPE_BF16)
+            ? forward_host_pipelined<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x_host), T,
+                                                    y_host, flags, st)
+            : forward_host_pipelined<float>(h, static_cast<const float*>(x_host), T, y_host, flags, st);
+        BEAM_TRY(r);
+        h->cur = own_routing(h);
+        h->last_T = T;
+        h->last_train = false;
+        h->last_pipelined = true;
+        BEAM_CUDA(cudaEventRecord(h->done, st));
+        BEAM_CUDA(cudaStreamSynchronize(st));
+        return BEAM_OK;
+    }
     const size_t xb = (size_t)T * h->D * h->esz, yb = (size_t)T * h->D * sizeof(float);
     if (T > 0) BEAM_CUDA(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st));
-    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, h->y_stage, flags, stream));
+    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, h->y_stage, flags & ~BEAM_HOST_PIPELINE, stream));
     if (T > 0) BEAM_CUDA(cudaMemcpyAsync(y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, st));
     BEAM_CUDA(cudaStreamSynchronize(st));
     return BEAM_OK;
@@ -2081,6 +2245,9 @@ beam_status_t beam_moe_get_routing(beam_moe_t* h, int32_t* topk_id, float* gate,
         if (offsets) memset(offsets, 0, sizeof(int32_t) * (h->E + 1));
         return BEAM_OK;
     }
+    if (h->last_pipelined && (offsets || perm || inv))
+        return fail(BEAM_ERR_UNSUPPORTED, "after a pipelined host call (BEAM_HOST_PIPELINE) only "
+                    "topk_id, gate, mask_logit and keep are available: the compaction ran per chunk");
     // the arrays the last forward read: its own, or those given to beam_moe_forward_routed
     const RouteIn& c = h->cur;
     if ((gate && !c.gate) || (mask_logit && !c.mlogit))

@@ -138,11 +138,13 @@ class BeamMoE:
         return out
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, mask_off: bool = False,
-                     path: str | None = None, stream=None) -> torch.Tensor:
-        """Host-buffer variant: copies x in, runs the layer, copies y out, synchronises."""
+                     path: str | None = None, stream=None, pipeline: bool = False) -> torch.Tensor:
+        """Host-buffer variant: copies x in, runs the layer, copies y out, synchronises.
+        pipeline=True (batches of >= 1024 tokens) runs chunks whose copies overlap the
+        forwards of the others (see BEAM_HOST_PIPELINE)."""
         T = x_host.shape[0]
-        check(_lib.load().beam_moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host),
-                                                self.flags(mask_off, path),
+        flags = self.flags(mask_off, path) | (_lib.BEAM_HOST_PIPELINE if pipeline else 0)
+        check(_lib.load().beam_moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host), flags,
                                                 ctypes.c_void_p(_stream_handle(stream))))
         return y_host
 
@@ -156,17 +158,20 @@ class BeamMoE:
                     n_tokens_all_masked=s.n_tokens_all_masked, tokens=s.tokens,
                     n_kept=s.n_kept, counts=counts)
 
-    def routing(self, T: int) -> dict:
-        """Routing of the last forward (T must be that forward's token count)."""
+    def routing(self, T: int, compaction: bool = True) -> dict:
+        """Routing of the last forward (T must be that forward's token count); compaction=False
+        leaves out offsets, perm and inv (not kept by a pipelined host call)."""
         K, E = self.top_k, self.n_experts
         out = dict(topk_id=np.zeros((T, K), np.int32), gate=np.zeros((T, K), np.float32),
-                   mask_logit=np.zeros((T, K), np.float32), keep=np.zeros((T, K), np.uint8),
-                   offsets=np.zeros(E + 1, np.int32), perm=np.zeros(max(1, T * K), np.int32),
-                   inv=np.zeros((T, K), np.int32))
+                   mask_logit=np.zeros((T, K), np.float32), keep=np.zeros((T, K), np.uint8))
+        if compaction:
+            out.update(offsets=np.zeros(E + 1, np.int32), perm=np.zeros(max(1, T * K), np.int32),
+                       inv=np.zeros((T, K), np.int32))
         p = {k: v.ctypes.data_as(ctypes.c_void_p) for k, v in out.items()}
         check(_lib.load().beam_moe_get_routing(self._h, p["topk_id"], p["gate"], p["mask_logit"],
-                                               p["keep"], p["offsets"], p["perm"], p["inv"]))
-        out["perm"] = out["perm"][: int(out["offsets"][E])].copy()
+                                               p["keep"], p.get("offsets"), p.get("perm"), p.get("inv")))
+        if compaction:
+            out["perm"] = out["perm"][: int(out["offsets"][E])].copy()
         return out
 
     def profile_begin(self, max_forwards: int) -> None:

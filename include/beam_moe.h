@@ -58,6 +58,9 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_TRAIN        0x20u /* training forward: every Top-K slot's expert is evaluated
                                    and the mask only scales the gates (g_hat = g * m), so that
                                    beam_moe_backward_router can follow (see there) */
+#define BEAM_HOST_PIPELINE 0x40u /* beam_moe_forward_host only: run a batch of >= 1024 tokens
+                                   as chunks whose copies overlap the forwards of the others
+                                   (see beam_moe_forward_host) */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
@@ -140,6 +143,15 @@ beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, floa
  * beam_moe_forward with host buffers: copies x_host (T*D elements of the storage type) to a
  * handle-owned device buffer, runs the forward and copies y back to y_host (T*D float32),
  * then synchronises `stream`.  Pinned host memory gives full-bandwidth copies.
+ * BEAM_HOST_PIPELINE (T >= 1024; flags may add BEAM_MASK_OFF, BEAM_PATH_* and BEAM_NO_GRAPH):
+ * the batch runs as 2 to 4 chunks of whole segments (about 1366 tokens each); chunk c's x copy,
+ * forward and y copy are ordered on two copy streams and `stream`, so the copies of one chunk
+ * overlap the forwards of its neighbours.  Each chunk is a complete forward of its tokens (the
+ * same arithmetic per token; a token near a Top-K or mask tie may resolve differently from a
+ * whole-batch forward, within the 1e-3 margin).  beam_moe_stats then describes the whole call
+ * (statistics and counts added up over the chunks on the device); beam_moe_get_routing gives
+ * topk_id, gate, mask_logit and keep of every token and returns BEAM_ERR_UNSUPPORTED if asked
+ * for offsets, perm or inv (the compaction ran per chunk).  Direct launches (no graph replay).
  */
 beam_status_t beam_moe_forward_host(beam_moe_t *h, const void *x_host, int32_t T, float *y_host,
                                     uint32_t flags, void *stream);

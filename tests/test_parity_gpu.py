@@ -539,8 +539,8 @@ def test_fp16_overflow_of_h_is_reported(T, path, fused):
 
 # ------------------------------------------------------------------ short-K down projection
 @pytest.mark.parametrize("F,T,E,K", [(256, 1600, 8, 2), (128, 900, 16, 4), (256, 3000, 60, 4),
-                                     (64, 600, 8, 1), (256, 2000, 212, 16)],
-                         ids=["f256_e8", "f128_e16", "f256_e60", "f64_one_kstep", "f256_e212"])
+                                     (128, 600, 8, 1), (256, 2000, 212, 16)],
+                         ids=["f256_e8", "f128_e16", "f256_e60", "f128_k1", "f256_e212"])
 def test_short_k_down_projection(F, T, E, K):
     """Routed down projections with F <= 256 (at most 4 k-steps per tile) run the kernel that
     keeps a unit's H rows in shared memory for all of its N-tiles (groups of more than 64 rows on
@@ -556,4 +556,50 @@ def test_short_k_down_projection(F, T, E, K):
     y2 = layer.forward(info["x"].cuda(), path="tensor", graph=False)
     torch.cuda.synchronize()
     assert torch.equal(y2, info["y"])
+    layer.close()
+
+
+# ------------------------------------------------------------------ pipelined host call
+@pytest.mark.parametrize("T,seg", [(3000, 0), (2500, 16), (1100, 0)], ids=["t3000", "segments", "two_chunks"])
+def test_pipelined_host_call(T, seg):
+    """BEAM_HOST_PIPELINE: the batch runs as chunks whose copies overlap the other chunks'
+    forwards.  y against the oracle on a spread sample; the routing of every token (clean tokens
+    bit-exact); the statistics describe the whole call (added over the chunks on the device)
+    and agree with the returned routing exactly; offsets / perm / inv are refused."""
+    from dynamic_expert_routing_b200 import BeamMoE, BeamError, _lib
+    spec = _small(n_shared=1, d_ff_shared=128, segment_len=seg)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=T, segment_len=seg)
+    x = synth.make_tokens(spec, T, seed=17)
+    yh = torch.full((T, spec.d_model), float("nan"), dtype=torch.float32).pin_memory()
+    layer.forward_host(x.pin_memory(), yh, pipeline=True)
+    gr = layer.routing(T, compaction=False)
+    orr = oracle.route(x, w["w_router"], w["w_mask"], spec.top_k, segment_len=seg)
+    clean = orr.clean()
+    for t in np.nonzero(clean)[0]:
+        assert set(gr["topk_id"][t].tolist()) == set(orr.topk_id[t].tolist())
+    same = clean & np.array([{int(e): int(k) for e, k in zip(gr["topk_id"][t], gr["keep"][t])} ==
+                             {int(e): int(k) for e, k in zip(orr.topk_id[t], orr.keep[t])} for t in range(T)])
+    sel = np.nonzero(same)[0][::7]
+    y_ref = oracle.layer(x, w, orr, tokens=sel)
+    parity.compare_y(yh.numpy()[sel], y_ref, spec.storage)
+    st = layer.stats()
+    assert st["tokens"] == T
+    keep = gr["keep"].astype(bool)
+    assert st["n_kept"] == int(keep.sum())
+    assert st["avg_k"] == keep.sum() / T
+    counts = np.bincount(gr["topk_id"][keep], minlength=spec.n_experts)
+    np.testing.assert_array_equal(st["counts"], counts)
+    assert st["n_active_experts"] == int((counts > 0).sum())
+    assert st["n_tokens_all_masked"] == int((keep.sum(axis=1) == 0).sum())
+    with pytest.raises(BeamError) as ei:
+        layer.routing(T)
+    assert ei.value.status == _lib.BEAM_ERR_UNSUPPORTED
+    # a second call on the same buffers gives the same bits; an ordinary forward afterwards
+    # restores the full routing
+    y1 = yh.clone()
+    layer.forward_host(x.pin_memory(), yh, pipeline=True)
+    assert torch.equal(y1, yh)
+    layer.forward(x.cuda())
+    layer.routing(T)
     layer.close()
