@@ -310,6 +310,54 @@ def gen_point(torch, name, steps, warmup, device, peaks):
                 l2="flushed (256 MB written, then read) between timed calls")
 
 
+# SoftTopK points (the relaxation of the mask generator's top-k): name -> (rows, experts, K, tau)
+SOFTTOPK_POINTS = {"softtopk-fine8192": (8192, 212, 16, 1.0),
+                   "softtopk-fine44-decode": (44, 212, 16, 1.0)}
+
+
+def softtopk_point(torch, name, steps, warmup, device, peaks):
+    """SoftTopK forward (y, hard mask, nu) and backward on `rows` logit rows, each call timed with
+    its own event pair after an L2 flush.  Algorithmic bytes: forward 4 B read + 4 B (y) + 1 B
+    (mask) written per logit and 4 B of nu per row; backward 8 B read + 4 B written per logit."""
+    from dynamic_expert_routing_b200 import softtopk, softtopk_backward
+    T, E, K, tau = SOFTTOPK_POINTS[name]
+    g = torch.Generator(device=device)
+    g.manual_seed(3)
+    r = torch.randn((T, E), generator=g, device=device, dtype=torch.float32)
+    dy = torch.randn((T, E), generator=g, device=device, dtype=torch.float32)
+    flush = L2Flush(torch, device)
+    for _ in range(warmup):
+        out = softtopk(r, K, tau, nu=True)
+        softtopk_backward(out["y"], dy, tau)
+    st = torch.cuda.current_stream()
+    fw, bw = [], []
+    for _ in range(steps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        out = softtopk(r, K, tau, nu=True)
+        b.record(st)
+        fw.append((a, b))
+        flush()
+        c, d = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c.record(st)
+        softtopk_backward(out["y"], dy, tau)
+        d.record(st)
+        bw.append((c, d))
+    torch.cuda.synchronize()
+    ms_f = sum(p.elapsed_time(q) for p, q in fw) / steps
+    ms_b = sum(p.elapsed_time(q) for p, q in bw) / steps
+    bytes_f = T * E * 9 + T * 4
+    bytes_b = T * E * 12
+    return dict(workload=name, metric="SoftTopK rows/s", unit="rows/s", rows=T, experts=E, top_k=K,
+                tau=tau, value=round(T / (ms_f * 1e-3), 2), ms_forward=round(ms_f, 5),
+                ms_backward=round(ms_b, 5),
+                forward_hbm_frac=round(bytes_f / (peaks["hbm"] * 1e9) / (ms_f * 1e-3), 4),
+                backward_hbm_frac=round(bytes_b / (peaks["hbm"] * 1e9) / (ms_b * 1e-3), 4),
+                algorithmic_bytes_forward=bytes_f, algorithmic_bytes_backward=bytes_b,
+                l2=L2_LABEL_FLUSHED)
+
+
 def grad_work(spec, T, tc_path=True) -> dict:
     """Algorithmic bytes of the routing gradient's kernels (all HBM-bound; their FLOPs are a
     few per byte).  route_grad: dy and dx rows (fp32), every Top-K slot's expert output row
@@ -797,6 +845,9 @@ def _run_ours(args):
                 gen_points.append(gen_point(torch, p, max(10, args.steps), args.warmup, device, peaks))
             train_points.append(train_point(torch, "train-mixtral-prefill", max(10, args.steps),
                                             args.warmup, device, peaks))
+            for p in SOFTTOPK_POINTS:
+                train_points.append(softtopk_point(torch, p, max(10, args.steps), args.warmup,
+                                                   device, peaks))
 
     if rank == 0:
         line = {
@@ -864,6 +915,8 @@ def run_sweep(args):
         if name != "train-profile":
             print(json.dumps(train_point(torch, name, args.steps, args.warmup, device, peaks)),
                   flush=True)
+    for name in SOFTTOPK_POINTS:
+        print(json.dumps(softtopk_point(torch, name, args.steps, args.warmup, device, peaks)), flush=True)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
