@@ -9,10 +9,11 @@
 // through nu, is dr_j = h_j (dy_j - sum_i h_i dy_i / sum_i h_i) with h_i = y_i (1 - y_i) / tau.
 //
 // One warp per token row; lane l holds logits l, l + 32, ... (EPL = ceil(E/32) per lane).
-//   forward:  nu by bisection in fp32 on f(nu) = sum_i sigmoid((r_i - nu)/tau) - K (strictly
-//             decreasing) from [min r - 40 tau, max r + 40 tau] until the midpoint equals an
-//             end of the bracket; every lane evaluates f with the same xor-butterfly sum, so the
-//             bracket is bitwise identical across the warp.  Then y, and the hard Top-K
+//   forward:  nu by safeguarded Newton in fp32 on f(nu) = sum_i sigmoid((r_i - nu)/tau) - K
+//             (strictly decreasing) inside the sign bracket [min r - 40 tau, max r + 40 tau],
+//             bisecting whenever a step leaves the bracket, until |f| reaches the float32
+//             resolution of the sum; every lane evaluates f with the same xor-butterfly sum, so
+//             the iteration is bitwise identical across the warp.  Then y, and the hard Top-K
 //             indicator (K rounds of a warp arg-max under (value desc, index asc)).
 //   backward: two butterfly sums per row (sum h, sum h dy), then dr.
 // Deterministic: fixed reduction order, no atomics.  HBM-bound: 4 B per logit read, 4 + 1 B
@@ -53,19 +54,36 @@ softtopk_fwd_kernel(const float* __restrict__ r, int T, int E, int K, float tau,
         if (K >= E) {
             nu = -INFINITY;   // y = 1 everywhere: the constraint leaves no freedom
         } else {
+            // safeguarded Newton on f(nu) = sum_i sigmoid((r_i - nu)/tau) - K, which is strictly
+            // decreasing with f' = -sum_i h_i: a Newton step that leaves the sign bracket
+            // [lo, hi] is replaced by the bisection of the bracket.  It stops once |f| is below
+            // the float32 resolution of the sum (K 2^-21), the step no longer moves nu, or the
+            // bracket is two adjacent floats; every lane computes the same sums (xor butterfly),
+            // so the iteration is identical across the warp.
             lo -= 40.f * tau;
             hi += 40.f * tau;
-            for (int it = 0; it < 200; ++it) {
-                const float mid = 0.5f * (lo + hi);
-                if (mid <= lo || mid >= hi) break;   // the bracket is two adjacent floats
-                float s = 0.f;
-#pragma unroll
-                for (int j = 0; j < EPL; ++j)
-                    if (lane + 32 * j < E) s += sigmoid_f((v[j] - mid) * inv_tau);
-                s = warp_sum(s);
-                if (s > (float)K) lo = mid; else hi = mid;
-            }
+            const float tol = (float)K * 4.76837158e-7f;   // K * 2^-21
             nu = 0.5f * (lo + hi);
+            for (int it = 0; it < 100; ++it) {
+                float s = 0.f, hs = 0.f;
+#pragma unroll
+                for (int j = 0; j < EPL; ++j) {
+                    if (lane + 32 * j < E) {
+                        const float y = sigmoid_f((v[j] - nu) * inv_tau);
+                        s += y;
+                        hs += y * (1.f - y);
+                    }
+                }
+                s = warp_sum(s);
+                hs = warp_sum(hs) * inv_tau;
+                const float f = s - (float)K;
+                if (f > 0.f) lo = nu; else hi = nu;
+                if (fabsf(f) <= tol) break;
+                float nn = nu + f / hs;
+                if (!(nn > lo && nn < hi)) nn = 0.5f * (lo + hi);
+                if (nn == nu || nn <= lo || nn >= hi) break;   // converged to the float grid
+                nu = nn;
+            }
         }
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
