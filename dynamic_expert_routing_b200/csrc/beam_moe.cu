@@ -202,6 +202,8 @@ struct beam_moe {
     // counters (cleared by the compaction scan of every forward)
     float* tail_ws = nullptr;
     int* tail_cnt = nullptr;     // [kTailCntRegions][num_sms][kEpiWarps]
+    int* fold_cnt = nullptr;     // split-K gate/up with SwiGLU folded in: arrival counters
+                                 // [E * 2F/256 + 2Fsh/256][4], zero between launches
     int* zero_int = nullptr;     // two zeros: an empty group table
     int* range_flag = nullptr;
     unsigned* rcnt = nullptr;    // arrival counters of the small-batch router, one per block of
@@ -545,6 +547,13 @@ static beam_status_t setup_tc(beam_moe* h)
         c.out_shared = h->g1part_sh; c.ld_shared = (int)(2 * Fsh);
         c.split_stride_routed = (long long)sr * h->K * 2 * F;
         c.split_stride_shared = (long long)sr * 2 * Fsh;
+    }
+    // split-K gate/up launches finish SwiGLU in the epilogue: one counter per (tile, lane
+    // quadrant); a split launch has at most one 128-row tile per group (<= 64 rows each)
+    {
+        const size_t n = ((size_t)E * (2 * F / tc::BN) + (Fsh ? 2 * Fsh / tc::BN : 0)) * 4;
+        BEAM_TRY(dalloc(h, &h->fold_cnt, n * sizeof(int)));
+        BEAM_CUDA(cudaMemset(h->fold_cnt, 0, n * sizeof(int)));
     }
     // tail split: at most kTailMaxSubWaves * num_sms piece slots per launch
     {
@@ -904,15 +913,16 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
     p.tail_cnt = tail1 ? h->tail_cnt : nullptr;
     p.tail_ws = tail1 ? h->tail_ws : nullptr;
     if (split1) {
+        // f32 partial slices; the warp that completes a tile quadrant's slices adds them in
+        // slice order and writes H (SwiGLU), so no finishing launch follows
+        p.fold_cnt = h->fold_cnt;
+        p.fold_h_routed = static_cast<__half*>(h->hbuf);
+        p.fold_h_shared = static_cast<__half*>(h->hsh);
+        p.fold_f_routed = F;
+        p.fold_f_shared = Fsh;
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
-        const long long work = (routed ? (long long)T_ * K * F : 0) + (shared ? (long long)T_ * Fsh : 0);
-        BEAM_CUDA(launch(h, st_fin, tc::swiglu_finish_kernel,
-                         dim3((unsigned)std::max<long long>(1, std::min<long long>(h->num_sms * 4, ceil_div(work, 256)))),
-                         dim3(256), 0, st, (const float*)h->g1part, s1n, p.split_stride_routed,
-                         (const int*)(routed ? h->offsets + E : h->zero_int), F, (__half*)h->hbuf,
-                         (const float*)h->g1part_sh, s1n, p.split_stride_shared, rows_sh, Fsh,
-                         (__half*)h->hsh, &h->dstats->err));
+        (void)st_fin;
     } else if (swap1) {
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_SWAP>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));

@@ -103,6 +103,13 @@ struct TcParams {
     // [kTailMaxSubWaves * grid slots][kEpiWarps][kTailSlotFloats].
     int* tail_cnt;
     float* tail_ws;
+    // SwiGLU folded into a split-K gate/up launch (EPI_STORE_F32 with the gate/up layout; null =
+    // off): arrival counters [tiles][4 lane quadrants], zero between launches (the warp that
+    // finishes a quadrant resets its counter), and the fp16 H outputs with their row lengths.
+    int* fold_cnt;
+    __half* fold_h_routed;
+    __half* fold_h_shared;
+    int fold_f_routed, fold_f_shared;
 };
 
 // Number of K pieces for the tail wave: rem whole-K tiles of ksteps k steps are left over after
@@ -266,6 +273,7 @@ struct Tile {
     int brow;     // first weight row of the tile
     int k0, k1;   // k steps [k0, k1) of this tile (its K split)
     int ks;       // K split index (selects the output slice)
+    int gmt;      // m tile index across the launch's groups (routed), or inside the shared problem
     int swap;     // 0, or N (32 / 64): a swapped tail tile (weights = M operand, rows = N)
     int pieces;   // tail split: K pieces of this tile (1 = a whole tile)
     int tail;     // tail split: index of the tile among the split ones
@@ -346,6 +354,7 @@ struct TileWalker {
             const int r = (int)(i % per_n);
             t.ks = r / mts_sh;
             t.mt = r % mts_sh;
+            t.gmt = t.mt;
             t.row0 = 0;
             t.m = p->shared_rows;
             t.brow = t.n * BN;
@@ -370,6 +379,7 @@ struct TileWalker {
         const int rr = (int)(rl % per_n);
         t.ks = rr / cg_mts;
         t.mt = rr % cg_mts;
+        t.gmt = cg.mt0 + t.mt;
         t.row0 = cg.row0;
         t.m = cg.m;
         t.brow = cg.expert * p->b_rows_per_expert + t.n * BN;
@@ -802,6 +812,50 @@ __device__ __forceinline__ void gemm_roles(const TcParams& p, const GemmSmem& sm
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tempty_bar(acc));
                 if (++acc == 2) { acc = 0; aph ^= 1u; }
+            }
+            if (EPI == EPI_STORE_F32 && p.fold_cnt != nullptr) {
+                // SwiGLU folded into the split-K gate/up launch: the 2 warps of this lane
+                // quadrant x the launch's K slices each store a partial; the warp whose arrival
+                // completes the count (the atomic only elects it) adds the slices in slice order
+                // and writes H = silu(gate) * up for the quadrant's rows and the tile's 128
+                // features -- the same sums, in the same order, as the SwiGLU finishing kernel.
+                const int splits = t.shared ? p.k_splits_shared : p.k_splits_routed;
+                const long long mts_routed = p.n_groups[1];
+                const long long tile = t.shared
+                    ? mts_routed * p.n_tiles_routed + (long long)t.gmt * p.n_tiles_shared + t.n
+                    : (long long)t.gmt * p.n_tiles_routed + t.n;
+                int* cnt = p.fold_cnt + tile * 4 + (warp & 3);
+                __threadfence();
+                __syncwarp();
+                int prev = 0;
+                if (lane == 0) prev = atomicAdd(cnt, 1);
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == 2 * splits - 1) {
+                    __threadfence();   // the other partials of the quadrant are visible
+                    const float* part = static_cast<const float*>(t.shared ? p.out_shared : p.out_routed);
+                    const long long st = t.shared ? p.split_stride_shared : p.split_stride_routed;
+                    __half* hout = t.shared ? p.fold_h_shared : p.fold_h_routed;
+                    const int FF = t.shared ? p.fold_f_shared : p.fold_f_routed;
+                    for (int i = 0; i < nrows; ++i) {
+                        const size_t row = row_base + i;
+                        const float* src = part + row * ld + (size_t)t.n * BN + 4 * lane;
+                        float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
+                        for (int q = 0; q < splits; ++q) {
+                            const float4 a = __ldcg(reinterpret_cast<const float4*>(src + q * st));
+                            const float4 b = __ldcg(reinterpret_cast<const float4*>(src + q * st + BN / 2));
+                            g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
+                            u.x += b.x; u.y += b.y; u.z += b.z; u.w += b.w;
+                        }
+                        const float h0 = silu_f(g.x) * u.x, h1 = silu_f(g.y) * u.y;
+                        const float h2 = silu_f(g.z) * u.z, h3 = silu_f(g.w) * u.w;
+                        bad |= fp16_out_of_range(h0) | fp16_out_of_range(h1) |
+                               fp16_out_of_range(h2) | fp16_out_of_range(h3);
+                        __half2 hv[2] = {__floats2half2_rn(h0, h1), __floats2half2_rn(h2, h3)};
+                        *reinterpret_cast<uint2*>(hout + row * FF + (size_t)t.n * (BN / 2) + 4 * lane) =
+                            *reinterpret_cast<const uint2*>(hv);
+                    }
+                    if (lane == 0) *cnt = 0;   // ready for the next launch
+                }
             }
         }
         if (bad) atomicOr(p.err, ERR_FP16_RANGE);

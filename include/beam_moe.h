@@ -446,8 +446,8 @@ beam_status_t beam_ep_recv_routing(const int32_t *recv_counts_dev, int32_t P, in
  * beam_softtopk_forward: logits_dev [T][E] float32 -> y_dev [T][E] float32, and optionally
  *   mask_dev [T][E] uint8 (the hard Top-K indicator, ties to the lower index, as the layer's
  *   router) and nu_dev [T] float32.  nu is found by safeguarded Newton iteration in float32
- *   (bisection inside the sign bracket whenever a step leaves it) until the constraint holds
- *   to the float32 resolution of the sum; y agrees with a float64 solution to about 1e-5.
+ *   (bisection inside the sign bracket whenever a step leaves it) until a step is below
+ *   2^-16 tau; y agrees with a float64 solution to about 1e-5.
  * beam_softtopk_backward: dlogits_dev [T][E] = the Jacobian of y (through nu) applied to
  *   dy_dev [T][E]: with h_i = y_i (1 - y_i) / tau,
  *   dlogits_j = h_j (dy_j - sum_i h_i dy_i / sum_i h_i)   (0 when sum_i h_i = 0);

@@ -272,7 +272,8 @@ def test_profiling_stages_count_every_launch(T):
     up to the handle's launch counter (so a roofline that divides a stage's time by its
     launches is consistent).  T = 300 runs the shared experts on the second stream, timed
     under stages of their own; T = 4 splits K and runs them inside the routed launches (as
-    separate kernels: fused=False, not the one-launch decode path)."""
+    separate kernels: fused=False, not the one-launch decode path), with SwiGLU finished inside
+    the split gate/up launch."""
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=256)
     w = synth.make_layer(spec, keep_rate=0.5)
@@ -290,11 +291,12 @@ def test_profiling_stages_count_every_launch(T):
     stages = {k: v for k, v in prof.items() if k != "forwards"}
     assert sum(c for _, c in stages.values()) == layer.launch_count() - n0
     split = T <= 64
-    expect = ["tc_gateup", "tc_down"] + (["swiglu_finish"] if split else ["tc_shared_gateup", "tc_shared_down"])
+    # split K: SwiGLU is finished inside the gate/up launch (no finishing kernel)
+    expect = ["tc_gateup", "tc_down"] + ([] if split else ["tc_shared_gateup", "tc_shared_down"])
     for s_ in expect:
         assert stages[s_][1] == n, (s_, stages[s_])
         assert stages[s_][0] > 0
-    absent = ["tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish"] if split else ["swiglu_finish"]
+    absent = ["swiglu_finish", "shared_swiglu_finish"] + (["tc_shared_gateup", "tc_shared_down"] if split else [])
     for s_ in absent:
         assert s_ not in stages, (s_, stages)
     layer.close()
