@@ -61,23 +61,29 @@ softtopk_fwd_kernel(const float* __restrict__ r, int T, int E, int K, float tau,
             // under the float32 rounding noise of the sum f itself, which a tighter test could
             // only chase.  Every lane computes the same sums (xor butterfly), so the iteration is
             // identical across the warp.
+            // With K > E/2 the sum is taken over the complements, f = (E - K) - sum_i
+            // sigmoid((nu - r_i)/tau): the terms are then the small ones, and f keeps its
+            // precision instead of being a difference of two numbers near K.
             lo -= 40.f * tau;
             hi += 40.f * tau;
             const float eps = 1.52587890625e-5f * tau;   // 2^-16 tau
+            const bool comp = 2 * K > E;
+            const float target = comp ? (float)(E - K) : (float)K;
             nu = 0.5f * (lo + hi);
             for (int it = 0; it < 100; ++it) {
                 float s = 0.f, hs = 0.f;
 #pragma unroll
                 for (int j = 0; j < EPL; ++j) {
                     if (lane + 32 * j < E) {
-                        const float y = sigmoid_f((v[j] - nu) * inv_tau);
+                        const float zz = (v[j] - nu) * inv_tau;
+                        const float y = sigmoid_f(comp ? -zz : zz);
                         s += y;
                         hs += y * (1.f - y);
                     }
                 }
                 s = warp_sum(s);
                 hs = warp_sum(hs) * inv_tau;
-                const float f = s - (float)K;
+                const float f = comp ? target - s : s - target;
                 if (f > 0.f) lo = nu; else hi = nu;
                 const float step = f / hs;
                 float nn = nu + step;
