@@ -253,14 +253,14 @@ enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
     ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE,
-    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_COUNT
+    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_CHUNK_STATS, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
     "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish",
-    "fused_decode", "route_grad", "route_dw"};
+    "fused_decode", "route_grad", "route_dw", "chunk_stats"};
 
 static void prof_release(beam_moe* h)
 {
@@ -1760,7 +1760,7 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
         h->ghat = const_cast<float*>(base.ghat); h->nkeep_tok = const_cast<int*>(base.nkeep);
         h->lreg_tok = const_cast<float*>(base.lreg);
         BEAM_TRY(r);
-        BEAM_CUDA(launch(h, ST_COMPACT_SCAN, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
+        BEAM_CUDA(launch(h, ST_CHUNK_STATS, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
                          h->dstats, (const int*)h->counts, h->acc_stats, h->acc_counts, E, c == 0 ? 0 : 1));
         BEAM_CUDA(cudaEventRecord(h->ev_out[c], st));
         BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_out[c], 0));
@@ -1768,7 +1768,7 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
                                   cudaMemcpyDeviceToHost, h->copy_out));
         ++nchunks;
     }
-    BEAM_CUDA(launch(h, ST_COMPACT_SCAN, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
+    BEAM_CUDA(launch(h, ST_CHUNK_STATS, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
                      h->dstats, (const int*)h->counts, h->acc_stats, h->acc_counts, E, 2));
     BEAM_CUDA(cudaEventRecord(h->ev_copied, h->copy_out));
     BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_copied, 0));

@@ -188,9 +188,10 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * the shared experts' GEMMs run on a second stream, overlapping the routing; they are timed
  * under stages of their own (tc_shared_gateup, tc_shared_down, shared_swiglu_finish), so that
  * each stage's time covers the work of one problem.  A fused decode forward is one launch,
- * timed as the stage fused_decode.
+ * timed as the stage fused_decode; the per-chunk statistics of a pipelined host call as
+ * chunk_stats.
  */
-#define BEAM_N_STAGES 18
+#define BEAM_N_STAGES 19
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);
