@@ -991,14 +991,6 @@ static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, co
                       (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
                       (const int*)h->inv, ghat, T_, h->K, h->D, y);
     }
-    if (T_ >= h->num_sms && h->K >= 8 && r.splits == 1 && sh.splits == 1) {
-        // many slots: the loads of 8 slots in flight at once (same sums, same order)
-        const int passes = ceil_div(d4, 256);
-        const int nthr = std::min(256, ceil_div(ceil_div(d4, passes), 32) * 32);
-        return launch(h, ST_COMBINE, combine_wide_kernel<TR, TS>, dim3(T_, 1), dim3(nthr), 0, st,
-                      (const TR*)r.base, (const TS*)sh.base, (const int*)h->inv, ghat, T_, h->K,
-                      h->D, y);
-    }
     const bool split_cols = T_ < h->num_sms;
     const int passes = ceil_div(d4, 256);
     const int nthr = split_cols ? 256 : std::min(256, ceil_div(ceil_div(d4, passes), 32) * 32);
@@ -1114,7 +1106,7 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
                          h->n_groups, h->dstats, h->tail_cnt, tail_cnt_ints(h->num_sms), h->tile_group,
                          h->scan_part, &h->dstats->grid_bar));
         BEAM_CUDA(launch(h, ST_SCATTER_GATHER, compact_scatter_gather_kernel<T>,
-                         dim3(ceil_div((long long)T_ * K, 8LL * kScatterPairsPerWarp)), dim3(256), 0, st,
+                         dim3(ceil_div((long long)T_ * K, 8)), dim3(256), 0, st,
                          rt.topk_id, rt.keep, T_, K, D, nch,
                          (const uint32_t*)h->bits, (const int*)h->offsets,
                          (const int*)h->chunk_base, x, h->perm, h->inv, (T*)h->xperm, 1));

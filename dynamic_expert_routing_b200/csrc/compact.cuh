@@ -307,13 +307,8 @@ compact_scan_kernel(const uint32_t* __restrict__ bits, int nch, int E, int T,
     pdl_launch_dependents();
 }
 
-// One warp per 32 consecutive (token, slot) pairs: lane l places pair i0 + l (its position
-// chain of dependent loads runs beside the other 31 lanes' chains), writes inv (-1 for a masked
-// slot) and perm; then the warp copies the batch's kept rows into X_perm as one stream of
-// 16-byte vectors over all of them (flattened row x vector index), 8 vectors per lane in flight,
-// so a warp keeps several rows' copies going at once.
-constexpr int kScatterPairsPerWarp = 32;
-
+// One warp per (token, slot).  Kept slots get their position, write perm / inv and copy the
+// token's activation row into X_perm; masked slots write inv = -1.
 template <typename TW>
 __global__ void __launch_bounds__(256)
 compact_scatter_gather_kernel(const int* __restrict__ topk_id, const uint8_t* __restrict__ keep,
@@ -322,58 +317,27 @@ compact_scatter_gather_kernel(const int* __restrict__ topk_id, const uint8_t* __
                               const TW* __restrict__ x, int* __restrict__ perm,
                               int* __restrict__ inv, TW* __restrict__ xperm, int gather)
 {
-    __shared__ int s_tok[8][kScatterPairsPerWarp];
-    __shared__ int s_pos[8][kScatterPairsPerWarp];
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long n = (long long)T * K;
-    const long long i0 = ((long long)blockIdx.x * 8 + warp) * kScatterPairsPerWarp;
-    if (i0 < n) {
-        const long long i = i0 + lane;
-        int pos = -1, t = 0;
-        if (i < n) {
-            t = (int)(i / K);
-            if (keep[i]) {
-                const int e = topk_id[i];
-                const int c = t >> 5, b = t & 31;
-                const uint32_t w = bits[(size_t)e * nch + c];
-                pos = offsets[e] + chunk_base[(size_t)e * nch + c] + __popc(w & ((1u << b) - 1u));
-            }
+    const long long i = (long long)blockIdx.x * 8 + warp;
+    if (i < (long long)T * K) {
+        const int t = (int)(i / K);
+        int pos = -1;
+        if (keep[i]) {
+            const int e = topk_id[i];
+            const int c = t >> 5, b = t & 31;
+            const uint32_t w = bits[(size_t)e * nch + c];
+            pos = offsets[e] + chunk_base[(size_t)e * nch + c] + __popc(w & ((1u << b) - 1u));
+        }
+        if (lane == 0) {
             inv[i] = pos;
             if (pos >= 0) perm[pos] = (int)i;
         }
-        if (gather) {
-            // the batch's kept pairs in lane order: entry q of the warp's list is the q-th
-            // kept lane's (token, position)
-            const uint32_t kept = __ballot_sync(0xffffffffu, pos >= 0);
-            if (pos >= 0) {
-                const int q = __popc(kept & ((1u << lane) - 1u));
-                s_tok[warp][q] = t;
-                s_pos[warp][q] = pos;
-            }
-            __syncwarp();
-            const int nk = __popc(kept);
+        if (gather && pos >= 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
+            uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)pos * D);
             const int nv = D * (int)sizeof(TW) / 16;
-            const int total = nk * nv;
-            for (int f0 = 0; f0 < total; f0 += 32 * 8) {
-                uint4 r[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int f = f0 + u * 32 + lane;
-                    if (f < total) {
-                        const int q = f / nv, v = f - q * nv;
-                        r[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)s_tok[warp][q] * D) + v);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int f = f0 + u * 32 + lane;
-                    if (f < total) {
-                        const int q = f / nv, v = f - q * nv;
-                        reinterpret_cast<uint4*>(xperm + (size_t)s_pos[warp][q] * D)[v] = r[u];
-                    }
-                }
-            }
+            copy_row_warp(dst, src, nv, lane);
         }
     }
     pdl_launch_dependents();

@@ -562,57 +562,6 @@ combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
     pdl_launch_dependents();
 }
 
-// combine_kernel for many slots (K >= 8) and unsplit outputs: the same sums in the same order,
-// with the loads of 8 slots issued before any of them is accumulated (combine_kernel keeps 4 in
-// flight), so a column's K = 16 rows take two load round trips instead of four.
-template <typename TY, typename TS>
-__global__ void __launch_bounds__(256)
-combine_wide_kernel(const TY* __restrict__ yperm, const TS* __restrict__ ysh,
-                    const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K,
-                    int D, float* __restrict__ y)
-{
-    __shared__ int s_inv[32];
-    __shared__ float s_g[32];
-    pdl_wait();
-    const int t = blockIdx.x;
-    if (t >= T) return;
-    if (threadIdx.x < K) {
-        s_inv[threadIdx.x] = inv[(size_t)t * K + threadIdx.x];
-        s_g[threadIdx.x] = ghat[(size_t)t * K + threadIdx.x];
-    }
-    __syncthreads();
-    const int D4 = D >> 2;
-    const int chunk = (D4 + gridDim.y - 1) / gridDim.y;
-    const int c_end = min(D4, (int)(blockIdx.y + 1) * chunk);
-    for (int c = blockIdx.y * chunk + threadIdx.x; c < c_end; c += blockDim.x) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k0 = 0; k0 < K; k0 += 8) {
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int k = k0 + u;
-                const int p = k < K ? s_inv[k] : -1;
-                if (p >= 0) v[u] = load4(yperm, (size_t)p * D4 + c);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int k = k0 + u;
-                if (k < K && s_inv[k] >= 0) {
-                    const float g = s_g[k];
-                    acc.x = fmaf(g, v[u].x, acc.x); acc.y = fmaf(g, v[u].y, acc.y);
-                    acc.z = fmaf(g, v[u].z, acc.z); acc.w = fmaf(g, v[u].w, acc.w);
-                }
-            }
-        }
-        if (ysh) {
-            const float4 w = load4(ysh, (size_t)t * D4 + c);
-            acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
-        }
-        __stcs(reinterpret_cast<float4*>(y) + (size_t)t * D4 + c, acc);
-    }
-    pdl_launch_dependents();
-}
-
 // The combine of a small batch (fewer tokens than SMs) whose expert outputs are split-K slices:
 // the per-column chain of slot x slice loads of combine_kernel is a long dependent walk there.
 // CTA (token t, 16-column block) has 16 x (K + 1) threads: thread (c, k < K) adds the slices of
