@@ -795,9 +795,11 @@ def _run_ours(args):
     xh = x.cpu().pin_memory()
     yh = torch.empty((T, spec.d_model), dtype=torch.float32).pin_memory()
 
-    def e2e_time(pipeline):
+    yh16 = torch.empty((T, spec.d_model), dtype=torch.bfloat16).pin_memory()
+
+    def e2e_time(pipeline, out=yh):
         for _ in range(max(1, args.warmup)):
-            layer.forward_host(xh, yh, mask_off=mask_off, pipeline=pipeline)
+            layer.forward_host(xh, out, mask_off=mask_off, pipeline=pipeline)
         if world > 1:
             dist.barrier()
         a = torch.cuda.Event(enable_timing=True)
@@ -805,7 +807,7 @@ def _run_ours(args):
         n = max(3, args.steps // 2)
         a.record()
         for _ in range(n):
-            layer.forward_host(xh, yh, mask_off=mask_off, pipeline=pipeline)
+            layer.forward_host(xh, out, mask_off=mask_off, pipeline=pipeline)
         b.record()
         torch.cuda.synchronize()
         return max_over_ranks(torch, dist, a.elapsed_time(b) / n, world, device)
@@ -813,6 +815,8 @@ def _run_ours(args):
     pipelined = T >= 1024
     e2e_ms = e2e_time(pipelined)
     e2e_plain_ms = e2e_time(False) if pipelined else e2e_ms
+    # the same call with y delivered in bf16 (rounded on the device), half the D2H bytes
+    e2e16_ms = e2e_time(pipelined, yh16) if spec.storage == "bf16" else None
 
     # mask off through the same library at the headline shape: the layer speedup from skipping
     y.zero_()
@@ -878,7 +882,12 @@ def _run_ours(args):
                     "h2d_bytes_per_step": T * spec.d_model * es,
                     "d2h_bytes_per_step": T * spec.d_model * 4,
                     "call": "beam_moe_forward_host" + (" with BEAM_HOST_PIPELINE" if pipelined else ""),
-                    "unpipelined_value": round(job_throughput(T, world, e2e_plain_ms), 2)},
+                    "unpipelined_value": round(job_throughput(T, world, e2e_plain_ms), 2),
+                    "y_bf16": None if e2e16_ms is None else {
+                        "value": round(job_throughput(T, world, e2e16_ms), 2),
+                        "d2h_bytes_per_step": T * spec.d_model * 2,
+                        "call": "the same call with a bf16 y_host (BEAM_HOST_Y_BF16: y rounded to "
+                                "bf16 on the device before the copy)"}},
             "gpu_launches": launches,
             "clocks": clocks,
             "cpu_baseline": cpu,

@@ -26,8 +26,9 @@ BEAM_NO_GRAPH = 0x8
 BEAM_FUSED_DECODE = 0x10
 BEAM_TRAIN = 0x20
 BEAM_HOST_PIPELINE = 0x40
+BEAM_HOST_Y_BF16 = 0x80
 
-BEAM_N_STAGES = 19
+BEAM_N_STAGES = 20
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 STATUS_NAMES = {0: "BEAM_OK", 1: "BEAM_ERR_INVALID_ARG", 2: "BEAM_ERR_OOM", 3: "BEAM_ERR_CUDA",

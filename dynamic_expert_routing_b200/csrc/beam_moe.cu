@@ -178,6 +178,7 @@ struct beam_moe {
     // host-call staging
     void* x_stage = nullptr;
     float* y_stage = nullptr;
+    __nv_bfloat16* y16_stage = nullptr;   // y rounded to bf16 for a BEAM_HOST_Y_BF16 host call
     // pipelined host calls (BEAM_HOST_PIPELINE): copy streams, per-chunk events, statistics
     // accumulated over the chunks
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
@@ -253,14 +254,14 @@ enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
     ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE,
-    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_CHUNK_STATS, ST_COUNT
+    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_CHUNK_STATS, ST_Y_BF16, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
     "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish",
-    "fused_decode", "route_grad", "route_dw", "chunk_stats"};
+    "fused_decode", "route_grad", "route_dw", "chunk_stats", "y_bf16"};
 
 static void prof_release(beam_moe* h)
 {
@@ -675,6 +676,7 @@ static beam_status_t create_impl(const beam_moe_config_t* cfg, const beam_moe_we
     BEAM_TRY(dalloc(h, &h->yperm, rows * D * sizeof(float)));
     BEAM_TRY(dalloc(h, &h->x_stage, Tm * D * es));
     BEAM_TRY(dalloc(h, &h->y_stage, Tm * D * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->y16_stage, Tm * D * sizeof(__nv_bfloat16)));
     BEAM_TRY(dalloc(h, &h->acc_stats, sizeof(DevStats)));
     BEAM_TRY(dalloc(h, &h->acc_counts, E * sizeof(int)));
     BEAM_TRY(dalloc(h, &h->pair_grad, rows * sizeof(float2)));
@@ -1721,8 +1723,49 @@ constexpr int kHostChunkTokens = 1366;   // about 3 chunks for a 4096-token batc
 constexpr int kHostMaxChunks = 4;
 constexpr int kHostPipelineMinTokens = 1024;   // smaller batches are copied and run whole
 
+// y [n] float32 -> bf16, round to nearest even (the host copy of a BEAM_HOST_Y_BF16 call);
+// 4 elements per thread, n a multiple of 4 (D is).
+__global__ void __launch_bounds__(256)
+y_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, long long n4)
+{
+    pdl_wait();
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        const float4 v = __ldcs(in + i);
+        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t*>(&a);
+        o.y = *reinterpret_cast<const uint32_t*>(&b);
+        __stcs(out + i, o);
+    }
+    pdl_launch_dependents();
+}
+
+// Host copy of n rows of y from the device staging buffers at row offset `off`: float32, or
+// rounded to bf16 on the device first (y16).
+static cudaError_t copy_y_out(beam_moe* h, void* y_host, long long off, int n, bool y16,
+                              cudaStream_t conv_st, cudaStream_t copy_st, cudaEvent_t after_conv)
+{
+    const size_t e0 = (size_t)off * h->D, ne = (size_t)n * h->D;
+    if (!y16)
+        return cudaMemcpyAsync(static_cast<float*>(y_host) + e0, h->y_stage + e0, ne * sizeof(float),
+                               cudaMemcpyDeviceToHost, copy_st);
+    const long long n4 = (long long)ne / 4;
+    cudaError_t e = launch(h, ST_Y_BF16, y_to_bf16_kernel, dim3((unsigned)std::min<long long>(
+                               ceil_div(n4, 256LL), 8LL * h->num_sms)), dim3(256), 0, conv_st,
+                           reinterpret_cast<const float4*>(h->y_stage + e0),
+                           reinterpret_cast<uint2*>(h->y16_stage + e0), n4);
+    if (e != cudaSuccess) return e;
+    if (after_conv) {
+        if ((e = cudaEventRecord(after_conv, conv_st)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(copy_st, after_conv, 0)) != cudaSuccess) return e;
+    }
+    return cudaMemcpyAsync(static_cast<__nv_bfloat16*>(y_host) + e0, h->y16_stage + e0,
+                           ne * sizeof(__nv_bfloat16), cudaMemcpyDeviceToHost, copy_st);
+}
+
 template <typename T>
-static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_, float* y_host,
+static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_, void* y_host,
                                             uint32_t flags, cudaStream_t st)
 {
     const int D = h->D, K = h->K, E = h->E;
@@ -1731,7 +1774,8 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
     const int tc = ceil_div(ceil_div(T_, C), align) * align;
     const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false
                                                                                         : h->tc_ok;
-    const uint32_t fflags = flags & ~(BEAM_HOST_PIPELINE | BEAM_NO_GRAPH);
+    const uint32_t fflags = flags & ~(BEAM_HOST_PIPELINE | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16);
+    const bool y16 = (flags & BEAM_HOST_Y_BF16) != 0;
     // the copy streams start after the work already on `st` (x_stage / y_stage are free)
     BEAM_CUDA(cudaEventRecord(h->ev_copied, st));
     BEAM_CUDA(cudaStreamWaitEvent(h->copy_in, h->ev_copied, 0));
@@ -1762,10 +1806,14 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
         BEAM_TRY(r);
         BEAM_CUDA(launch(h, ST_CHUNK_STATS, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
                          h->dstats, (const int*)h->counts, h->acc_stats, h->acc_counts, E, c == 0 ? 0 : 1));
-        BEAM_CUDA(cudaEventRecord(h->ev_out[c], st));
-        BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_out[c], 0));
-        BEAM_CUDA(cudaMemcpyAsync(y_host + xo, h->y_stage + xo, (size_t)n * D * sizeof(float),
-                                  cudaMemcpyDeviceToHost, h->copy_out));
+        if (y16) {
+            // rounded on `st`, after the chunk's forward; copied once the rounding is done
+            BEAM_CUDA(copy_y_out(h, y_host, off, n, true, st, h->copy_out, h->ev_out[c]));
+        } else {
+            BEAM_CUDA(cudaEventRecord(h->ev_out[c], st));
+            BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_out[c], 0));
+            BEAM_CUDA(copy_y_out(h, y_host, off, n, false, st, h->copy_out, nullptr));
+        }
         ++nchunks;
     }
     BEAM_CUDA(launch(h, ST_CHUNK_STATS, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
@@ -2173,7 +2221,7 @@ beam_status_t beam_moe_forward_routed(beam_moe_t* h, const void* x, int32_t T,
     return forward_entry(h, x, T, y, flags, &rin, stream);
 }
 
-beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T, float* y_host,
+beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T, void* y_host,
                                     uint32_t flags, void* stream)
 {
     g_err[0] = 0;
@@ -2184,7 +2232,8 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
     if ((flags & BEAM_HOST_PIPELINE) && T >= kHostPipelineMinTokens && h->Ew > 0) {
         if (flags & (BEAM_TRAIN | BEAM_FUSED_DECODE))
             return fail(BEAM_ERR_INVALID_ARG, "BEAM_HOST_PIPELINE excludes BEAM_TRAIN and BEAM_FUSED_DECODE");
-        if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_HOST_PIPELINE))
+        if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_HOST_PIPELINE |
+                      BEAM_HOST_Y_BF16))
             return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
         if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
             return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
@@ -2206,10 +2255,11 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
         BEAM_CUDA(cudaStreamSynchronize(st));
         return BEAM_OK;
     }
-    const size_t xb = (size_t)T * h->D * h->esz, yb = (size_t)T * h->D * sizeof(float);
+    const size_t xb = (size_t)T * h->D * h->esz;
     if (T > 0) BEAM_CUDA(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st));
-    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, h->y_stage, flags & ~BEAM_HOST_PIPELINE, stream));
-    if (T > 0) BEAM_CUDA(cudaMemcpyAsync(y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, st));
+    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, h->y_stage, flags & ~(BEAM_HOST_PIPELINE | BEAM_HOST_Y_BF16),
+                              stream));
+    if (T > 0) BEAM_CUDA(copy_y_out(h, y_host, 0, T, (flags & BEAM_HOST_Y_BF16) != 0, st, st, nullptr));
     BEAM_CUDA(cudaStreamSynchronize(st));
     return BEAM_OK;
 }

@@ -141,9 +141,13 @@ class BeamMoE:
                      path: str | None = None, stream=None, pipeline: bool = False) -> torch.Tensor:
         """Host-buffer variant: copies x in, runs the layer, copies y out, synchronises.
         pipeline=True (batches of >= 1024 tokens) runs chunks whose copies overlap the
-        forwards of the others (see BEAM_HOST_PIPELINE)."""
+        forwards of the others (see BEAM_HOST_PIPELINE).  A bfloat16 y_host receives y rounded
+        to bf16 on the device (BEAM_HOST_Y_BF16); otherwise y_host is float32."""
         T = x_host.shape[0]
-        flags = self.flags(mask_off, path) | (_lib.BEAM_HOST_PIPELINE if pipeline else 0)
+        if y_host.dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("y_host must be float32 or bfloat16")
+        flags = self.flags(mask_off, path) | (_lib.BEAM_HOST_PIPELINE if pipeline else 0) | \
+            (_lib.BEAM_HOST_Y_BF16 if y_host.dtype == torch.bfloat16 else 0)
         check(_lib.load().beam_moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host), flags,
                                                 ctypes.c_void_p(_stream_handle(stream))))
         return y_host

@@ -61,6 +61,9 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_HOST_PIPELINE 0x40u /* beam_moe_forward_host only: run a batch of >= 1024 tokens
                                    as chunks whose copies overlap the forwards of the others
                                    (see beam_moe_forward_host) */
+#define BEAM_HOST_Y_BF16  0x80u  /* beam_moe_forward_host only: y_host receives y rounded to
+                                   bf16 (round to nearest even) instead of float32, half the
+                                   device-to-host bytes (see beam_moe_forward_host) */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
@@ -141,9 +144,11 @@ beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, floa
 
 /*
  * beam_moe_forward with host buffers: copies x_host (T*D elements of the storage type) to a
- * handle-owned device buffer, runs the forward and copies y back to y_host (T*D float32),
- * then synchronises `stream`.  Pinned host memory gives full-bandwidth copies.
- * BEAM_HOST_PIPELINE (T >= 1024; flags may add BEAM_MASK_OFF, BEAM_PATH_* and BEAM_NO_GRAPH):
+ * handle-owned device buffer, runs the forward and copies y back to y_host (T*D float32, or
+ * with BEAM_HOST_Y_BF16 T*D bf16: the float32 y rounded to nearest even on the device before
+ * the copy), then synchronises `stream`.  Pinned host memory gives full-bandwidth copies.
+ * BEAM_HOST_PIPELINE (T >= 1024; flags may add BEAM_MASK_OFF, BEAM_PATH_*, BEAM_NO_GRAPH and
+ * BEAM_HOST_Y_BF16):
  * the batch runs as 2 to 4 chunks of whole segments (about 1366 tokens each); chunk c's x copy,
  * forward and y copy are ordered on two copy streams and `stream`, so the copies of one chunk
  * overlap the forwards of its neighbours.  Each chunk is a complete forward of its tokens (the
@@ -153,7 +158,7 @@ beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, floa
  * topk_id, gate, mask_logit and keep of every token and returns BEAM_ERR_UNSUPPORTED if asked
  * for offsets, perm or inv (the compaction ran per chunk).  Direct launches (no graph replay).
  */
-beam_status_t beam_moe_forward_host(beam_moe_t *h, const void *x_host, int32_t T, float *y_host,
+beam_status_t beam_moe_forward_host(beam_moe_t *h, const void *x_host, int32_t T, void *y_host,
                                     uint32_t flags, void *stream);
 
 /*
@@ -189,9 +194,9 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * under stages of their own (tc_shared_gateup, tc_shared_down, shared_swiglu_finish), so that
  * each stage's time covers the work of one problem.  A fused decode forward is one launch,
  * timed as the stage fused_decode; the per-chunk statistics of a pipelined host call as
- * chunk_stats.
+ * chunk_stats, and the rounding of y to bf16 of a BEAM_HOST_Y_BF16 host call as y_bf16.
  */
-#define BEAM_N_STAGES 19
+#define BEAM_N_STAGES 20
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);

@@ -605,3 +605,24 @@ def test_pipelined_host_call(T, seg):
     layer.forward(x.cuda())
     layer.routing(T)
     layer.close()
+
+
+@pytest.mark.parametrize("T,pipeline", [(1500, True), (1500, False), (3, False)],
+                         ids=["pipelined", "plain", "decode"])
+def test_host_bf16_output(T, pipeline):
+    """BEAM_HOST_Y_BF16: the host receives y rounded to bf16 on the device.  The bits are the
+    float32 y of the same call form, rounded to nearest even (torch's conversion), so the
+    output loses nothing beyond that rounding."""
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=T)
+    x = synth.make_tokens(spec, T, seed=23).pin_memory()
+    y32 = torch.full((T, spec.d_model), float("nan"), dtype=torch.float32).pin_memory()
+    y16 = torch.full((T, spec.d_model), float("nan"), dtype=torch.bfloat16).pin_memory()
+    layer.forward_host(x, y32, pipeline=pipeline)
+    layer.forward_host(x, y16, pipeline=pipeline)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    with pytest.raises(ValueError):
+        layer.forward_host(x, torch.empty((T, spec.d_model), dtype=torch.float16), pipeline=pipeline)
+    layer.close()
