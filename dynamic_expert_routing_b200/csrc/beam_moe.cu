@@ -1719,9 +1719,39 @@ static beam_status_t softtopk_check(int32_t T, int32_t E, float tau, const void*
 // routing arrays of chunk c are written at the chunk's offset (the handle's pointers are
 // shifted for the call), so the routing of every token is kept; the statistics are added up
 // over the chunks on the device.
-constexpr int kHostChunkTokens = 1366;   // about 3 chunks for a 4096-token batch
 constexpr int kHostMaxChunks = 4;
 constexpr int kHostPipelineMinTokens = 1024;   // smaller batches are copied and run whole
+// Chunk plan of a pipelined host call, in quarters of the batch: the first chunk's copy in
+// and the last chunk's copy out are the only copies nothing overlaps, so those two chunks are
+// small; the middle is one chunk, because every chunk reads all the kept experts' weights.
+// (Relative sizes; batches below 2048 tokens run as two halves.)
+constexpr int kHostPlan[] = {1, 2, 1};
+static_assert(sizeof(kHostPlan) / sizeof(kHostPlan[0]) <= kHostMaxChunks, "one event pair per chunk");
+
+// Token counts of the chunks of a pipelined host call (whole segments of `align` tokens,
+// none empty).
+static int host_chunk_plan(int T_, int align, int* sizes)
+{
+    const int units = ceil_div(T_, align);
+    int n = 0;
+    if (T_ < 2048 || units < 4) {
+        const int a = ceil_div(units, 2) * align;
+        sizes[n++] = std::min(a, T_);
+        if (T_ > a) sizes[n++] = T_ - a;
+        return n;
+    }
+    int q = 0;
+    for (int w : kHostPlan) q += w;
+    int done = 0, acc = 0;
+    for (size_t i = 0; i < sizeof(kHostPlan) / sizeof(kHostPlan[0]); ++i) {
+        acc += kHostPlan[i];
+        const int end = (i + 1 == sizeof(kHostPlan) / sizeof(kHostPlan[0]))
+                            ? T_ : std::min(T_, (int)((long long)units * acc / q) * align);
+        if (end > done) sizes[n++] = end - done;
+        done = std::max(done, end);
+    }
+    return n;
+}
 
 // y [n] float32 -> bf16, round to nearest even (the host copy of a BEAM_HOST_Y_BF16 call);
 // 4 elements per thread, n a multiple of 4 (D is).
@@ -1770,8 +1800,8 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
 {
     const int D = h->D, K = h->K, E = h->E;
     const int align = h->S > 1 ? h->S : 32;
-    const int C = std::min(kHostMaxChunks, std::max(2, ceil_div(T_, kHostChunkTokens)));
-    const int tc = ceil_div(ceil_div(T_, C), align) * align;
+    int sizes[kHostMaxChunks];
+    const int C = host_chunk_plan(T_, align, sizes);
     const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false
                                                                                         : h->tc_ok;
     const uint32_t fflags = flags & ~(BEAM_HOST_PIPELINE | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16);
@@ -1782,8 +1812,8 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
     BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_copied, 0));
     const RouteIn base = own_routing(h);
     int nchunks = 0;
-    for (int c = 0, off = 0; off < T_; ++c, off += tc) {
-        const int n = std::min(tc, T_ - off);
+    for (int c = 0, off = 0; c < C; off += sizes[c], ++c) {
+        const int n = sizes[c];
         const size_t xo = (size_t)off * D;
         BEAM_CUDA(cudaMemcpyAsync(static_cast<T*>(h->x_stage) + xo, x_host + xo, (size_t)n * D * sizeof(T),
                                   cudaMemcpyHostToDevice, h->copy_in));
