@@ -1045,8 +1045,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
     ap.add_argument("--sweep", action="store_true",
                     help="measure every workload (one JSON line each) instead of the headline")
-    ap.add_argument("--train", choices=sorted(TRAIN_POINTS), action="append",
-                    help="measure only these training points (one JSON line each)")
+    ap.add_argument("--train", choices=sorted(TRAIN_POINTS) + sorted(SOFTTOPK_POINTS), action="append",
+                    help="measure only these training points (routing gradient or SoftTopK; one JSON line each)")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="store a kernel's DRAM bytes per launch from an ncu CSV log (no GPU work)")
     ap.add_argument("--traffic-kernel", default=r"tc_grouped_gemm_kernel<(\(int\))?0,",
@@ -1069,8 +1069,12 @@ def main():
         torch.cuda.set_device(device)
         with torch.cuda.stream(torch.cuda.Stream(device)):
             for name in args.train:
-                print(json.dumps(train_point(torch, name, args.steps, args.warmup, device,
-                                             load_peaks())), flush=True)
+                if name in SOFTTOPK_POINTS:
+                    print(json.dumps(softtopk_point(torch, name, args.steps, args.warmup, device,
+                                                    load_peaks())), flush=True)
+                else:
+                    print(json.dumps(train_point(torch, name, args.steps, args.warmup, device,
+                                                 load_peaks())), flush=True)
     elif args.sweep:
         run_sweep(args)
     else:

@@ -9,12 +9,14 @@
 // through nu, is dr_j = h_j (dy_j - sum_i h_i dy_i / sum_i h_i) with h_i = y_i (1 - y_i) / tau.
 //
 // One warp per token row; lane l holds logits l, l + 32, ... (EPL = ceil(E/32) per lane).
-//   forward:  nu by safeguarded Newton in fp32 on f(nu) = sum_i sigmoid((r_i - nu)/tau) - K
-//             (strictly decreasing) inside the sign bracket [min r - 40 tau, max r + 40 tau],
-//             bisecting whenever a step leaves the bracket, until a Newton step is below
-//             2^-16 tau; every lane evaluates f with the same xor-butterfly sum, so the
-//             iteration is bitwise identical across the warp.  Then y, and the hard Top-K
-//             indicator (K rounds of a warp arg-max under (value desc, index asc)).
+//   forward:  the hard Top-K indicator first (K rounds of a warp arg-max under (value desc,
+//             index asc), and one more round for the (K+1)-th value); then nu by safeguarded
+//             Newton in fp32 on f(nu) = sum_i sigmoid((r_i - nu)/tau) - K (strictly
+//             decreasing), started halfway between the K-th and the (K+1)-th largest logit
+//             (the root when tau is small against their gap) inside the sign bracket
+//             [min r - 40 tau, max r + 40 tau], bisecting whenever a step leaves the bracket,
+//             until a Newton step is below 2^-16 tau; every lane evaluates f with the same
+//             xor-butterfly sum, so the iteration is bitwise identical across the warp.  Then y.
 //   backward: two butterfly sums per row (sum h, sum h dy), then dr.
 // Deterministic: fixed reduction order, no atomics.  HBM-bound: 4 B per logit read, 4 + 1 B
 // written (y, mask) forward; 8 B read and 4 B written per logit backward.
@@ -50,6 +52,28 @@ softtopk_fwd_kernel(const float* __restrict__ r, int T, int E, int K, float tau,
             hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
         }
         const float inv_tau = 1.0f / tau;
+        // hard Top-K indicator: K rounds, each taking the largest remaining value, the lowest
+        // expert among equal ones; a (K+1)-th round gives the next value, for the start of nu
+        uint32_t ord[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) ord[j] = (lane + 32 * j < E) ? topk_ord(v[j]) : 0u;
+        uint32_t sel = 0u;   // bit j: this lane's expert lane + 32 j is selected
+        uint32_t kth = 0u, next = 0u;
+        const int rounds = K < E ? K + 1 : K;
+        for (int k = 0; k < rounds; ++k) {
+            uint32_t best = 0u, bidx = 0xffffffffu;
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const uint32_t e = (uint32_t)(lane + 32 * j);
+                if (!((sel >> j) & 1u) && e < (uint32_t)E && ord[j] > best) { best = ord[j]; bidx = e; }
+                else if (!((sel >> j) & 1u) && e < (uint32_t)E && ord[j] == best && e < bidx) bidx = e;
+            }
+            const uint32_t wbest = __reduce_max_sync(0xffffffffu, best);
+            if (k == K) { next = wbest; break; }
+            const uint32_t widx = __reduce_min_sync(0xffffffffu, best == wbest ? bidx : 0xffffffffu);
+            if ((widx & 31u) == (uint32_t)lane) sel |= 1u << (widx >> 5);
+            kth = wbest;
+        }
         float nu;
         if (K >= E) {
             nu = -INFINITY;   // y = 1 everywhere: the constraint leaves no freedom
@@ -69,7 +93,7 @@ softtopk_fwd_kernel(const float* __restrict__ r, int T, int E, int K, float tau,
             const float eps = 1.52587890625e-5f * tau;   // 2^-16 tau
             const bool comp = 2 * K > E;
             const float target = comp ? (float)(E - K) : (float)K;
-            nu = 0.5f * (lo + hi);
+            nu = 0.5f * (topk_value(kth) + topk_value(next));
             for (int it = 0; it < 100; ++it) {
                 float s = 0.f, hs = 0.f;
 #pragma unroll
@@ -103,24 +127,6 @@ softtopk_fwd_kernel(const float* __restrict__ r, int T, int E, int K, float tau,
         }
         if (nu_out && lane == 0) nu_out[t] = nu;
         if (mask) {
-            // hard Top-K indicator: K rounds, each taking the largest remaining value, the
-            // lowest expert among equal ones
-            uint32_t ord[EPL];
-#pragma unroll
-            for (int j = 0; j < EPL; ++j) ord[j] = (lane + 32 * j < E) ? topk_ord(v[j]) : 0u;
-            uint32_t sel = 0u;   // bit j: this lane's expert lane + 32 j is selected
-            for (int k = 0; k < K; ++k) {
-                uint32_t best = 0u, bidx = 0xffffffffu;
-#pragma unroll
-                for (int j = 0; j < EPL; ++j) {
-                    const uint32_t e = (uint32_t)(lane + 32 * j);
-                    if (!((sel >> j) & 1u) && e < (uint32_t)E && ord[j] > best) { best = ord[j]; bidx = e; }
-                    else if (!((sel >> j) & 1u) && e < (uint32_t)E && ord[j] == best && e < bidx) bidx = e;
-                }
-                const uint32_t wbest = __reduce_max_sync(0xffffffffu, best);
-                const uint32_t widx = __reduce_min_sync(0xffffffffu, best == wbest ? bidx : 0xffffffffu);
-                if ((widx & 31u) == (uint32_t)lane) sel |= 1u << (widx >> 5);
-            }
 #pragma unroll
             for (int j = 0; j < EPL; ++j) {
                 const int e = lane + 32 * j;
