@@ -27,6 +27,7 @@ BEAM_FUSED_DECODE = 0x10
 BEAM_TRAIN = 0x20
 BEAM_HOST_PIPELINE = 0x40
 BEAM_HOST_Y_BF16 = 0x80
+BEAM_HOST_ASYNC = 0x100
 
 BEAM_N_STAGES = 20
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.beam_moe_forward.argtypes = [P, P, I, P, U, P]
     lib.beam_moe_forward_host.argtypes = [P, P, I, P, U, P]
     lib.beam_moe_stats.argtypes = [P, ctypes.POINTER(BeamStats), P]
+    lib.beam_moe_host_wait.argtypes = [P]
+    lib.beam_moe_host_wait.restype = ctypes.c_int
     lib.beam_moe_get_routing.argtypes = [P, P, P, P, P, P, P, P]
     lib.beam_moe_route_noalloc.argtypes = [P, P, I, P, P, P, P, P, U, P]
     lib.beam_moe_route_noalloc.restype = ctypes.c_int

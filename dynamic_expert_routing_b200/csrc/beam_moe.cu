@@ -184,6 +184,17 @@ struct beam_moe {
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
     cudaEvent_t ev_in[4] = {}, ev_out[4] = {};
     cudaEvent_t ev_copied = nullptr;
+    // asynchronous host calls (BEAM_HOST_ASYNC): a second staging set, allocated on the first
+    // such call; call k uses set k % 2.  ev_ax_free[b]: the forward that read x set b and
+    // wrote y set b is done; ev_ay_free[b]: the copy out of y set b is done; ev_async_last: the
+    // last asynchronous call's copy out.
+    void* x_stage2 = nullptr;
+    float* y_stage2 = nullptr;
+    __nv_bfloat16* y16_stage2 = nullptr;
+    cudaEvent_t ev_ax_ready[2] = {}, ev_ax_free[2] = {}, ev_ay_free[2] = {}, ev_async_last = nullptr;
+    bool async_used[2] = {false, false};
+    int async_next = 0;
+    bool async_pending = false;
     DevStats* acc_stats = nullptr;
     int* acc_counts = nullptr;
     bool last_pipelined = false;
@@ -298,6 +309,14 @@ static void free_all(beam_moe* h)
         h->ev_in[i] = h->ev_out[i] = nullptr;
     }
     if (h->ev_copied) cudaEventDestroy(h->ev_copied);
+    for (int b = 0; b < 2; ++b) {
+        if (h->ev_ax_ready[b]) cudaEventDestroy(h->ev_ax_ready[b]);
+        if (h->ev_ax_free[b]) cudaEventDestroy(h->ev_ax_free[b]);
+        if (h->ev_ay_free[b]) cudaEventDestroy(h->ev_ay_free[b]);
+        h->ev_ax_ready[b] = h->ev_ax_free[b] = h->ev_ay_free[b] = nullptr;
+    }
+    if (h->ev_async_last) cudaEventDestroy(h->ev_async_last);
+    h->ev_async_last = nullptr;
     if (h->copy_in) cudaStreamDestroy(h->copy_in);
     if (h->copy_out) cudaStreamDestroy(h->copy_out);
     h->ev_copied = nullptr;
@@ -1858,6 +1877,82 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
     return BEAM_OK;
 }
 
+// beam_moe_forward_host with BEAM_HOST_ASYNC: one whole-batch forward per call, on staging
+// set b = the call's parity, and no wait at the end.  The input copy (copy_in) waits for the
+// forward that last read set b; the forward (on `st`) waits for its input copy and for the copy
+// out that last read y set b; the output copy (copy_out) waits for the forward.  So call k+1's
+// input copy and call k-1's output copy run during call k's forward.
+static beam_status_t async_setup(beam_moe* h)
+{
+    if (h->x_stage2) return BEAM_OK;
+    const size_t n = (size_t)h->Tmax * h->D;
+    BEAM_TRY(dalloc(h, &h->x_stage2, n * h->esz));
+    BEAM_TRY(dalloc(h, &h->y_stage2, n * sizeof(float)));
+    BEAM_TRY(dalloc(h, &h->y16_stage2, n * sizeof(__nv_bfloat16)));
+    for (int b = 0; b < 2; ++b) {
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_ax_ready[b], cudaEventDisableTiming));
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_ax_free[b], cudaEventDisableTiming));
+        BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_ay_free[b], cudaEventDisableTiming));
+    }
+    BEAM_CUDA(cudaEventCreateWithFlags(&h->ev_async_last, cudaEventDisableTiming));
+    return BEAM_OK;
+}
+
+template <typename T>
+static beam_status_t forward_host_async(beam_moe* h, const T* x_host, int T_, void* y_host,
+                                        uint32_t flags, cudaStream_t st)
+{
+    BEAM_TRY(async_setup(h));
+    const int b = h->async_next;
+    T* xs = static_cast<T*>(b ? h->x_stage2 : h->x_stage);
+    float* ys = b ? h->y_stage2 : h->y_stage;
+    __nv_bfloat16* y16 = b ? h->y16_stage2 : h->y16_stage;
+    const size_t n = (size_t)T_ * h->D;
+    const bool y16_out = (flags & BEAM_HOST_Y_BF16) != 0;
+    const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false : h->tc_ok;
+    const uint32_t fflags = flags & ~(BEAM_HOST_ASYNC | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16);
+    if (!h->async_used[b]) {
+        // first use of this set: after everything already on `st`
+        BEAM_CUDA(cudaEventRecord(h->ev_ax_free[b], st));
+    }
+    BEAM_CUDA(cudaStreamWaitEvent(h->copy_in, h->ev_ax_free[b], 0));
+    BEAM_CUDA(cudaMemcpyAsync(xs, x_host, n * sizeof(T), cudaMemcpyHostToDevice, h->copy_in));
+    BEAM_CUDA(cudaEventRecord(h->ev_ax_ready[b], h->copy_in));
+    BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_ax_ready[b], 0));
+    if (h->async_used[b]) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_ay_free[b], 0));
+    BEAM_TRY(forward_impl<T>(h, xs, T_, ys, fflags, use_tc, st));
+    if (y16_out) {
+        const long long n4 = (long long)n / 4;
+        BEAM_CUDA(launch(h, ST_Y_BF16, y_to_bf16_kernel,
+                         dim3((unsigned)std::min<long long>(ceil_div(n4, 256LL), 8LL * h->num_sms)),
+                         dim3(256), 0, st, reinterpret_cast<const float4*>(ys), reinterpret_cast<uint2*>(y16), n4));
+    }
+    BEAM_CUDA(cudaEventRecord(h->ev_ax_free[b], st));
+    BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_ax_free[b], 0));
+    if (y16_out)
+        BEAM_CUDA(cudaMemcpyAsync(y_host, y16, n * sizeof(__nv_bfloat16), cudaMemcpyDeviceToHost, h->copy_out));
+    else
+        BEAM_CUDA(cudaMemcpyAsync(y_host, ys, n * sizeof(float), cudaMemcpyDeviceToHost, h->copy_out));
+    BEAM_CUDA(cudaEventRecord(h->ev_ay_free[b], h->copy_out));
+    BEAM_CUDA(cudaEventRecord(h->ev_async_last, h->copy_out));
+    h->async_used[b] = true;
+    h->async_next = b ^ 1;
+    h->async_pending = true;
+    return BEAM_OK;
+}
+
+// Before a synchronous host call reuses staging set 0: the asynchronous calls' copies are done.
+static cudaError_t join_async(beam_moe* h, cudaStream_t st)
+{
+    if (!h->async_pending) return cudaSuccess;
+    h->async_pending = false;
+    cudaError_t e = cudaStreamWaitEvent(st, h->ev_async_last, 0);
+    if (e != cudaSuccess) return e;
+    // and the next input copy of set 0 or 1 starts after this call's forward (copy_in waits
+    // on ev_ax_free, which that call records again)
+    return cudaSuccess;
+}
+
 extern "C" {
 
 beam_status_t beam_moe_route_noalloc(beam_moe_t* h, const void* x, int32_t T, int32_t* topk_id,
@@ -2263,6 +2358,32 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
     if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
     if (T > 0 && (!x_host || !y_host)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (flags & BEAM_HOST_ASYNC) {
+        if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16 |
+                      BEAM_HOST_ASYNC))
+            return fail(BEAM_ERR_INVALID_ARG, "BEAM_HOST_ASYNC takes only BEAM_MASK_OFF, BEAM_PATH_*, "
+                        "BEAM_NO_GRAPH and BEAM_HOST_Y_BF16 (flags 0x%x)", flags);
+        if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
+            return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
+        if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
+            return fail(BEAM_ERR_UNSUPPORTED, "the tensor-core expert path needs a bf16 layer with "
+                        "d_model a multiple of 256");
+        if (h->Ew == 0) return fail(BEAM_ERR_UNSUPPORTED, "a routing-only handle has no expert forward");
+        if (T == 0) return BEAM_OK;
+        if (h->prof && h->prof_forwards >= h->prof_max) h->prof = false;
+        if (h->prof) ++h->prof_forwards;
+        beam_status_t r = (h->cfg.dtype == BEAM_DTYPE_BF16)
+            ? forward_host_async<__nv_bfloat16>(h, static_cast<const __nv_bfloat16*>(x_host), T, y_host, flags, st)
+            : forward_host_async<float>(h, static_cast<const float*>(x_host), T, y_host, flags, st);
+        BEAM_TRY(r);
+        h->cur = own_routing(h);
+        h->last_T = T;
+        h->last_train = false;
+        h->last_pipelined = false;
+        BEAM_CUDA(cudaEventRecord(h->done, st));
+        return BEAM_OK;
+    }
+    BEAM_CUDA(join_async(h, st));
     if ((flags & BEAM_HOST_PIPELINE) && T >= kHostPipelineMinTokens && h->Ew > 0) {
         if (flags & (BEAM_TRAIN | BEAM_FUSED_DECODE))
             return fail(BEAM_ERR_INVALID_ARG, "BEAM_HOST_PIPELINE excludes BEAM_TRAIN and BEAM_FUSED_DECODE");
@@ -2295,6 +2416,16 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
                               stream));
     if (T > 0) BEAM_CUDA(copy_y_out(h, y_host, 0, T, (flags & BEAM_HOST_Y_BF16) != 0, st, st, nullptr));
     BEAM_CUDA(cudaStreamSynchronize(st));
+    return BEAM_OK;
+}
+
+beam_status_t beam_moe_host_wait(beam_moe_t* h)
+{
+    g_err[0] = 0;
+    if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
+    if (h->copy_in) BEAM_CUDA(cudaStreamSynchronize(h->copy_in));
+    if (h->copy_out) BEAM_CUDA(cudaStreamSynchronize(h->copy_out));
+    if (h->done) BEAM_CUDA(cudaEventSynchronize(h->done));
     return BEAM_OK;
 }
 
@@ -2525,6 +2656,9 @@ void beam_moe_destroy(beam_moe_t* h)
 {
     if (!h) return;
     if (h->done) cudaEventSynchronize(h->done);
+    // copies of asynchronous host calls may still read the staging buffers
+    if (h->copy_in) cudaStreamSynchronize(h->copy_in);
+    if (h->copy_out) cudaStreamSynchronize(h->copy_out);
     free_all(h);
     delete h;
 }

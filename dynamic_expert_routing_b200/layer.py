@@ -138,19 +138,30 @@ class BeamMoE:
         return out
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, mask_off: bool = False,
-                     path: str | None = None, stream=None, pipeline: bool = False) -> torch.Tensor:
+                     path: str | None = None, stream=None, pipeline: bool = False,
+                     asynchronous: bool = False) -> torch.Tensor:
         """Host-buffer variant: copies x in, runs the layer, copies y out, synchronises.
         pipeline=True (batches of >= 1024 tokens) runs chunks whose copies overlap the
-        forwards of the others (see BEAM_HOST_PIPELINE).  A bfloat16 y_host receives y rounded
-        to bf16 on the device (BEAM_HOST_Y_BF16); otherwise y_host is float32."""
+        forwards of the others (see BEAM_HOST_PIPELINE).  asynchronous=True returns once the
+        copies and the forward are queued (BEAM_HOST_ASYNC): consecutive calls overlap one
+        call's forward with the neighbours' copies; call host_wait() before reading y_host or
+        reusing x_host.  A bfloat16 y_host receives y rounded to bf16 on the device
+        (BEAM_HOST_Y_BF16); otherwise y_host is float32."""
         T = x_host.shape[0]
         if y_host.dtype not in (torch.float32, torch.bfloat16):
             raise ValueError("y_host must be float32 or bfloat16")
+        if pipeline and asynchronous:
+            raise ValueError("pipeline and asynchronous are exclusive")
         flags = self.flags(mask_off, path) | (_lib.BEAM_HOST_PIPELINE if pipeline else 0) | \
+            (_lib.BEAM_HOST_ASYNC if asynchronous else 0) | \
             (_lib.BEAM_HOST_Y_BF16 if y_host.dtype == torch.bfloat16 else 0)
         check(_lib.load().beam_moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host), flags,
                                                 ctypes.c_void_p(_stream_handle(stream))))
         return y_host
+
+    def host_wait(self) -> None:
+        """Wait for every queued host call's copies and the last forward (BEAM_HOST_ASYNC)."""
+        check(_lib.load().beam_moe_host_wait(self._h))
 
     # -------------------------------------------------------------- inspection
     def stats(self) -> dict:

@@ -64,6 +64,9 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_HOST_Y_BF16  0x80u  /* beam_moe_forward_host only: y_host receives y rounded to
                                    bf16 (round to nearest even) instead of float32, half the
                                    device-to-host bytes (see beam_moe_forward_host) */
+#define BEAM_HOST_ASYNC   0x100u /* beam_moe_forward_host only: return once the copies and the
+                                   forward are queued, without waiting (see beam_moe_forward_host
+                                   and beam_moe_host_wait) */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */
@@ -160,6 +163,22 @@ beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, floa
  */
 beam_status_t beam_moe_forward_host(beam_moe_t *h, const void *x_host, int32_t T, void *y_host,
                                     uint32_t flags, void *stream);
+
+/*
+ * BEAM_HOST_ASYNC (flags may add BEAM_MASK_OFF, BEAM_PATH_*, BEAM_NO_GRAPH, BEAM_HOST_Y_BF16):
+ * beam_moe_forward_host queues the input copy, the whole-batch forward and the output copy and
+ * returns without waiting.  Consecutive asynchronous calls on a handle alternate between two
+ * handle-owned staging sets (the second is allocated by the first such call), so call k+1's
+ * input copy and call k-1's output copy run while call k's forward does.  The forward runs on
+ * `stream`, the copies on the handle's two copy streams, ordered by events.  x_host must stay
+ * unchanged, and y_host unread, until beam_moe_host_wait returns.  beam_moe_stats and
+ * beam_moe_get_routing describe the last call (they wait for its forward).  A later
+ * synchronous host call waits for the asynchronous calls' copies first.
+ *
+ * beam_moe_host_wait: blocks until every queued host call's copies and the last forward are
+ * done.
+ */
+beam_status_t beam_moe_host_wait(beam_moe_t *h);
 
 /*
  * Statistics of the last forward; waits for it to finish.  counts_host, if not NULL,

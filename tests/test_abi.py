@@ -60,6 +60,7 @@ def test_null_handle_calls(lib):
     from dynamic_expert_routing_b200._lib import BeamStats, BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_forward(None, None, 1, None, 0, None) == BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_forward_host(None, None, 1, None, 0, None) == BEAM_ERR_INVALID_ARG
+    assert lib.beam_moe_host_wait(None) == BEAM_ERR_INVALID_ARG
     s = BeamStats()
     assert lib.beam_moe_stats(None, ctypes.byref(s), None) == BEAM_ERR_INVALID_ARG
     assert lib.beam_moe_get_routing(None, None, None, None, None, None, None, None) == BEAM_ERR_INVALID_ARG

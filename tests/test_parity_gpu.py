@@ -607,6 +607,39 @@ def test_pipelined_host_call(T, seg):
     layer.close()
 
 
+@pytest.mark.parametrize("T,y_dtype", [(700, torch.float32), (700, torch.bfloat16), (5, torch.float32)],
+                         ids=["f32", "bf16", "decode"])
+def test_host_async_calls(T, y_dtype):
+    """BEAM_HOST_ASYNC: consecutive calls on alternating staging sets, queued without waits and
+    finished by host_wait, give the bits of the same synchronous calls (four calls, so each
+    staging set is reused with a new input); statistics describe the last call; a synchronous
+    call afterwards waits for the queued copies and is itself unchanged."""
+    from dynamic_expert_routing_b200 import BeamMoE
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    layer = BeamMoE(to_dev(w), spec.top_k, max_tokens=T)
+    xs = [synth.make_tokens(spec, T, seed=40 + i).pin_memory() for i in range(3)]
+    order = [0, 1, 2, 0]
+    ref = []
+    for i in order:
+        y = torch.empty((T, spec.d_model), dtype=y_dtype).pin_memory()
+        layer.forward_host(xs[i], y)
+        ref.append(y)
+    st_ref = layer.stats()
+    ys = [torch.full((T, spec.d_model), float("nan"), dtype=y_dtype).pin_memory() for _ in order]
+    for i, y in zip(order, ys):
+        layer.forward_host(xs[i], y, asynchronous=True)
+    layer.host_wait()
+    for a, b in zip(ys, ref):
+        assert torch.equal(a, b)
+    st = layer.stats()
+    for k in ("avg_k", "n_kept", "n_active_experts", "tokens"):
+        assert st[k] == st_ref[k], k
+    y2 = torch.empty((T, spec.d_model), dtype=y_dtype).pin_memory()
+    layer.forward_host(xs[1], y2)
+    assert torch.equal(y2, ref[1])
+    layer.close()
+
 @pytest.mark.parametrize("T,pipeline", [(1500, True), (1500, False), (3, False)],
                          ids=["pipelined", "plain", "decode"])
 def test_host_bf16_output(T, pipeline):
