@@ -884,43 +884,5 @@ tc_grouped_gemm_kernel(const __grid_constant__ TcParams p)
     pdl_launch_dependents();
 }
 
-// Finishing step of a split-K gate/up GEMM: H[r][f] = silu(sum_s G[s][r][gate f]) *
-// (sum_s G[s][r][up f]), with the per-split partials G [splits][rows][2F] laid out like the
-// gate/up weight rows (128 gate columns, then the same 128 up columns).  Splits are added in
-// index order.  Routed rows: n_rows = offsets[E] read on the device; shared rows: T.
-__global__ void __launch_bounds__(256)
-swiglu_finish_kernel(const float* __restrict__ g, int splits, long long stride,
-                     const int* __restrict__ n_rows_ptr, int F, __half* __restrict__ h,
-                     const float* __restrict__ gsh, int splits_sh, long long stride_sh,
-                     int rows_sh, int Fsh, __half* __restrict__ hsh, int* __restrict__ err)
-{
-    pdl_wait();
-    bool bad = false;
-    const long long nr = (long long)(*n_rows_ptr) * F;
-    const long long ns = (long long)rows_sh * Fsh;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nr + ns;
-         i += (long long)gridDim.x * blockDim.x) {
-        const bool shared = i >= nr;
-        const long long j = shared ? i - nr : i;
-        const int FF = shared ? Fsh : F;
-        const long long r = j / FF;
-        const int f = (int)(j % FF);
-        const long long base = r * 2 * FF + (long long)(f >> 7) * 256 + (f & 127);
-        const float* src = shared ? gsh : g;
-        const int ns_ = shared ? splits_sh : splits;
-        const long long st = shared ? stride_sh : stride;
-        float gate = 0.f, up = 0.f;
-        for (int s = 0; s < ns_; ++s) {
-            gate += src[s * st + base];
-            up += src[s * st + base + 128];
-        }
-        const float hv = silu_f(gate) * up;
-        bad |= fp16_out_of_range(hv);
-        (shared ? hsh : h)[r * FF + f] = __float2half_rn(hv);
-    }
-    if (bad) atomicOr(err, ERR_FP16_RANGE);
-    pdl_launch_dependents();
-}
-
 }  // namespace tc
 }  // namespace beam
