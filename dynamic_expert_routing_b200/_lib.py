@@ -28,6 +28,7 @@ BEAM_TRAIN = 0x20
 BEAM_HOST_PIPELINE = 0x40
 BEAM_HOST_Y_BF16 = 0x80
 BEAM_HOST_ASYNC = 0x100
+BEAM_Y_BF16 = 0x200
 
 BEAM_N_STAGES = 20
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20

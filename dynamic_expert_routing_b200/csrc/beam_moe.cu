@@ -999,9 +999,9 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
     return BEAM_OK;
 }
 
-template <typename TR, typename TS>
-static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, const float* ghat,
-                                  int T_, float* y, cudaStream_t st)
+template <typename TR, typename TS, typename TO>
+static cudaError_t launch_combine_to(beam_moe* h, const YOut& r, const YOut& sh, const float* ghat,
+                                     int T_, TO* y, cudaStream_t st)
 {
     // few tokens: split each token's columns over several CTAs so the combine spans the SMs;
     // otherwise one CTA per token whose threads take the row's float4 columns in equal passes
@@ -1010,7 +1010,7 @@ static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, co
     if (T_ < h->num_sms && (r.splits > 1 || sh.splits > 1) && h->K <= 32 &&
         r.splits <= kCombineMaxSplits && sh.splits <= kCombineMaxSplits) {
         // a small batch with split-K slices: slots and slices read in parallel
-        return launch(h, ST_COMBINE, combine_small_kernel<TR, TS>,
+        return launch(h, ST_COMBINE, combine_small_kernel<TR, TS, TO>,
                       dim3(T_, ceil_div(d4, kCombineSmallCols)),
                       dim3(kCombineSmallCols, h->K + 1), 0, st,
                       (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
@@ -1020,9 +1020,19 @@ static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, co
     const int passes = ceil_div(d4, 256);
     const int nthr = split_cols ? 256 : std::min(256, ceil_div(ceil_div(d4, passes), 32) * 32);
     const dim3 cgrid(T_, split_cols ? ceil_div(d4, 256) : 1);
-    return launch(h, ST_COMBINE, combine_kernel<TR, TS>, cgrid, dim3(nthr), 0, st,
+    return launch(h, ST_COMBINE, combine_kernel<TR, TS, TO>, cgrid, dim3(nthr), 0, st,
                   (const TR*)r.base, r.splits, r.stride, (const TS*)sh.base, sh.splits, sh.stride,
                   (const int*)h->inv, ghat, T_, h->K, h->D, y);
+}
+
+// y: float32 [T][D], or bf16 [T][D] (the same pointer, BEAM_Y_BF16) when y16 is set
+template <typename TR, typename TS>
+static cudaError_t launch_combine(beam_moe* h, const YOut& r, const YOut& sh, const float* ghat,
+                                  int T_, float* y, cudaStream_t st, bool y16 = false)
+{
+    if (y16)
+        return launch_combine_to<TR, TS>(h, r, sh, ghat, T_, reinterpret_cast<__nv_bfloat16*>(y), st);
+    return launch_combine_to<TR, TS>(h, r, sh, ghat, T_, y, st);
 }
 
 // ep_dispatch: stop after the compaction (expert parallelism, beam_moe_ep_dispatch): the kept
@@ -1179,10 +1189,11 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
     if (fork) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_join, 0));
     if (!h->Fsh) ysh_out.f16 = yr.f16;  // no shared term: only its (unused) type must match
     cudaError_t ce;
-    if (yr.f16 && ysh_out.f16) ce = launch_combine<__half, __half>(h, yr, ysh_out, rt.ghat, T_, y, st);
-    else if (yr.f16) ce = launch_combine<__half, float>(h, yr, ysh_out, rt.ghat, T_, y, st);
-    else if (ysh_out.f16) ce = launch_combine<float, __half>(h, yr, ysh_out, rt.ghat, T_, y, st);
-    else ce = launch_combine<float, float>(h, yr, ysh_out, rt.ghat, T_, y, st);
+    const bool y16 = (flags & BEAM_Y_BF16) != 0;
+    if (yr.f16 && ysh_out.f16) ce = launch_combine<__half, __half>(h, yr, ysh_out, rt.ghat, T_, y, st, y16);
+    else if (yr.f16) ce = launch_combine<__half, float>(h, yr, ysh_out, rt.ghat, T_, y, st, y16);
+    else if (ysh_out.f16) ce = launch_combine<float, __half>(h, yr, ysh_out, rt.ghat, T_, y, st, y16);
+    else ce = launch_combine<float, float>(h, yr, ysh_out, rt.ghat, T_, y, st, y16);
     BEAM_CUDA(ce);
     return BEAM_OK;
 }
@@ -2230,8 +2241,12 @@ static beam_status_t forward_entry(beam_moe* h, const void* x, int32_t T, float*
     if ((flags & BEAM_PATH_STREAM) && (flags & BEAM_PATH_TENSOR))
         return fail(BEAM_ERR_INVALID_ARG, "BEAM_PATH_STREAM and BEAM_PATH_TENSOR are exclusive");
     if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH |
-                  BEAM_FUSED_DECODE | BEAM_TRAIN))
+                  BEAM_FUSED_DECODE | BEAM_TRAIN | BEAM_Y_BF16))
         return fail(BEAM_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & BEAM_Y_BF16) && (flags & BEAM_FUSED_DECODE))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_Y_BF16 excludes BEAM_FUSED_DECODE");
+    if (T > 0 && (flags & BEAM_Y_BF16) && (reinterpret_cast<uintptr_t>(y) & 7))
+        return fail(BEAM_ERR_INVALID_ARG, "a bf16 y must be 8-byte aligned");
     if ((flags & BEAM_TRAIN) && (flags & (BEAM_MASK_OFF | BEAM_FUSED_DECODE)))
         return fail(BEAM_ERR_INVALID_ARG, "BEAM_TRAIN excludes BEAM_MASK_OFF and BEAM_FUSED_DECODE");
     if ((flags & BEAM_PATH_TENSOR) && !h->tc_ok)
@@ -2357,6 +2372,8 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
     if (!h) return fail(BEAM_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0 || T > h->Tmax) return fail(BEAM_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, h->Tmax);
     if (T > 0 && (!x_host || !y_host)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
+    if (flags & BEAM_Y_BF16)
+        return fail(BEAM_ERR_INVALID_ARG, "host calls take BEAM_HOST_Y_BF16 for a bf16 y, not BEAM_Y_BF16");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (flags & BEAM_HOST_ASYNC) {
         if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16 |

@@ -513,12 +513,27 @@ __device__ __forceinline__ float4 load4(const __half* p, size_t i) {
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
-template <typename TY, typename TS>
+// y stores of 4 columns (streaming): float32, or rounded to bf16 (nearest even) for a
+// BEAM_Y_BF16 forward.
+__device__ __forceinline__ void store_y4(float* y, size_t i, float4 v)
+{
+    __stcs(reinterpret_cast<float4*>(y) + i, v);
+}
+__device__ __forceinline__ void store_y4(__nv_bfloat16* y, size_t i, float4 v)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&a);
+    o.y = *reinterpret_cast<const uint32_t*>(&b);
+    __stcs(reinterpret_cast<uint2*>(y) + i, o);
+}
+
+template <typename TY, typename TS, typename TO = float>
 __global__ void __launch_bounds__(256)
 combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
                const TS* __restrict__ ysh, int splits_sh, long long stride_sh,
                const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K, int D,
-               float* __restrict__ y)
+               TO* __restrict__ y)
 {
     __shared__ int s_inv[32];
     __shared__ float s_g[32];
@@ -557,7 +572,7 @@ combine_kernel(const TY* __restrict__ yperm, int splits, long long stride,
                 acc.x += w.x; acc.y += w.y; acc.z += w.z; acc.w += w.w;
             }
         }
-        __stcs(reinterpret_cast<float4*>(y) + (size_t)t * D4 + c, acc);
+        store_y4(y, (size_t)t * D4 + c, acc);
     }
     pdl_launch_dependents();
 }
@@ -586,12 +601,12 @@ __device__ __forceinline__ float4 sum_slices(const TY* base, int splits, long lo
     return a;
 }
 
-template <typename TY, typename TS>
+template <typename TY, typename TS, typename TO = float>
 __global__ void __launch_bounds__(kCombineSmallCols * 33)
 combine_small_kernel(const TY* __restrict__ yperm, int splits, long long stride,
                      const TS* __restrict__ ysh, int splits_sh, long long stride_sh,
                      const int* __restrict__ inv, const float* __restrict__ ghat, int T, int K,
-                     int D, float* __restrict__ y)
+                     int D, TO* __restrict__ y)
 {
     __shared__ float4 red[33][kCombineSmallCols];
     __shared__ int s_inv[32];
@@ -632,7 +647,7 @@ combine_small_kernel(const TY* __restrict__ yperm, int splits, long long stride,
             const float4 v = red[K][cx];
             acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
-        __stcs(reinterpret_cast<float4*>(y) + (size_t)t * D4 + c, acc);
+        store_y4(y, (size_t)t * D4 + c, acc);
     }
     pdl_launch_dependents();
 }

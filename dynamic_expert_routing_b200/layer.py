@@ -28,6 +28,15 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _y_flag(out: torch.Tensor, T: int, D: int) -> int:
+    """BEAM_Y_BF16 for a bfloat16 output tensor; the output must be a contiguous CUDA tensor
+    of float32 or bfloat16 with room for [T][D]."""
+    if not (out.is_cuda and out.is_contiguous() and out.numel() >= T * D
+            and out.dtype in (torch.float32, torch.bfloat16)):
+        raise ValueError("out must be a contiguous CUDA float32 or bfloat16 tensor of at least T*D values")
+    return _lib.BEAM_Y_BF16 if out.dtype == torch.bfloat16 else 0
+
+
 class BeamMoE:
     """A BEAM masked MoE layer held by the CUDA library.
 
@@ -77,14 +86,16 @@ class BeamMoE:
         graph=False launches the kernels directly instead of replaying a captured graph;
         fused=True runs a bf16 batch of <= 32 tokens as one cooperative launch (opt-in);
         train=True evaluates every Top-K slot's expert (the mask only scales the gates) so
-        that backward_router can follow."""
+        that backward_router can follow.  A bfloat16 `out` receives y rounded to bf16
+        (BEAM_Y_BF16)."""
         if not (x.is_cuda and x.is_contiguous() and x.dtype == self.dtype):
             raise ValueError("x must be a contiguous CUDA tensor of the layer's storage dtype")
         T = x.shape[0]
         if out is None:
             out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
         check(_lib.load().beam_moe_forward(self._h, _ptr(x), T, _ptr(out),
-                                           self.flags(mask_off, path, graph, fused, train),
+                                           self.flags(mask_off, path, graph, fused, train) |
+                                           _y_flag(out, T, self.d_model),
                                            ctypes.c_void_p(_stream_handle(stream))))
         return out
 
@@ -133,7 +144,8 @@ class BeamMoE:
             out = torch.empty((T, self.d_model), dtype=torch.float32, device=x.device)
         r = _routing_struct(routing)
         check(_lib.load().beam_moe_forward_routed(self._h, _ptr(x), T, ctypes.byref(r), _ptr(out),
-                                                  self.flags(False, path, graph),
+                                                  self.flags(False, path, graph) |
+                                                  _y_flag(out, T, self.d_model),
                                                   ctypes.c_void_p(_stream_handle(stream))))
         return out
 

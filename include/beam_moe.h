@@ -67,6 +67,10 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
 #define BEAM_HOST_ASYNC   0x100u /* beam_moe_forward_host only: return once the copies and the
                                    forward are queued, without waiting (see beam_moe_forward_host
                                    and beam_moe_host_wait) */
+#define BEAM_Y_BF16       0x200u /* beam_moe_forward / _forward_routed: y is written as bf16
+                                   (the float32 sum rounded to nearest even), T*D values at an
+                                   8-byte aligned y; excludes BEAM_FUSED_DECODE (host calls use
+                                   BEAM_HOST_Y_BF16) */
 
 typedef struct {
     int32_t d_model;      /* D. bf16: multiple of 64; fp32: multiple of 4. <= 8192 (4096 fp32) */

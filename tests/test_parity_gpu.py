@@ -640,6 +640,43 @@ def test_host_async_calls(T, y_dtype):
     assert torch.equal(y2, ref[1])
     layer.close()
 
+@pytest.mark.parametrize("T", [1, 40, 700], ids=["decode", "small", "prefill"])
+def test_bf16_y_is_the_rounded_float32_y(T):
+    """BEAM_Y_BF16 (a bfloat16 `out`): the combine writes the float32 sum rounded to nearest
+    even, so y equals the float32 forward's y converted by torch, bit for bit; the same through
+    forward_routed; and the flag is refused with the fused decode launch and on host calls."""
+    from dynamic_expert_routing_b200 import BeamMoE, BeamGenerator, BeamError, _lib
+    spec = _small(n_shared=1, d_ff_shared=128)
+    w = synth.make_layer(spec, keep_rate=0.5)
+    wd = to_dev(w)
+    layer = BeamMoE(wd, spec.top_k, max_tokens=T)
+    x = synth.make_tokens(spec, T, seed=71).cuda()
+    y32 = layer.forward(x)
+    y16 = layer.forward(x, out=torch.empty((T, spec.d_model), dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    gen = BeamGenerator(wd["w_router"][None].contiguous(), wd["w_mask"][None].contiguous(),
+                        spec.top_k, max_tokens=T)
+    one = gen.layer(gen.route(x), 0)
+    r32 = layer.forward_routed(x, one)
+    r16 = layer.forward_routed(x, one, out=torch.empty((T, spec.d_model), dtype=torch.bfloat16,
+                                                        device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(r16, r32.to(torch.bfloat16))
+    lib = _lib.load()
+    import ctypes
+    yb = torch.empty((T, spec.d_model), dtype=torch.bfloat16, device="cuda")
+    assert lib.beam_moe_forward(layer._h, ctypes.c_void_p(x.data_ptr()), T, ctypes.c_void_p(yb.data_ptr()),
+                                _lib.BEAM_Y_BF16 | _lib.BEAM_FUSED_DECODE, None) == _lib.BEAM_ERR_INVALID_ARG
+    xh = x.cpu().pin_memory()
+    with pytest.raises(BeamError):
+        _lib.check(lib.beam_moe_forward_host(layer._h, ctypes.c_void_p(xh.data_ptr()), T,
+                                             ctypes.c_void_p(yb.cpu().pin_memory().data_ptr()),
+                                             _lib.BEAM_Y_BF16, None))
+    torch.cuda.synchronize()
+    gen.close()
+    layer.close()
+
 def test_host_call_forms_interleaved():
     """Host calls of every form on one handle, interleaved: asynchronous calls of different
     batch sizes and mask settings, a pipelined synchronous call between them, and asynchronous
