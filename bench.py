@@ -235,8 +235,6 @@ def layer_work(spec, T, st, tc_path=True, joint=False):
     w["combine"] = dict(bytes=nk * D * ys + Tsh * D * ys + T * D * 4 + T * K * 8,
                         flops=2 * nk * D)
     w["scatter_gather"] = dict(bytes=2 * nk * D * es + T * K * 12, flops=0)
-    w["swiglu_finish"] = dict(bytes=(nk * F + (Tsh * Fsh if joint else 0)) * hs, flops=0)
-    w["shared_swiglu_finish"] = dict(bytes=Tsh * Fsh * hs, flops=0)
     total_bytes = (na * 3 * F * D + 3 * Fsh * D + 2 * E * D) * es + T * D * es + T * D * 4
     total_flops = 2 * (nk * 3 * F * D + T * 3 * Fsh * D + Tr * D * 2 * E)
     return w, dict(bytes=total_bytes, flops=total_flops)

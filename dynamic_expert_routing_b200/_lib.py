@@ -30,7 +30,7 @@ BEAM_HOST_Y_BF16 = 0x80
 BEAM_HOST_ASYNC = 0x100
 BEAM_Y_BF16 = 0x200
 
-BEAM_N_STAGES = 20
+BEAM_N_STAGES = 17
 BEAM_ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 STATUS_NAMES = {0: "BEAM_OK", 1: "BEAM_ERR_INVALID_ARG", 2: "BEAM_ERR_OOM", 3: "BEAM_ERR_CUDA",

@@ -178,7 +178,7 @@ struct beam_moe {
     // host-call staging
     void* x_stage = nullptr;
     float* y_stage = nullptr;
-    __nv_bfloat16* y16_stage = nullptr;   // y rounded to bf16 for a BEAM_HOST_Y_BF16 host call
+    __nv_bfloat16* y16_stage = nullptr;   // bf16 y of a BEAM_HOST_Y_BF16 host call
     // pipelined host calls (BEAM_HOST_PIPELINE): copy streams, per-chunk events, statistics
     // accumulated over the chunks
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
@@ -264,15 +264,15 @@ struct beam_moe {
 enum Stage {
     ST_ROUTER_LOGITS = 0, ST_ROUTE_SELECT, ST_COMPACT_BITS, ST_COMPACT_SCAN, ST_SCATTER_GATHER,
     ST_STREAM_GATEUP, ST_STREAM_DOWN, ST_COMBINE, ST_TC_GATEUP, ST_TC_DOWN, ST_TC_ROUTER,
-    ST_SWIGLU_FINISH, ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_SH_SWIGLU_FINISH, ST_FUSED_DECODE,
-    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_CHUNK_STATS, ST_Y_BF16, ST_COUNT
+    ST_TC_SH_GATEUP, ST_TC_SH_DOWN, ST_FUSED_DECODE,
+    ST_ROUTE_GRAD, ST_ROUTE_DW, ST_CHUNK_STATS, ST_COUNT
 };
 static_assert(ST_COUNT == BEAM_N_STAGES, "stage table out of sync with the header");
 static const char* kStageNames[ST_COUNT] = {
     "router_logits", "route_select", "compact_bits", "compact_scan", "scatter_gather",
     "stream_gateup", "stream_down", "combine", "tc_gateup", "tc_down", "tc_router",
-    "swiglu_finish", "tc_shared_gateup", "tc_shared_down", "shared_swiglu_finish",
-    "fused_decode", "route_grad", "route_dw", "chunk_stats", "y_bf16"};
+    "tc_shared_gateup", "tc_shared_down",
+    "fused_decode", "route_grad", "route_dw", "chunk_stats"};
 
 static void prof_release(beam_moe* h)
 {
@@ -914,7 +914,6 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
     const bool sh_only = which == PROB_SHARED;
     const int st_gu = sh_only ? ST_TC_SH_GATEUP : ST_TC_GATEUP;
     const int st_dn = sh_only ? ST_TC_SH_DOWN : ST_TC_DOWN;
-    const int st_fin = sh_only ? ST_SH_SWIGLU_FINISH : ST_SWIGLU_FINISH;
     const int* ngroups = routed ? h->n_groups : h->zero_int;
 
     // GEMM1: gate/up, SwiGLU in the epilogue, or f32 partials + the finishing kernel
@@ -947,7 +946,6 @@ static beam_status_t tc_problem(beam_moe* h, const T* x, int T_, int which, cuda
         p.fold_f_shared = Fsh;
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_STORE_F32, 1, tc::MODE_PLAIN>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
-        (void)st_fin;
     } else if (swap1) {
         BEAM_CUDA(launch(h, st_gu, tc::tc_grouped_gemm_kernel<tc::EPI_SWIGLU, 1, tc::MODE_SWAP>,
                          dim3(h->num_sms), dim3(tc::kThreads), (size_t)tc::SMEM_BYTES, st, p));
@@ -1787,45 +1785,24 @@ static int host_chunk_plan(int T_, int align, int* sizes)
     return n;
 }
 
-// y [n] float32 -> bf16, round to nearest even (the host copy of a BEAM_HOST_Y_BF16 call);
-// 4 elements per thread, n a multiple of 4 (D is).
-__global__ void __launch_bounds__(256)
-y_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out, long long n4)
-{
-    pdl_wait();
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
-         i += (long long)gridDim.x * blockDim.x) {
-        const float4 v = __ldcs(in + i);
-        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
-        uint2 o;
-        o.x = *reinterpret_cast<const uint32_t*>(&a);
-        o.y = *reinterpret_cast<const uint32_t*>(&b);
-        __stcs(out + i, o);
-    }
-    pdl_launch_dependents();
-}
-
-// Host copy of n rows of y from the device staging buffers at row offset `off`: float32, or
-// rounded to bf16 on the device first (y16).
+// Host copy of n rows of y at row offset `off` from the device staging buffer: float32, or
+// (y16) the bf16 rows the combine wrote under BEAM_Y_BF16.
 static cudaError_t copy_y_out(beam_moe* h, void* y_host, long long off, int n, bool y16,
-                              cudaStream_t conv_st, cudaStream_t copy_st, cudaEvent_t after_conv)
+                              cudaStream_t copy_st)
 {
     const size_t e0 = (size_t)off * h->D, ne = (size_t)n * h->D;
     if (!y16)
         return cudaMemcpyAsync(static_cast<float*>(y_host) + e0, h->y_stage + e0, ne * sizeof(float),
                                cudaMemcpyDeviceToHost, copy_st);
-    const long long n4 = (long long)ne / 4;
-    cudaError_t e = launch(h, ST_Y_BF16, y_to_bf16_kernel, dim3((unsigned)std::min<long long>(
-                               ceil_div(n4, 256LL), 8LL * h->num_sms)), dim3(256), 0, conv_st,
-                           reinterpret_cast<const float4*>(h->y_stage + e0),
-                           reinterpret_cast<uint2*>(h->y16_stage + e0), n4);
-    if (e != cudaSuccess) return e;
-    if (after_conv) {
-        if ((e = cudaEventRecord(after_conv, conv_st)) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(copy_st, after_conv, 0)) != cudaSuccess) return e;
-    }
     return cudaMemcpyAsync(static_cast<__nv_bfloat16*>(y_host) + e0, h->y16_stage + e0,
                            ne * sizeof(__nv_bfloat16), cudaMemcpyDeviceToHost, copy_st);
+}
+
+// The device y of a host call: the float32 staging rows, or the bf16 ones (written through the
+// same float* argument with BEAM_Y_BF16 set).
+static float* host_y_dev(beam_moe* h, float* y32, __nv_bfloat16* y16, bool bf16)
+{
+    return bf16 ? reinterpret_cast<float*>(y16) : y32;
 }
 
 template <typename T>
@@ -1838,8 +1815,9 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
     const int C = host_chunk_plan(T_, align, sizes);
     const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false
                                                                                         : h->tc_ok;
-    const uint32_t fflags = flags & ~(BEAM_HOST_PIPELINE | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16);
     const bool y16 = (flags & BEAM_HOST_Y_BF16) != 0;
+    const uint32_t fflags = (flags & ~(BEAM_HOST_PIPELINE | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16)) |
+                            (y16 ? BEAM_Y_BF16 : 0u);
     // the copy streams start after the work already on `st` (x_stage / y_stage are free)
     BEAM_CUDA(cudaEventRecord(h->ev_copied, st));
     BEAM_CUDA(cudaStreamWaitEvent(h->copy_in, h->ev_copied, 0));
@@ -1861,7 +1839,8 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
         h->ghat = const_cast<float*>(base.ghat) + (size_t)off * K;
         h->nkeep_tok = const_cast<int*>(base.nkeep) + off;
         h->lreg_tok = const_cast<float*>(base.lreg) + off;
-        beam_status_t r = forward_impl<T>(h, static_cast<const T*>(h->x_stage) + xo, n, h->y_stage + xo,
+        beam_status_t r = forward_impl<T>(h, static_cast<const T*>(h->x_stage) + xo, n,
+                                          host_y_dev(h, h->y_stage + xo, h->y16_stage + xo, y16),
                                           fflags, use_tc, st);
         h->topk_id = const_cast<int*>(base.topk_id); h->gate = const_cast<float*>(base.gate);
         h->mlogit = const_cast<float*>(base.mlogit); h->keep = const_cast<uint8_t*>(base.keep);
@@ -1870,14 +1849,9 @@ static beam_status_t forward_host_pipelined(beam_moe* h, const T* x_host, int T_
         BEAM_TRY(r);
         BEAM_CUDA(launch(h, ST_CHUNK_STATS, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
                          h->dstats, (const int*)h->counts, h->acc_stats, h->acc_counts, E, c == 0 ? 0 : 1));
-        if (y16) {
-            // rounded on `st`, after the chunk's forward; copied once the rounding is done
-            BEAM_CUDA(copy_y_out(h, y_host, off, n, true, st, h->copy_out, h->ev_out[c]));
-        } else {
-            BEAM_CUDA(cudaEventRecord(h->ev_out[c], st));
-            BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_out[c], 0));
-            BEAM_CUDA(copy_y_out(h, y_host, off, n, false, st, h->copy_out, nullptr));
-        }
+        BEAM_CUDA(cudaEventRecord(h->ev_out[c], st));
+        BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_out[c], 0));
+        BEAM_CUDA(copy_y_out(h, y_host, off, n, y16, h->copy_out));
         ++nchunks;
     }
     BEAM_CUDA(launch(h, ST_CHUNK_STATS, stats_accumulate_kernel, dim3(1), dim3(256), 0, st,
@@ -1921,7 +1895,8 @@ static beam_status_t forward_host_async(beam_moe* h, const T* x_host, int T_, vo
     const size_t n = (size_t)T_ * h->D;
     const bool y16_out = (flags & BEAM_HOST_Y_BF16) != 0;
     const bool use_tc = (flags & BEAM_PATH_TENSOR) ? true : (flags & BEAM_PATH_STREAM) ? false : h->tc_ok;
-    const uint32_t fflags = flags & ~(BEAM_HOST_ASYNC | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16);
+    const uint32_t fflags = (flags & ~(BEAM_HOST_ASYNC | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16)) |
+                            (y16_out ? BEAM_Y_BF16 : 0u);
     if (!h->async_used[b]) {
         // first use of this set: after everything already on `st`
         BEAM_CUDA(cudaEventRecord(h->ev_ax_free[b], st));
@@ -1931,13 +1906,7 @@ static beam_status_t forward_host_async(beam_moe* h, const T* x_host, int T_, vo
     BEAM_CUDA(cudaEventRecord(h->ev_ax_ready[b], h->copy_in));
     BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_ax_ready[b], 0));
     if (h->async_used[b]) BEAM_CUDA(cudaStreamWaitEvent(st, h->ev_ay_free[b], 0));
-    BEAM_TRY(forward_impl<T>(h, xs, T_, ys, fflags, use_tc, st));
-    if (y16_out) {
-        const long long n4 = (long long)n / 4;
-        BEAM_CUDA(launch(h, ST_Y_BF16, y_to_bf16_kernel,
-                         dim3((unsigned)std::min<long long>(ceil_div(n4, 256LL), 8LL * h->num_sms)),
-                         dim3(256), 0, st, reinterpret_cast<const float4*>(ys), reinterpret_cast<uint2*>(y16), n4));
-    }
+    BEAM_TRY(forward_impl<T>(h, xs, T_, host_y_dev(h, ys, y16, y16_out), fflags, use_tc, st));
     BEAM_CUDA(cudaEventRecord(h->ev_ax_free[b], st));
     BEAM_CUDA(cudaStreamWaitEvent(h->copy_out, h->ev_ax_free[b], 0));
     if (y16_out)
@@ -2374,6 +2343,8 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
     if (T > 0 && (!x_host || !y_host)) return fail(BEAM_ERR_INVALID_ARG, "x or y is NULL");
     if (flags & BEAM_Y_BF16)
         return fail(BEAM_ERR_INVALID_ARG, "host calls take BEAM_HOST_Y_BF16 for a bf16 y, not BEAM_Y_BF16");
+    if ((flags & BEAM_HOST_Y_BF16) && (flags & BEAM_FUSED_DECODE))
+        return fail(BEAM_ERR_INVALID_ARG, "BEAM_HOST_Y_BF16 excludes BEAM_FUSED_DECODE");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (flags & BEAM_HOST_ASYNC) {
         if (flags & ~(BEAM_MASK_OFF | BEAM_PATH_STREAM | BEAM_PATH_TENSOR | BEAM_NO_GRAPH | BEAM_HOST_Y_BF16 |
@@ -2428,10 +2399,12 @@ beam_status_t beam_moe_forward_host(beam_moe_t* h, const void* x_host, int32_t T
         return BEAM_OK;
     }
     const size_t xb = (size_t)T * h->D * h->esz;
+    const bool y16 = (flags & BEAM_HOST_Y_BF16) != 0;
     if (T > 0) BEAM_CUDA(cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, st));
-    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, h->y_stage, flags & ~(BEAM_HOST_PIPELINE | BEAM_HOST_Y_BF16),
+    BEAM_TRY(beam_moe_forward(h, h->x_stage, T, host_y_dev(h, h->y_stage, h->y16_stage, y16),
+                              (flags & ~(BEAM_HOST_PIPELINE | BEAM_HOST_Y_BF16)) | (y16 ? BEAM_Y_BF16 : 0u),
                               stream));
-    if (T > 0) BEAM_CUDA(copy_y_out(h, y_host, 0, T, (flags & BEAM_HOST_Y_BF16) != 0, st, st, nullptr));
+    if (T > 0) BEAM_CUDA(copy_y_out(h, y_host, 0, T, y16, st));
     BEAM_CUDA(cudaStreamSynchronize(st));
     return BEAM_OK;
 }

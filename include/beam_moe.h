@@ -63,7 +63,8 @@ enum { BEAM_DTYPE_F32 = 0, BEAM_DTYPE_BF16 = 1 };
                                    (see beam_moe_forward_host) */
 #define BEAM_HOST_Y_BF16  0x80u  /* beam_moe_forward_host only: y_host receives y rounded to
                                    bf16 (round to nearest even) instead of float32, half the
-                                   device-to-host bytes (see beam_moe_forward_host) */
+                                   device-to-host bytes; excludes BEAM_FUSED_DECODE (see
+                                   beam_moe_forward_host) */
 #define BEAM_HOST_ASYNC   0x100u /* beam_moe_forward_host only: return once the copies and the
                                    forward are queued, without waiting (see beam_moe_forward_host
                                    and beam_moe_host_wait) */
@@ -152,8 +153,9 @@ beam_status_t beam_moe_forward(beam_moe_t *h, const void *x_dev, int32_t T, floa
 /*
  * beam_moe_forward with host buffers: copies x_host (T*D elements of the storage type) to a
  * handle-owned device buffer, runs the forward and copies y back to y_host (T*D float32, or
- * with BEAM_HOST_Y_BF16 T*D bf16: the float32 y rounded to nearest even on the device before
- * the copy), then synchronises `stream`.  Pinned host memory gives full-bandwidth copies.
+ * with BEAM_HOST_Y_BF16 T*D bf16: the combine stores y rounded to nearest even, as under
+ * BEAM_Y_BF16, and the bf16 rows are copied; excludes BEAM_FUSED_DECODE), then synchronises
+ * `stream`.  Pinned host memory gives full-bandwidth copies.
  * BEAM_HOST_PIPELINE (T >= 1024; flags may add BEAM_MASK_OFF, BEAM_PATH_*, BEAM_NO_GRAPH and
  * BEAM_HOST_Y_BF16):
  * the batch runs as 2 to 4 chunks of whole segments (about 1366 tokens each); chunk c's x copy,
@@ -214,12 +216,11 @@ beam_status_t beam_moe_get_routing(beam_moe_t *h, int32_t *topk_id, float *gate,
  * stage_launches[BEAM_N_STAGES] (either may be NULL), sets *n_forwards, and switches timing
  * off.  beam_moe_stage_name(i) names stage i ("" when out of range).  On the tensor-core path
  * the shared experts' GEMMs run on a second stream, overlapping the routing; they are timed
- * under stages of their own (tc_shared_gateup, tc_shared_down, shared_swiglu_finish), so that
- * each stage's time covers the work of one problem.  A fused decode forward is one launch,
- * timed as the stage fused_decode; the per-chunk statistics of a pipelined host call as
- * chunk_stats, and the rounding of y to bf16 of a BEAM_HOST_Y_BF16 host call as y_bf16.
+ * under stages of their own (tc_shared_gateup, tc_shared_down), so that each stage's time
+ * covers the work of one problem.  A fused decode forward is one launch, timed as the stage
+ * fused_decode; the per-chunk statistics of a pipelined host call as chunk_stats.
  */
-#define BEAM_N_STAGES 20
+#define BEAM_N_STAGES 17
 beam_status_t beam_moe_profile_begin(beam_moe_t *h, int32_t max_forwards);
 beam_status_t beam_moe_profile_end(beam_moe_t *h, float *stage_ms, int32_t *stage_launches,
                                    int32_t *n_forwards);

@@ -113,7 +113,8 @@ def test_stage_table_matches_the_header(lib):
     names = [lib.beam_moe_stage_name(i).decode() for i in range(_lib.BEAM_N_STAGES)]
     assert all(names) and len(set(names)) == len(names)
     assert lib.beam_moe_stage_name(_lib.BEAM_N_STAGES) == b""
-    assert names[-4:] == ["route_grad", "route_dw", "chunk_stats", "y_bf16"]
+    assert names[-4:] == ["fused_decode", "route_grad", "route_dw", "chunk_stats"]
+    assert "swiglu_finish" not in names and "shared_swiglu_finish" not in names
 
 
 def test_missing_library_fails_loudly(tmp_path):

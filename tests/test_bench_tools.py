@@ -47,7 +47,6 @@ def test_layer_work_joint_launches_carry_both_problems():
     jnt, _ = bench.layer_work(spec, T, STATS, tc_path=True, joint=True)
     for s in ("gateup", "down"):
         assert jnt["tc_" + s] == _sum(sep["tc_" + s], sep["tc_shared_" + s])
-    assert jnt["swiglu_finish"]["bytes"] == sep["swiglu_finish"]["bytes"] + sep["shared_swiglu_finish"]["bytes"]
 
 
 def test_grad_work_counts_each_array_once():
@@ -83,7 +82,6 @@ def test_layer_work_without_shared_experts_has_empty_shared_problem():
     w, _ = bench.layer_work(spec, 64, STATS)
     assert w["tc_shared_gateup"] == {"bytes": 0, "flops": 0}
     assert w["tc_shared_down"] == {"bytes": 0, "flops": 0}
-    assert w["shared_swiglu_finish"] == {"bytes": 0, "flops": 0}
 
 
 def _ncu_csv(path, rows):

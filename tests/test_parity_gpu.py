@@ -296,7 +296,7 @@ def test_profiling_stages_count_every_launch(T):
     for s_ in expect:
         assert stages[s_][1] == n, (s_, stages[s_])
         assert stages[s_][0] > 0
-    absent = ["swiglu_finish", "shared_swiglu_finish"] + (["tc_shared_gateup", "tc_shared_down"] if split else [])
+    absent = ["tc_shared_gateup", "tc_shared_down"] if split else []
     for s_ in absent:
         assert s_ not in stages, (s_, stages)
     layer.close()
@@ -712,12 +712,12 @@ def test_host_call_forms_interleaved():
         layer.forward_host(xs[0], out[0], pipeline=True, asynchronous=True)
     layer.close()
 
-@pytest.mark.parametrize("T,pipeline", [(1500, True), (1500, False), (3, False)],
-                         ids=["pipelined", "plain", "decode"])
-def test_host_bf16_output(T, pipeline):
-    """BEAM_HOST_Y_BF16: the host receives y rounded to bf16 on the device.  The bits are the
+@pytest.mark.parametrize("T,form", [(1500, "pipeline"), (1500, "plain"), (3, "plain"), (1500, "async")],
+                         ids=["pipelined", "plain", "decode", "async"])
+def test_host_bf16_output(T, form):
+    """BEAM_HOST_Y_BF16: the host receives y rounded to bf16 by the combine.  The bits are the
     float32 y of the same call form, rounded to nearest even (torch's conversion), so the
-    output loses nothing beyond that rounding."""
+    output loses nothing beyond that rounding; the fused decode launch is refused with it."""
     from dynamic_expert_routing_b200 import BeamMoE
     spec = _small(n_shared=1, d_ff_shared=128)
     w = synth.make_layer(spec, keep_rate=0.5)
@@ -725,9 +725,18 @@ def test_host_bf16_output(T, pipeline):
     x = synth.make_tokens(spec, T, seed=23).pin_memory()
     y32 = torch.full((T, spec.d_model), float("nan"), dtype=torch.float32).pin_memory()
     y16 = torch.full((T, spec.d_model), float("nan"), dtype=torch.bfloat16).pin_memory()
-    layer.forward_host(x, y32, pipeline=pipeline)
-    layer.forward_host(x, y16, pipeline=pipeline)
+    pipeline, asynchronous = form == "pipeline", form == "async"
+    layer.forward_host(x, y32, pipeline=pipeline, asynchronous=asynchronous)
+    layer.forward_host(x, y16, pipeline=pipeline, asynchronous=asynchronous)
+    layer.host_wait()
     assert torch.equal(y16, y32.to(torch.bfloat16))
     with pytest.raises(ValueError):
         layer.forward_host(x, torch.empty((T, spec.d_model), dtype=torch.float16), pipeline=pipeline)
+    if form == "plain":
+        from dynamic_expert_routing_b200 import BeamError, _lib
+        import ctypes
+        with pytest.raises(BeamError):
+            _lib.check(_lib.load().beam_moe_forward_host(
+                layer._h, ctypes.c_void_p(x.data_ptr()), T, ctypes.c_void_p(y16.data_ptr()),
+                _lib.BEAM_HOST_Y_BF16 | _lib.BEAM_FUSED_DECODE, None))
     layer.close()
