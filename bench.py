@@ -910,8 +910,8 @@ def _run_ours(args):
                     "y_bf16": None if e2e16_ms is None else {
                         "value": round(job_throughput(T, world, e2e16_ms), 2),
                         "d2h_bytes_per_step": T * spec.d_model * 2,
-                        "call": "the same asynchronous calls with a bf16 y_host (BEAM_HOST_Y_BF16: y "
-                                "rounded to bf16 on the device before the copy)"}},
+                        "call": "the same asynchronous calls with a bf16 y_host (BEAM_HOST_Y_BF16: the "
+                                "combine stores y rounded to bf16, and the bf16 rows are copied)"}},
             "gpu_launches": launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
