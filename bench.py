@@ -12,6 +12,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import functools
 import hashlib
 import json
 import math
@@ -754,6 +755,9 @@ def _run_ours(args):
 
     name = args.workload
     spec, T, keep, layer, x = build_layer(torch, name, device)
+    if args.path:
+        # every forward of this run on one expert path (for profiling that path's kernels)
+        layer.forward = functools.partial(type(layer).forward, layer, path=args.path)
     y = torch.empty((T, spec.d_model), dtype=torch.float32, device=device)
     mask_off = keep is None
     sb = step_bytes(torch, layer, x, y, spec, T, mask_off)
@@ -885,7 +889,8 @@ def _run_ours(args):
             "vs_baseline": None,
             "dtype": "bf16" if spec.storage == "bf16" else "f32",
             "data": "synthetic (seeded; random-init weights of the layer shape)",
-            "config": workload_config(spec, T, keep, world, sb),
+            "config": dict(workload_config(spec, T, keep, world, sb),
+                           **({"expert_path": args.path} if args.path else {})),
             "routing_stats": {"avg_k": round(st["avg_k"], 4), "l_reg": round(st["l_reg"], 6),
                               "n_active_experts": st["n_active_experts"], "n_kept": st["n_kept"],
                               "n_tokens_all_masked": st["n_tokens_all_masked"]},
@@ -1065,6 +1070,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-points", action="store_true", help="skip the supplementary points")
+    ap.add_argument("--path", choices=["stream", "tensor"], default=None,
+                    help="run the workload's forwards on this expert path (default: the library's choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU work")
     ap.add_argument("--sweep", action="store_true",

@@ -1153,9 +1153,9 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
             a.h = h->hbuf; a.hsh = h->hsh; a.yperm = h->yperm; a.ysh = h->ysh;
             a.groups = h->groups; a.n_groups = h->zero_int; a.err = &h->dstats->err;
             a.D = D; a.F = h->F; a.Fsh = h->Fsh; a.T = T_;
-            BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(h->num_sms), dim3(256),
+            BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(h->num_sms), dim3(kStreamThreads),
                              (size_t)stream_gateup_smem(), st, a));
-            BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(h->num_sms), dim3(256),
+            BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(h->num_sms), dim3(kStreamThreads),
                              (size_t)stream_down_smem(), st, a));
             ysh_out.base = h->ysh; ysh_out.f16 = false;
         }
@@ -1174,10 +1174,10 @@ static beam_status_t forward_impl(beam_moe* h, const T* x, int T_, float* y, uin
         a.h = h->hbuf; a.hsh = h->hsh; a.yperm = h->yperm; a.ysh = h->ysh;
         a.groups = h->groups; a.n_groups = h->n_groups; a.err = &h->dstats->err;
         a.D = D; a.F = h->F; a.Fsh = h->Fsh; a.T = T_;
-        const int grid = h->num_sms;  // one 256-thread CTA per SM (shared-memory rings)
-        BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(grid), dim3(256),
+        const int grid = h->num_sms;  // one CTA per SM (shared-memory rings)
+        BEAM_CUDA(launch(h, ST_STREAM_GATEUP, stream_gateup_kernel<T, TH>, dim3(grid), dim3(kStreamThreads),
                          (size_t)stream_gateup_smem(), st, a));
-        BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(grid), dim3(256),
+        BEAM_CUDA(launch(h, ST_STREAM_DOWN, stream_down_kernel<TH>, dim3(grid), dim3(kStreamThreads),
                          (size_t)stream_down_smem(), st, a));
         yr.base = h->yperm; yr.f16 = false;
         if (h->Fsh) { ysh_out.base = h->ysh; ysh_out.f16 = false; }

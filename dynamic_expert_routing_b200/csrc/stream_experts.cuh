@@ -17,9 +17,14 @@
 
 namespace beam {
 
-constexpr int kStreamMT = 8;   // tokens per pass over a weight row
-constexpr int kStreamR = 16;   // weight rows per work item (2 per warp, 8 warps)
-constexpr int kStreamNR = 2;   // rows a warp streams at once
+constexpr int kStreamMT = 8;       // tokens per pass over a weight row
+constexpr int kStreamR = 16;       // weight rows per work item
+constexpr int kStreamWarps = 16;   // warps per CTA (one CTA per SM)
+constexpr int kStreamThreads = 32 * kStreamWarps;
+constexpr int kStreamNR = kStreamR / kStreamWarps;   // rows a warp streams at once
+constexpr int kGuStreams = 2 * kStreamNR;            // gate/up: a gate and an up row per row
+constexpr int kDnStreams = kStreamNR;                // down: one weight row per output row
+static_assert(kStreamNR * kStreamWarps == kStreamR, "items split evenly over the warps");
 
 struct StreamArgs {
     const void* xperm;   // routed activations, row g.row0 + i = i-th kept pair of group g
@@ -144,26 +149,26 @@ __device__ __forceinline__ void ring_drain(uint32_t bars, long long issued, long
     }
 }
 
-constexpr int kGuSegBytes = 1024;    // bytes per row segment, gate/up kernel (4 rows per stage)
-constexpr int kDnSegBytes = 2048;    // bytes per row segment, down kernel (2 rows per stage)
+constexpr int kGuSegBytes = 1024;    // bytes per row segment, gate/up kernel (kGuStreams per stage)
+constexpr int kDnSegBytes = 2048;    // bytes per row segment, down kernel (kDnStreams per stage)
 constexpr int kXTileBytes = 65536;   // activation tile of the gate/up kernel
 constexpr int kHTileBytes = 81920;   // H tile of the down kernel
 
 __host__ __device__ constexpr int stream_gateup_smem() {
-    return kXTileBytes + 8 * kRingNS * 4 * kGuSegBytes + 8 * kRingNS * 8 + 16;
+    return kXTileBytes + kStreamWarps * kRingNS * kGuStreams * kGuSegBytes + kStreamWarps * kRingNS * 8 + 16;
 }
 __host__ __device__ constexpr int stream_down_smem() {
-    return kHTileBytes + 8 * kRingNS * 2 * kDnSegBytes + 8 * kRingNS * 8 + 16;
+    return kHTileBytes + kStreamWarps * kRingNS * kDnStreams * kDnSegBytes + kStreamWarps * kRingNS * 8 + 16;
 }
 
 // Producer cursor of the gate/up kernel: position (item, pass p0, segment c) in the warp's
-// segment stream, with the item's four weight rows.  The consumer walks the same sequence,
+// segment stream, with the warp's kGuStreams weight rows of the item.  The consumer walks the same sequence,
 // so the producer can run kRingNS segments ahead across item and pass boundaries.
 template <typename T>
 struct GuCursor {
     long item;
     int p0, c, m;
-    const T* rows[4];
+    const T* rows[kGuStreams];
     bool valid;
 };
 
@@ -183,20 +188,20 @@ __device__ __forceinline__ void gu_rows(const StreamArgs& a, const ItemView& v, 
 }
 
 // H[i][f] = silu(sum_d Wg[f][d] x_i[d]) * (sum_d Wu[f][d] x_i[d]) for the group's tokens i.
-// T: storage type of x and the gate/up weights; TH: type of H.  Each warp owns two
-// intermediate rows of an item (four weight streams: gate f, up f, gate f+1, up f+1).
+// T: storage type of x and the gate/up weights; TH: type of H.  Each warp owns kStreamNR
+// intermediate rows of an item (kGuStreams weight streams: gate f, up f, ...).
 template <typename T, typename TH>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kStreamThreads, 1)
 stream_gateup_kernel(StreamArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     constexpr int VN = Vec<T>::N;
     constexpr int SEG = kGuSegBytes / (int)sizeof(T);
-    constexpr int STAGE = 4 * kGuSegBytes;
+    constexpr int STAGE = kGuStreams * kGuSegBytes;
     T* xs = reinterpret_cast<T*>(smem_raw);
     unsigned char* ring_p = smem_raw + kXTileBytes;
-    uint64_t* bars_p = reinterpret_cast<uint64_t*>(ring_p + 8 * kRingNS * STAGE);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_p + 8 * kRingNS);
+    uint64_t* bars_p = reinterpret_cast<uint64_t*>(ring_p + kStreamWarps * kRingNS * STAGE);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_p + kStreamWarps * kRingNS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t ring = smem_addr(ring_p) + (uint32_t)(warp * kRingNS * STAGE);
     const uint32_t bars = smem_addr(bars_p) + (uint32_t)(warp * kRingNS * 8);
@@ -238,8 +243,8 @@ stream_gateup_kernel(StreamArgs a)
         if (!ok || !pc.valid) return;
         if (lane == 0) {
             ring_release();
-            ring_issue<T, 4>(ring, bars, STAGE, kGuSegBytes, k_issue, pc.rows, pc.c, SEG,
-                             min(SEG, D - pc.c * SEG));
+            ring_issue<T, kGuStreams>(ring, bars, STAGE, kGuSegBytes, k_issue, pc.rows, pc.c, SEG,
+                                      min(SEG, D - pc.c * SEG));
         }
         ++k_issue;
         if (++pc.c == nseg) {
@@ -267,9 +272,9 @@ stream_gateup_kernel(StreamArgs a)
                 cached = src;
                 cached_rows = mp;
             }
-            float acc[4][kStreamMT];
+            float acc[kGuStreams][kStreamMT];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < kGuStreams; ++q)
 #pragma unroll
                 for (int i = 0; i < kStreamMT; ++i) acc[q][i] = 0.f;
             for (int c = 0; c < nseg && ok; ++c) {
@@ -280,9 +285,9 @@ stream_gateup_kernel(StreamArgs a)
                 const unsigned char* st = ring_g + (k % kRingNS) * STAGE;
                 const int len = min(SEG, D - c * SEG);
                 for (int e = lane * VN; e < len; e += 32 * VN) {
-                    float w[4][VN];
+                    float w[kGuStreams][VN];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
+                    for (int q = 0; q < kGuStreams; ++q)
                         Vec<T>::widen(*reinterpret_cast<const uint4*>(st + q * kGuSegBytes + e * sizeof(T)), w[q]);
 #pragma unroll
                     for (int i = 0; i < kStreamMT; ++i) {
@@ -290,7 +295,7 @@ stream_gateup_kernel(StreamArgs a)
                             float xv[VN];
                             Vec<T>::widen(*reinterpret_cast<const uint4*>(xs + (size_t)i * D + c * SEG + e), xv);
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
+                            for (int q = 0; q < kGuStreams; ++q) {
                                 float sacc = 0.f;
 #pragma unroll
                                 for (int j = 0; j < VN; ++j) sacc = fmaf(w[q][j], xv[j], sacc);
@@ -335,23 +340,23 @@ __device__ __forceinline__ int down_chunk(int mp, int SEG) {
     return max(SEG, (kHTileBytes / (mp * (int)sizeof(T))) / SEG * SEG);
 }
 
-// Y[i][j] = sum_f Wd[j][f] H[i][f] for the group's tokens i.  Each warp owns two output rows
-// of an item (two weight streams).  H is staged in shared memory in chunks of up to
+// Y[i][j] = sum_f Wd[j][f] H[i][f] for the group's tokens i.  Each warp owns kDnStreams
+// output rows of an item (one weight stream each).  H is staged in shared memory in chunks of up to
 // kHTileBytes; the producer cursor runs across chunk, pass and item boundaries, so the next
 // weight segments are already in flight while a chunk of H is being staged.
 // T: type of H and of the down weights.
 template <typename T>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kStreamThreads, 1)
 stream_down_kernel(StreamArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     constexpr int VN = Vec<T>::N;
     constexpr int SEG = kDnSegBytes / (int)sizeof(T);
-    constexpr int STAGE = 2 * kDnSegBytes;
+    constexpr int STAGE = kDnStreams * kDnSegBytes;
     T* hs = reinterpret_cast<T*>(smem_raw);
     unsigned char* ring_p = smem_raw + kHTileBytes;
-    uint64_t* bars_p = reinterpret_cast<uint64_t*>(ring_p + 8 * kRingNS * STAGE);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_p + 8 * kRingNS);
+    uint64_t* bars_p = reinterpret_cast<uint64_t*>(ring_p + kStreamWarps * kRingNS * STAGE);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars_p + kStreamWarps * kRingNS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t ring = smem_addr(ring_p) + (uint32_t)(warp * kRingNS * STAGE);
     const uint32_t bars = smem_addr(bars_p) + (uint32_t)(warp * kRingNS * 8);
@@ -374,7 +379,7 @@ stream_down_kernel(StreamArgs a)
     struct {
         long item;
         int p0, c0, c, m, FF, cap;
-        const T* rows[2];
+        const T* rows[kDnStreams];
         bool valid;
     } pc;
     pc.item = blockIdx.x; pc.p0 = 0; pc.c0 = 0; pc.c = 0; pc.m = 0; pc.FF = 0; pc.cap = SEG;
@@ -388,8 +393,8 @@ stream_down_kernel(StreamArgs a)
             const int j0 = v.rb * kStreamR + warp * kStreamNR;
             pc.m = v.m;
             pc.FF = v.FF;
-            pc.rows[0] = wbase + (size_t)j0 * v.FF;
-            pc.rows[1] = wbase + (size_t)(j0 + 1) * v.FF;
+#pragma unroll
+            for (int q = 0; q < kDnStreams; ++q) pc.rows[q] = wbase + (size_t)(j0 + q) * v.FF;
             pc.p0 = 0; pc.c0 = 0; pc.c = 0;
             pc.cap = down_chunk<T>(min(kStreamMT, pc.m), SEG);
         }
@@ -401,10 +406,12 @@ stream_down_kernel(StreamArgs a)
         const int fl = min(pc.cap, pc.FF - pc.c0);
         const int nseg = (fl + SEG - 1) / SEG;
         if (lane == 0) {
-            const T* crow[2] = {pc.rows[0] + pc.c0, pc.rows[1] + pc.c0};
+            const T* crow[kDnStreams];
+#pragma unroll
+            for (int q = 0; q < kDnStreams; ++q) crow[q] = pc.rows[q] + pc.c0;
             ring_release();
-            ring_issue<T, 2>(ring, bars, STAGE, kDnSegBytes, k_issue, crow, pc.c, SEG,
-                             min(SEG, fl - pc.c * SEG));
+            ring_issue<T, kDnStreams>(ring, bars, STAGE, kDnSegBytes, k_issue, crow, pc.c, SEG,
+                                      min(SEG, fl - pc.c * SEG));
         }
         ++k_issue;
         if (++pc.c == nseg) {
@@ -429,9 +436,9 @@ stream_down_kernel(StreamArgs a)
             const int mp = min(kStreamMT, v.m - p0);
             const int cap = down_chunk<T>(mp, SEG);
             const T* hsrc = static_cast<const T*>(v.hrow) + (size_t)p0 * FF;
-            float acc[2][kStreamMT];
+            float acc[kDnStreams][kStreamMT];
 #pragma unroll
-            for (int q = 0; q < 2; ++q)
+            for (int q = 0; q < kDnStreams; ++q)
 #pragma unroll
                 for (int i = 0; i < kStreamMT; ++i) acc[q][i] = 0.f;
             for (int c0 = 0; c0 < FF; c0 += cap) {
@@ -453,9 +460,9 @@ stream_down_kernel(StreamArgs a)
                     const unsigned char* st = ring_g + (k % kRingNS) * STAGE;
                     const int len = min(SEG, fl - c * SEG);
                     for (int e = lane * VN; e < len; e += 32 * VN) {
-                        float w[2][VN];
+                        float w[kDnStreams][VN];
 #pragma unroll
-                        for (int q = 0; q < 2; ++q)
+                        for (int q = 0; q < kDnStreams; ++q)
                             Vec<T>::widen(*reinterpret_cast<const uint4*>(st + q * kDnSegBytes + e * sizeof(T)), w[q]);
 #pragma unroll
                         for (int i = 0; i < kStreamMT; ++i) {
@@ -463,7 +470,7 @@ stream_down_kernel(StreamArgs a)
                                 float hv[VN];
                                 Vec<T>::widen(*reinterpret_cast<const uint4*>(hs + (size_t)i * cap + c * SEG + e), hv);
 #pragma unroll
-                                for (int q = 0; q < 2; ++q) {
+                                for (int q = 0; q < kDnStreams; ++q) {
                                     float sacc = 0.f;
 #pragma unroll
                                     for (int j = 0; j < VN; ++j) sacc = fmaf(w[q][j], hv[j], sacc);
@@ -479,7 +486,7 @@ stream_down_kernel(StreamArgs a)
             }
             if (!ok) continue;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
+            for (int q = 0; q < kDnStreams; ++q) {
 #pragma unroll
                 for (int i = 0; i < kStreamMT; ++i) {
                     if (i < mp) {
