@@ -125,3 +125,30 @@ def test_missing_library_fails_loudly(tmp_path):
             _lib.load(str(tmp_path / "nope.so"))
         finally:
             _lib._lib = None
+
+
+def test_binding_constants_match_the_header():
+    """Every flag, status code, dtype and size the header defines has the same value in the
+    binding, so a flag added on one side only fails here."""
+    from dynamic_expert_routing_b200 import _lib
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    found = {}
+    for name, val, shift in re.findall(r"#define\s+(BEAM_[A-Z0-9_]+)\s+\(?(0x[0-9a-fA-F]+|\d+)u?(?:\s*<<\s*(\d+))?", text):
+        found[name] = int(val, 0) << (int(shift) if shift else 0)
+    for name, val in re.findall(r"\b(BEAM_[A-Z0-9_]+)\s*=\s*(\d+)", text):
+        found[name] = int(val)
+    found.pop("BEAM_MOE_H", None)
+    assert len(found) >= 20
+    for name, val in found.items():
+        assert getattr(_lib, name) == val, name
+
+
+def test_output_dtype_flag_of_the_binding():
+    """forward(out=...) takes a CUDA float32 or bfloat16 tensor of at least T*D values and sets
+    BEAM_Y_BF16 for bfloat16; anything else is refused before the library is called."""
+    import torch
+    from dynamic_expert_routing_b200.layer import _y_flag
+    with pytest.raises(ValueError):
+        _y_flag(torch.empty((4, 8)), 4, 8)                       # host memory
+    with pytest.raises(ValueError):
+        _y_flag(torch.empty((4, 8), dtype=torch.float16), 4, 8)  # neither float32 nor bf16
